@@ -1,0 +1,209 @@
+"""CPU oracle for Reduced Matrix Multiplication (RMM) -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+legs of ``bench.py`` may import this package.  The product library never
+loads it, and it never loads the product library: the two share nothing but
+the seeded input generators of ``rmm_synth``.
+
+The arithmetic lives in ``rmm_oracle.c`` (plain single-threaded C, fp64
+accumulation); this module compiles it with gcc on first use (``build()``)
+and marshals numpy arrays of bf16 bit patterns (uint16) into it.
+
+Every function follows the method as the pages describe it:
+
+* Reduced Matrix Multiplication: Input-Adaptive Matrix-Product Reduction for
+  LLM Inference (Lan, Li, Zhou), abstract -- keep informative slices along the
+  contraction dimension at retention ratio r;
+* Input-adaptive matrix-product reduction for LLM inference (cf-1.com post),
+  §2 (Y ~= X @ W_sub^T), §5.1-§5.3 (score, top-k, gather + smaller product),
+  §6.1 (top-k then sort; keep ratio 1 reproduces the full product),
+  §3.3 (reduce inside attention heads).
+
+Pins (tests/test_oracle_pins.py): closed forms for k, brute force over all
+subsets for the kept set on H <= 12, r = 1 against a library dense product,
+kept + dropped = full, exact scaling, attention against a library softmax
+attention on a Q whose dropped head dimensions are zeroed, and hand-worked
+golden fixtures under tests/golden/.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rmm_oracle.c")
+_LIB = os.path.join(_HERE, "_build", "liboracle.so")
+
+ERR_ARG = -1
+ERR_NONFINITE = -2
+ERR_NOMEM = -3
+
+_u16p = np.ctypeslib.ndpointer(dtype=np.uint16, flags="C_CONTIGUOUS")
+_i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+_f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+
+
+def build(force: bool = False) -> str:
+    """Compile rmm_oracle.c into _build/liboracle.so (plain gcc, no fast-math, no FMA contraction)."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    os.makedirs(os.path.dirname(_LIB), exist_ok=True)
+    tmp = _LIB + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+           _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    L, D, I, P = ctypes.c_long, ctypes.c_double, ctypes.c_int, ctypes.c_void_p
+    lib.oracle_k_for.argtypes = [L, D]
+    lib.oracle_k_for.restype = I
+    lib.oracle_score.argtypes = [_u16p, L, L, _u16p]
+    lib.oracle_score.restype = I
+    lib.oracle_select.argtypes = [_u16p, L, L, _i32p]
+    lib.oracle_select.restype = I
+    lib.oracle_reduced_product.argtypes = [_u16p, _u16p, L, L, L, _i32p, L, P, L, _f64p]
+    lib.oracle_reduced_product.restype = I
+    lib.oracle_linear.argtypes = [_u16p, _u16p, L, L, L, D, P, L, _f64p, _i32p]
+    lib.oracle_linear.restype = I
+    lib.oracle_attention.argtypes = [_u16p, _u16p, _u16p, L, L, L, L, L, L, L, I, D, I, P, L,
+                                     _f64p, _i32p]
+    lib.oracle_attention.restype = I
+    lib.oracle_rmsnorm.argtypes = [_u16p, L, L, D, _f64p]
+    lib.oracle_rmsnorm.restype = I
+    lib.oracle_swiglu.argtypes = [_u16p, _u16p, L, _f64p]
+    lib.oracle_swiglu.restype = I
+    _lib = lib
+    return lib
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise OracleError(f"{what} failed with code {rc}")
+
+
+def _bits(a) -> np.ndarray:
+    """Accept a bf16 torch tensor or a uint16 numpy array; return contiguous uint16 bits."""
+    if isinstance(a, np.ndarray):
+        assert a.dtype == np.uint16
+        return np.ascontiguousarray(a)
+    import torch  # local: the oracle itself needs only numpy
+
+    assert a.dtype == torch.bfloat16
+    return a.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _rows(rows):
+    if rows is None:
+        return None, 0, None
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    return r.ctypes.data_as(ctypes.c_void_p), len(r), r
+
+
+def k_for(H: int, r: float) -> int:
+    """k = ceil(r*H) clamped to [1, H]; -1 for r outside (0, 1]."""
+    return int(_load().oracle_k_for(int(H), float(r)))
+
+
+def score(X) -> np.ndarray:
+    """s[h] = max_t |X[t,h]| as the bf16 magnitude key (uint16)."""
+    x = _bits(X)
+    T, H = x.shape
+    s = np.zeros(H, dtype=np.uint16)
+    _check(_load().oracle_score(x, T, H, s), "oracle_score")
+    return s
+
+
+def select(s, k: int) -> np.ndarray:
+    """Top-k of s under (score desc, index asc), in ascending index order (int32)."""
+    s = np.ascontiguousarray(np.asarray(s, dtype=np.uint16))
+    idx = np.zeros(int(k), dtype=np.int32)
+    _check(_load().oracle_select(s, len(s), int(k), idx), "oracle_select")
+    return idx
+
+
+def reduced_product(X, W, idx, rows=None) -> np.ndarray:
+    """Y[r, n] = sum_{j} X[t_r, idx_j] * W[n, idx_j] in fp64.  W is [N, H]."""
+    x, w = _bits(X), _bits(W)
+    T, H = x.shape
+    N = w.shape[0]
+    assert w.shape[1] == H
+    idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int32))
+    rp, nr, _keep = _rows(rows)
+    Y = np.zeros((nr if rows is not None else T, N), dtype=np.float64)
+    _check(_load().oracle_reduced_product(x, w, T, H, N, idx, len(idx), rp, nr, Y),
+           "oracle_reduced_product")
+    return Y
+
+
+def linear(X, W, r: float, rows=None):
+    """(Y fp64 [nrows, N], idx int32 [k]) of the reduced linear map Y ~= X[:,S] W[:,S]^T."""
+    x, w = _bits(X), _bits(W)
+    T, H = x.shape
+    N = w.shape[0]
+    k = k_for(H, r)
+    if k < 1:
+        raise OracleError("r must lie in (0, 1]")
+    rp, nr, _keep = _rows(rows)
+    Y = np.zeros((nr if rows is not None else T, N), dtype=np.float64)
+    idx = np.zeros(k, dtype=np.int32)
+    _check(_load().oracle_linear(x, w, T, H, N, float(r), rp, nr, Y, idx), "oracle_linear")
+    return Y, idx
+
+
+def attention(Q, K, V, k: int, causal: bool = True, scale: float | None = None,
+              per_query_head: bool = False, t_rows=None):
+    """Reduced attention.  Q [B,Hq,T,d], K/V [B,Hkv,L,d] (bf16).
+
+    Returns (O fp64 [B,Hq,nrows,d], idx int32 [B,Hkv|Hq,k]).
+    """
+    q, kk, v = _bits(Q), _bits(K), _bits(V)
+    B, Hq, T, d = q.shape
+    _, Hkv, L, _ = kk.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rp, nr, _keep = _rows(t_rows)
+    nrows = nr if t_rows is not None else T
+    O = np.zeros((B, Hq, nrows, d), dtype=np.float64)
+    nsets = Hq if per_query_head else Hkv
+    idx = np.zeros((B, nsets, int(k)), dtype=np.int32)
+    _check(_load().oracle_attention(q, kk, v, B, Hq, Hkv, T, L, d, int(k), int(bool(causal)),
+                                    float(scale), int(bool(per_query_head)), rp, nr, O, idx),
+           "oracle_attention")
+    return O, idx
+
+
+def rmsnorm(x, eps: float = 1e-5) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) row-wise (norm weight 1), fp64."""
+    b = _bits(x)
+    T, H = b.shape
+    y = np.zeros((T, H), dtype=np.float64)
+    _check(_load().oracle_rmsnorm(b, T, H, float(eps), y), "oracle_rmsnorm")
+    return y
+
+
+def swiglu(g, u) -> np.ndarray:
+    """silu(g) * u elementwise, fp64."""
+    gb, ub = _bits(g), _bits(u)
+    assert gb.shape == ub.shape
+    out = np.zeros(gb.shape, dtype=np.float64)
+    _check(_load().oracle_swiglu(gb.reshape(-1), ub.reshape(-1), gb.size, out.reshape(-1)),
+           "oracle_swiglu")
+    return out

@@ -1,0 +1,292 @@
+"""Pins of the CPU oracle against facts the method and the mathematics fix.
+
+Nothing here compares the oracle with itself or retypes its formulas: every
+check goes through another route -- hand-worked golden fixtures, exhaustive
+brute force over all subsets, library dense products and library softmax
+attention (numpy), exact algebraic identities.  Each plausible mistake (a
+floor for the ceil, the wrong tie rule, a transposed weight, a dropped
+scale, an off-by-one causal mask, the wrong GQA group) fails at least one.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rmm_synth
+from input_adaptive_reduced_rmm_b200 import metrics
+
+
+def f64(t):
+    return t.to(torch.float64).numpy()
+
+
+def key_to_float(keys):
+    """bf16 magnitude keys (sign cleared) back to their float values."""
+    k = np.asarray(keys, dtype=np.uint16).astype(np.uint32) << 16
+    return k.view(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------- k = ceil(r H)
+
+def test_k_for_golden(golden):
+    g = golden("k_for.json")
+    for H, r, k in g["cases"]:
+        assert oracle.k_for(H, r) == k, (H, r)
+        assert metrics.k_for(H, r) == k, (H, r)
+    for H, r in g["rejected"]:
+        assert oracle.k_for(H, r) == -1
+
+
+def test_flop_formula_golden(golden):
+    g = golden("flops_gemm_example.json")
+    f = metrics.gemm_flops(g["m"], g["n"], g["k"])
+    assert f == g["flops_exact"]
+    assert abs(f - g["flops_quoted_approx"]) / g["flops_quoted_approx"] < 1e-3
+
+
+# ---------------------------------------------------------------- score
+
+def test_score_matches_float_brute_force():
+    X = rmm_synth.activations(9, 37, seed=11)
+    xs = X.to(torch.float64).tolist()
+    want = [max(abs(xs[t][h]) for t in range(9)) for h in range(37)]
+    got = key_to_float(oracle.score(X))
+    assert got.tolist() == want
+
+
+def test_score_signed_zero_and_ties():
+    X = rmm_synth.tie_heavy((5, 64), seed=3)
+    xs = X.to(torch.float64).tolist()
+    want = [max(abs(xs[t][h]) for t in range(5)) for h in range(64)]
+    assert key_to_float(oracle.score(X)).tolist() == want
+    z = torch.tensor([[-0.0, 0.0, -0.0]], dtype=torch.bfloat16)
+    assert oracle.score(z).tolist() == [0, 0, 0]
+
+
+def test_score_rejects_nonfinite():
+    X = torch.tensor([[1.0, float("inf")]], dtype=torch.bfloat16)
+    with pytest.raises(oracle.OracleError):
+        oracle.score(X)
+
+
+# ---------------------------------------------------------------- select
+
+def brute_force_kept_set(scores, k):
+    """The unique k-subset whose every member beats every non-member under (score desc, index asc)."""
+    H = len(scores)
+    found = []
+    for sub in itertools.combinations(range(H), k):
+        inside = set(sub)
+        ok = True
+        for a in inside:
+            for b in range(H):
+                if b in inside:
+                    continue
+                # a must beat b: larger score, or equal score and lower index
+                if not (scores[a] > scores[b] or (scores[a] == scores[b] and a < b)):
+                    ok = False
+                    break
+            if not ok:
+                break
+        if ok:
+            found.append(list(sub))
+    assert len(found) == 1, found
+    return found[0]
+
+
+@pytest.mark.parametrize("H", [1, 2, 3, 5, 7, 8, 10, 12])
+def test_select_brute_force(H):
+    rng = np.random.default_rng(H)
+    for trial in range(4):
+        if trial % 2 == 0:
+            s = rng.integers(0, 4, size=H).astype(np.uint16)  # heavy ties
+        else:
+            s = rng.integers(0, 0x7F80, size=H).astype(np.uint16)
+        for k in range(1, H + 1):
+            assert oracle.select(s, k).tolist() == brute_force_kept_set(s.tolist(), k)
+
+
+def test_select_nested_over_r():
+    X = rmm_synth.activations(4, 300, seed=5)
+    s = oracle.score(X)
+    prev = set()
+    for k in range(1, 301):
+        cur = set(oracle.select(s, k).tolist())
+        assert prev < cur and len(cur) == k
+        prev = cur
+
+
+def test_select_all_zero_and_dominant():
+    s = np.zeros(50, dtype=np.uint16)
+    for k in (1, 7, 50):
+        assert oracle.select(s, k).tolist() == list(range(k))
+    s[33] = 0x4000
+    assert oracle.select(s, 1).tolist() == [33]
+    assert oracle.select(s, 3).tolist() == [0, 1, 33]
+
+
+def test_select_output_ascending_and_size():
+    X = rmm_synth.activations(3, 777, seed=8)
+    s = oracle.score(X)
+    for r in (0.125, 0.5, 0.9, 1.0):
+        k = oracle.k_for(777, r)
+        idx = oracle.select(s, k)
+        assert len(idx) == k == math.ceil(r * 777)
+        assert np.all(np.diff(idx) > 0)
+
+
+# ---------------------------------------------------------------- reduced product
+
+def test_tiny_linear_golden(golden):
+    g = golden("tiny_linear.json")
+    X = torch.tensor(g["X"], dtype=torch.bfloat16)
+    W = torch.tensor(g["W"], dtype=torch.bfloat16)
+    for case in g["cases"]:
+        Y, idx = oracle.linear(X, W, case["r"])
+        assert idx.tolist() == case["idx"]
+        assert Y.tolist() == case["Y"]
+    t = g["ties"]
+    Xt = torch.tensor(t["X"], dtype=torch.bfloat16)
+    _, idx = oracle.linear(Xt, W, t["r"])
+    assert idx.tolist() == t["idx"]
+
+
+def test_r1_equals_library_dense_product():
+    X = rmm_synth.activations(13, 96, seed=21)
+    W = rmm_synth.weights(40, 96, seed=22)
+    Y, idx = oracle.linear(X, W, 1.0)
+    assert idx.tolist() == list(range(96))
+    ref = f64(X) @ f64(W).T
+    assert np.max(np.abs(Y - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_kept_plus_dropped_is_full():
+    X = rmm_synth.activations(7, 130, seed=31)
+    W = rmm_synth.weights(33, 130, seed=32)
+    Yk, idx = oracle.linear(X, W, 0.4)
+    drop = np.setdiff1d(np.arange(130), idx).astype(np.int32)
+    Yd = oracle.reduced_product(X, W, drop)
+    full = f64(X) @ f64(W).T
+    assert np.max(np.abs(Yk + Yd - full)) <= 1e-12 * np.max(np.abs(full))
+    # the kept set alone equals the library product of the gathered operands
+    ref = f64(X)[:, idx] @ f64(W)[:, idx].T
+    assert np.max(np.abs(Yk - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_exact_scaling_and_row_subset():
+    X = rmm_synth.activations(6, 64, seed=41)
+    W = rmm_synth.weights(20, 64, seed=42)
+    Y, idx = oracle.linear(X, W, 0.5)
+    Y2, idx2 = oracle.linear((X.float() * 2).to(torch.bfloat16), W, 0.5)
+    assert idx.tolist() == idx2.tolist()
+    assert np.array_equal(Y2, 2 * Y)
+    rows = [5, 0, 3]
+    Ys, _ = oracle.linear(X, W, 0.5, rows=rows)
+    assert np.array_equal(Ys, Y[rows])
+
+
+def test_outlier_channels_are_kept():
+    # the 2 % outlier columns (x20) dominate the max-magnitude score
+    X = rmm_synth.activations(32, 512, seed=0)
+    _, idx = oracle.linear(X, rmm_synth.weights(8, 512, seed=1), 0.5)
+    xs = f64(X)
+    colmax = np.abs(xs).max(axis=0)
+    top10 = np.argsort(-colmax, kind="stable")[:10]
+    assert set(top10.tolist()) <= set(idx.tolist())
+
+
+# ---------------------------------------------------------------- attention
+
+def numpy_attention(q, K, V, scale, causal):
+    """Library softmax attention for one head: q [T,d], K/V [L,d]."""
+    T, L = q.shape[0], K.shape[0]
+    logits = scale * (q @ K.T)
+    if causal:
+        pos = np.arange(T)[:, None] + (L - T)
+        logits = np.where(np.arange(L)[None, :] <= pos, logits, -np.inf)
+    logits = logits - logits.max(axis=1, keepdims=True)
+    p = np.exp(logits)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ V
+
+
+def test_attention_golden(golden):
+    g = golden("tiny_attention.json")
+    Q = torch.tensor(g["Q"], dtype=torch.bfloat16).reshape(1, 1, 1, 4)
+    K = torch.tensor(g["K"], dtype=torch.bfloat16).reshape(1, 1, 2, 4)
+    V = torch.tensor(g["V"], dtype=torch.bfloat16).reshape(1, 1, 2, 4)
+    O, idx = oracle.attention(Q, K, V, g["k"], causal=True, scale=1.0)
+    assert idx.reshape(-1).tolist() == g["idx"]
+    assert np.allclose(O.reshape(-1), g["O_reduced"], rtol=0, atol=1e-15)
+    O4, _ = oracle.attention(Q, K, V, 4, causal=True, scale=1.0)
+    assert np.allclose(O4.reshape(-1), g["O_full"], rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("per_head", [False, True])
+@pytest.mark.parametrize("T,L,causal", [(1, 37, True), (5, 23, True), (4, 19, False)])
+def test_attention_equals_library_attention_on_masked_q(T, L, causal, per_head):
+    B, Hq, Hkv, d, k = 2, 6, 2, 16, 6
+    Q = rmm_synth.normal((B, Hq, T, d), seed=51)
+    K = rmm_synth.normal((B, Hkv, L, d), seed=52)
+    V = rmm_synth.normal((B, Hkv, L, d), seed=53)
+    scale = 1.0 / math.sqrt(d)
+    O, idx = oracle.attention(Q, K, V, k, causal=causal, scale=scale, per_query_head=per_head)
+    q, Kf, Vf = f64(Q), f64(K), f64(V)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            heads = [h] if per_head else list(range(g * G, (g + 1) * G))
+            s = np.abs(q[b, heads]).max(axis=(0, 1))
+            order = np.lexsort((np.arange(d), -s))  # score desc, index asc
+            S = np.sort(order[:k])
+            assert idx[b, h if per_head else g].tolist() == S.tolist()
+            qm = np.zeros_like(q[b, h])
+            qm[:, S] = q[b, h][:, S]
+            ref = numpy_attention(qm, Kf[b, g], Vf[b, g], scale, causal)
+            assert np.max(np.abs(O[b, h] - ref)) <= 1e-12
+
+
+def test_attention_full_head_dim_is_standard_attention():
+    B, Hq, Hkv, T, L, d = 1, 4, 1, 3, 11, 8
+    Q = rmm_synth.normal((B, Hq, T, d), seed=61)
+    K = rmm_synth.normal((B, Hkv, L, d), seed=62)
+    V = rmm_synth.normal((B, Hkv, L, d), seed=63)
+    O, _ = oracle.attention(Q, K, V, d, causal=True)
+    for h in range(Hq):
+        ref = numpy_attention(f64(Q)[0, h], f64(K)[0, 0], f64(V)[0, 0], 1 / math.sqrt(d), True)
+        assert np.max(np.abs(O[0, h] - ref)) <= 1e-12
+
+
+def test_attention_decode_mask_is_noop_and_rows_subset():
+    Q = rmm_synth.normal((1, 4, 1, 16), seed=71)
+    K = rmm_synth.normal((1, 2, 29, 16), seed=72)
+    V = rmm_synth.normal((1, 2, 29, 16), seed=73)
+    Oc, ic = oracle.attention(Q, K, V, 8, causal=True)
+    On, inn = oracle.attention(Q, K, V, 8, causal=False)
+    assert np.array_equal(Oc, On) and np.array_equal(ic, inn)
+    Q5 = rmm_synth.normal((1, 4, 5, 16), seed=74)
+    Of, _ = oracle.attention(Q5, K, V, 8, causal=True)
+    Os, _ = oracle.attention(Q5, K, V, 8, causal=True, t_rows=[4, 1])
+    assert np.array_equal(Os, Of[:, :, [4, 1]])
+
+
+# ---------------------------------------------------------------- layer glue
+
+def test_rmsnorm_closed_form():
+    x = torch.full((2, 8), 2.0, dtype=torch.bfloat16)
+    x[1] = -0.5
+    y = oracle.rmsnorm(x, eps=1e-5)
+    assert np.allclose(y[0], 2.0 / math.sqrt(4.0 + 1e-5), rtol=0, atol=1e-15)
+    assert np.allclose(y[1], -0.5 / math.sqrt(0.25 + 1e-5), rtol=0, atol=1e-15)
+
+
+def test_swiglu_closed_form():
+    g = torch.tensor([0.0, 1.0, -2.0, 3.0], dtype=torch.bfloat16)
+    u = torch.tensor([5.0, 2.0, 1.0, -1.0], dtype=torch.bfloat16)
+    out = oracle.swiglu(g, u)
+    want = [0.0, 2.0 / (1 + math.exp(-1.0)), -2.0 / (1 + math.exp(2.0)), -3.0 / (1 + math.exp(-3.0))]
+    assert np.allclose(out, want, rtol=0, atol=1e-15)
