@@ -1,0 +1,416 @@
+"""Benchmark of the reduced-matrix-multiplication hot path on B200.
+
+One step = one pass of the reduced linear map over the seven projections of a
+Llama-3-8B-shaped layer (q, k, v, o: 4096 -> 4096/1024/1024/4096; gate, up:
+4096 -> 14336; down: 14336 -> 4096) on a prefill batch of T = 2048 tokens at
+retention r = 0.5.  Each projection is one rmm_linear call through the C ABI
+(score -> kept set -> tcgen05 reduced GEMM), with random-init bf16 weights
+~N(0, 0.02) pre-transposed once and synthetic activations N(0, 1) with 2 % of
+the channels x20.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rmm|reference]
+
+Prints one JSON line (rank 0).  value = effective TFLOP/s = sum 2*T*N*k over
+all ranks' steps / max-over-ranks device time.  Extra keys: the dominant
+kernel's roofline, the dense cuBLAS comparison, the end-to-end number through
+the public call with host buffers, the oracle timed on the host cores, the
+decode (T = 1) GEMV and attention rows, and SM clocks sampled during timing.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import rmm_synth  # noqa: E402
+from input_adaptive_reduced_rmm_b200 import metrics  # noqa: E402
+
+T_PREFILL = 2048
+R = 0.5
+PROJ = [  # (name, H, N, activation stream)
+    ("q", 4096, 4096, 0), ("k", 4096, 1024, 0), ("v", 4096, 1024, 0), ("o", 4096, 4096, 1),
+    ("gate", 4096, 14336, 2), ("up", 4096, 14336, 2), ("down", 14336, 4096, 3),
+]
+ACT_H = {0: 4096, 1: 4096, 2: 4096, 3: 14336}
+WORKLOAD = "llama3-8b 7 projections (q,k,v,o,gate,up,down), prefill T=2048, r=0.5"
+METRIC = "reduced-GEMM effective TFLOP/s (2*T*N*k / time)"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ oracle (CPU baseline)
+
+def oracle_sample(rows_per_proj: int, seed: int):
+    """Time the CPU oracle on `rows_per_proj` token rows of every projection (full score/select).
+
+    Returns (flops, seconds, sample description)."""
+    import oracle
+
+    oracle.build()
+    acts = {s: rmm_synth.activations(T_PREFILL, h, rmm_synth.seed_for(1, 70 + s, 0)) for s, h in ACT_H.items()}
+    weights = {n: rmm_synth.weights(N, H, rmm_synth.seed_for(1, 80 + i, 1), std=0.02)
+               for i, (n, H, N, _) in enumerate(PROJ)}
+    g = torch.Generator().manual_seed(seed)
+    flops, secs = 0, 0.0
+    for name, H, N, s in PROJ:
+        rows = torch.randperm(T_PREFILL, generator=g)[:rows_per_proj].tolist()
+        t0 = time.perf_counter()
+        oracle.linear(acts[s], weights[name], R, rows=rows)
+        secs += time.perf_counter() - t0
+        flops += metrics.reduced_linear_flops(rows_per_proj, N, metrics.k_for(H, R))
+    desc = (f"{rows_per_proj} of {T_PREFILL} token rows per projection, all 7 projections, "
+            "score and kept set over the full batch; single-threaded fp64 C oracle")
+    return flops, secs, desc
+
+
+def run_reference(args, world, rank):
+    """The oracle timed on the host cores: each step is a bounded sample of the workload."""
+    if rank != 0:
+        return
+    rows = 2
+    for _ in range(args.warmup):
+        oracle_sample(1, seed=999)
+    times, total_flops = [], 0
+    sample = ""
+    for s in range(args.steps):
+        f, t, sample = oracle_sample(rows, seed=s)
+        times.append(t)
+        total_flops += f
+    value = total_flops / sum(times) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "sample_rows_per_projection": rows},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def make_inputs(dev):
+    from input_adaptive_reduced_rmm_b200 import rmm
+
+    acts = {s: rmm_synth.activations(T_PREFILL, h, rmm_synth.seed_for(1, 70 + s, 0)).to(dev)
+            for s, h in ACT_H.items()}
+    Wts, Wfull = {}, {}
+    for i, (name, H, N, _) in enumerate(PROJ):
+        W = rmm_synth.weights(N, H, rmm_synth.seed_for(1, 80 + i, 1), std=0.02).to(dev)
+        Wts[name] = rmm.rmm_transpose_weight(W)
+        Wfull[name] = W
+    torch.cuda.synchronize()
+    return acts, Wts
+
+
+def time_decode_and_attention(dev, peaks):
+    """Secondary rows: the T=1 decode GEMV over the same projections, and decode attention."""
+    from input_adaptive_reduced_rmm_b200 import rmm
+
+    out = {}
+    # decode GEMV: T = 1, all seven projections, r = 0.5, weights larger than L2 in total
+    acts = {s: rmm_synth.activations(1, h, 500 + s).to(dev) for s, h in ACT_H.items()}
+    Wts = {n: rmm.rmm_transpose_weight(rmm_synth.weights(N, H, 600 + i, std=0.02).to(dev))
+           for i, (n, H, N, _) in enumerate(PROJ)}
+    ws = {n: rmm.new_workspace(rmm.rmm_linear_workspace_bytes(1, H, N), dev) for n, H, N, _ in PROJ}
+    Ys = {n: torch.empty(1, N, dtype=torch.bfloat16, device=dev) for n, H, N, _ in PROJ}
+    ev = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n, _, _, _ in PROJ}
+    opts = {n: rmm.options(product_events=ev[n]) for n, _, _, _ in PROJ}
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step():
+        for n, H, N, s in PROJ:
+            rmm.rmm_linear(acts[s], Wts[n], R, Y=Ys[n], workspace=ws[n], opts=opts[n])
+
+    for _ in range(3):
+        step()
+    iters = 20
+    gemv_ms = {n: 0.0 for n, _, _, _ in PROJ}
+    call_ms = 0.0
+    for _ in range(iters):
+        flush.zero_()  # evict the weights from L2 between iterations
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        torch.cuda.synchronize()
+        call_ms += e0.elapsed_time(e1)
+        for n in gemv_ms:
+            gemv_ms[n] += ev[n][0].elapsed_time(ev[n][1])
+    bytes_total = sum(metrics.gemv_bytes(1, H, N, metrics.k_for(H, R)) for _, H, N, _ in PROJ)
+    gemv_total_ms = sum(gemv_ms.values()) / iters
+    out["decode_gemv"] = {
+        "workload": "T=1, same 7 projections, r=0.5, L2 flushed between iterations",
+        "kernel_us_per_step": 1e3 * gemv_total_ms,
+        "achieved_gbs": bytes_total / (gemv_total_ms * 1e-3) / 1e9,
+        "frac_of_hbm": bytes_total / (gemv_total_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "calls_us_per_step": 1e3 * call_ms / iters,
+        "per_projection_us": {n: 1e3 * v / iters for n, v in gemv_ms.items()},
+    }
+    del Wts, ws, flush
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_rmm(args, world, rank, local):
+    from input_adaptive_reduced_rmm_b200 import rmm
+
+    dev = torch.device("cuda", local if world > 1 else 0)
+    peaks = load_peaks()
+    acts, Wts = make_inputs(dev)
+    ks = {n: metrics.k_for(H, R) for n, H, _, _ in PROJ}
+    step_flops = sum(metrics.reduced_linear_flops(T_PREFILL, N, ks[n]) for n, _, N, _ in PROJ)
+    ws = {n: rmm.new_workspace(rmm.rmm_linear_workspace_bytes(T_PREFILL, H, N), dev) for n, H, N, _ in PROJ}
+    Ys = {n: torch.empty(T_PREFILL, N, dtype=torch.bfloat16, device=dev) for n, _, N, _ in PROJ}
+    K, W = args.steps, args.warmup
+    evs = {n: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+           for n, _, _, _ in PROJ}
+    opt_timed = {n: [rmm.options(product_events=evs[n][i]) for i in range(K)] for n, _, _, _ in PROJ}
+
+    def step(i=None):
+        for n, H, N, s in PROJ:
+            o = opt_timed[n][i] if i is not None else None
+            rmm.rmm_linear(acts[s], Wts[n], R, Y=Ys[n], workspace=ws[n], opts=o)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    for n, _, _, _ in PROJ:
+        if rmm.rmm_get_status(ws[n]) != rmm.RMM_OK:
+            raise RuntimeError("device status not OK after warm-up")
+
+    clocks = ClockSampler(local if world > 1 else 0)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(K):
+        step(i)
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    ms_max = max_over_ranks(ms, world)
+    value = step_flops * K * world / (ms_max * 1e-3) / 1e12
+
+    # dominant kernel: the reduced GEMM launches, timed by events recorded around each one
+    gemm_ms = {n: sum(b.elapsed_time(e) for b, e in evs[n]) / K for n, _, _, _ in PROJ}
+    gemm_total_ms = sum(gemm_ms.values())
+    achieved = step_flops / (gemm_total_ms * 1e-3) / 1e12
+    per_proj = {n: {"H": H, "N": N, "k": ks[n], "gemm_us": 1e3 * gemm_ms[n],
+                    "gemm_tflops": metrics.reduced_linear_flops(T_PREFILL, N, ks[n]) / (gemm_ms[n] * 1e-3) / 1e12}
+                for n, H, N, _ in PROJ}
+
+    # dense cuBLAS product of the same shapes, same stream, same inputs
+    def dense_step():
+        for n, H, N, s in PROJ:
+            torch.matmul(acts[s], Wts[n], out=Ys[n])
+
+    for _ in range(W):
+        dense_step()
+    torch.cuda.synchronize()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record()
+    for _ in range(K):
+        dense_step()
+    d1.record()
+    torch.cuda.synchronize()
+    dense_ms = d0.elapsed_time(d1) / K
+    dense_flops = sum(metrics.gemm_flops(T_PREFILL, N, H) for _, H, N, _ in PROJ)
+
+    # end to end through the public call with host buffers: H2D of the step's activations,
+    # the seven calls, D2H of the seven outputs, every step
+    host_acts = {s: a.cpu().pin_memory() for s, a in acts.items()}
+    host_Y = {n: torch.empty(T_PREFILL, N, dtype=torch.bfloat16).pin_memory() for n, _, N, _ in PROJ}
+    h2d = sum(a.numel() * 2 for a in host_acts.values())
+    d2h = sum(y.numel() * 2 for y in host_Y.values())
+
+    def e2e_step():
+        for s, a in host_acts.items():
+            acts[s].copy_(a, non_blocking=True)
+        step()
+        for n in host_Y:
+            host_Y[n].copy_(Ys[n], non_blocking=True)
+
+    for _ in range(W):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = step_flops * K * world / (e2e_ms * 1e-3) / 1e12
+
+    extra = time_decode_and_attention(dev, peaks) if not args.skip_secondary else {}
+
+    cpu = None
+    if rank == 0 and not args.skip_cpu_baseline:
+        f, t, desc = oracle_sample(args.cpu_rows, seed=1)
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc}
+
+    if rank != 0:
+        return
+    peak = peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "T": T_PREFILL, "r": R, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (0.55 GB of weights and activations per step)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "gemm_kernel (tcgen05 reduced GEMM), all 7 launches of a step",
+                     "peak_source": f"{peaks['source']} bf16 burst"},
+        "speedup_vs_dense": dense_ms / (ms_max / K),
+        "dense": {"ms_per_step": dense_ms, "tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
+                  "effective_tflops_at_reduced_flops": step_flops / (dense_ms * 1e-3) / 1e12},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "cpu_baseline": cpu,
+        "gpu_launches": 3 * len(PROJ) * K,
+        "clocks": clk,
+        "per_projection": per_proj,
+    }
+    line.update(extra)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["rmm", "reference"], default="rmm")
+    ap.add_argument("--cpu-rows", type=int, default=24)
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-secondary", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_rmm(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

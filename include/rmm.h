@@ -1,0 +1,173 @@
+/*
+ * rmm.h -- C ABI of librmm: Reduced Matrix Multiplication (RMM) on B200 (sm_100a).
+ *
+ * The method (Reduced Matrix Multiplication: Input-Adaptive Matrix-Product
+ * Reduction for LLM Inference, Lan, Li, Zhou -- abstract): a training-free,
+ * input-adaptive reduction of each Transformer matrix product that keeps
+ * only informative slices along the contraction dimension, controlled by one
+ * retention ratio r.  For a projection Y = X W^T (X [T,H] activations,
+ * W [N,H] weights; cf-1.com post on input-adaptive matrix-product reduction,
+ * §2) the library
+ *   1. scores every contraction index h by s_h = max_t |X[t,h]| (post §5.1:
+ *      a cheap score from the current activations),
+ *   2. keeps the top k = ceil(r*H) indices S, ties going to the lower index,
+ *      emitted in ascending order (post §5.2, and the §6.1 demo's sort after
+ *      top-k),
+ *   3. computes Y ~= X[:,S] W[:,S]^T (post §5.3: the smaller dense product)
+ *      without writing any compacted copy of X or W to memory.
+ * Attention's Q K^T is reduced the same way along the head dimension (post
+ * §3.3: reduce inside heads), followed by an unreduced softmax(.) V.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are device pointers owned by the caller; the library never
+ *     allocates or frees memory and never synchronises, except
+ *     rmm_get_status().  Work is enqueued on `stream` (a cudaStream_t; NULL =
+ *     the legacy default stream) and runs asynchronously.
+ *   - bf16 tensors are passed as `void*` holding IEEE bfloat16 bit patterns,
+ *     row-major with the stated leading dimension.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and returned as RMM_ERR_INVALID_ARG / RMM_ERR_UNSUPPORTED /
+ *     RMM_ERR_WORKSPACE; a failed launch returns RMM_ERR_CUDA.
+ *   - Device-side errors (a bounded wait that ran out) are written to a status
+ *     word at the start of the workspace and read by rmm_get_status().
+ *   - Inputs must be finite; NaN or Inf in X or Q gives an unspecified kept set.
+ *   - Workspaces must be zero-filled once before first use (rmm_workspace_init
+ *     does this); the library leaves them reusable after every successful call.
+ *     One workspace must not be used by two calls that may run concurrently.
+ */
+#ifndef RMM_H_
+#define RMM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, passed opaquely so that this header needs no CUDA headers. */
+typedef void* rmm_stream_t;
+
+typedef enum {
+    RMM_OK = 0,
+    RMM_ERR_INVALID_ARG = 1, /* null pointer, bad size, r outside (0,1], misaligned pointer */
+    RMM_ERR_UNSUPPORTED = 2, /* a valid shape this build does not handle (e.g. d != 128) */
+    RMM_ERR_WORKSPACE = 3,   /* workspace null or smaller than the *_workspace_bytes() query */
+    RMM_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
+    RMM_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (reported by rmm_get_status) */
+} rmm_status;
+
+/* Optional knobs; pass NULL for the defaults. */
+typedef struct rmm_options {
+    /* Largest T that takes the split-K GEMV (decode) path; larger T takes the
+     * tcgen05 GEMM.  Default 16; valid range 0..16. */
+    int t_gemv;
+    /* Attention kept-set granularity: 0 (default) = one set per (batch, KV
+     * head) over the stacked queries of its group; 1 = one set per query head. */
+    int attn_per_query_head;
+    /* Split count of the decode GEMV; 0 = automatic. */
+    int gemv_splits;
+    /* Watchdog self-test: nonzero makes the reduced GEMM wait, with a 50 ms
+     * limit, on a barrier that nothing signals; the call then reports
+     * RMM_ERR_TIMEOUT through rmm_get_status() and leaves Y unspecified. */
+    int debug_timeout_test;
+    int reserved[4]; /* must be zero */
+    /* Optional pair of cudaEvent_t handles (NULL: none) recorded on the
+     * stream immediately before and after the reduced-product kernel (GEMV or
+     * GEMM) of rmm_linear / rmm_gemm_reduced, so that a caller can time that
+     * kernel alone inside a longer sequence of calls. */
+    void* product_event_begin;
+    void* product_event_end;
+} rmm_options;
+
+/* Human-readable name of a status code (static storage). */
+const char* rmm_status_string(rmm_status status);
+
+/* Number of kept slices for retention ratio r: ceil(r*H) in double, clamped
+ * to [1, H].  Returns -1 if r is not in (0, 1] or H < 1. */
+int rmm_k_for(int H, double r);
+
+/* Zero-fill a workspace (device memory, `bytes` long) on `stream`.  Needed
+ * once before the first call that uses it. */
+rmm_status rmm_workspace_init(void* workspace, size_t bytes, rmm_stream_t stream);
+
+/* Read and clear the device status word of a workspace: synchronises
+ * `stream`, returns RMM_OK or the first device-side error recorded since the
+ * last call (RMM_ERR_TIMEOUT), or RMM_ERR_CUDA if the stream itself failed. */
+rmm_status rmm_get_status(void* workspace, rmm_stream_t stream);
+
+/* W^T from W: W bf16 [N, H] row-major -> Wt bf16 [H, N] row-major, so that a
+ * kept slice h of the weight is one contiguous row of N elements.  Done once
+ * per weight (outside any timed region).  W and Wt must not overlap. */
+rmm_status rmm_transpose_weight(const void* W, void* Wt, int N, int H, rmm_stream_t stream);
+
+/* Workspace bytes needed by rmm_linear / rmm_gemm_reduced / rmm_score /
+ * rmm_select for these sizes and options. */
+size_t rmm_linear_workspace_bytes(int T, int H, int N, const rmm_options* options);
+
+/* The reduced linear map Y ~= X[:,S] W[:,S]^T with S the k = ceil(r*H) kept
+ * slices (cf-1.com post §2, §5.1-§5.3; paper abstract).
+ *   X        bf16 [T, H] row-major (leading dimension H), 16-byte aligned
+ *   Wt       bf16 [H, N] row-major (leading dimension N) = W^T, 16-byte aligned
+ *   T        tokens, 1 <= T <= 2^20
+ *   H        contraction size, 1 <= H <= 65535
+ *   N        output features, 8 <= N, N % 8 == 0
+ *   r        retention ratio in (0, 1]
+ *   Y        bf16 [T, N] row-major, 16-byte aligned (written)
+ *   idx_out  int32 [k] or NULL: receives the kept set S, ascending
+ *   workspace, workspace_bytes: >= rmm_linear_workspace_bytes(T, H, N, options)
+ * T <= options.t_gemv runs score -> select -> split-K GEMV; larger T runs
+ * score (+ X^T) -> select -> tcgen05 GEMM.  Accumulation is fp32, Y is
+ * rounded to bf16 (round to nearest even). */
+rmm_status rmm_linear(const void* X, const void* Wt, int T, int H, int N, double r, void* Y,
+                      int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                      rmm_stream_t stream, const rmm_options* options);
+
+/* Step 1 alone: s_out[h] = max_t |X[t,h]| as the bf16 magnitude key
+ * (bit pattern with the sign cleared; -0 and +0 both give 0).  X bf16 [T, H],
+ * s_out uint32 [H].  T >= 1. */
+rmm_status rmm_score(const void* X, int T, int H, uint32_t* s_out, void* workspace,
+                     size_t workspace_bytes, rmm_stream_t stream);
+
+/* Step 2 alone: the k indices of the largest scores under (score desc, index
+ * asc), written to idx_out [k] in ascending order.  s: uint32 [H], each
+ * < 65536; 1 <= k <= H <= 65535. */
+rmm_status rmm_select(const uint32_t* s, int H, int k, int32_t* idx_out, void* workspace,
+                      size_t workspace_bytes, rmm_stream_t stream);
+
+/* Step 3 alone, for a given kept set: Y[t,n] = sum_{j<k} X[t,idx[j]] * Wt[idx[j],n].
+ * idx: int32 [k], distinct values in [0, H) (any order).  Same layouts and
+ * path choice as rmm_linear. */
+rmm_status rmm_gemm_reduced(const void* X, const void* Wt, const int32_t* idx, int k, int T,
+                            int H, int N, void* Y, void* workspace, size_t workspace_bytes,
+                            rmm_stream_t stream, const rmm_options* options);
+
+/* Workspace bytes needed by rmm_attn_qk for these sizes. */
+size_t rmm_attn_workspace_bytes(int B, int Hq, int Hkv, int T, int L, int d,
+                                const rmm_options* options);
+
+/* Reduced attention (cf-1.com post §3.3; paper abstract: attention products
+ * reduced along their contraction dimension).  For each (batch b, KV head g):
+ *   s_j = max over the group's query heads q and all t < T of |Q[b,q,t,j]|,
+ *   S_g = top-k of s (k = ceil(r*d), ties to the lower index),
+ *   logit[q,t,l] = scale * sum_{j in S_g} Q[b,q,t,j] * Kt[b,g,j,l],
+ *   O[b,q,t,:] = softmax_l(logit) . V[b,g,l,:]   (full d, fp32 softmax).
+ * Queries sit at positions L-T .. L-1; with causal != 0 query t sees keys
+ * l <= L-T+t.
+ *   Q   bf16 [B, Hq, T, d]
+ *   Kt  bf16 [B, Hkv, d, ldL]  (d-major key cache: a kept dim is one row)
+ *   V   bf16 [B, Hkv, ldL, d]
+ *   O   bf16 [B, Hq, T, d] (written)
+ *   idx_out int32 [B, Hkv, k] (or [B, Hq, k] with attn_per_query_head) or NULL
+ * Requirements: d == 128, Hq % Hkv == 0, 1 <= T <= L <= ldL, ldL % 8 == 0,
+ * 16-byte aligned pointers. */
+rmm_status rmm_attn_qk(const void* Q, const void* Kt, const void* V, int B, int Hq, int Hkv,
+                       int T, int L, int ldL, int d, double r, int causal, float scale, void* O,
+                       int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                       rmm_stream_t stream, const rmm_options* options);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RMM_H_ */

@@ -1,0 +1,370 @@
+// rmm_api.cu -- the extern "C" entry points of librmm (declared in rmm.h):
+// argument validation, workspace layout, path choice, tensor-map cache and
+// launches.  Everything here is host code; all arithmetic runs in the kernels.
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+#include <unordered_map>
+
+#include "rmm_common.cuh"
+#include "rmm_internal.h"
+
+namespace rmm {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;  // status word (int32 at offset 0) + reserved
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int num_sms_current() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    static int cache[64] = {0};
+    if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev >= 0 && dev < 64) cache[dev] = n;
+    return n;
+}
+
+const rmm_options& opts_or_default(const rmm_options* o) {
+    static const rmm_options d = {16, 0, 0, 0, {0, 0, 0, 0}, nullptr, nullptr};
+    return o ? *o : d;
+}
+
+bool opts_valid(const rmm_options* o) {
+    if (!o) return true;
+    if (o->t_gemv < 0 || o->t_gemv > kGemvMaxT) return false;
+    if (o->gemv_splits < 0) return false;
+    for (int i = 0; i < 4; ++i)
+        if (o->reserved[i] != 0) return false;
+    return true;
+}
+
+// ---------------------------------------------------------------- layout
+
+struct LinearLayout {
+    bool gemv;
+    int P;       // score partial rows
+    int ldT;     // leading dimension of X^T (GEMM path)
+    GemvPlan plan;
+    size_t part, idx, counters, partials, xt, total;
+};
+
+// Workspace layout of the reduced linear map for kept count k (k = H gives
+// the largest layout, used by the size query).
+LinearLayout linear_layout(int T, int H, int N, int k, const rmm_options& o, int sms) {
+    LinearLayout L{};
+    L.gemv = T <= o.t_gemv;
+    L.P = score_partials_for(T, H, sms);
+    size_t off = kStatusBytes;
+    L.part = off;
+    off += align_up((size_t)L.P * H * sizeof(uint16_t), kAlign);
+    L.idx = off;
+    off += align_up(((size_t)H + 2 * kGemmBK) * sizeof(int32_t), kAlign);
+    if (L.gemv) {
+        L.plan = gemv_plan(T, N, k, sms, o.gemv_splits);
+        L.counters = off;
+        off += align_up((size_t)L.plan.col_blocks * sizeof(unsigned), kAlign);
+        L.partials = off;
+        off += align_up(gemv_partials_bytes(L.plan, T, N), kAlign);
+    } else {
+        L.ldT = (T + 7) / 8 * 8;
+        L.xt = off;
+        off += align_up((size_t)H * L.ldT * sizeof(uint16_t), kAlign);
+    }
+    L.total = off;
+    return L;
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+struct MapKey {
+    const void* ptr;
+    uint64_t rows, cols, ld;
+    bool operator==(const MapKey& o) const {
+        return ptr == o.ptr && rows == o.rows && cols == o.cols && ld == o.ld;
+    }
+};
+struct MapKeyHash {
+    size_t operator()(const MapKey& k) const {
+        size_t h = std::hash<const void*>()(k.ptr);
+        h ^= std::hash<uint64_t>()(k.rows * 1000003ull + k.cols * 7919ull + k.ld) + 0x9e3779b9 + (h << 6) + (h >> 2);
+        return h;
+    }
+};
+
+// A row-gather map over a bf16 matrix [rows, cols] (leading dimension ld
+// elements): box = 1 row x 64 columns, 128-byte swizzle, out-of-range
+// elements read as zero.  Cached by (pointer, shape).
+bool row_gather_map(const void* base, uint64_t rows, uint64_t cols, uint64_t ld, CUtensorMap* out) {
+    static std::mutex mu;
+    static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+    const MapKey key{base, rows, cols, ld};
+    {
+        std::lock_guard<std::mutex> g(mu);
+        auto it = cache.find(key);
+        if (it != cache.end()) {
+            *out = it->second;
+            return true;
+        }
+    }
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    CUtensorMap m;
+    memset(&m, 0, sizeof m);
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {ld * sizeof(uint16_t)};
+    const cuuint32_t box[2] = {64, 1};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    std::lock_guard<std::mutex> g(mu);
+    if (cache.size() > 4096) cache.clear();
+    cache[key] = m;
+    *out = m;
+    return true;
+}
+
+rmm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RMM_OK : RMM_ERR_CUDA; }
+
+bool linear_args_ok(const void* X, const void* Wt, int T, int H, int N, const void* Y) {
+    if (!X || !Wt || !Y) return false;
+    if (T < 1 || T > (1 << 20) || H < 1 || H > 65535 || N < 8 || N % 8 != 0) return false;
+    if (!aligned16(X) || !aligned16(Wt) || !aligned16(Y)) return false;
+    return true;
+}
+
+// Shared tail of rmm_linear and rmm_gemm_reduced: the product on the chosen path.
+rmm_status run_product_kernel(const void* X, const void* Wt, const int32_t* idx_padded, int k,
+                              int T, int H, int N, void* Y, uint8_t* ws, const LinearLayout& L,
+                              const rmm_options& o, cudaStream_t s) {
+    int* status = reinterpret_cast<int*>(ws);
+    if (L.gemv) {
+        return cuda_status(launch_gemv(static_cast<const uint16_t*>(X), T, H,
+                                       static_cast<const uint16_t*>(Wt), N, idx_padded, k,
+                                       static_cast<uint16_t*>(Y),
+                                       reinterpret_cast<float*>(ws + L.partials),
+                                       reinterpret_cast<unsigned*>(ws + L.counters), L.plan, status,
+                                       s));
+    }
+    CUtensorMap mx, mw;
+    if (!row_gather_map(ws + L.xt, (uint64_t)H, (uint64_t)T, (uint64_t)L.ldT, &mx)) return RMM_ERR_CUDA;
+    if (!row_gather_map(Wt, (uint64_t)H, (uint64_t)N, (uint64_t)N, &mw)) return RMM_ERR_CUDA;
+    return cuda_status(launch_gemm(mx, mw, idx_padded, k, T, H, N, static_cast<uint16_t*>(Y), status,
+                                   o.debug_timeout_test, num_sms_current(), s));
+}
+
+rmm_status run_product(const void* X, const void* Wt, const int32_t* idx_padded, int k, int T,
+                       int H, int N, void* Y, uint8_t* ws, const LinearLayout& L,
+                       const rmm_options& o, cudaStream_t s) {
+    if (o.product_event_begin &&
+        cudaEventRecord(static_cast<cudaEvent_t>(o.product_event_begin), s) != cudaSuccess)
+        return RMM_ERR_CUDA;
+    rmm_status st = run_product_kernel(X, Wt, idx_padded, k, T, H, N, Y, ws, L, o, s);
+    if (st == RMM_OK && o.product_event_end &&
+        cudaEventRecord(static_cast<cudaEvent_t>(o.product_event_end), s) != cudaSuccess)
+        return RMM_ERR_CUDA;
+    return st;
+}
+
+}  // namespace
+}  // namespace rmm
+
+using namespace rmm;
+
+extern "C" {
+
+const char* rmm_status_string(rmm_status s) {
+    switch (s) {
+        case RMM_OK: return "RMM_OK";
+        case RMM_ERR_INVALID_ARG: return "RMM_ERR_INVALID_ARG";
+        case RMM_ERR_UNSUPPORTED: return "RMM_ERR_UNSUPPORTED";
+        case RMM_ERR_WORKSPACE: return "RMM_ERR_WORKSPACE";
+        case RMM_ERR_CUDA: return "RMM_ERR_CUDA";
+        case RMM_ERR_TIMEOUT: return "RMM_ERR_TIMEOUT";
+    }
+    return "RMM_ERR_UNKNOWN";
+}
+
+int rmm_k_for(int H, double r) {
+    if (H < 1 || !(r > 0.0) || !(r <= 1.0)) return -1;
+    double kk = ceil(r * (double)H);
+    long k = (long)kk;
+    if (k < 1) k = 1;
+    if (k > H) k = H;
+    return (int)k;
+}
+
+rmm_status rmm_workspace_init(void* ws, size_t bytes, rmm_stream_t stream) {
+    if (!ws || bytes < kStatusBytes) return RMM_ERR_INVALID_ARG;
+    return cuda_status(cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream)));
+}
+
+rmm_status rmm_get_status(void* ws, rmm_stream_t stream) {
+    if (!ws) return RMM_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return RMM_ERR_CUDA;
+    int code = 0;
+    if (cudaMemcpy(&code, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return RMM_ERR_CUDA;
+    if (code != 0) {
+        if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess) return RMM_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return RMM_ERR_CUDA;
+    }
+    return static_cast<rmm_status>(code);
+}
+
+rmm_status rmm_transpose_weight(const void* W, void* Wt, int N, int H, rmm_stream_t stream) {
+    if (!W || !Wt || N < 1 || H < 1) return RMM_ERR_INVALID_ARG;
+    const char* a = static_cast<const char*>(W);
+    const char* b = static_cast<const char*>(Wt);
+    const size_t bytes = (size_t)N * H * sizeof(uint16_t);
+    if (a < b + bytes && b < a + bytes) return RMM_ERR_INVALID_ARG;
+    return cuda_status(launch_transpose(static_cast<const uint16_t*>(W), static_cast<uint16_t*>(Wt),
+                                        N, H, static_cast<cudaStream_t>(stream)));
+}
+
+size_t rmm_linear_workspace_bytes(int T, int H, int N, const rmm_options* options) {
+    if (T < 1 || H < 1 || N < 1 || !opts_valid(options)) return 0;
+    const rmm_options& o = opts_or_default(options);
+    return linear_layout(T, H, N, H, o, num_sms_current()).total;
+}
+
+rmm_status rmm_linear(const void* X, const void* Wt, int T, int H, int N, double r, void* Y,
+                      int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                      rmm_stream_t stream, const rmm_options* options) {
+    if (!linear_args_ok(X, Wt, T, H, N, Y) || !opts_valid(options)) return RMM_ERR_INVALID_ARG;
+    const int k = rmm_k_for(H, r);
+    if (k < 1) return RMM_ERR_INVALID_ARG;
+    const rmm_options& o = opts_or_default(options);
+    const int sms = num_sms_current();
+    const LinearLayout L = linear_layout(T, H, N, k, o, sms);
+    if (!workspace || workspace_bytes < L.total || !aligned16(workspace)) return RMM_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    uint16_t* part = reinterpret_cast<uint16_t*>(ws + L.part);
+    int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+    cudaError_t e = launch_score(static_cast<const uint16_t*>(X), T, H, part, L.P,
+                                 L.gemv ? nullptr : reinterpret_cast<uint16_t*>(ws + L.xt), L.ldT, s);
+    if (e != cudaSuccess) return RMM_ERR_CUDA;
+    const int pad_to = (k + kGemmBK - 1) / kGemmBK * kGemmBK;
+    e = launch_select(part, L.P, nullptr, H, k, idx, pad_to, idx_out, nullptr, s);
+    if (e != cudaSuccess) return RMM_ERR_CUDA;
+    return run_product(X, Wt, idx, k, T, H, N, Y, ws, L, o, s);
+}
+
+rmm_status rmm_score(const void* X, int T, int H, uint32_t* s_out, void* workspace,
+                     size_t workspace_bytes, rmm_stream_t stream) {
+    if (!X || !s_out || T < 1 || H < 1 || H > 65535 || !aligned16(X)) return RMM_ERR_INVALID_ARG;
+    const int sms = num_sms_current();
+    const int P = score_partials_for(T, H, sms);
+    const size_t need = kStatusBytes + align_up((size_t)P * H * 2, kAlign) +
+                        align_up(((size_t)H + 2 * kGemmBK) * 4, kAlign);
+    if (!workspace || workspace_bytes < need) return RMM_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint16_t* part = reinterpret_cast<uint16_t*>(ws + kStatusBytes);
+    int32_t* idx = reinterpret_cast<int32_t*>(ws + kStatusBytes + align_up((size_t)P * H * 2, kAlign));
+    cudaError_t e = launch_score(static_cast<const uint16_t*>(X), T, H, part, P, nullptr, 0, s);
+    if (e != cudaSuccess) return RMM_ERR_CUDA;
+    return cuda_status(launch_select(part, P, nullptr, H, H, idx, H, nullptr, s_out, s));
+}
+
+rmm_status rmm_select(const uint32_t* sc, int H, int k, int32_t* idx_out, void* /*workspace*/,
+                      size_t /*workspace_bytes*/, rmm_stream_t stream) {
+    if (!sc || !idx_out || H < 1 || H > 65535 || k < 1 || k > H) return RMM_ERR_INVALID_ARG;
+    return cuda_status(launch_select(nullptr, 0, sc, H, k, idx_out, k, nullptr, nullptr,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+rmm_status rmm_gemm_reduced(const void* X, const void* Wt, const int32_t* idx, int k, int T, int H,
+                            int N, void* Y, void* workspace, size_t workspace_bytes,
+                            rmm_stream_t stream, const rmm_options* options) {
+    if (!linear_args_ok(X, Wt, T, H, N, Y) || !idx || k < 1 || k > H || !opts_valid(options))
+        return RMM_ERR_INVALID_ARG;
+    const rmm_options& o = opts_or_default(options);
+    const int sms = num_sms_current();
+    const LinearLayout L = linear_layout(T, H, N, k, o, sms);
+    if (!workspace || workspace_bytes < L.total || !aligned16(workspace)) return RMM_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (L.gemv) return run_product(X, Wt, idx, k, T, H, N, Y, ws, L, o, s);
+    // GEMM path: X^T (written by the score pass) and the kept list padded to the K-block
+    cudaError_t e = launch_score(static_cast<const uint16_t*>(X), T, H,
+                                 reinterpret_cast<uint16_t*>(ws + L.part), L.P,
+                                 reinterpret_cast<uint16_t*>(ws + L.xt), L.ldT, s);
+    if (e != cudaSuccess) return RMM_ERR_CUDA;
+    int32_t* idx_pad = reinterpret_cast<int32_t*>(ws + L.idx);
+    const int pad_to = (k + kGemmBK - 1) / kGemmBK * kGemmBK;
+    e = launch_pad_idx(idx, k, H, idx_pad, pad_to, s);
+    if (e != cudaSuccess) return RMM_ERR_CUDA;
+    return run_product(X, Wt, idx_pad, k, T, H, N, Y, ws, L, o, s);
+}
+
+size_t rmm_attn_workspace_bytes(int B, int Hq, int Hkv, int T, int L, int d,
+                                const rmm_options* options) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || L < T || d != 128 || Hq % Hkv != 0 ||
+        !opts_valid(options))
+        return 0;
+    const rmm_options& o = opts_or_default(options);
+    const AttnPlan p = attn_plan(B, Hq, Hkv, T, L, o.attn_per_query_head, num_sms_current());
+    return kStatusBytes + align_up((size_t)B * p.nsets * d * sizeof(int32_t), kAlign) +
+           align_up(attn_partials_bytes(p, B, Hq, T), kAlign);
+}
+
+rmm_status rmm_attn_qk(const void* Q, const void* Kt, const void* V, int B, int Hq, int Hkv, int T,
+                       int L, int ldL, int d, double r, int causal, float scale, void* O,
+                       int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                       rmm_stream_t stream, const rmm_options* options) {
+    if (!Q || !Kt || !V || !O || B < 1 || Hq < 1 || Hkv < 1 || T < 1 || L < T || ldL < L ||
+        ldL % 8 != 0 || Hq % Hkv != 0 || !opts_valid(options))
+        return RMM_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(Kt) || !aligned16(V) || !aligned16(O)) return RMM_ERR_INVALID_ARG;
+    if (!(scale > 0.0f) || !isfinite(scale)) return RMM_ERR_INVALID_ARG;
+    if (d != 128) return RMM_ERR_UNSUPPORTED;
+    const int k = rmm_k_for(d, r);
+    if (k < 1) return RMM_ERR_INVALID_ARG;
+    const rmm_options& o = opts_or_default(options);
+    if (!o.attn_per_query_head && Hq / Hkv > 8) return RMM_ERR_UNSUPPORTED;
+    const AttnPlan p = attn_plan(B, Hq, Hkv, T, L, o.attn_per_query_head, num_sms_current());
+    const size_t idx_bytes = align_up((size_t)B * p.nsets * d * sizeof(int32_t), kAlign);
+    const size_t need = kStatusBytes + idx_bytes + align_up(attn_partials_bytes(p, B, Hq, T), kAlign);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return RMM_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + kStatusBytes);
+    float* partials = reinterpret_cast<float*>(ws + kStatusBytes + idx_bytes);
+    return cuda_status(launch_attn(static_cast<const uint16_t*>(Q), static_cast<const uint16_t*>(Kt),
+                                   static_cast<const uint16_t*>(V), B, Hq, Hkv, T, L, ldL, k,
+                                   causal ? 1 : 0, scale, o.attn_per_query_head,
+                                   static_cast<uint16_t*>(O), idx, partials, p,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,327 @@
+// rmm_attn.cu -- attention with Q K^T reduced along the head dimension.
+//
+// For each (batch b, KV head g) -- or each query head, on request:
+//   s_j   = max over the group's query heads q and all t < T of |Q[b,q,t,j]|
+//   S_g   = top-k of s, k = ceil(r*d), ties to the lower index, ascending
+//   logit = scale * sum_{j in S_g} Q[b,q,t,j] * Kt[b,g,j,l]
+//   O     = softmax_l(logit) . V[b,g,l,:]          (all d dims, fp32 softmax)
+// (cf-1.com post on input-adaptive matrix-product reduction, §3.3: reduce
+// inside a head rather than dropping heads; paper abstract: attention-side
+// products reduced along their contraction dimension.)
+//
+// The key cache is stored d-major (Kt [B, Hkv, d, ldL]) so a kept head
+// dimension is one contiguous row of L keys: the logits pass reads exactly
+// k of the d rows, and V is read in full.
+//
+// Kernels:
+//   attn_select_kernel  one CTA per kept set: column max over the set's query
+//                       rows, then an exact rank-based top-k of the d scores
+//   attn_split_kernel   one CTA per (set, split of L, block of query tokens):
+//                       logits for a 1024-key sub-block (each thread 4 keys,
+//                       8-byte loads of kept K^T rows), online softmax in fp32,
+//                       P.V with 16-byte loads of V rows; writes the split's
+//                       running max, sum and unnormalised output
+//   attn_combine_kernel merges the splits (flash-decoding style) into bf16 O.
+#include <math.h>
+
+#include "rmm_common.cuh"
+#include "rmm_internal.h"
+
+namespace rmm {
+
+namespace {
+
+constexpr int D = 128;        // head dimension handled by this build
+constexpr int kThreads = 256;
+constexpr int SB = 1024;      // keys per sub-block
+constexpr int RMAX = 8;       // query rows per CTA
+constexpr int PSTRIDE = D + 2;  // floats per split partial: m, l, O[d]
+
+// ---------------------------------------------------------------- selection
+
+__global__ void __launch_bounds__(D)
+    attn_select_kernel(const uint16_t* __restrict__ Q, int Hq, int Hkv, int T, int k,
+                       int per_query_head, int32_t* __restrict__ idx) {
+    __shared__ uint32_t sv[D];
+    __shared__ int warp_cnt[D / 32];
+    const int nsets = per_query_head ? Hq : Hkv;
+    const int set = blockIdx.x % nsets;
+    const int b = blockIdx.x / nsets;
+    const int G = Hq / Hkv;
+    const int q_lo = per_query_head ? set : set * G;
+    const int q_hi = per_query_head ? set + 1 : (set + 1) * G;
+    const int j = threadIdx.x;
+
+    uint32_t m = 0;
+    for (int q = q_lo; q < q_hi; ++q) {
+        const uint16_t* row = Q + ((size_t)(b * Hq + q) * T) * D + j;
+        for (int t = 0; t < T; ++t) m = max(m, (uint32_t)(row[(size_t)t * D] & 0x7FFF));
+    }
+    sv[j] = m;
+    __syncthreads();
+    // rank under (score desc, index asc): number of entries that beat j
+    int rank = 0;
+    for (int i = 0; i < D; ++i) {
+        const uint32_t v = sv[i];
+        rank += (v > m) || (v == m && i < j);
+    }
+    const bool keep = rank < k;
+    const unsigned ball = __ballot_sync(0xffffffffu, keep);
+    const int lane = j & 31, w = j >> 5;
+    if (lane == 0) warp_cnt[w] = __popc(ball);
+    __syncthreads();
+    int pos = __popc(ball & ((1u << lane) - 1u));
+    for (int i = 0; i < w; ++i) pos += warp_cnt[i];
+    if (keep) idx[(size_t)blockIdx.x * k + pos] = j;
+}
+
+// ---------------------------------------------------------------- split pass
+
+__global__ void __launch_bounds__(kThreads)
+    attn_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ Kt,
+                      const uint16_t* __restrict__ V, int Hq, int Hkv, int T, int L, int ldL, int k,
+                      int causal, float scale, int per_query_head, const int32_t* __restrict__ idx,
+                      float* __restrict__ partials, int chunk, int tq) {
+    __shared__ float qs[RMAX][D];      // scaled kept query values
+    __shared__ int sidx[D];
+    // One buffer, two uses: logits/probabilities of the current sub-block
+    // [RMAX][SB] inside the key loop, the cross-warp fold of P.V [8][RMAX][D]
+    // after it (both 32 KB).
+    __shared__ float buf[RMAX * SB];
+    float (*lg)[SB] = reinterpret_cast<float (*)[SB]>(buf);
+    float (*red)[RMAX][D] = reinterpret_cast<float (*)[RMAX][D]>(buf);
+    static_assert(8 * RMAX * D <= RMAX * SB, "fold buffer must fit in the logits buffer");
+    __shared__ float m_run[RMAX], l_run[RMAX], alpha[RMAX];
+
+    const int nsets = per_query_head ? Hq : Hkv;
+    const int set = blockIdx.x % nsets;
+    const int b = blockIdx.x / nsets;
+    const int G = Hq / Hkv;
+    const int g = per_query_head ? set / G : set;
+    const int q_lo = per_query_head ? set : set * G;
+    const int nq = per_query_head ? 1 : G;
+    const int split = blockIdx.y;
+    const int nsplit = gridDim.y;
+    const int t0 = blockIdx.z * tq;
+    const int l_begin = split * chunk;
+    const int l_end = min(L, l_begin + chunk);
+    const int R = nq * tq;  // rows: r = qi * tq + ti
+    const int tid = threadIdx.x;
+
+    for (int i = tid; i < k; i += kThreads) sidx[i] = idx[(size_t)blockIdx.x * k + i];
+    __syncthreads();
+    for (int e = tid; e < RMAX * D; e += kThreads) {
+        const int r = e / D, jj = e % D;
+        float v = 0.0f;
+        if (r < R && jj < k) {
+            const int qi = r / tq, ti = r % tq, t = t0 + ti;
+            if (t < T) v = scale * bf16_bits_to_float(Q[(((size_t)(b * Hq + q_lo + qi)) * T + t) * D + sidx[jj]]);
+        }
+        qs[r][jj] = v;
+    }
+    if (tid < RMAX) {
+        m_run[tid] = -INFINITY;
+        l_run[tid] = 0.0f;
+    }
+    __syncthreads();
+
+    // last key each row may see
+    int last[RMAX];
+#pragma unroll
+    for (int r = 0; r < RMAX; ++r) {
+        const int ti = (r < R) ? r % tq : 0;
+        const int t = t0 + ti;
+        last[r] = (r < R && t < T) ? (causal ? (L - T + t) : (L - 1)) : -1;
+    }
+
+    const uint16_t* kbase = Kt + ((size_t)(b * Hkv + g) * D) * ldL;
+    const uint16_t* vbase = V + ((size_t)(b * Hkv + g) * ldL) * D;
+
+    // P.V mapping: 16 column groups of 8 dims x 16 key groups
+    const int cgp = tid & 15, kg = tid >> 4;
+    float acc[RMAX][8];
+#pragma unroll
+    for (int r = 0; r < RMAX; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[r][c] = 0.0f;
+
+    for (int l0 = l_begin; l0 < l_end; l0 += SB) {
+        // ---- logits: thread owns keys l0 + 4*tid .. +3
+        const int l = l0 + tid * 4;
+        float s4[RMAX][4];
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) s4[r][c] = 0.0f;
+        if (l < l_end) {
+            for (int jj = 0; jj < k; ++jj) {
+                const uint2 kv = ld_nc_v2(kbase + (size_t)sidx[jj] * ldL + l);
+                const float k0 = __uint_as_float(kv.x << 16), k1 = __uint_as_float(kv.x & 0xFFFF0000u);
+                const float k2 = __uint_as_float(kv.y << 16), k3 = __uint_as_float(kv.y & 0xFFFF0000u);
+#pragma unroll
+                for (int r = 0; r < RMAX; ++r) {
+                    const float qv = qs[r][jj];
+                    s4[r][0] = fmaf(qv, k0, s4[r][0]);
+                    s4[r][1] = fmaf(qv, k1, s4[r][1]);
+                    s4[r][2] = fmaf(qv, k2, s4[r][2]);
+                    s4[r][3] = fmaf(qv, k3, s4[r][3]);
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int lc = l + c;
+                lg[r][tid * 4 + c] = (lc < l_end && lc <= last[r]) ? s4[r][c] : -INFINITY;
+            }
+        __syncthreads();
+
+        // ---- online softmax, one warp per row
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int r = warp; r < RMAX; r += kThreads / 32) {
+            float mx = -INFINITY;
+            for (int i = lane; i < SB; i += 32) mx = fmaxf(mx, lg[r][i]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const float m_old = m_run[r];
+            const float m_new = fmaxf(m_old, mx);
+            float sum = 0.0f;
+            if (m_new == -INFINITY) {
+                for (int i = lane; i < SB; i += 32) lg[r][i] = 0.0f;
+            } else {
+                for (int i = lane; i < SB; i += 32) {
+                    const float p = __expf(lg[r][i] - m_new);
+                    lg[r][i] = p;
+                    sum += p;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            if (lane == 0) {
+                const float a = (m_old == -INFINITY) ? 0.0f : __expf(m_old - m_new);
+                alpha[r] = (m_new == -INFINITY) ? 1.0f : a;
+                l_run[r] = l_run[r] * alpha[r] + sum;
+                m_run[r] = m_new;
+            }
+        }
+        __syncthreads();
+
+        // ---- P.V
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r) {
+            const float a = alpha[r];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[r][c] *= a;
+        }
+        const int nkeys = min(SB, l_end - l0);
+        for (int i = kg; i < nkeys; i += 16) {
+            const uint4 v = ld_nc_v4(vbase + (size_t)(l0 + i) * D + cgp * 8);
+            float vf[8];
+            vf[0] = __uint_as_float(v.x << 16); vf[1] = __uint_as_float(v.x & 0xFFFF0000u);
+            vf[2] = __uint_as_float(v.y << 16); vf[3] = __uint_as_float(v.y & 0xFFFF0000u);
+            vf[4] = __uint_as_float(v.z << 16); vf[5] = __uint_as_float(v.z & 0xFFFF0000u);
+            vf[6] = __uint_as_float(v.w << 16); vf[7] = __uint_as_float(v.w & 0xFFFF0000u);
+#pragma unroll
+            for (int r = 0; r < RMAX; ++r) {
+                const float p = lg[r][i];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(p, vf[c], acc[r][c]);
+            }
+        }
+        __syncthreads();  // lg is rewritten by the next sub-block
+    }
+
+    // fold the 16 key groups: pairs within a warp by shuffle, then 8 warps via smem
+#pragma unroll
+    for (int r = 0; r < RMAX; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[r][c] += __shfl_xor_sync(0xffffffffu, acc[r][c], 16);
+    const int warp = tid >> 5, lane = tid & 31;
+    if (lane < 16) {
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) red[warp][r][cgp * 8 + c] = acc[r][c];
+    }
+    __syncthreads();
+    for (int e = tid; e < R * D; e += kThreads) {
+        const int r = e / D, c = e % D;
+        const int qi = r / tq, ti = r % tq, t = t0 + ti;
+        if (t >= T) continue;
+        float o = 0.0f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) o += red[w][r][c];
+        const size_t row = ((size_t)(b * Hq + q_lo + qi)) * T + t;
+        float* dst = partials + (row * nsplit + split) * PSTRIDE;
+        dst[2 + c] = o;
+        if (c == 0) {
+            dst[0] = m_run[r];
+            dst[1] = l_run[r];
+        }
+    }
+}
+
+// ---------------------------------------------------------------- combine
+
+__global__ void __launch_bounds__(D)
+    attn_combine_kernel(const float* __restrict__ partials, int nsplit, uint16_t* __restrict__ O) {
+    const size_t row = blockIdx.x;
+    const float* p = partials + row * nsplit * PSTRIDE;
+    float M = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, p[s * PSTRIDE]);
+    float num = 0.0f, den = 0.0f;
+    for (int s = 0; s < nsplit; ++s) {
+        const float m = p[s * PSTRIDE];
+        if (m == -INFINITY) continue;
+        const float w = __expf(m - M);
+        den += w * p[s * PSTRIDE + 1];
+        num += w * p[s * PSTRIDE + 2 + threadIdx.x];
+    }
+    O[row * D + threadIdx.x] = float_to_bf16_bits(num / den);
+}
+
+}  // namespace
+
+AttnPlan attn_plan(int B, int Hq, int Hkv, int T, int L, int per_query_head, int num_sms) {
+    AttnPlan p;
+    p.nsets = per_query_head ? Hq : Hkv;
+    const int nq = per_query_head ? 1 : Hq / Hkv;
+    p.tq = RMAX / nq;
+    if (p.tq < 1) p.tq = 1;
+    if (p.tq > T) p.tq = T;
+    const long long base = (long long)B * p.nsets * ((T + p.tq - 1) / p.tq);
+    const long long target = 2LL * num_sms;
+    long long ns = (target + base - 1) / base;
+    if (ns < 1) ns = 1;
+    int chunk = (int)((L + ns - 1) / ns);
+    if (chunk < 256) chunk = 256;
+    chunk = (chunk + 3) & ~3;
+    p.chunk = chunk;
+    p.nsplit = (L + chunk - 1) / chunk;
+    return p;
+}
+
+size_t attn_partials_bytes(const AttnPlan& p, int B, int Hq, int T) {
+    return (size_t)B * Hq * T * p.nsplit * PSTRIDE * sizeof(float);
+}
+
+cudaError_t launch_attn(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq,
+                        int Hkv, int T, int L, int ldL, int k, int causal, float scale,
+                        int per_query_head, uint16_t* O, int32_t* idx, float* partials,
+                        const AttnPlan& p, cudaStream_t stream) {
+    attn_select_kernel<<<B * p.nsets, D, 0, stream>>>(Q, Hq, Hkv, T, k, per_query_head, idx);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int nq = per_query_head ? 1 : Hq / Hkv;
+    if (nq > RMAX) return cudaErrorInvalidValue;
+    dim3 grid(B * p.nsets, p.nsplit, (T + p.tq - 1) / p.tq);
+    attn_split_kernel<<<grid, kThreads, 0, stream>>>(Q, Kt, V, Hq, Hkv, T, L, ldL, k, causal, scale,
+                                                     per_query_head, idx, partials, p.chunk, p.tq);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_combine_kernel<<<B * Hq * T, D, 0, stream>>>(partials, p.nsplit, O);
+    return cudaGetLastError();
+}
+
+}  // namespace rmm

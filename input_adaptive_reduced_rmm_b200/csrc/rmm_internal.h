@@ -1,0 +1,68 @@
+// rmm_internal.h -- host-side launchers shared between the library's .cu files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace rmm {
+
+constexpr int kMaxScorePartials = 32;  // partial-maximum rows written by the score pass
+constexpr int kGemvMaxT = 16;          // largest T of the split-K GEMV
+constexpr int kGemmBK = 64;            // kept slices per GEMM pipeline stage (idx padded to this)
+
+// ---- score (rmm_score.cu)
+int score_partials_for(int T, int H, int num_sms);
+cudaError_t launch_score(const uint16_t* X, int T, int H, uint16_t* part, int P, uint16_t* Xt,
+                         int ldT, cudaStream_t stream);
+
+// ---- select (rmm_select.cu)
+// Folds P partial rows (part, u16 [P][H]) -- or reads s32 (u32 [H]) when part is
+// null -- into the score, optionally stores it to s_out, and writes the k best
+// indices ascending to idx[0..k), then idx[k..pad_to) = H; idx_copy (if not
+// null) receives the same k indices without padding.
+cudaError_t launch_select(const uint16_t* part, int P, const uint32_t* s32, int H, int k,
+                          int32_t* idx, int pad_to, int32_t* idx_copy, uint32_t* s_out,
+                          cudaStream_t stream);
+
+// ---- split-K GEMV (rmm_gemv.cu)
+struct GemvPlan {
+    int cols_per_cta;  // 256 or 512
+    int splits;
+    int rows_per_split;
+    int col_blocks;
+};
+GemvPlan gemv_plan(int T, int N, int k, int num_sms, int forced_splits);
+size_t gemv_partials_bytes(const GemvPlan& p, int T, int N);
+cudaError_t launch_gemv(const uint16_t* X, int T, int H, const uint16_t* Wt, int N,
+                        const int32_t* idx, int k, uint16_t* Y, float* partials,
+                        unsigned* counters, const GemvPlan& plan, int* status,
+                        cudaStream_t stream);
+
+// ---- tcgen05 GEMM (rmm_gemm.cu)
+cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt,
+                        const int32_t* idx, int k, int T, int H, int N, uint16_t* Y,
+                        int* status, int debug_timeout, int num_sms, cudaStream_t stream);
+size_t gemm_smem_bytes();
+
+// ---- attention (rmm_attn.cu)
+struct AttnPlan {
+    int chunk;    // keys per split
+    int nsplit;   // splits over L
+    int tq;       // query tokens per CTA
+    int nsets;    // kept sets per batch (Hkv or Hq)
+};
+AttnPlan attn_plan(int B, int Hq, int Hkv, int T, int L, int per_query_head, int num_sms);
+size_t attn_partials_bytes(const AttnPlan& p, int B, int Hq, int T);
+cudaError_t launch_attn(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq,
+                        int Hkv, int T, int L, int ldL, int k, int causal, float scale,
+                        int per_query_head, uint16_t* O, int32_t* idx, float* partials,
+                        const AttnPlan& plan, cudaStream_t stream);
+
+// ---- glue (rmm_glue.cu)
+cudaError_t launch_transpose(const uint16_t* W, uint16_t* Wt, int N, int H, cudaStream_t stream);
+cudaError_t launch_pad_idx(const int32_t* src, int k, int H, int32_t* dst, int pad_to,
+                           cudaStream_t stream);
+
+}  // namespace rmm

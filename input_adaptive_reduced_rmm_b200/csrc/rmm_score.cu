@@ -1,0 +1,148 @@
+// rmm_score.cu -- step 1 of the reduced product: the per-slice input score.
+//
+// s_h = max over tokens t of |X[t,h]|  (cf-1.com post on input-adaptive
+// matrix-product reduction, §5.1: a cheap score taken from the current
+// activations; one common score for all tokens of the call, §8).
+//
+// |x| is taken on the bf16 bit pattern with the sign cleared, an integer that
+// orders exactly like the magnitude of a finite value, so the maximum is
+// exact and independent of the reduction order.
+//
+// One pass over X [T, H] (HBM-bound: T*H*2 bytes read).  Each CTA owns a
+// 64-wide channel strip and a strided subset of 64-token tiles; it writes its
+// strip's partial maximum to part[blockIdx.y][h] and the select kernel folds
+// the gridDim.y partials.  On the GEMM path the same pass also writes the
+// full transpose X^T [H, ldT] (through a shared-memory tile) so that a kept
+// slice of X is one contiguous row that TMA can gather; this is a transposed
+// copy of all of X, never a compacted copy of the kept part.
+#include "rmm_common.cuh"
+#include "rmm_internal.h"
+
+namespace rmm {
+
+namespace {
+
+constexpr int kTileT = 64;  // tokens per tile
+constexpr int kTileH = 64;  // channels per strip
+constexpr int kThreads = 256;
+
+template <bool kWriteXt, bool kVec>
+__global__ void __launch_bounds__(kThreads)
+    score_kernel(const uint16_t* __restrict__ X, int T, int H, uint16_t* __restrict__ part,
+                 uint16_t* __restrict__ Xt, int ldT) {
+    // Rows of 66 elements (33 words): the transposed reads of 8 rows that are
+    // 8 apart then fall on distinct bank groups (2-way conflicts at most).
+    __shared__ __align__(16) uint16_t tile[kTileT][kTileH + 2];
+    __shared__ uint16_t red[32][kTileH];
+
+    const int tid = threadIdx.x;
+    const int cg = tid & 7;    // 8-channel group within the strip
+    const int row = tid >> 3;  // 0..31
+    const int h0 = blockIdx.x * kTileH;
+    const int hc = h0 + cg * 8;
+
+    uint32_t mx[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = 0;
+
+    for (int t0 = blockIdx.y * kTileT; t0 < T; t0 += gridDim.y * kTileT) {
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const int r = p * 32 + row;
+            const int t = t0 + r;
+            uint16_t v[8];
+            if (kVec && t < T && hc + 8 <= H) {
+                uint4 q = ld_nc_v4(X + (size_t)t * H + hc);
+                v[0] = q.x & 0xFFFF; v[1] = q.x >> 16;
+                v[2] = q.y & 0xFFFF; v[3] = q.y >> 16;
+                v[4] = q.z & 0xFFFF; v[5] = q.z >> 16;
+                v[6] = q.w & 0xFFFF; v[7] = q.w >> 16;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    v[i] = (t < T && hc + i < H) ? X[(size_t)t * H + hc + i] : (uint16_t)0;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx[i] = max(mx[i], (uint32_t)(v[i] & 0x7FFF));
+            if (kWriteXt) {
+                uint32_t* d = reinterpret_cast<uint32_t*>(&tile[r][cg * 8]);
+                d[0] = v[0] | ((uint32_t)v[1] << 16);
+                d[1] = v[2] | ((uint32_t)v[3] << 16);
+                d[2] = v[4] | ((uint32_t)v[5] << 16);
+                d[3] = v[6] | ((uint32_t)v[7] << 16);
+            }
+        }
+        if (kWriteXt) {
+            __syncthreads();
+            // transposed write-out: 8 threads per channel row, 8 tokens each
+            const int tc = tid & 7;
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const int hl = p * 32 + (tid >> 3);
+                const int h = h0 + hl;
+                const int tt = t0 + tc * 8;
+                if (h < H && tt < T) {
+                    uint16_t w[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) w[i] = tile[tc * 8 + i][hl];
+                    uint16_t* dst = Xt + (size_t)h * ldT + tt;
+                    if (tt + 8 <= T) {
+                        uint4 q;
+                        q.x = w[0] | ((uint32_t)w[1] << 16);
+                        q.y = w[2] | ((uint32_t)w[3] << 16);
+                        q.z = w[4] | ((uint32_t)w[5] << 16);
+                        q.w = w[6] | ((uint32_t)w[7] << 16);
+                        *reinterpret_cast<uint4*>(dst) = q;
+                    } else {
+                        for (int i = 0; i < 8 && tt + i < T; ++i) dst[i] = w[i];
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+
+    // fold the 32 row-threads that share each channel group
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[row][cg * 8 + i] = (uint16_t)mx[i];
+    __syncthreads();
+    if (tid < kTileH) {
+        uint32_t m = 0;
+#pragma unroll 8
+        for (int r = 0; r < 32; ++r) m = max(m, (uint32_t)red[r][tid]);
+        const int h = h0 + tid;
+        if (h < H) part[(size_t)blockIdx.y * H + h] = (uint16_t)m;
+    }
+}
+
+}  // namespace
+
+int score_partials_for(int T, int H, int num_sms) {
+    const int strips = (H + kTileH - 1) / kTileH;
+    const int tiles = (T + kTileT - 1) / kTileT;
+    int p = (4 * num_sms + strips - 1) / strips;
+    if (p > tiles) p = tiles;
+    if (p > kMaxScorePartials) p = kMaxScorePartials;
+    if (p < 1) p = 1;
+    return p;
+}
+
+cudaError_t launch_score(const uint16_t* X, int T, int H, uint16_t* part, int P, uint16_t* Xt,
+                         int ldT, cudaStream_t stream) {
+    dim3 grid((H + kTileH - 1) / kTileH, P);
+    const bool vec = (H % 8 == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
+    if (Xt) {
+        if (vec)
+            score_kernel<true, true><<<grid, kThreads, 0, stream>>>(X, T, H, part, Xt, ldT);
+        else
+            score_kernel<true, false><<<grid, kThreads, 0, stream>>>(X, T, H, part, Xt, ldT);
+    } else {
+        if (vec)
+            score_kernel<false, true><<<grid, kThreads, 0, stream>>>(X, T, H, part, nullptr, 0);
+        else
+            score_kernel<false, false><<<grid, kThreads, 0, stream>>>(X, T, H, part, nullptr, 0);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace rmm

@@ -1,0 +1,253 @@
+"""Thin ctypes binding of librmm (C ABI in include/rmm.h), with the same names.
+
+Argument marshalling only: tensors become device pointers and sizes, the
+current torch stream becomes the cudaStream_t, a non-OK status becomes an
+exception.  Every step of the computation runs in librmm's CUDA kernels;
+there is no fallback path, and a missing library raises on first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librmm.so")
+
+RMM_OK = 0
+RMM_ERR_INVALID_ARG = 1
+RMM_ERR_UNSUPPORTED = 2
+RMM_ERR_WORKSPACE = 3
+RMM_ERR_CUDA = 4
+RMM_ERR_TIMEOUT = 5
+
+# every symbol include/rmm.h declares
+EXPORTED = (
+    "rmm_status_string", "rmm_k_for", "rmm_workspace_init", "rmm_get_status",
+    "rmm_transpose_weight", "rmm_linear_workspace_bytes", "rmm_linear", "rmm_score",
+    "rmm_select", "rmm_gemm_reduced", "rmm_attn_workspace_bytes", "rmm_attn_qk",
+)
+
+
+class RmmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {rmm_status_string(status)} ({status})")
+        self.status = status
+
+
+class rmm_options(ctypes.Structure):
+    _fields_ = [
+        ("t_gemv", ctypes.c_int),
+        ("attn_per_query_head", ctypes.c_int),
+        ("gemv_splits", ctypes.c_int),
+        ("debug_timeout_test", ctypes.c_int),
+        ("reserved", ctypes.c_int * 4),
+        ("product_event_begin", ctypes.c_void_p),
+        ("product_event_end", ctypes.c_void_p),
+    ]
+
+
+def options(t_gemv: int = 16, attn_per_query_head: bool = False, gemv_splits: int = 0,
+            debug_timeout_test: bool = False, product_events=None) -> rmm_options:
+    """An rmm_options struct; product_events = (begin, end) torch.cuda.Event pair (enable_timing)."""
+    o = rmm_options(int(t_gemv), int(bool(attn_per_query_head)), int(gemv_splits),
+                    int(bool(debug_timeout_test)), (ctypes.c_int * 4)(0, 0, 0, 0), None, None)
+    if product_events is not None:
+        b, e = product_events
+        o.product_event_begin = ctypes.c_void_p(b.cuda_event)
+        o.product_event_end = ctypes.c_void_p(e.cuda_event)
+    return o
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load librmm.so (built in-tree by input_adaptive_reduced_rmm_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m input_adaptive_reduced_rmm_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, D, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_float, ctypes.c_size_t
+    OP = ctypes.POINTER(rmm_options)
+    sig = {
+        "rmm_status_string": (ctypes.c_char_p, [I]),
+        "rmm_k_for": (I, [I, D]),
+        "rmm_workspace_init": (I, [P, Z, P]),
+        "rmm_get_status": (I, [P, P]),
+        "rmm_transpose_weight": (I, [P, P, I, I, P]),
+        "rmm_linear_workspace_bytes": (Z, [I, I, I, OP]),
+        "rmm_linear": (I, [P, P, I, I, I, D, P, P, P, Z, P, OP]),
+        "rmm_score": (I, [P, I, I, P, P, Z, P]),
+        "rmm_select": (I, [P, I, I, P, P, Z, P]),
+        "rmm_gemm_reduced": (I, [P, P, P, I, I, I, I, P, P, Z, P, OP]),
+        "rmm_attn_workspace_bytes": (Z, [I, I, I, I, I, I, OP]),
+        "rmm_attn_qk": (I, [P, P, P, I, I, I, I, I, I, I, D, I, F, P, P, P, Z, P, OP]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _opt(o):
+    return None if o is None else ctypes.byref(o)
+
+
+def _check(rc: int, what: str):
+    if rc != RMM_OK:
+        raise RmmError(rc, what)
+
+
+def _bf16_cuda(t, name):
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+
+
+def rmm_status_string(status: int) -> str:
+    return lib().rmm_status_string(int(status)).decode()
+
+
+def rmm_k_for(H: int, r: float) -> int:
+    return int(lib().rmm_k_for(int(H), float(r)))
+
+
+def new_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zero-filled device workspace (the status word must start at zero)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def rmm_workspace_init(workspace: torch.Tensor, stream=None):
+    _check(lib().rmm_workspace_init(_ptr(workspace), workspace.numel(), _stream(stream)),
+           "rmm_workspace_init")
+
+
+def rmm_get_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the device status word."""
+    return int(lib().rmm_get_status(_ptr(workspace), _stream(stream)))
+
+
+def rmm_transpose_weight(W: torch.Tensor, Wt: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """W [N, H] -> W^T [H, N] (bf16)."""
+    _bf16_cuda(W, "W")
+    N, H = W.shape
+    if Wt is None:
+        Wt = torch.empty(H, N, dtype=torch.bfloat16, device=W.device)
+    _check(lib().rmm_transpose_weight(_ptr(W), _ptr(Wt), N, H, _stream(stream)), "rmm_transpose_weight")
+    return Wt
+
+
+def rmm_linear_workspace_bytes(T: int, H: int, N: int, opts: rmm_options | None = None) -> int:
+    return int(lib().rmm_linear_workspace_bytes(int(T), int(H), int(N), _opt(opts)))
+
+
+def rmm_linear(X: torch.Tensor, Wt: torch.Tensor, r: float, Y: torch.Tensor | None = None,
+               idx_out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+               opts: rmm_options | None = None, stream=None) -> torch.Tensor:
+    """Y ~= X[:,S] W[:,S]^T with S the ceil(r*H) kept slices.  X [T,H], Wt [H,N] bf16."""
+    _bf16_cuda(X, "X")
+    _bf16_cuda(Wt, "Wt")
+    T, H = X.shape
+    H2, N = Wt.shape
+    if H2 != H:
+        raise ValueError("X and Wt disagree on H")
+    if Y is None:
+        Y = torch.empty(T, N, dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = new_workspace(rmm_linear_workspace_bytes(T, H, N, opts), X.device)
+    if idx_out is not None and (idx_out.dtype != torch.int32 or not idx_out.is_cuda):
+        raise ValueError("idx_out must be an int32 CUDA tensor")
+    _check(lib().rmm_linear(_ptr(X), _ptr(Wt), T, H, N, float(r), _ptr(Y), _ptr(idx_out),
+                            _ptr(workspace), workspace.numel(), _stream(stream), _opt(opts)),
+           "rmm_linear")
+    return Y
+
+
+def rmm_score(X: torch.Tensor, s_out: torch.Tensor | None = None,
+              workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """s[h] = max_t |X[t,h]| as the bf16 magnitude key (int32 tensor holding uint32 values)."""
+    _bf16_cuda(X, "X")
+    T, H = X.shape
+    if s_out is None:
+        s_out = torch.empty(H, dtype=torch.int32, device=X.device)
+    if workspace is None:
+        workspace = new_workspace(rmm_linear_workspace_bytes(T, H, 8), X.device)
+    _check(lib().rmm_score(_ptr(X), T, H, _ptr(s_out), _ptr(workspace), workspace.numel(),
+                           _stream(stream)), "rmm_score")
+    return s_out
+
+
+def rmm_select(s: torch.Tensor, k: int, idx_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The k best indices of s under (score desc, index asc), ascending (int32)."""
+    if s.dtype != torch.int32 or not s.is_cuda:
+        raise ValueError("s must be an int32 CUDA tensor (uint32 scores)")
+    H = s.numel()
+    if idx_out is None:
+        idx_out = torch.empty(int(k), dtype=torch.int32, device=s.device)
+    _check(lib().rmm_select(_ptr(s), H, int(k), _ptr(idx_out), None, 0, _stream(stream)), "rmm_select")
+    return idx_out
+
+
+def rmm_gemm_reduced(X: torch.Tensor, Wt: torch.Tensor, idx: torch.Tensor, Y: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, opts: rmm_options | None = None,
+                     stream=None) -> torch.Tensor:
+    """Y[t,n] = sum_j X[t, idx_j] * Wt[idx_j, n] for a given kept list."""
+    _bf16_cuda(X, "X")
+    _bf16_cuda(Wt, "Wt")
+    if idx.dtype != torch.int32 or not idx.is_cuda:
+        raise ValueError("idx must be an int32 CUDA tensor")
+    T, H = X.shape
+    N = Wt.shape[1]
+    if Y is None:
+        Y = torch.empty(T, N, dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = new_workspace(rmm_linear_workspace_bytes(T, H, N, opts), X.device)
+    _check(lib().rmm_gemm_reduced(_ptr(X), _ptr(Wt), _ptr(idx), idx.numel(), T, H, N, _ptr(Y),
+                                  _ptr(workspace), workspace.numel(), _stream(stream), _opt(opts)),
+           "rmm_gemm_reduced")
+    return Y
+
+
+def rmm_attn_workspace_bytes(B: int, Hq: int, Hkv: int, T: int, L: int, d: int = 128,
+                             opts: rmm_options | None = None) -> int:
+    return int(lib().rmm_attn_workspace_bytes(B, Hq, Hkv, T, L, d, _opt(opts)))
+
+
+def rmm_attn_qk(Q: torch.Tensor, Kt: torch.Tensor, V: torch.Tensor, L: int, r: float,
+                causal: bool = True, scale: float | None = None, O: torch.Tensor | None = None,
+                idx_out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                opts: rmm_options | None = None, stream=None) -> torch.Tensor:
+    """Reduced attention.  Q [B,Hq,T,d]; Kt [B,Hkv,d,ldL] (d-major keys); V [B,Hkv,ldL,d]."""
+    for t, n in ((Q, "Q"), (Kt, "Kt"), (V, "V")):
+        _bf16_cuda(t, n)
+    B, Hq, T, d = Q.shape
+    _, Hkv, d2, ldL = Kt.shape
+    if d2 != d or V.shape != (B, Hkv, ldL, d):
+        raise ValueError("Q, Kt, V shapes disagree")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(Q)
+    if workspace is None:
+        workspace = new_workspace(rmm_attn_workspace_bytes(B, Hq, Hkv, T, L, d, opts), Q.device)
+    _check(lib().rmm_attn_qk(_ptr(Q), _ptr(Kt), _ptr(V), B, Hq, Hkv, T, int(L), ldL, d, float(r),
+                             int(bool(causal)), float(scale), _ptr(O), _ptr(idx_out), _ptr(workspace),
+                             workspace.numel(), _stream(stream), _opt(opts)), "rmm_attn_qk")
+    return O

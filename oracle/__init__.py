@@ -75,9 +75,9 @@ def _load():
     lib.oracle_score.restype = I
     lib.oracle_select.argtypes = [_u16p, L, L, _i32p]
     lib.oracle_select.restype = I
-    lib.oracle_reduced_product.argtypes = [_u16p, _u16p, L, L, L, _i32p, L, P, L, _f64p]
+    lib.oracle_reduced_product.argtypes = [_u16p, _u16p, L, L, L, _i32p, L, P, L, P, L, _f64p]
     lib.oracle_reduced_product.restype = I
-    lib.oracle_linear.argtypes = [_u16p, _u16p, L, L, L, D, P, L, _f64p, _i32p]
+    lib.oracle_linear.argtypes = [_u16p, _u16p, L, L, L, D, P, L, P, L, _f64p, _i32p]
     lib.oracle_linear.restype = I
     lib.oracle_attention.argtypes = [_u16p, _u16p, _u16p, L, L, L, L, L, L, L, I, D, I, P, L,
                                      _f64p, _i32p]
@@ -139,32 +139,37 @@ def select(s, k: int) -> np.ndarray:
     return idx
 
 
-def reduced_product(X, W, idx, rows=None) -> np.ndarray:
-    """Y[r, n] = sum_{j} X[t_r, idx_j] * W[n, idx_j] in fp64.  W is [N, H]."""
+def reduced_product(X, W, idx, rows=None, cols=None) -> np.ndarray:
+    """Y[r, c] = sum_{j} X[t_r, idx_j] * W[n_c, idx_j] in fp64.  W is [N, H].
+
+    rows / cols (optional) select the token rows and output features computed.
+    """
     x, w = _bits(X), _bits(W)
     T, H = x.shape
     N = w.shape[0]
     assert w.shape[1] == H
     idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int32))
-    rp, nr, _keep = _rows(rows)
-    Y = np.zeros((nr if rows is not None else T, N), dtype=np.float64)
-    _check(_load().oracle_reduced_product(x, w, T, H, N, idx, len(idx), rp, nr, Y),
+    rp, nr, _kr = _rows(rows)
+    cp, nc, _kc = _rows(cols)
+    Y = np.zeros((nr if rows is not None else T, nc if cols is not None else N), dtype=np.float64)
+    _check(_load().oracle_reduced_product(x, w, T, H, N, idx, len(idx), rp, nr, cp, nc, Y),
            "oracle_reduced_product")
     return Y
 
 
-def linear(X, W, r: float, rows=None):
-    """(Y fp64 [nrows, N], idx int32 [k]) of the reduced linear map Y ~= X[:,S] W[:,S]^T."""
+def linear(X, W, r: float, rows=None, cols=None):
+    """(Y fp64 [nrows, ncols], idx int32 [k]) of the reduced linear map Y ~= X[:,S] W[:,S]^T."""
     x, w = _bits(X), _bits(W)
     T, H = x.shape
     N = w.shape[0]
     k = k_for(H, r)
     if k < 1:
         raise OracleError("r must lie in (0, 1]")
-    rp, nr, _keep = _rows(rows)
-    Y = np.zeros((nr if rows is not None else T, N), dtype=np.float64)
+    rp, nr, _kr = _rows(rows)
+    cp, nc, _kc = _rows(cols)
+    Y = np.zeros((nr if rows is not None else T, nc if cols is not None else N), dtype=np.float64)
     idx = np.zeros(k, dtype=np.int32)
-    _check(_load().oracle_linear(x, w, T, H, N, float(r), rp, nr, Y, idx), "oracle_linear")
+    _check(_load().oracle_linear(x, w, T, H, N, float(r), rp, nr, cp, nc, Y, idx), "oracle_linear")
     return Y, idx
 
 

@@ -145,58 +145,58 @@ int oracle_select(const uint16_t* s, long H, long k, int32_t* idx) {
 
 /* ---- §5.3 gather + smaller dense product ---------------------------------- */
 
-/* Y[r, n] = sum over j < k of X[t_r, idx[j]] * W[n, idx[j]], in fp64, summed
- * over ascending j.  X is [T, H], W is [N, H] (the layer's weight as stored
- * by the model: one row per output feature).  rows selects which token rows
- * t_r to compute (NULL: all T rows, in order); Y is [nrows, N].
+/* Y[r, c] = sum over j < k of X[t_r, idx[j]] * W[n_c, idx[j]], in fp64,
+ * summed over ascending j.  X is [T, H], W is [N, H] (the layer's weight as
+ * stored by the model: one row per output feature).  rows selects which
+ * token rows t_r to compute (NULL: all T rows, in order) and cols which
+ * output features n_c (NULL: all N, in order); Y is [nrows, ncols].
  * idx may hold any list of distinct in-range indices (used by the tests to
  * form complementary sets). */
 int oracle_reduced_product(const uint16_t* X, const uint16_t* W, long T, long H, long N,
                            const int32_t* idx, long k, const int64_t* rows, long nrows,
-                           double* Y) {
+                           const int64_t* cols, long ncols, double* Y) {
     if (!X || !W || !idx || !Y || T < 1 || H < 1 || N < 1 || k < 1 || k > H) return ORACLE_ERR_ARG;
     if (!rows) nrows = T;
-    if (nrows < 0) return ORACLE_ERR_ARG;
+    if (!cols) ncols = N;
+    if (nrows < 0 || ncols < 0) return ORACLE_ERR_ARG;
     for (long j = 0; j < k; ++j)
         if (idx[j] < 0 || idx[j] >= H) return ORACLE_ERR_ARG;
+    for (long r = 0; r < nrows; ++r)
+        if (rows && (rows[r] < 0 || rows[r] >= T)) return ORACLE_ERR_ARG;
+    for (long c = 0; c < ncols; ++c)
+        if (cols && (cols[c] < 0 || cols[c] >= N)) return ORACLE_ERR_ARG;
     if (!all_finite(X, T * H) || !all_finite(W, N * H)) return ORACLE_ERR_NONFINITE;
 
-    /* gather the kept slices of W into a compact [N, k] fp64 operand */
-    double* Wk = (double*)malloc(sizeof(double) * (size_t)N * (size_t)k);
     double* xk = (double*)malloc(sizeof(double) * (size_t)k);
-    if (!Wk || !xk) {
-        free(Wk);
+    double* wk = (double*)malloc(sizeof(double) * (size_t)k);
+    if (!xk || !wk) {
         free(xk);
+        free(wk);
         return ORACLE_ERR_NOMEM;
     }
-    for (long n = 0; n < N; ++n)
-        for (long j = 0; j < k; ++j) Wk[n * k + j] = bf16_to_double(W[n * H + idx[j]]);
-
     for (long r = 0; r < nrows; ++r) {
         long t = rows ? (long)rows[r] : r;
-        if (t < 0 || t >= T) {
-            free(Wk);
-            free(xk);
-            return ORACLE_ERR_ARG;
-        }
         /* gather the kept slices of this activation row */
         for (long j = 0; j < k; ++j) xk[j] = bf16_to_double(X[t * H + idx[j]]);
-        for (long n = 0; n < N; ++n) {
+        for (long c = 0; c < ncols; ++c) {
+            long n = cols ? (long)cols[c] : c;
+            /* gather the same kept slices of the weight row, then the smaller dot product */
+            for (long j = 0; j < k; ++j) wk[j] = bf16_to_double(W[n * H + idx[j]]);
             double acc = 0.0;
-            const double* w = Wk + n * k;
-            for (long j = 0; j < k; ++j) acc += xk[j] * w[j];
-            Y[r * N + n] = acc;
+            for (long j = 0; j < k; ++j) acc += xk[j] * wk[j];
+            Y[r * ncols + c] = acc;
         }
     }
-    free(Wk);
     free(xk);
+    free(wk);
     return 0;
 }
 
 /* The whole reduced linear map: k = ceil(r*H); score; select; gather and
  * product.  idx_out (k entries, may be NULL) receives the kept set. */
 int oracle_linear(const uint16_t* X, const uint16_t* W, long T, long H, long N, double r,
-                  const int64_t* rows, long nrows, double* Y, int32_t* idx_out) {
+                  const int64_t* rows, long nrows, const int64_t* cols, long ncols, double* Y,
+                  int32_t* idx_out) {
     int k = oracle_k_for(H, r);
     if (k < 1) return ORACLE_ERR_ARG;
     if (!X || !W || !Y || T < 1 || N < 1) return ORACLE_ERR_ARG;
@@ -209,7 +209,7 @@ int oracle_linear(const uint16_t* X, const uint16_t* W, long T, long H, long N, 
     }
     int rc = oracle_score(X, T, H, s);
     if (rc == 0) rc = oracle_select(s, H, k, idx);
-    if (rc == 0) rc = oracle_reduced_product(X, W, T, H, N, idx, k, rows, nrows, Y);
+    if (rc == 0) rc = oracle_reduced_product(X, W, T, H, N, idx, k, rows, nrows, cols, ncols, Y);
     if (rc == 0 && idx_out) memcpy(idx_out, idx, sizeof(int32_t) * (size_t)k);
     free(s);
     free(idx);

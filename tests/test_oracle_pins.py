@@ -290,3 +290,13 @@ def test_swiglu_closed_form():
     out = oracle.swiglu(g, u)
     want = [0.0, 2.0 / (1 + math.exp(-1.0)), -2.0 / (1 + math.exp(2.0)), -3.0 / (1 + math.exp(-3.0))]
     assert np.allclose(out, want, rtol=0, atol=1e-15)
+
+
+def test_row_and_column_subsets():
+    X = rmm_synth.activations(9, 70, seed=81)
+    W = rmm_synth.weights(30, 70, seed=82)
+    Y, idx = oracle.linear(X, W, 0.3)
+    rows, cols = [8, 2, 5], [29, 0, 13, 7]
+    Ys, idx2 = oracle.linear(X, W, 0.3, rows=rows, cols=cols)
+    assert idx.tolist() == idx2.tolist()
+    assert np.array_equal(Ys, Y[np.ix_(rows, cols)])
