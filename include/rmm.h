@@ -71,7 +71,11 @@ typedef struct rmm_options {
      * limit, on a barrier that nothing signals; the call then reports
      * RMM_ERR_TIMEOUT through rmm_get_status() and leaves Y unspecified. */
     int debug_timeout_test;
-    int reserved[4]; /* must be zero */
+    /* Operand producer of the reduced GEMM: 0 (default) = four warps gather
+     * the kept rows with 16-byte cp.async into the swizzled layout; 1 = TMA
+     * tile::gather4 (one instruction per four kept rows x 64 columns). */
+    int gemm_producer;
+    int reserved[3]; /* must be zero */
     /* Optional pair of cudaEvent_t handles (NULL: none) recorded on the
      * stream immediately before and after the reduced-product kernel (GEMV or
      * GEMM) of rmm_linear / rmm_gemm_reduced, so that a caller can time that

@@ -33,7 +33,7 @@ int num_sms_current() {
 }
 
 const rmm_options& opts_or_default(const rmm_options* o) {
-    static const rmm_options d = {16, 0, 0, 0, {0, 0, 0, 0}, nullptr, nullptr};
+    static const rmm_options d = {16, 0, 0, 0, 0, {0, 0, 0}, nullptr, nullptr};
     return o ? *o : d;
 }
 
@@ -41,7 +41,8 @@ bool opts_valid(const rmm_options* o) {
     if (!o) return true;
     if (o->t_gemv < 0 || o->t_gemv > kGemvMaxT) return false;
     if (o->gemv_splits < 0) return false;
-    for (int i = 0; i < 4; ++i)
+    if (o->gemm_producer < 0 || o->gemm_producer > 1) return false;
+    for (int i = 0; i < 3; ++i)
         if (o->reserved[i] != 0) return false;
     return true;
 }
@@ -175,10 +176,16 @@ rmm_status run_product_kernel(const void* X, const void* Wt, const int32_t* idx_
                                        s));
     }
     CUtensorMap mx, mw;
-    if (!row_gather_map(ws + L.xt, (uint64_t)H, (uint64_t)T, (uint64_t)L.ldT, &mx)) return RMM_ERR_CUDA;
-    if (!row_gather_map(Wt, (uint64_t)H, (uint64_t)N, (uint64_t)N, &mw)) return RMM_ERR_CUDA;
-    return cuda_status(launch_gemm(mx, mw, idx_padded, k, T, H, N, static_cast<uint16_t*>(Y), status,
-                                   o.debug_timeout_test, num_sms_current(), s));
+    memset(&mx, 0, sizeof mx);
+    memset(&mw, 0, sizeof mw);
+    const uint16_t* xt = reinterpret_cast<const uint16_t*>(ws + L.xt);
+    if (o.gemm_producer == 1) {
+        if (!row_gather_map(xt, (uint64_t)H, (uint64_t)T, (uint64_t)L.ldT, &mx)) return RMM_ERR_CUDA;
+        if (!row_gather_map(Wt, (uint64_t)H, (uint64_t)N, (uint64_t)N, &mw)) return RMM_ERR_CUDA;
+    }
+    return cuda_status(launch_gemm(mx, mw, xt, L.ldT, static_cast<const uint16_t*>(Wt), idx_padded, k,
+                                   T, H, N, static_cast<uint16_t*>(Y), status, o.debug_timeout_test,
+                                   o.gemm_producer, num_sms_current(), s));
 }
 
 rmm_status run_product(const void* X, const void* Wt, const int32_t* idx_padded, int k, int T,

@@ -6,27 +6,42 @@
 // The reduced product is a dense contraction over the k kept slices
 // (cf-1.com post on input-adaptive matrix-product reduction, §5.3: the
 // smaller dense product; paper abstract: slices along the contraction
-// dimension).  Instead of gathering the kept slices into compacted copies
-// in memory (the post's demo does this, and §8 of the post names the copy
-// traffic as the method's first cost), the producer warp gathers them straight
-// into shared memory with TMA tile::gather4: each instruction brings four
-// kept rows (of X^T or of W^T) x 64 elements, so a K-block of 64 kept slices is
-// 16 gathers per 64-wide column group.  Both operands land MN-major in the
-// 128-byte-swizzled canonical layout that tcgen05.mma reads directly.
+// dimension).  The post's demo gathers the kept slices into compacted copies
+// in memory, and its §8 names that copy traffic as the method's first cost;
+// here the kept slices go straight from their home rows into shared memory,
+// and no compacted copy exists anywhere in HBM.
 //
-// Persistent, warp-specialised, one CTA per SM:
-//   warp 0     TMA producer (all 32 lanes issue gathers; 4-stage ring)
-//   warp 1     TMEM allocator and MMA issuer (one thread issues
-//              tcgen05.mma 128x256x16; tcgen05.commit frees ring slots and
+// A kept slice h is one contiguous row of W^T [H, N] and one contiguous row of
+// X^T [H, T] (written by the score pass).  For a 128 x 256 output tile and a
+// K-block of 64 kept slices the operands are 64 rows x 256 columns of W^T
+// (512 B per row) and 64 rows x 128 columns of X^T (256 B per row), placed
+// MN-major in the 128-byte-swizzled canonical layout that tcgen05.mma reads:
+// each 64-column group is a block of 64 rows x 128 B, and 16-byte chunk c of
+// row j sits at chunk position c ^ (j mod 8).
+//
+// Two producers fill that layout (template parameter):
+//   cp.async (default)  many warps; one warp instruction moves one 512-B row
+//                       segment (16 B per lane) into its swizzled place; each
+//                       thread's copies arrive on the stage barrier through
+//                       cp.async.mbarrier.arrive.  Padded slices (index H) and
+//                       columns past N or T are zero-filled.
+//   TMA tile::gather4   one warp; each instruction brings four kept rows x 64
+//                       columns (measured on B200: ~75 SM cycles of TMA time
+//                       per instruction, 96 per stage, which caps this
+//                       producer near 155 TFLOP/s -- kept for comparison).
+//
+// Persistent, warp-specialised, one CTA per SM (21 warps):
+//   warps 0-15   producer (measured: the copy-issue rate per warp is the
+//                limit, so the 96 row copies of a stage are spread over 16
+//                warps, 6 per warp, fully unrolled with precomputed offsets)
+//   warps 16-19  epilogue: tcgen05.ld 32 lanes x 32 columns -> bf16 -> global
+//                (warp w reads TMEM lanes 32*(w%4) .. +31)
+//   warp 20      TMEM allocator and MMA issuer (one thread issues
+//              tcgen05.mma 128x256x16, tcgen05.commit frees ring slots and
 //              signals finished accumulators)
-//   warps 2-5  epilogue: tcgen05.ld 32 lanes x 32 columns -> bf16 -> global
 // Two 256-column fp32 accumulators (all 512 TMEM columns) let the epilogue of
 // one tile overlap the main loop of the next.  Tiles are walked M-fastest so
 // CTAs running at the same time share W^T column blocks in L2.
-//
-// Tail handling: the kept list is padded with the index H (out of range) to a
-// multiple of 64; TMA zero-fills out-of-range rows, so padded slices add 0.
-// Rows t >= T of the last M tile are zero-filled the same way and not stored.
 //
 // Every wait is bounded (rmm_common.cuh): a stalled pipeline reports
 // RMM_ERR_TIMEOUT through the status word and the CTA drains its in-flight
@@ -42,13 +57,20 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = kGemmBK;  // 64
 constexpr int STAGES = 4;
-constexpr int CHUNK_BYTES = BK * 128;           // BK rows x 64 bf16 (one swizzle-atom column)
+constexpr int CHUNK_BYTES = BK * 128;                   // BK rows x 64 bf16 (one swizzle-atom column)
 constexpr int A_STAGE_BYTES = (BM / 64) * CHUNK_BYTES;  // 16 KB
 constexpr int B_STAGE_BYTES = (BN / 64) * CHUNK_BYTES;  // 32 KB
 constexpr uint32_t STAGE_TX = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int kThreads = 192;
+constexpr int kProducerWarps = 16;
+constexpr int kRowsB = BK / kProducerWarps;        // W^T row copies per producer warp and stage
+constexpr int kRowsA = BK / (2 * kProducerWarps);  // X^T double-row copies per producer warp and stage
+static_assert(BK % (2 * kProducerWarps) == 0, "row copies must divide evenly over the producer warps");
+constexpr int kProducerThreads = 32 * kProducerWarps;
 constexpr int kEpilogueWarps = 4;
+constexpr int kFirstEpilogueWarp = kProducerWarps;
+constexpr int kMmaWarp = kProducerWarps + kEpilogueWarps;
+constexpr int kThreads = 32 * (kMmaWarp + 1);
 
 struct __align__(8) Barriers {
     uint64_t full[STAGES];
@@ -60,11 +82,20 @@ struct __align__(8) Barriers {
     int abort_flag;
 };
 
-constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + (size_t)STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) +
-                              sizeof(Barriers);
+constexpr size_t kSmemBytes =
+    1024 /*alignment slack*/ + (size_t)STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + sizeof(Barriers);
 
+// Byte offset, inside a stage's operand block, of 16-byte chunk c16 (counted
+// along M/N from the tile start) of kept row j, in the 128-byte-swizzled
+// MN-major canonical layout.
+__device__ __forceinline__ uint32_t swz_offset(int j, int c16) {
+    return (uint32_t)((c16 >> 3) * CHUNK_BYTES + j * 128 + (((c16 & 7) ^ (j & 7)) << 4));
+}
+
+template <bool kTmaGather>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_xt, const __grid_constant__ CUtensorMap map_wt,
+                const uint16_t* __restrict__ Xt, int ldT, const uint16_t* __restrict__ Wt,
                 const int32_t* __restrict__ idx, int k, int T, int H, int N,
                 uint16_t* __restrict__ Y, int* status, int debug_timeout) {
     extern __shared__ uint8_t smem_raw[];
@@ -84,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_addr(&bars->full[s]), 1);
+            mbar_init(smem_addr(&bars->full[s]), kTmaGather ? 1 : kProducerThreads);
             mbar_init(smem_addr(&bars->empty[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -95,11 +126,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         bars->abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
+    if (kTmaGather && warp == 0 && lane == 0) {
         tma_prefetch_desc(&map_xt);
         tma_prefetch_desc(&map_wt);
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(smem_addr(&bars->tmem_base), TMEM_COLS);
         tmem_relinquish();
     }
@@ -108,38 +139,93 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = bars->tmem_base;
 
-    if (warp == 0) {
+    if (warp < kProducerWarps) {
         // ------------------------------------------------------------ producer
         int stage = 0;
         uint32_t phase = 0;
-        uint32_t armed_mask = 0, armed_parity = 0;  // per stage: armed at least once / parity armed
+        uint32_t armed_mask = 0, armed_parity = 0;  // TMA producer: stages armed / parity armed
         bool ok = true;
-        const int g = lane & 15;     // group of 4 kept slices within the K-block
-        const int half = lane >> 4;  // which 64-wide column groups this lane gathers
+        // Kept indices of a K-block live in registers, two per lane
+        // (idx[kb*64 + lane], idx[kb*64 + 32 + lane]); they are fetched two
+        // K-blocks ahead so their latency never sits on the copy-issue path.
+        // The K-block sequence repeats 0..nkb-1 for every tile.
+        int q0a = 0, q1a = 0, q0b = 0, q1b = 0, next_kb = 0;
+        if (!kTmaGather) {
+            q0a = __ldg(idx + lane);
+            q1a = __ldg(idx + 32 + lane);
+            next_kb = (1 < nkb) ? 1 : 0;
+            q0b = __ldg(idx + next_kb * BK + lane);
+            q1b = __ldg(idx + next_kb * BK + 32 + lane);
+            next_kb = (next_kb + 1 < nkb) ? next_kb + 1 : 0;
+        }
+        // swizzled shared-memory offsets of this thread's copies: fixed for every stage
+        uint32_t b_off[kRowsB], a_off[kRowsA];
+#pragma unroll
+        for (int i = 0; i < kRowsB; ++i) b_off[i] = swz_offset(warp + kProducerWarps * i, lane);
+#pragma unroll
+        for (int i = 0; i < kRowsA; ++i)
+            a_off[i] = swz_offset(2 * (warp + kProducerWarps * i) + (lane >> 4), lane & 15);
         for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
             const int m0 = (tile % m_tiles) * BM;
             const int n0 = (tile / m_tiles) * BN;
+            if (kTmaGather && warp != 0) break;
+            const int b_col = n0 + lane * 8;          // this lane's W^T columns
+            const int a_col = m0 + (lane & 15) * 8;   // this lane's X^T columns (tokens)
+            const bool b_col_ok = b_col < N;
+            const bool a_col_ok = a_col < T;
             for (int kb = 0; kb < nkb; ++kb) {
                 const uint32_t full = smem_addr(&bars->full[stage]);
                 if (!mbar_wait(smem_addr(&bars->empty[stage]), phase ^ 1, status, abort_flag)) {
                     ok = false;
                     break;
                 }
-                if (lane == 0) mbar_arrive_expect_tx(full, STAGE_TX);
-                __syncwarp();
-                armed_mask |= 1u << stage;
-                armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-                const int j = kb * BK + g * 4;
-                const int r0 = __ldg(idx + j), r1 = __ldg(idx + j + 1);
-                const int r2 = __ldg(idx + j + 2), r3 = __ldg(idx + j + 3);
-                const uint32_t a_dst =
-                    smem_addr(sA + stage * A_STAGE_BYTES + half * CHUNK_BYTES + g * 512);
-                tma_gather4(a_dst, &map_xt, full, m0 + half * 64, r0, r1, r2, r3);
+                const uint32_t a_stage = smem_addr(sA + stage * A_STAGE_BYTES);
+                const uint32_t b_stage = smem_addr(sB + stage * B_STAGE_BYTES);
+                if constexpr (kTmaGather) {
+                    if (lane == 0) mbar_arrive_expect_tx(full, STAGE_TX);
+                    __syncwarp();
+                    armed_mask |= 1u << stage;
+                    armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                    const int g = lane & 15, half = lane >> 4;
+                    const int j = kb * BK + g * 4;
+                    const int r0 = __ldg(idx + j), r1 = __ldg(idx + j + 1);
+                    const int r2 = __ldg(idx + j + 2), r3 = __ldg(idx + j + 3);
+                    tma_gather4(a_stage + half * CHUNK_BYTES + g * 512, &map_xt, full, m0 + half * 64, r0,
+                                r1, r2, r3);
 #pragma unroll
-                for (int c = half; c < BN / 64; c += 2) {
-                    const uint32_t b_dst =
-                        smem_addr(sB + stage * B_STAGE_BYTES + c * CHUNK_BYTES + g * 512);
-                    tma_gather4(b_dst, &map_wt, full, n0 + c * 64, r0, r1, r2, r3);
+                    for (int c = half; c < BN / 64; c += 2)
+                        tma_gather4(b_stage + c * CHUNK_BYTES + g * 512, &map_wt, full, n0 + c * 64, r0, r1,
+                                    r2, r3);
+                } else {
+                    // kept indices of this K-block (the list is padded with H)
+                    const int v0 = q0a, v1 = q1a;
+                    q0a = q0b;
+                    q1a = q1b;
+                    q0b = __ldg(idx + next_kb * BK + lane);
+                    q1b = __ldg(idx + next_kb * BK + 32 + lane);
+                    next_kb = (next_kb + 1 < nkb) ? next_kb + 1 : 0;
+                    // W^T: 64 rows x 32 chunks; warp w copies rows w + PW*i (one
+                    // 512-B row segment per warp instruction, lane = 16-B chunk)
+#pragma unroll
+                    for (int i = 0; i < kRowsB; ++i) {
+                        const int jr = warp + kProducerWarps * i;  // warp-uniform
+                        const int h = __shfl_sync(0xffffffffu, jr < 32 ? v0 : v1, jr & 31);
+                        const bool ok_copy = b_col_ok && h < H;
+                        const uint16_t* src = ok_copy ? Wt + (size_t)h * N + b_col : Wt;
+                        cp_async_16(b_stage + b_off[i], src, ok_copy ? 16u : 0u);
+                    }
+                    // X^T: 64 rows x 16 chunks; a warp instruction covers two rows
+#pragma unroll
+                    for (int i = 0; i < kRowsA; ++i) {
+                        const int jr = 2 * (warp + kProducerWarps * i) + (lane >> 4);
+                        const int h0v = __shfl_sync(0xffffffffu, v0, jr & 31);
+                        const int h1v = __shfl_sync(0xffffffffu, v1, jr & 31);
+                        const int h = jr < 32 ? h0v : h1v;
+                        const bool ok_copy = a_col_ok && h < H;
+                        const uint16_t* src = ok_copy ? Xt + (size_t)h * ldT + a_col : Xt;
+                        cp_async_16(a_stage + a_off[i], src, ok_copy ? 16u : 0u);
+                    }
+                    cp_async_arrive_noinc(full);
                 }
                 if (++stage == STAGES) {
                     stage = 0;
@@ -147,18 +233,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-        // Drain: every armed stage's copies must land before the CTA exits
-        // (a no-op on the normal path, where the MMA warp consumed them all).
-        if (lane == 0) {
-            for (int s = 0; s < STAGES; ++s) {
-                if (armed_mask & (1u << s)) {
-                    int tmp_abort = 0;  // drain even after an abort
-                    mbar_wait(smem_addr(&bars->full[s]), (armed_parity >> s) & 1u, status,
-                              &tmp_abort, kDebugWaitLimitNs);
+        if constexpr (kTmaGather) {
+            // Drain: every armed stage's copies must land before the CTA exits
+            // (a no-op on the normal path, where the MMA warp consumed them all).
+            if (warp == 0 && lane == 0) {
+                for (int s = 0; s < STAGES; ++s) {
+                    if (armed_mask & (1u << s)) {
+                        int tmp_abort = 0;  // drain even after an abort
+                        mbar_wait(smem_addr(&bars->full[s]), (armed_parity >> s) & 1u, status, &tmp_abort,
+                                  kDebugWaitLimitNs);
+                    }
                 }
             }
+        } else {
+            cp_async_wait_all();
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc = idesc_bf16_f32_mn_mn(BM, BN);
         int stage = 0;
@@ -180,6 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
+                if (!kTmaGather) fence_proxy_async_smem();  // cp.async wrote the stage
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t a_base = smem_addr(sA + stage * A_STAGE_BYTES);
@@ -209,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int q = warp & 3;  // TMEM lane quarter (four consecutive warps cover all four)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -252,23 +343,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+    if (warp == kMmaWarp) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
 }  // namespace
 
 size_t gemm_smem_bytes() { return kSmemBytes; }
 
-cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt, const int32_t* idx,
-                        int k, int T, int H, int N, uint16_t* Y, int* status, int debug_timeout,
-                        int num_sms, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt, const uint16_t* Xt,
+                        int ldT, const uint16_t* Wt, const int32_t* idx, int k, int T, int H, int N,
+                        uint16_t* Y, int* status, int debug_timeout, int tma_gather, int num_sms,
+                        cudaStream_t stream) {
+    auto kern = tma_gather ? gemm_kernel<true> : gemm_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const int tiles = ((T + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = tiles < num_sms ? tiles : num_sms;
-    gemm_kernel<<<grid, kThreads, kSmemBytes, stream>>>(map_xt, map_wt, idx, k, T, H, N, Y, status,
-                                                         debug_timeout);
+    kern<<<grid, kThreads, kSmemBytes, stream>>>(map_xt, map_wt, Xt, ldT, Wt, idx, k, T, H, N, Y, status,
+                                                  debug_timeout);
     return cudaGetLastError();
 }
 

@@ -41,9 +41,11 @@ cudaError_t launch_gemv(const uint16_t* X, int T, int H, const uint16_t* Wt, int
                         cudaStream_t stream);
 
 // ---- tcgen05 GEMM (rmm_gemm.cu)
-cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt,
-                        const int32_t* idx, int k, int T, int H, int N, uint16_t* Y,
-                        int* status, int debug_timeout, int num_sms, cudaStream_t stream);
+// map_xt / map_wt are used only by the TMA tile::gather4 producer (tma_gather != 0).
+cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt, const uint16_t* Xt,
+                        int ldT, const uint16_t* Wt, const int32_t* idx, int k, int T, int H, int N,
+                        uint16_t* Y, int* status, int debug_timeout, int tma_gather, int num_sms,
+                        cudaStream_t stream);
 size_t gemm_smem_bytes();
 
 // ---- attention (rmm_attn.cu)

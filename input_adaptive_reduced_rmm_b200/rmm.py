@@ -43,19 +43,24 @@ class rmm_options(ctypes.Structure):
         ("attn_per_query_head", ctypes.c_int),
         ("gemv_splits", ctypes.c_int),
         ("debug_timeout_test", ctypes.c_int),
-        ("reserved", ctypes.c_int * 4),
+        ("gemm_producer", ctypes.c_int),
+        ("reserved", ctypes.c_int * 3),
         ("product_event_begin", ctypes.c_void_p),
         ("product_event_end", ctypes.c_void_p),
     ]
 
 
 def options(t_gemv: int = 16, attn_per_query_head: bool = False, gemv_splits: int = 0,
-            debug_timeout_test: bool = False, product_events=None) -> rmm_options:
+            debug_timeout_test: bool = False, gemm_producer: int = 0, product_events=None) -> rmm_options:
     """An rmm_options struct; product_events = (begin, end) torch.cuda.Event pair (enable_timing)."""
     o = rmm_options(int(t_gemv), int(bool(attn_per_query_head)), int(gemv_splits),
-                    int(bool(debug_timeout_test)), (ctypes.c_int * 4)(0, 0, 0, 0), None, None)
+                    int(bool(debug_timeout_test)), int(gemm_producer), (ctypes.c_int * 3)(0, 0, 0),
+                    None, None)
     if product_events is not None:
         b, e = product_events
+        for ev in (b, e):
+            if ev.cuda_event == 0:  # torch creates the CUDA event on its first record
+                ev.record()
         o.product_event_begin = ctypes.c_void_p(b.cuda_event)
         o.product_event_end = ctypes.c_void_p(e.cuda_event)
     return o
