@@ -128,13 +128,20 @@ def dist_setup():
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The largest of the ranks' values (device time of a multi-GPU run is the slowest rank's)."""
     if world == 1:
         return v
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job rate: the units all ranks processed over the slowest rank's time (per second)."""
+    return units_per_rank * world / (ms_max * 1e-3)
 
 
 def barrier(world):
@@ -146,6 +153,20 @@ def barrier(world):
 
 # ------------------------------------------------------------------ oracle (CPU baseline)
 
+_host_inputs = None
+
+
+def host_inputs():
+    """The step's activations and weights on the host (bf16), generated once."""
+    global _host_inputs
+    if _host_inputs is None:
+        acts = {s: rmm_synth.activations(T_PREFILL, h, rmm_synth.seed_for(1, 70 + s, 0)) for s, h in ACT_H.items()}
+        weights = {n: rmm_synth.weights(N, H, rmm_synth.seed_for(1, 80 + i, 1), std=0.02)
+                   for i, (n, H, N, _) in enumerate(PROJ)}
+        _host_inputs = (acts, weights)
+    return _host_inputs
+
+
 def oracle_sample(rows_per_proj: int, seed: int):
     """Time the CPU oracle on `rows_per_proj` token rows of every projection (full score/select).
 
@@ -153,9 +174,7 @@ def oracle_sample(rows_per_proj: int, seed: int):
     import oracle
 
     oracle.build()
-    acts = {s: rmm_synth.activations(T_PREFILL, h, rmm_synth.seed_for(1, 70 + s, 0)) for s, h in ACT_H.items()}
-    weights = {n: rmm_synth.weights(N, H, rmm_synth.seed_for(1, 80 + i, 1), std=0.02)
-               for i, (n, H, N, _) in enumerate(PROJ)}
+    acts, weights = host_inputs()
     g = torch.Generator().manual_seed(seed)
     flops, secs = 0, 0.0
     for name, H, N, s in PROJ:
@@ -199,13 +218,11 @@ def run_reference(args, world, rank):
 def make_inputs(dev):
     from input_adaptive_reduced_rmm_b200 import rmm
 
-    acts = {s: rmm_synth.activations(T_PREFILL, h, rmm_synth.seed_for(1, 70 + s, 0)).to(dev)
-            for s, h in ACT_H.items()}
-    Wts, Wfull = {}, {}
-    for i, (name, H, N, _) in enumerate(PROJ):
-        W = rmm_synth.weights(N, H, rmm_synth.seed_for(1, 80 + i, 1), std=0.02).to(dev)
-        Wts[name] = rmm.rmm_transpose_weight(W)
-        Wfull[name] = W
+    hacts, hweights = host_inputs()
+    acts = {s: a.to(dev) for s, a in hacts.items()}
+    Wts = {}
+    for name, H, N, _ in PROJ:
+        Wts[name] = rmm.rmm_transpose_weight(hweights[name].to(dev))
     torch.cuda.synchronize()
     return acts, Wts
 
@@ -300,7 +317,7 @@ def run_rmm(args, world, rank, local):
     clk = clocks.stop()
     ms = t0.elapsed_time(t1)
     ms_max = max_over_ranks(ms, world)
-    value = step_flops * K * world / (ms_max * 1e-3) / 1e12
+    value = job_throughput(step_flops * K, world, ms_max) / 1e12
 
     # dominant kernel: the reduced GEMM launches, timed by events recorded around each one
     gemm_ms = {n: sum(b.elapsed_time(e) for b, e in evs[n]) / K for n, _, _, _ in PROJ}
@@ -352,7 +369,7 @@ def run_rmm(args, world, rank, local):
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = step_flops * K * world / (e2e_ms * 1e-3) / 1e12
+    e2e_value = job_throughput(step_flops * K, world, e2e_ms) / 1e12
 
     extra = time_decode_and_attention(dev, peaks) if not args.skip_secondary else {}
 

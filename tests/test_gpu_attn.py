@@ -1,0 +1,131 @@
+"""GPU parity of the reduced attention (Q K^T reduced along the head dimension, then softmax . V).
+
+Every call goes through the C ABI.  Kept head-dimension sets are compared bit
+for bit with the oracle; outputs within the float bar of tests/parity.py.
+The key cache is handed to the library d-major (K^T [B, Hkv, d, ldL]) with a
+padded leading dimension; the oracle takes K in its natural [B, Hkv, L, d].
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rmm_synth
+from parity import assert_close, sample_indices
+
+pytestmark = pytest.mark.gpu
+D = 128
+
+
+@pytest.fixture(scope="module")
+def rmm():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from input_adaptive_reduced_rmm_b200 import rmm as _rmm
+
+    _rmm.lib()
+    return _rmm
+
+
+def to_device_cache(K, V, pad=8):
+    """K, V [B, Hkv, L, d] (CPU) -> d-major K^T [B, Hkv, d, ldL] and V [B, Hkv, ldL, d] on the GPU."""
+    B, Hkv, L, d = K.shape
+    ldL = (L + pad - 1) // pad * pad
+    Kt = torch.zeros(B, Hkv, d, ldL, dtype=torch.bfloat16)
+    Kt[..., :L] = K.transpose(-1, -2)
+    Vp = torch.zeros(B, Hkv, ldL, d, dtype=torch.bfloat16)
+    Vp[:, :, :L] = V
+    return Kt.cuda(), Vp.cuda()
+
+
+def run_attn(rmm, Q, K, V, r, causal=True, per_head=False, opts=None):
+    B, Hq, T, d = Q.shape
+    Hkv, L = K.shape[1], K.shape[2]
+    Kt, Vp = to_device_cache(K, V)
+    k = rmm.rmm_k_for(d, r)
+    nsets = Hq if per_head else Hkv
+    idx = torch.full((B, nsets, k), -1, dtype=torch.int32, device="cuda")
+    o = opts if opts is not None else rmm.options(attn_per_query_head=per_head)
+    ws = rmm.new_workspace(rmm.rmm_attn_workspace_bytes(B, Hq, Hkv, T, L, d, o))
+    O = rmm.rmm_attn_qk(Q.cuda(), Kt, Vp, L, r, causal=causal, idx_out=idx, workspace=ws, opts=o)
+    torch.cuda.synchronize()
+    assert rmm.rmm_get_status(ws) == rmm.RMM_OK
+    return O.cpu(), idx.cpu().numpy(), k
+
+
+@pytest.mark.parametrize("T,L", [(1, 37), (1, 1000), (5, 5), (5, 300), (33, 2100), (64, 64)])
+@pytest.mark.parametrize("r", [0.25, 0.5, 1.0])
+@pytest.mark.parametrize("causal", [True, False])
+def test_attention_small(rmm, T, L, r, causal):
+    B, Hq, Hkv = 2, 8, 2
+    seed = rmm_synth.seed_for(7, T, L % 10)
+    Q = rmm_synth.normal((B, Hq, T, D), seed)
+    K = rmm_synth.normal((B, Hkv, L, D), seed + 1)
+    V = rmm_synth.normal((B, Hkv, L, D), seed + 2)
+    O, idx, k = run_attn(rmm, Q, K, V, r, causal)
+    Oo, io = oracle.attention(Q, K, V, k, causal=causal)
+    assert np.array_equal(idx, io)
+    assert_close(O, Oo, f"T={T} L={L} r={r} causal={causal}")
+
+
+@pytest.mark.parametrize("T", [1, 7])
+def test_attention_per_query_head(rmm, T):
+    B, Hq, Hkv, L = 1, 12, 3, 513
+    Q = rmm_synth.normal((B, Hq, T, D), 41)
+    K = rmm_synth.normal((B, Hkv, L, D), 42)
+    V = rmm_synth.normal((B, Hkv, L, D), 43)
+    O, idx, k = run_attn(rmm, Q, K, V, 0.25, True, per_head=True)
+    Oo, io = oracle.attention(Q, K, V, k, causal=True, per_query_head=True)
+    assert np.array_equal(idx, io)
+    assert_close(O, Oo, "per-query-head")
+
+
+def test_attention_tie_heavy_queries(rmm):
+    B, Hq, Hkv, T, L = 1, 4, 1, 3, 200
+    Q = rmm_synth.tie_heavy((B, Hq, T, D), 5)
+    K = rmm_synth.normal((B, Hkv, L, D), 6)
+    V = rmm_synth.normal((B, Hkv, L, D), 7)
+    O, idx, k = run_attn(rmm, Q, K, V, 0.5, True)
+    Oo, io = oracle.attention(Q, K, V, k, causal=True)
+    assert np.array_equal(idx, io)
+    assert_close(O, Oo, "ties")
+
+
+def check_large(rmm, cfg, B, Hq, Hkv, T, L, r, nrows):
+    seed = rmm_synth.seed_for(cfg, T % 100, L % 97)
+    Q = rmm_synth.normal((B, Hq, T, D), seed)
+    K = rmm_synth.normal((B, Hkv, L, D), seed + 1)
+    V = rmm_synth.normal((B, Hkv, L, D), seed + 2)
+    O, idx, k = run_attn(rmm, Q, K, V, r, True)
+    rows = sample_indices(T, nrows, seed=L + T)
+    Oo, io = oracle.attention(Q, K, V, k, causal=True, t_rows=rows)
+    assert np.array_equal(idx, io)
+    assert_close(O[:, :, rows], Oo, f"cfg{cfg} T={T} L={L} r={r}")
+
+
+@pytest.mark.parametrize("L", [4096, 16384, 32768])
+@pytest.mark.parametrize("T", [1, 512])
+@pytest.mark.parametrize("r", [0.25, 0.5])
+def test_attention_llama3_8b(rmm, L, T, r):
+    """Batch 1, 32 query / 8 KV heads, d = 128, decode and a prefill chunk of 512."""
+    check_large(rmm, 2, 1, 32, 8, T, L, r, nrows=3)
+
+
+@pytest.mark.parametrize("T", [1, 512])
+def test_attention_llama3_70b(rmm, T):
+    """64 query / 8 KV heads, d = 128, KV length 65536."""
+    check_large(rmm, 4, 1, 64, 8, T, 65536, 0.5, nrows=2)
+
+
+def test_attention_rejects_bad_head_dim(rmm):
+    L = rmm.lib()
+    Q = torch.zeros(1, 2, 1, 64, dtype=torch.bfloat16, device="cuda")
+    Kt = torch.zeros(1, 1, 64, 16, dtype=torch.bfloat16, device="cuda")
+    V = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16, device="cuda")
+    ws = rmm.new_workspace(4096)
+    p = rmm._ptr
+    rc = L.rmm_attn_qk(p(Q), p(Kt), p(V), 1, 2, 1, 1, 16, 16, 64, 0.5, 1, 1.0 / math.sqrt(64), p(Q), None,
+                       p(ws), ws.numel(), rmm._stream(None), None)
+    assert rc == rmm.RMM_ERR_UNSUPPORTED
