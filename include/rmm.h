@@ -170,6 +170,29 @@ rmm_status rmm_attn_qk(const void* Q, const void* Kt, const void* V, int B, int 
                        int32_t* idx_out, void* workspace, size_t workspace_bytes,
                        rmm_stream_t stream, const rmm_options* options);
 
+/* The decode-sized reduced linear map without a workspace.  The pages have
+ * no counterpart to this entry point; it exists for callers that cannot give
+ * the library device memory of its own: a plugin whose host framework owns
+ * every allocation and only lends it input and output buffers, a serving loop
+ * with a fixed memory budget, code being recorded into a CUDA graph (where a
+ * cudaMalloc would break the capture).
+ * Computes exactly what rmm_linear computes on its split-K GEMV path
+ * (score -> kept set -> reduced product), but all intermediates live in a
+ * fixed 4 MiB array inside the library: every GPU that loads the library
+ * holds that array until the process exits.  Nothing is allocated or freed.
+ *   X, Wt, T, H, N, r, Y, idx_out: as for rmm_linear.
+ * Limits: T <= 16 (decode sizes), H <= 65535, N % 8 == 0, N <= 2^20; sizes
+ * beyond these return RMM_ERR_UNSUPPORTED with nothing launched.  Large T*N
+ * use fewer splits so that the partial sums fit in the array.
+ * The first call on a device (with that device current) looks up the array's
+ * device address once; make that first call before any stream capture.
+ * Every call uses the same array: calls that may overlap on the GPU (on
+ * different streams, or from different threads) race and must not be
+ * issued; calls in one stream are ordered and safe.  The array keeps the
+ * previous call's contents; each call clears what must start at zero. */
+rmm_status rmm_linear_decode_noalloc(const void* X, const void* Wt, int T, int H, int N, double r,
+                                     void* Y, int32_t* idx_out, rmm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -227,6 +227,12 @@ GemvPlan gemv_plan(int T, int N, int k, int num_sms, int forced_splits) {
     return p;
 }
 
+size_t gemv_smem_bytes(const GemvPlan& p, int T) {
+    const int TT = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : T <= 8 ? 8 : 16;
+    return (size_t)p.rows_per_split * TT * sizeof(float) + (size_t)p.rows_per_split * sizeof(int) +
+           (size_t)TT * p.cols_per_cta * sizeof(float);
+}
+
 size_t gemv_partials_bytes(const GemvPlan& p, int T, int N) {
     return p.splits > 1 ? (size_t)p.splits * T * N * sizeof(float) : 0;
 }

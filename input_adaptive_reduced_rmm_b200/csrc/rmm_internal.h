@@ -35,6 +35,8 @@ struct GemvPlan {
 };
 GemvPlan gemv_plan(int T, int N, int k, int num_sms, int forced_splits);
 size_t gemv_partials_bytes(const GemvPlan& p, int T, int N);
+size_t gemv_smem_bytes(const GemvPlan& p, int T);  // dynamic shared memory of one CTA
+constexpr size_t kGemvMaxSmemBytes = 200 * 1024;
 cudaError_t launch_gemv(const uint16_t* X, int T, int H, const uint16_t* Wt, int N,
                         const int32_t* idx, int k, uint16_t* Y, float* partials,
                         unsigned* counters, const GemvPlan& plan, int* status,

@@ -1,0 +1,115 @@
+// rmm_noalloc.cu -- the decode-sized reduced linear map with library-owned scratch.
+//
+// Some callers cannot hand the library a workspace: they run where allocating
+// device memory is not allowed or not safe -- a plugin whose host framework owns
+// every allocation and only lends it input and output buffers, an inference
+// loop with a fixed memory budget that must not grow at run time, or code that
+// is being recorded into a CUDA graph, where a cudaMalloc would break the
+// capture.  rmm_linear_decode_noalloc serves them: the same score -> kept set ->
+// split-K GEMV path as rmm_linear for T <= 16, but every intermediate (partial
+// maxima, the kept list, the split partial sums, the split counters) lives in
+// one file-scope __device__ array of fixed size that every GPU loading the
+// library holds until the process exits.  Nothing is allocated or freed.
+//
+// Host code never uses the array's name as a device address: on first use on
+// a device (with that device current) the address is obtained once with
+// cudaGetSymbolAddress, checked, cached per device, and passed to the kernels.
+#include <mutex>
+
+#include "rmm_common.cuh"
+#include "rmm_internal.h"
+
+namespace rmm {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB per device
+constexpr size_t kNoAllocStatusBytes = 256;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+size_t up256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Device address of the scratch array on the current device (set up once per device).
+rmm_status noalloc_scratch(uint8_t** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RMM_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return RMM_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> g(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RMM_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = static_cast<uint8_t*>(g_noalloc_ptr[dev]);
+    return RMM_OK;
+}
+
+// Zero the words a call needs to start at zero (split counters, status word);
+// the scratch keeps whatever the previous call left there.
+__global__ void noalloc_clear_kernel(unsigned* words, int n) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) words[i] = 0;
+}
+
+}  // namespace
+}  // namespace rmm
+
+using namespace rmm;
+
+extern "C" rmm_status rmm_linear_decode_noalloc(const void* X, const void* Wt, int T, int H, int N,
+                                                double r, void* Y, int32_t* idx_out,
+                                                rmm_stream_t stream) {
+    if (!X || !Wt || !Y || T < 1 || H < 1 || H > 65535 || N < 8 || N % 8 != 0) return RMM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(Wt) | reinterpret_cast<uintptr_t>(Y)) & 15)
+        return RMM_ERR_INVALID_ARG;
+    if (T > kGemvMaxT || N > (1 << 20)) return RMM_ERR_UNSUPPORTED;  // beyond the scratch's sizing
+    const int k = rmm_k_for(H, r);
+    if (k < 1) return RMM_ERR_INVALID_ARG;
+
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RMM_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return RMM_ERR_CUDA;
+    uint8_t* scratch = nullptr;
+    rmm_status st = noalloc_scratch(&scratch);
+    if (st != RMM_OK) return st;
+
+    // scratch layout: status | score partials | kept list | split counters | split partials
+    const int P = score_partials_for(T, H, sms);
+    GemvPlan plan = gemv_plan(T, N, k, sms, 0);
+    const size_t off_part = kNoAllocStatusBytes;
+    const size_t off_idx = off_part + up256((size_t)P * H * sizeof(uint16_t));
+    const size_t off_cnt = off_idx + up256(((size_t)H + 2 * kGemmBK) * sizeof(int32_t));
+    const size_t off_partials = off_cnt + up256((size_t)plan.col_blocks * sizeof(unsigned));
+    if (off_partials > kNoAllocScratchBytes) return RMM_ERR_UNSUPPORTED;
+    const size_t room = kNoAllocScratchBytes - off_partials;
+    if (gemv_partials_bytes(plan, T, N) > room) {
+        // fewer splits so that the partial sums fit; one split needs none
+        const size_t per_split = (size_t)T * N * sizeof(float);
+        int splits = (int)(room / per_split);
+        if (splits < 2) splits = 1;
+        plan = gemv_plan(T, N, k, sms, splits);
+        if (gemv_partials_bytes(plan, T, N) > room) return RMM_ERR_UNSUPPORTED;
+    }
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (gemv_smem_bytes(plan, T) > kGemvMaxSmemBytes) return RMM_ERR_UNSUPPORTED;
+    noalloc_clear_kernel<<<1, 256, 0, s>>>(reinterpret_cast<unsigned*>(scratch), (int)(kNoAllocStatusBytes / 4));
+    noalloc_clear_kernel<<<(plan.col_blocks + 255) / 256, 256, 0, s>>>(
+        reinterpret_cast<unsigned*>(scratch + off_cnt), plan.col_blocks);
+    if (cudaGetLastError() != cudaSuccess) return RMM_ERR_CUDA;
+
+    uint16_t* part = reinterpret_cast<uint16_t*>(scratch + off_part);
+    int32_t* idx = reinterpret_cast<int32_t*>(scratch + off_idx);
+    if (launch_score(static_cast<const uint16_t*>(X), T, H, part, P, nullptr, 0, s) != cudaSuccess)
+        return RMM_ERR_CUDA;
+    if (launch_select(part, P, nullptr, H, k, idx, k, idx_out, nullptr, s) != cudaSuccess) return RMM_ERR_CUDA;
+    if (launch_gemv(static_cast<const uint16_t*>(X), T, H, static_cast<const uint16_t*>(Wt), N, idx, k,
+                    static_cast<uint16_t*>(Y), reinterpret_cast<float*>(scratch + off_partials),
+                    reinterpret_cast<unsigned*>(scratch + off_cnt), plan,
+                    reinterpret_cast<int*>(scratch), s) != cudaSuccess)
+        return RMM_ERR_CUDA;
+    return RMM_OK;
+}

@@ -28,6 +28,7 @@ EXPORTED = (
     "rmm_status_string", "rmm_k_for", "rmm_workspace_init", "rmm_get_status",
     "rmm_transpose_weight", "rmm_linear_workspace_bytes", "rmm_linear", "rmm_score",
     "rmm_select", "rmm_gemm_reduced", "rmm_attn_workspace_bytes", "rmm_attn_qk",
+    "rmm_linear_decode_noalloc",
 )
 
 
@@ -93,6 +94,7 @@ def lib() -> ctypes.CDLL:
         "rmm_gemm_reduced": (I, [P, P, P, I, I, I, I, P, P, Z, P, OP]),
         "rmm_attn_workspace_bytes": (Z, [I, I, I, I, I, I, OP]),
         "rmm_attn_qk": (I, [P, P, P, I, I, I, I, I, I, I, D, I, F, P, P, P, Z, P, OP]),
+        "rmm_linear_decode_noalloc": (I, [P, P, I, I, I, D, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -256,3 +258,17 @@ def rmm_attn_qk(Q: torch.Tensor, Kt: torch.Tensor, V: torch.Tensor, L: int, r: f
                              int(bool(causal)), float(scale), _ptr(O), _ptr(idx_out), _ptr(workspace),
                              workspace.numel(), _stream(stream), _opt(opts)), "rmm_attn_qk")
     return O
+
+
+def rmm_linear_decode_noalloc(X: torch.Tensor, Wt: torch.Tensor, r: float, Y: torch.Tensor,
+                              idx_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The decode-sized reduced linear map (T <= 16) with no workspace: for callers that
+    cannot allocate device memory.  Y must be given (the binding allocates nothing)."""
+    _bf16_cuda(X, "X")
+    _bf16_cuda(Wt, "Wt")
+    _bf16_cuda(Y, "Y")
+    T, H = X.shape
+    N = Wt.shape[1]
+    _check(lib().rmm_linear_decode_noalloc(_ptr(X), _ptr(Wt), T, H, N, float(r), _ptr(Y), _ptr(idx_out),
+                                           _stream(stream)), "rmm_linear_decode_noalloc")
+    return Y
