@@ -3,10 +3,12 @@
 One step = one pass of the reduced linear map over the seven projections of a
 Llama-3-8B-shaped layer (q, k, v, o: 4096 -> 4096/1024/1024/4096; gate, up:
 4096 -> 14336; down: 14336 -> 4096) on a prefill batch of T = 2048 tokens at
-retention r = 0.5.  Each projection is one rmm_linear call through the C ABI
-(score -> kept set -> tcgen05 reduced GEMM), with random-init bf16 weights
-~N(0, 0.02) pre-transposed once and synthetic activations N(0, 1) with 2 % of
-the channels x20.
+retention r = 0.5, with random-init bf16 weights ~N(0, 0.02) pre-transposed
+once and synthetic activations N(0, 1) with 2 % of the channels x20.  As in
+the layer, q/k/v read one activation matrix and gate/up another, so each of
+those sets is one rmm_linear_group call (one score, one kept set, one grouped
+tcgen05 GEMM launch); o and down are rmm_linear calls: four C-ABI calls, three
+kernels each, per step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rmm|reference]
 
@@ -43,6 +45,8 @@ PROJ = [  # (name, H, N, activation stream)
     ("gate", 4096, 14336, 2), ("up", 4096, 14336, 2), ("down", 14336, 4096, 3),
 ]
 ACT_H = {0: 4096, 1: 4096, 2: 4096, 3: 14336}
+CALLS = [(0, ["q", "k", "v"]), (1, ["o"]), (2, ["gate", "up"]), (3, ["down"])]  # (activation, members)
+PROJ_BY_NAME = {n: (H, N) for n, H, N, _ in PROJ}
 WORKLOAD = "llama3-8b 7 projections (q,k,v,o,gate,up,down), prefill T=2048, r=0.5"
 METRIC = "reduced-GEMM effective TFLOP/s (2*T*N*k / time)"
 
@@ -284,23 +288,27 @@ def run_rmm(args, world, rank, local):
     acts, Wts = make_inputs(dev)
     ks = {n: metrics.k_for(H, R) for n, H, _, _ in PROJ}
     step_flops = sum(metrics.reduced_linear_flops(T_PREFILL, N, ks[n]) for n, _, N, _ in PROJ)
-    ws = {n: rmm.new_workspace(rmm.rmm_linear_workspace_bytes(T_PREFILL, H, N), dev) for n, H, N, _ in PROJ}
     Ys = {n: torch.empty(T_PREFILL, N, dtype=torch.bfloat16, device=dev) for n, _, N, _ in PROJ}
+    ws = {}
+    for c, (s, names) in enumerate(CALLS):
+        ws[c] = rmm.new_workspace(rmm.rmm_linear_group_workspace_bytes(
+            T_PREFILL, ACT_H[s], [PROJ_BY_NAME[n][1] for n in names]), dev)
     K, W = args.steps, args.warmup
-    evs = {n: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-           for n, _, _, _ in PROJ}
-    opt_timed = {n: [rmm.options(product_events=evs[n][i]) for i in range(K)] for n, _, _, _ in PROJ}
+    evs = {c: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+           for c in range(len(CALLS))}
+    opt_timed = {c: [rmm.options(product_events=evs[c][i]) for i in range(K)] for c in range(len(CALLS))}
 
     def step(i=None):
-        for n, H, N, s in PROJ:
-            o = opt_timed[n][i] if i is not None else None
-            rmm.rmm_linear(acts[s], Wts[n], R, Y=Ys[n], workspace=ws[n], opts=o)
+        for c, (s, names) in enumerate(CALLS):
+            o = opt_timed[c][i] if i is not None else None
+            rmm.rmm_linear_group(acts[s], [Wts[n] for n in names], R, Ys=[Ys[n] for n in names],
+                                 workspace=ws[c], opts=o)
 
     for _ in range(W):
         step()
     torch.cuda.synchronize()
-    for n, _, _, _ in PROJ:
-        if rmm.rmm_get_status(ws[n]) != rmm.RMM_OK:
+    for c in ws:
+        if rmm.rmm_get_status(ws[c]) != rmm.RMM_OK:
             raise RuntimeError("device status not OK after warm-up")
 
     clocks = ClockSampler(local if world > 1 else 0)
@@ -319,13 +327,16 @@ def run_rmm(args, world, rank, local):
     ms_max = max_over_ranks(ms, world)
     value = job_throughput(step_flops * K, world, ms_max) / 1e12
 
-    # dominant kernel: the reduced GEMM launches, timed by events recorded around each one
-    gemm_ms = {n: sum(b.elapsed_time(e) for b, e in evs[n]) / K for n, _, _, _ in PROJ}
+    # dominant kernel: the reduced GEMM launches, timed by events the library
+    # records around each product launch inside the timed region
+    gemm_ms = {c: sum(b.elapsed_time(e) for b, e in evs[c]) / K for c in range(len(CALLS))}
     gemm_total_ms = sum(gemm_ms.values())
     achieved = step_flops / (gemm_total_ms * 1e-3) / 1e12
-    per_proj = {n: {"H": H, "N": N, "k": ks[n], "gemm_us": 1e3 * gemm_ms[n],
-                    "gemm_tflops": metrics.reduced_linear_flops(T_PREFILL, N, ks[n]) / (gemm_ms[n] * 1e-3) / 1e12}
-                for n, H, N, _ in PROJ}
+    per_call = {}
+    for c, (s, names) in enumerate(CALLS):
+        f = sum(metrics.reduced_linear_flops(T_PREFILL, PROJ_BY_NAME[n][1], ks[n]) for n in names)
+        per_call["+".join(names)] = {"H": ACT_H[s], "N": [PROJ_BY_NAME[n][1] for n in names], "k": ks[names[0]],
+                                     "gemm_us": 1e3 * gemm_ms[c], "gemm_tflops": f / (gemm_ms[c] * 1e-3) / 1e12}
 
     # dense cuBLAS product of the same shapes, same stream, same inputs
     def dense_step():
@@ -344,8 +355,8 @@ def run_rmm(args, world, rank, local):
     dense_ms = d0.elapsed_time(d1) / K
     dense_flops = sum(metrics.gemm_flops(T_PREFILL, N, H) for _, H, N, _ in PROJ)
 
-    # end to end through the public call with host buffers: H2D of the step's activations,
-    # the seven calls, D2H of the seven outputs, every step
+    # end to end through the public calls with host buffers: H2D of the step's
+    # activations, the four calls, D2H of the seven outputs, every step
     host_acts = {s: a.cpu().pin_memory() for s, a in acts.items()}
     host_Y = {n: torch.empty(T_PREFILL, N, dtype=torch.bfloat16).pin_memory() for n, _, N, _ in PROJ}
     h2d = sum(a.numel() * 2 for a in host_acts.values())
@@ -386,19 +397,20 @@ def run_rmm(args, world, rank, local):
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "T": T_PREFILL, "r": R, "parallelism": f"replicas x{world}",
+                   "calls_per_step": "q+k+v grouped, o, gate+up grouped, down",
                    "l2": "inputs larger than L2 (0.55 GB of weights and activations per step)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None,
-                     "kernel": "gemm_kernel (tcgen05 reduced GEMM), all 7 launches of a step",
+                     "kernel": "gemm_kernel (tcgen05 reduced GEMM), the 4 launches of a step",
                      "peak_source": f"{peaks['source']} bf16 burst"},
         "speedup_vs_dense": dense_ms / (ms_max / K),
         "dense": {"ms_per_step": dense_ms, "tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
                   "effective_tflops_at_reduced_flops": step_flops / (dense_ms * 1e-3) / 1e12},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "cpu_baseline": cpu,
-        "gpu_launches": 3 * len(PROJ) * K,
+        "gpu_launches": 3 * len(CALLS) * K,
         "clocks": clk,
-        "per_projection": per_proj,
+        "per_call": per_call,
     }
     line.update(extra)
     print(json.dumps(line), flush=True)

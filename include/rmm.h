@@ -127,6 +127,24 @@ rmm_status rmm_linear(const void* X, const void* Wt, int T, int H, int N, double
                       int32_t* idx_out, void* workspace, size_t workspace_bytes,
                       rmm_stream_t stream, const rmm_options* options);
 
+/* Several projections of the same activations (e.g. q, k, v of one layer, or
+ * gate and up): since the score depends only on X, they share one kept set
+ * (cf-1.com post §8: one common set per batch), so the score pass, the kept
+ * set and (GEMM path) X^T are computed once and the products of all members
+ * run in one launch.  Y_p ~= X[:,S] W_p[:,S]^T for p < count.
+ *   X, T, H, r: as for rmm_linear
+ *   count: 1..4 members
+ *   Wts[p]: bf16 W_p^T [H, Ns[p]], Ys[p]: bf16 [T, Ns[p]] (host arrays of
+ *           device pointers; Ns[p] % 8 == 0)
+ *   idx_out: int32 [k] or NULL (the shared kept set, ascending)
+ *   workspace_bytes >= rmm_linear_group_workspace_bytes(T, H, count, Ns, options)
+ * With options.gemm_producer == 1 only count == 1 is supported. */
+size_t rmm_linear_group_workspace_bytes(int T, int H, int count, const int* Ns,
+                                        const rmm_options* options);
+rmm_status rmm_linear_group(const void* X, int T, int H, double r, int count, const void* const* Wts,
+                            const int* Ns, void* const* Ys, int32_t* idx_out, void* workspace,
+                            size_t workspace_bytes, rmm_stream_t stream, const rmm_options* options);
+
 /* Step 1 alone: s_out[h] = max_t |X[t,h]| as the bf16 magnitude key
  * (bit pattern with the sign cleared; -0 and +0 both give 0).  X bf16 [T, H],
  * s_out uint32 [H].  T >= 1. */

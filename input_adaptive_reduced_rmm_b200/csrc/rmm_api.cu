@@ -51,29 +51,32 @@ bool opts_valid(const rmm_options* o) {
 
 struct LinearLayout {
     bool gemv;
-    int P;       // score partial rows
-    int ldT;     // leading dimension of X^T (GEMM path)
-    GemvPlan plan;
-    size_t part, idx, counters, partials, xt, total;
+    int ldT;           // leading dimension of X^T (GEMM path)
+    int col_blocks;    // GEMV: most column blocks of any product
+    size_t s32, idx, counters, partials, xt, total;
 };
 
-// Workspace layout of the reduced linear map for kept count k (k = H gives
-// the largest layout, used by the size query).
-LinearLayout linear_layout(int T, int H, int N, int k, const rmm_options& o, int sms) {
+// Workspace layout for `count` products of one activation matrix [T, H] with
+// kept count k (k = H gives the largest layout, used by the size queries).
+LinearLayout linear_layout(int T, int H, const int* Ns, int count, int k, const rmm_options& o, int sms) {
     LinearLayout L{};
     L.gemv = T <= o.t_gemv;
-    L.P = score_partials_for(T, H, sms);
     size_t off = kStatusBytes;
-    L.part = off;
-    off += align_up((size_t)L.P * H * sizeof(uint16_t), kAlign);
+    L.s32 = off;
+    off += align_up((size_t)H * sizeof(uint32_t), kAlign);
     L.idx = off;
     off += align_up(((size_t)H + 2 * kGemmBK) * sizeof(int32_t), kAlign);
     if (L.gemv) {
-        L.plan = gemv_plan(T, N, k, sms, o.gemv_splits);
+        size_t part = 0;
+        for (int p = 0; p < count; ++p) {
+            const GemvPlan plan = gemv_plan(T, Ns[p], k, sms, o.gemv_splits);
+            if (plan.col_blocks > L.col_blocks) L.col_blocks = plan.col_blocks;
+            if (gemv_partials_bytes(plan, T, Ns[p]) > part) part = gemv_partials_bytes(plan, T, Ns[p]);
+        }
         L.counters = off;
-        off += align_up((size_t)L.plan.col_blocks * sizeof(unsigned), kAlign);
+        off += align_up((size_t)L.col_blocks * sizeof(unsigned), kAlign);
         L.partials = off;
-        off += align_up(gemv_partials_bytes(L.plan, T, N), kAlign);
+        off += align_up(part, kAlign);
     } else {
         L.ldT = (T + 7) / 8 * 8;
         L.xt = off;
@@ -155,50 +158,93 @@ bool row_gather_map(const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
 
 rmm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RMM_OK : RMM_ERR_CUDA; }
 
-bool linear_args_ok(const void* X, const void* Wt, int T, int H, int N, const void* Y) {
-    if (!X || !Wt || !Y) return false;
-    if (T < 1 || T > (1 << 20) || H < 1 || H > 65535 || N < 8 || N % 8 != 0) return false;
-    if (!aligned16(X) || !aligned16(Wt) || !aligned16(Y)) return false;
+bool group_args_ok(const void* X, int T, int H, int count, const void* const* Wts, const int* Ns,
+                   void* const* Ys) {
+    if (!X || !Wts || !Ns || !Ys || count < 1 || count > kMaxGroup) return false;
+    if (T < 1 || T > (1 << 20) || H < 1 || H > 65535 || !aligned16(X)) return false;
+    for (int p = 0; p < count; ++p) {
+        if (!Wts[p] || !Ys[p] || Ns[p] < 8 || Ns[p] % 8 != 0) return false;
+        if (!aligned16(Wts[p]) || !aligned16(Ys[p])) return false;
+    }
     return true;
 }
 
-// Shared tail of rmm_linear and rmm_gemm_reduced: the product on the chosen path.
-rmm_status run_product_kernel(const void* X, const void* Wt, const int32_t* idx_padded, int k,
-                              int T, int H, int N, void* Y, uint8_t* ws, const LinearLayout& L,
-                              const rmm_options& o, cudaStream_t s) {
+// The product step for every member of the group, on the chosen path.
+rmm_status run_product_kernels(const void* X, int T, int H, int count, const void* const* Wts,
+                               const int* Ns, void* const* Ys, const int32_t* idx_padded, int k,
+                               uint8_t* ws, const LinearLayout& L, const rmm_options& o,
+                               cudaStream_t s) {
     int* status = reinterpret_cast<int*>(ws);
+    const int sms = num_sms_current();
     if (L.gemv) {
-        return cuda_status(launch_gemv(static_cast<const uint16_t*>(X), T, H,
-                                       static_cast<const uint16_t*>(Wt), N, idx_padded, k,
-                                       static_cast<uint16_t*>(Y),
-                                       reinterpret_cast<float*>(ws + L.partials),
-                                       reinterpret_cast<unsigned*>(ws + L.counters), L.plan, status,
-                                       s));
+        for (int p = 0; p < count; ++p) {
+            const GemvPlan plan = gemv_plan(T, Ns[p], k, sms, o.gemv_splits);
+            cudaError_t e = launch_gemv(static_cast<const uint16_t*>(X), T, H,
+                                        static_cast<const uint16_t*>(Wts[p]), Ns[p], idx_padded, k,
+                                        static_cast<uint16_t*>(Ys[p]),
+                                        reinterpret_cast<float*>(ws + L.partials),
+                                        reinterpret_cast<unsigned*>(ws + L.counters), plan, status, s);
+            if (e != cudaSuccess) return RMM_ERR_CUDA;
+        }
+        return RMM_OK;
     }
+    if (o.gemm_producer == 1 && count != 1) return RMM_ERR_UNSUPPORTED;
     CUtensorMap mx, mw;
     memset(&mx, 0, sizeof mx);
     memset(&mw, 0, sizeof mw);
     const uint16_t* xt = reinterpret_cast<const uint16_t*>(ws + L.xt);
     if (o.gemm_producer == 1) {
         if (!row_gather_map(xt, (uint64_t)H, (uint64_t)T, (uint64_t)L.ldT, &mx)) return RMM_ERR_CUDA;
-        if (!row_gather_map(Wt, (uint64_t)H, (uint64_t)N, (uint64_t)N, &mw)) return RMM_ERR_CUDA;
+        if (!row_gather_map(Wts[0], (uint64_t)H, (uint64_t)Ns[0], (uint64_t)Ns[0], &mw)) return RMM_ERR_CUDA;
     }
-    return cuda_status(launch_gemm(mx, mw, xt, L.ldT, static_cast<const uint16_t*>(Wt), idx_padded, k,
-                                   T, H, N, static_cast<uint16_t*>(Y), status, o.debug_timeout_test,
-                                   o.gemm_producer, num_sms_current(), s));
+    GemmGroup g;
+    memset(&g, 0, sizeof g);
+    g.count = count;
+    for (int p = 0; p < count; ++p) {
+        g.Wt[p] = static_cast<const uint16_t*>(Wts[p]);
+        g.Y[p] = static_cast<uint16_t*>(Ys[p]);
+        g.N[p] = Ns[p];
+    }
+    gemm_group_tiles(g, T);
+    return cuda_status(launch_gemm(mx, mw, xt, L.ldT, g, idx_padded, k, T, H, status,
+                                   o.debug_timeout_test, o.gemm_producer, sms, s));
 }
 
-rmm_status run_product(const void* X, const void* Wt, const int32_t* idx_padded, int k, int T,
-                       int H, int N, void* Y, uint8_t* ws, const LinearLayout& L,
-                       const rmm_options& o, cudaStream_t s) {
+rmm_status run_products(const void* X, int T, int H, int count, const void* const* Wts, const int* Ns,
+                        void* const* Ys, const int32_t* idx_padded, int k, uint8_t* ws,
+                        const LinearLayout& L, const rmm_options& o, cudaStream_t s) {
     if (o.product_event_begin &&
         cudaEventRecord(static_cast<cudaEvent_t>(o.product_event_begin), s) != cudaSuccess)
         return RMM_ERR_CUDA;
-    rmm_status st = run_product_kernel(X, Wt, idx_padded, k, T, H, N, Y, ws, L, o, s);
+    rmm_status st = run_product_kernels(X, T, H, count, Wts, Ns, Ys, idx_padded, k, ws, L, o, s);
     if (st == RMM_OK && o.product_event_end &&
         cudaEventRecord(static_cast<cudaEvent_t>(o.product_event_end), s) != cudaSuccess)
         return RMM_ERR_CUDA;
     return st;
+}
+
+// score (+ X^T) -> kept set -> products, shared by rmm_linear and rmm_linear_group.
+rmm_status linear_group(const void* X, int T, int H, double r, int count, const void* const* Wts,
+                        const int* Ns, void* const* Ys, int32_t* idx_out, void* workspace,
+                        size_t workspace_bytes, rmm_stream_t stream, const rmm_options* options) {
+    if (!group_args_ok(X, T, H, count, Wts, Ns, Ys) || !opts_valid(options)) return RMM_ERR_INVALID_ARG;
+    const int k = rmm_k_for(H, r);
+    if (k < 1) return RMM_ERR_INVALID_ARG;
+    const rmm_options& o = opts_or_default(options);
+    const int sms = num_sms_current();
+    const LinearLayout L = linear_layout(T, H, Ns, count, k, o, sms);
+    if (!workspace || workspace_bytes < L.total || !aligned16(workspace)) return RMM_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t* s32 = reinterpret_cast<uint32_t*>(ws + L.s32);
+    int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+    cudaError_t e = launch_score(static_cast<const uint16_t*>(X), T, H, s32,
+                                 L.gemv ? nullptr : reinterpret_cast<uint16_t*>(ws + L.xt), L.ldT, sms, s);
+    if (e != cudaSuccess) return RMM_ERR_CUDA;
+    const int pad_to = (k + kGemmBK - 1) / kGemmBK * kGemmBK;
+    e = launch_select(s32, 1, H, k, idx, pad_to, idx_out, nullptr, s);
+    if (e != cudaSuccess) return RMM_ERR_CUDA;
+    return run_products(X, T, H, count, Wts, Ns, Ys, idx, k, ws, L, o, s);
 }
 
 }  // namespace
@@ -260,79 +306,78 @@ rmm_status rmm_transpose_weight(const void* W, void* Wt, int N, int H, rmm_strea
 size_t rmm_linear_workspace_bytes(int T, int H, int N, const rmm_options* options) {
     if (T < 1 || H < 1 || N < 1 || !opts_valid(options)) return 0;
     const rmm_options& o = opts_or_default(options);
-    return linear_layout(T, H, N, H, o, num_sms_current()).total;
+    return linear_layout(T, H, &N, 1, H, o, num_sms_current()).total;
+}
+
+size_t rmm_linear_group_workspace_bytes(int T, int H, int count, const int* Ns, const rmm_options* options) {
+    if (T < 1 || H < 1 || count < 1 || count > kMaxGroup || !Ns || !opts_valid(options)) return 0;
+    for (int p = 0; p < count; ++p)
+        if (Ns[p] < 1) return 0;
+    const rmm_options& o = opts_or_default(options);
+    return linear_layout(T, H, Ns, count, H, o, num_sms_current()).total;
 }
 
 rmm_status rmm_linear(const void* X, const void* Wt, int T, int H, int N, double r, void* Y,
                       int32_t* idx_out, void* workspace, size_t workspace_bytes,
                       rmm_stream_t stream, const rmm_options* options) {
-    if (!linear_args_ok(X, Wt, T, H, N, Y) || !opts_valid(options)) return RMM_ERR_INVALID_ARG;
-    const int k = rmm_k_for(H, r);
-    if (k < 1) return RMM_ERR_INVALID_ARG;
-    const rmm_options& o = opts_or_default(options);
-    const int sms = num_sms_current();
-    const LinearLayout L = linear_layout(T, H, N, k, o, sms);
-    if (!workspace || workspace_bytes < L.total || !aligned16(workspace)) return RMM_ERR_WORKSPACE;
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const void* Wts[1] = {Wt};
+    void* Ys[1] = {Y};
+    return linear_group(X, T, H, r, 1, Wts, &N, Ys, idx_out, workspace, workspace_bytes, stream, options);
+}
 
-    uint16_t* part = reinterpret_cast<uint16_t*>(ws + L.part);
-    int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
-    cudaError_t e = launch_score(static_cast<const uint16_t*>(X), T, H, part, L.P,
-                                 L.gemv ? nullptr : reinterpret_cast<uint16_t*>(ws + L.xt), L.ldT, s);
-    if (e != cudaSuccess) return RMM_ERR_CUDA;
-    const int pad_to = (k + kGemmBK - 1) / kGemmBK * kGemmBK;
-    e = launch_select(part, L.P, nullptr, H, k, idx, pad_to, idx_out, nullptr, s);
-    if (e != cudaSuccess) return RMM_ERR_CUDA;
-    return run_product(X, Wt, idx, k, T, H, N, Y, ws, L, o, s);
+rmm_status rmm_linear_group(const void* X, int T, int H, double r, int count, const void* const* Wts,
+                            const int* Ns, void* const* Ys, int32_t* idx_out, void* workspace,
+                            size_t workspace_bytes, rmm_stream_t stream, const rmm_options* options) {
+    return linear_group(X, T, H, r, count, Wts, Ns, Ys, idx_out, workspace, workspace_bytes, stream, options);
 }
 
 rmm_status rmm_score(const void* X, int T, int H, uint32_t* s_out, void* workspace,
                      size_t workspace_bytes, rmm_stream_t stream) {
     if (!X || !s_out || T < 1 || H < 1 || H > 65535 || !aligned16(X)) return RMM_ERR_INVALID_ARG;
-    const int sms = num_sms_current();
-    const int P = score_partials_for(T, H, sms);
-    const size_t need = kStatusBytes + align_up((size_t)P * H * 2, kAlign) +
-                        align_up(((size_t)H + 2 * kGemmBK) * 4, kAlign);
+    const size_t off_s32 = kStatusBytes;
+    const size_t off_idx = off_s32 + align_up((size_t)H * 4, kAlign);
+    const size_t need = off_idx + align_up(((size_t)H + 2 * kGemmBK) * 4, kAlign);
     if (!workspace || workspace_bytes < need) return RMM_ERR_WORKSPACE;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint16_t* part = reinterpret_cast<uint16_t*>(ws + kStatusBytes);
-    int32_t* idx = reinterpret_cast<int32_t*>(ws + kStatusBytes + align_up((size_t)P * H * 2, kAlign));
-    cudaError_t e = launch_score(static_cast<const uint16_t*>(X), T, H, part, P, nullptr, 0, s);
+    uint32_t* s32 = reinterpret_cast<uint32_t*>(ws + off_s32);
+    int32_t* idx = reinterpret_cast<int32_t*>(ws + off_idx);
+    cudaError_t e = launch_score(static_cast<const uint16_t*>(X), T, H, s32, nullptr, 0, num_sms_current(), s);
     if (e != cudaSuccess) return RMM_ERR_CUDA;
-    return cuda_status(launch_select(part, P, nullptr, H, H, idx, H, nullptr, s_out, s));
+    return cuda_status(launch_select(s32, 1, H, H, idx, H, nullptr, s_out, s));
 }
 
 rmm_status rmm_select(const uint32_t* sc, int H, int k, int32_t* idx_out, void* /*workspace*/,
                       size_t /*workspace_bytes*/, rmm_stream_t stream) {
     if (!sc || !idx_out || H < 1 || H > 65535 || k < 1 || k > H) return RMM_ERR_INVALID_ARG;
-    return cuda_status(launch_select(nullptr, 0, sc, H, k, idx_out, k, nullptr, nullptr,
+    return cuda_status(launch_select(const_cast<uint32_t*>(sc), 0, H, k, idx_out, k, nullptr, nullptr,
                                      static_cast<cudaStream_t>(stream)));
 }
 
 rmm_status rmm_gemm_reduced(const void* X, const void* Wt, const int32_t* idx, int k, int T, int H,
                             int N, void* Y, void* workspace, size_t workspace_bytes,
                             rmm_stream_t stream, const rmm_options* options) {
-    if (!linear_args_ok(X, Wt, T, H, N, Y) || !idx || k < 1 || k > H || !opts_valid(options))
+    const void* Wts[1] = {Wt};
+    void* Ys[1] = {Y};
+    if (!group_args_ok(X, T, H, 1, Wts, &N, Ys) || !idx || k < 1 || k > H || !opts_valid(options))
         return RMM_ERR_INVALID_ARG;
     const rmm_options& o = opts_or_default(options);
     const int sms = num_sms_current();
-    const LinearLayout L = linear_layout(T, H, N, k, o, sms);
+    const LinearLayout L = linear_layout(T, H, &N, 1, k, o, sms);
     if (!workspace || workspace_bytes < L.total || !aligned16(workspace)) return RMM_ERR_WORKSPACE;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (L.gemv) return run_product(X, Wt, idx, k, T, H, N, Y, ws, L, o, s);
-    // GEMM path: X^T (written by the score pass) and the kept list padded to the K-block
-    cudaError_t e = launch_score(static_cast<const uint16_t*>(X), T, H,
-                                 reinterpret_cast<uint16_t*>(ws + L.part), L.P,
-                                 reinterpret_cast<uint16_t*>(ws + L.xt), L.ldT, s);
+    if (L.gemv) return run_products(X, T, H, 1, Wts, &N, Ys, idx, k, ws, L, o, s);
+    // GEMM path: X^T (written by the score pass, scores not accumulated) and
+    // the kept list padded to the K-block
+    cudaError_t e = launch_score(static_cast<const uint16_t*>(X), T, H, nullptr,
+                                 reinterpret_cast<uint16_t*>(ws + L.xt), L.ldT, sms, s);
     if (e != cudaSuccess) return RMM_ERR_CUDA;
     int32_t* idx_pad = reinterpret_cast<int32_t*>(ws + L.idx);
     const int pad_to = (k + kGemmBK - 1) / kGemmBK * kGemmBK;
     e = launch_pad_idx(idx, k, H, idx_pad, pad_to, s);
     if (e != cudaSuccess) return RMM_ERR_CUDA;
-    return run_product(X, Wt, idx_pad, k, T, H, N, Y, ws, L, o, s);
+    return run_products(X, T, H, 1, Wts, &N, Ys, idx_pad, k, ws, L, o, s);
 }
 
 size_t rmm_attn_workspace_bytes(int B, int Hq, int Hkv, int T, int L, int d,

@@ -92,12 +92,30 @@ __device__ __forceinline__ uint32_t swz_offset(int j, int c16) {
     return (uint32_t)((c16 >> 3) * CHUNK_BYTES + j * 128 + (((c16 & 7) ^ (j & 7)) << 4));
 }
 
+struct TileCoord {
+    int p, m0, n0;
+};
+
+// Tile t of the group: product p with tile_start[p] <= t < tile_start[p+1],
+// walked M-fastest inside the product so concurrent CTAs share W^T columns.
+__device__ __forceinline__ TileCoord decode_tile(const GemmGroup& g, int t, int m_tiles) {
+    int p = 0;
+#pragma unroll
+    for (int i = 1; i < kMaxGroup; ++i)
+        if (i < g.count && t >= g.tile_start[i]) p = i;
+    const int local = t - g.tile_start[p];
+    TileCoord c;
+    c.p = p;
+    c.m0 = (local % m_tiles) * BM;
+    c.n0 = (local / m_tiles) * BN;
+    return c;
+}
+
 template <bool kTmaGather>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_xt, const __grid_constant__ CUtensorMap map_wt,
-                const uint16_t* __restrict__ Xt, int ldT, const uint16_t* __restrict__ Wt,
-                const int32_t* __restrict__ idx, int k, int T, int H, int N,
-                uint16_t* __restrict__ Y, int* status, int debug_timeout) {
+                const uint16_t* __restrict__ Xt, int ldT, const __grid_constant__ GemmGroup group,
+                const int32_t* __restrict__ idx, int k, int T, int H, int* status, int debug_timeout) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -109,8 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int m_tiles = (T + BM - 1) / BM;
-    const int n_tiles = (N + BN - 1) / BN;
-    const int num_tiles = m_tiles * n_tiles;
+    const int num_tiles = group.tile_start[group.count];
     const int nkb = (k + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
@@ -166,8 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kRowsA; ++i)
             a_off[i] = swz_offset(2 * (warp + kProducerWarps * i) + (lane >> 4), lane & 15);
         for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-            const int m0 = (tile % m_tiles) * BM;
-            const int n0 = (tile / m_tiles) * BN;
+            const TileCoord tc = decode_tile(group, tile, m_tiles);
+            const int m0 = tc.m0, n0 = tc.n0;
+            const int N = group.N[tc.p];
+            const uint16_t* __restrict__ Wt = group.Wt[tc.p];
             if (kTmaGather && warp != 0) break;
             const int b_col = n0 + lane * 8;          // this lane's W^T columns
             const int a_col = m0 + (lane & 15) * 8;   // this lane's X^T columns (tokens)
@@ -304,8 +323,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            const int m0 = (tile % m_tiles) * BM;
-            const int n0 = (tile / m_tiles) * BN;
+            const TileCoord tc = decode_tile(group, tile, m_tiles);
+            const int m0 = tc.m0, n0 = tc.n0;
+            const int N = group.N[tc.p];
+            uint16_t* __restrict__ Y = group.Y[tc.p];
             if (!mbar_wait(smem_addr(&bars->tfull[acc]), acc_phase, status, abort_flag)) break;
             tc_fence_after();
             const int row = m0 + q * 32 + lane;
@@ -350,16 +371,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t gemm_smem_bytes() { return kSmemBytes; }
 
+int gemm_group_tiles(GemmGroup& g, int T) {
+    const int m_tiles = (T + BM - 1) / BM;
+    g.tile_start[0] = 0;
+    for (int p = 0; p < g.count; ++p) g.tile_start[p + 1] = g.tile_start[p] + m_tiles * ((g.N[p] + BN - 1) / BN);
+    for (int p = g.count + 1; p <= kMaxGroup; ++p) g.tile_start[p] = g.tile_start[g.count];
+    return g.tile_start[g.count];
+}
+
 cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt, const uint16_t* Xt,
-                        int ldT, const uint16_t* Wt, const int32_t* idx, int k, int T, int H, int N,
-                        uint16_t* Y, int* status, int debug_timeout, int tma_gather, int num_sms,
+                        int ldT, const GemmGroup& group, const int32_t* idx, int k, int T, int H,
+                        int* status, int debug_timeout, int tma_gather, int num_sms,
                         cudaStream_t stream) {
+    if (group.count < 1 || group.count > kMaxGroup || (tma_gather && group.count != 1))
+        return cudaErrorInvalidValue;
     auto kern = tma_gather ? gemm_kernel<true> : gemm_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    const int tiles = ((T + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int tiles = group.tile_start[group.count];
     const int grid = tiles < num_sms ? tiles : num_sms;
-    kern<<<grid, kThreads, kSmemBytes, stream>>>(map_xt, map_wt, Xt, ldT, Wt, idx, k, T, H, N, Y, status,
+    kern<<<grid, kThreads, kSmemBytes, stream>>>(map_xt, map_wt, Xt, ldT, group, idx, k, T, H, status,
                                                   debug_timeout);
     return cudaGetLastError();
 }

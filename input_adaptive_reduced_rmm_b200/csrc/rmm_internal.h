@@ -8,23 +8,22 @@
 
 namespace rmm {
 
-constexpr int kMaxScorePartials = 32;  // partial-maximum rows written by the score pass
 constexpr int kGemvMaxT = 16;          // largest T of the split-K GEMV
 constexpr int kGemmBK = 64;            // kept slices per GEMM pipeline stage (idx padded to this)
 
 // ---- score (rmm_score.cu)
-int score_partials_for(int T, int H, int num_sms);
-cudaError_t launch_score(const uint16_t* X, int T, int H, uint16_t* part, int P, uint16_t* Xt,
-                         int ldT, cudaStream_t stream);
+// Folds max_t |X[t,h]| into s32[h] (u32 [H], must hold zeros or smaller
+// keys on entry); on the GEMM path (Xt != null) also writes X^T [H, ldT].
+cudaError_t launch_score(const uint16_t* X, int T, int H, uint32_t* s32, uint16_t* Xt, int ldT,
+                         int num_sms, cudaStream_t stream);
 
 // ---- select (rmm_select.cu)
-// Folds P partial rows (part, u16 [P][H]) -- or reads s32 (u32 [H]) when part is
-// null -- into the score, optionally stores it to s_out, and writes the k best
-// indices ascending to idx[0..k), then idx[k..pad_to) = H; idx_copy (if not
-// null) receives the same k indices without padding.
-cudaError_t launch_select(const uint16_t* part, int P, const uint32_t* s32, int H, int k,
-                          int32_t* idx, int pad_to, int32_t* idx_copy, uint32_t* s_out,
-                          cudaStream_t stream);
+// Reads the scores s32 (u32 [H]; zeroed afterwards when clear_input != 0),
+// optionally stores them to s_out, and writes the k best indices ascending to
+// idx[0..k), then idx[k..pad_to) = H; idx_copy (if not null) receives the
+// same k indices without padding.
+cudaError_t launch_select(uint32_t* s32, int clear_input, int H, int k, int32_t* idx, int pad_to,
+                          int32_t* idx_copy, uint32_t* s_out, cudaStream_t stream);
 
 // ---- split-K GEMV (rmm_gemv.cu)
 struct GemvPlan {
@@ -43,10 +42,24 @@ cudaError_t launch_gemv(const uint16_t* X, int T, int H, const uint16_t* Wt, int
                         cudaStream_t stream);
 
 // ---- tcgen05 GEMM (rmm_gemm.cu)
-// map_xt / map_wt are used only by the TMA tile::gather4 producer (tma_gather != 0).
+// Up to kMaxGroup products that share the activations (X^T, T, H and the kept
+// list) and differ in the weight: one persistent launch walks the tiles of
+// all of them.
+constexpr int kMaxGroup = 4;
+struct GemmGroup {
+    const uint16_t* Wt[kMaxGroup];
+    uint16_t* Y[kMaxGroup];
+    int N[kMaxGroup];
+    int tile_start[kMaxGroup + 1];  // prefix sums of the products' tile counts
+    int count;
+};
+// Fills tile_start for the given T; returns the total tile count.
+int gemm_group_tiles(GemmGroup& g, int T);
+// map_xt / map_wt are used only by the TMA tile::gather4 producer
+// (tma_gather != 0), which handles a group of one.
 cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt, const uint16_t* Xt,
-                        int ldT, const uint16_t* Wt, const int32_t* idx, int k, int T, int H, int N,
-                        uint16_t* Y, int* status, int debug_timeout, int tma_gather, int num_sms,
+                        int ldT, const GemmGroup& group, const int32_t* idx, int k, int T, int H,
+                        int* status, int debug_timeout, int tma_gather, int num_sms,
                         cudaStream_t stream);
 size_t gemm_smem_bytes();
 

@@ -7,7 +7,7 @@
 // is being recorded into a CUDA graph, where a cudaMalloc would break the
 // capture.  rmm_linear_decode_noalloc serves them: the same score -> kept set ->
 // split-K GEMV path as rmm_linear for T <= 16, but every intermediate (partial
-// maxima, the kept list, the split partial sums, the split counters) lives in
+// score vector, the kept list, the split partial sums, the split counters) lives in
 // one file-scope __device__ array of fixed size that every GPU loading the
 // library holds until the process exits.  Nothing is allocated or freed.
 //
@@ -76,11 +76,10 @@ extern "C" rmm_status rmm_linear_decode_noalloc(const void* X, const void* Wt, i
     rmm_status st = noalloc_scratch(&scratch);
     if (st != RMM_OK) return st;
 
-    // scratch layout: status | score partials | kept list | split counters | split partials
-    const int P = score_partials_for(T, H, sms);
+    // scratch layout: status | score vector | kept list | split counters | split partials
     GemvPlan plan = gemv_plan(T, N, k, sms, 0);
-    const size_t off_part = kNoAllocStatusBytes;
-    const size_t off_idx = off_part + up256((size_t)P * H * sizeof(uint16_t));
+    const size_t off_s32 = kNoAllocStatusBytes;
+    const size_t off_idx = off_s32 + up256((size_t)H * sizeof(uint32_t));
     const size_t off_cnt = off_idx + up256(((size_t)H + 2 * kGemmBK) * sizeof(int32_t));
     const size_t off_partials = off_cnt + up256((size_t)plan.col_blocks * sizeof(unsigned));
     if (off_partials > kNoAllocScratchBytes) return RMM_ERR_UNSUPPORTED;
@@ -96,16 +95,18 @@ extern "C" rmm_status rmm_linear_decode_noalloc(const void* X, const void* Wt, i
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (gemv_smem_bytes(plan, T) > kGemvMaxSmemBytes) return RMM_ERR_UNSUPPORTED;
-    noalloc_clear_kernel<<<1, 256, 0, s>>>(reinterpret_cast<unsigned*>(scratch), (int)(kNoAllocStatusBytes / 4));
+    // status word and score vector: the score pass folds maxima into zeros
+    noalloc_clear_kernel<<<(int)((off_idx / 4 + 255) / 256), 256, 0, s>>>(reinterpret_cast<unsigned*>(scratch),
+                                                                         (int)(off_idx / 4));
     noalloc_clear_kernel<<<(plan.col_blocks + 255) / 256, 256, 0, s>>>(
         reinterpret_cast<unsigned*>(scratch + off_cnt), plan.col_blocks);
     if (cudaGetLastError() != cudaSuccess) return RMM_ERR_CUDA;
 
-    uint16_t* part = reinterpret_cast<uint16_t*>(scratch + off_part);
+    uint32_t* s32 = reinterpret_cast<uint32_t*>(scratch + off_s32);
     int32_t* idx = reinterpret_cast<int32_t*>(scratch + off_idx);
-    if (launch_score(static_cast<const uint16_t*>(X), T, H, part, P, nullptr, 0, s) != cudaSuccess)
+    if (launch_score(static_cast<const uint16_t*>(X), T, H, s32, nullptr, 0, sms, s) != cudaSuccess)
         return RMM_ERR_CUDA;
-    if (launch_select(part, P, nullptr, H, k, idx, k, idx_out, nullptr, s) != cudaSuccess) return RMM_ERR_CUDA;
+    if (launch_select(s32, 1, H, k, idx, k, idx_out, nullptr, s) != cudaSuccess) return RMM_ERR_CUDA;
     if (launch_gemv(static_cast<const uint16_t*>(X), T, H, static_cast<const uint16_t*>(Wt), N, idx, k,
                     static_cast<uint16_t*>(Y), reinterpret_cast<float*>(scratch + off_partials),
                     reinterpret_cast<unsigned*>(scratch + off_cnt), plan,

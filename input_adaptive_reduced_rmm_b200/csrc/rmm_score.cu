@@ -9,9 +9,10 @@
 // exact and independent of the reduction order.
 //
 // One pass over X [T, H] (HBM-bound: T*H*2 bytes read).  Each CTA owns a
-// 64-wide channel strip and a strided subset of 64-token tiles; it writes its
-// strip's partial maximum to part[blockIdx.y][h] and the select kernel folds
-// the gridDim.y partials.  On the GEMM path the same pass also writes the
+// 64-wide channel strip and a strided subset of 64-token tiles; it folds its
+// strip's maximum into the score vector s32[h] with atomicMax (the vector
+// starts at zero: the select kernel clears it after reading).  On the GEMM
+// path the same pass also writes the
 // full transpose X^T [H, ldT] (through a shared-memory tile) so that a kept
 // slice of X is one contiguous row that TMA can gather; this is a transposed
 // copy of all of X, never a compacted copy of the kept part.
@@ -28,7 +29,7 @@ constexpr int kThreads = 256;
 
 template <bool kWriteXt, bool kVec>
 __global__ void __launch_bounds__(kThreads)
-    score_kernel(const uint16_t* __restrict__ X, int T, int H, uint16_t* __restrict__ part,
+    score_kernel(const uint16_t* __restrict__ X, int T, int H, uint32_t* __restrict__ s32,
                  uint16_t* __restrict__ Xt, int ldT) {
     // Rows of 66 elements (33 words): the transposed reads of 8 rows that are
     // 8 apart then fall on distinct bank groups (2-way conflicts at most).
@@ -111,36 +112,33 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll 8
         for (int r = 0; r < 32; ++r) m = max(m, (uint32_t)red[r][tid]);
         const int h = h0 + tid;
-        if (h < H) part[(size_t)blockIdx.y * H + h] = (uint16_t)m;
+        if (s32 && h < H && m > 0) atomicMax(s32 + h, m);
     }
 }
 
 }  // namespace
 
-int score_partials_for(int T, int H, int num_sms) {
+cudaError_t launch_score(const uint16_t* X, int T, int H, uint32_t* s32, uint16_t* Xt, int ldT,
+                         int num_sms, cudaStream_t stream) {
+    // enough CTAs to keep ~16 per SM in flight; each takes one or more 64-token tiles
     const int strips = (H + kTileH - 1) / kTileH;
     const int tiles = (T + kTileT - 1) / kTileT;
-    int p = (4 * num_sms + strips - 1) / strips;
-    if (p > tiles) p = tiles;
-    if (p > kMaxScorePartials) p = kMaxScorePartials;
-    if (p < 1) p = 1;
-    return p;
-}
-
-cudaError_t launch_score(const uint16_t* X, int T, int H, uint16_t* part, int P, uint16_t* Xt,
-                         int ldT, cudaStream_t stream) {
-    dim3 grid((H + kTileH - 1) / kTileH, P);
+    int ty = (16 * num_sms + strips - 1) / strips;
+    if (ty > tiles) ty = tiles;
+    if (ty > 65535) ty = 65535;
+    if (ty < 1) ty = 1;
+    dim3 grid(strips, ty);
     const bool vec = (H % 8 == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
     if (Xt) {
         if (vec)
-            score_kernel<true, true><<<grid, kThreads, 0, stream>>>(X, T, H, part, Xt, ldT);
+            score_kernel<true, true><<<grid, kThreads, 0, stream>>>(X, T, H, s32, Xt, ldT);
         else
-            score_kernel<true, false><<<grid, kThreads, 0, stream>>>(X, T, H, part, Xt, ldT);
+            score_kernel<true, false><<<grid, kThreads, 0, stream>>>(X, T, H, s32, Xt, ldT);
     } else {
         if (vec)
-            score_kernel<false, true><<<grid, kThreads, 0, stream>>>(X, T, H, part, nullptr, 0);
+            score_kernel<false, true><<<grid, kThreads, 0, stream>>>(X, T, H, s32, nullptr, 0);
         else
-            score_kernel<false, false><<<grid, kThreads, 0, stream>>>(X, T, H, part, nullptr, 0);
+            score_kernel<false, false><<<grid, kThreads, 0, stream>>>(X, T, H, s32, nullptr, 0);
     }
     return cudaGetLastError();
 }

@@ -7,7 +7,8 @@
 // original order).
 //
 // One CTA of 1024 threads, scores resident in shared memory:
-//   1. fold the score pass's partial maxima into s[h] (15-bit keys);
+//   1. read the score vector into shared memory (and clear it for the next
+//      call when it is the library's own accumulator);
 //   2. radix select on the key: a 256-bin histogram of s>>8 finds the bin of
 //      the k-th largest score, a 256-bin histogram of s&255 inside that bin
 //      finds the threshold score s*; c_gt = #{s > s*}, need = k - c_gt;
@@ -86,9 +87,8 @@ __device__ __forceinline__ int warp_find_bin(const int* cnt, int nbins, int k, i
 }
 
 __global__ void __launch_bounds__(kThreads)
-    select_kernel(const uint16_t* __restrict__ part, int P, const uint32_t* __restrict__ s32, int H,
-                  int k, int32_t* __restrict__ idx, int pad_to, int32_t* __restrict__ idx_copy,
-                  uint32_t* __restrict__ s_out) {
+    select_kernel(uint32_t* __restrict__ s32, int clear_input, int H, int k, int32_t* __restrict__ idx,
+                  int pad_to, int32_t* __restrict__ idx_copy, uint32_t* __restrict__ s_out) {
     extern __shared__ uint16_t s[];  // H keys
     __shared__ int hist_hi[256];
     __shared__ int hist_fine[256];
@@ -99,14 +99,10 @@ __global__ void __launch_bounds__(kThreads)
     if (tid < 256) hist_hi[tid] = 0;
     if (tid < 256) hist_fine[tid] = 0;
 
-    // 1. fold partial maxima
+    // 1. load the scores
     for (int h = tid; h < H; h += kThreads) {
-        uint32_t m = 0;
-        if (part) {
-            for (int p = 0; p < P; ++p) m = max(m, (uint32_t)part[(size_t)p * H + h]);
-        } else {
-            m = s32[h] & 0xFFFFu;
-        }
+        const uint32_t m = s32[h] & 0xFFFFu;
+        if (clear_input) s32[h] = 0;
         s[h] = (uint16_t)m;
         if (s_out) s_out[h] = m;
     }
@@ -176,16 +172,15 @@ __global__ void __launch_bounds__(kThreads)
 
 }  // namespace
 
-cudaError_t launch_select(const uint16_t* part, int P, const uint32_t* s32, int H, int k,
-                          int32_t* idx, int pad_to, int32_t* idx_copy, uint32_t* s_out,
-                          cudaStream_t stream) {
+cudaError_t launch_select(uint32_t* s32, int clear_input, int H, int k, int32_t* idx, int pad_to,
+                          int32_t* idx_copy, uint32_t* s_out, cudaStream_t stream) {
     const size_t smem = ((size_t)H * sizeof(uint16_t) + 15) & ~(size_t)15;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(select_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    select_kernel<<<1, kThreads, smem, stream>>>(part, P, s32, H, k, idx, pad_to, idx_copy, s_out);
+    select_kernel<<<1, kThreads, smem, stream>>>(s32, clear_input, H, k, idx, pad_to, idx_copy, s_out);
     return cudaGetLastError();
 }
 

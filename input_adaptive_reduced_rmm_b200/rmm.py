@@ -28,7 +28,7 @@ EXPORTED = (
     "rmm_status_string", "rmm_k_for", "rmm_workspace_init", "rmm_get_status",
     "rmm_transpose_weight", "rmm_linear_workspace_bytes", "rmm_linear", "rmm_score",
     "rmm_select", "rmm_gemm_reduced", "rmm_attn_workspace_bytes", "rmm_attn_qk",
-    "rmm_linear_decode_noalloc",
+    "rmm_linear_decode_noalloc", "rmm_linear_group", "rmm_linear_group_workspace_bytes",
 )
 
 
@@ -95,6 +95,8 @@ def lib() -> ctypes.CDLL:
         "rmm_attn_workspace_bytes": (Z, [I, I, I, I, I, I, OP]),
         "rmm_attn_qk": (I, [P, P, P, I, I, I, I, I, I, I, D, I, F, P, P, P, Z, P, OP]),
         "rmm_linear_decode_noalloc": (I, [P, P, I, I, I, D, P, P, P]),
+        "rmm_linear_group_workspace_bytes": (Z, [I, I, I, P, OP]),
+        "rmm_linear_group": (I, [P, I, I, D, I, P, P, P, P, P, Z, P, OP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -185,6 +187,36 @@ def rmm_linear(X: torch.Tensor, Wt: torch.Tensor, r: float, Y: torch.Tensor | No
                             _ptr(workspace), workspace.numel(), _stream(stream), _opt(opts)),
            "rmm_linear")
     return Y
+
+
+def rmm_linear_group_workspace_bytes(T: int, H: int, Ns, opts: rmm_options | None = None) -> int:
+    arr = (ctypes.c_int * len(Ns))(*[int(n) for n in Ns])
+    return int(lib().rmm_linear_group_workspace_bytes(int(T), int(H), len(Ns), arr, _opt(opts)))
+
+
+def rmm_linear_group(X: torch.Tensor, Wts, r: float, Ys=None, idx_out: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, opts: rmm_options | None = None, stream=None):
+    """Projections of one activation matrix sharing one kept set: [X[:,S] W_p[:,S]^T for each W_p^T in Wts]."""
+    _bf16_cuda(X, "X")
+    T, H = X.shape
+    Ns = []
+    for i, Wt in enumerate(Wts):
+        _bf16_cuda(Wt, f"Wts[{i}]")
+        if Wt.shape[0] != H:
+            raise ValueError("X and a weight disagree on H")
+        Ns.append(Wt.shape[1])
+    if Ys is None:
+        Ys = [torch.empty(T, n, dtype=torch.bfloat16, device=X.device) for n in Ns]
+    if workspace is None:
+        workspace = new_workspace(rmm_linear_group_workspace_bytes(T, H, Ns, opts), X.device)
+    c = len(Ns)
+    w_arr = (ctypes.c_void_p * c)(*[W.data_ptr() for W in Wts])
+    y_arr = (ctypes.c_void_p * c)(*[Y.data_ptr() for Y in Ys])
+    n_arr = (ctypes.c_int * c)(*Ns)
+    _check(lib().rmm_linear_group(_ptr(X), T, H, float(r), c, w_arr, n_arr, y_arr, _ptr(idx_out),
+                                  _ptr(workspace), workspace.numel(), _stream(stream), _opt(opts)),
+           "rmm_linear_group")
+    return Ys
 
 
 def rmm_score(X: torch.Tensor, s_out: torch.Tensor | None = None,

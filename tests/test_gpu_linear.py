@@ -171,6 +171,28 @@ def test_llama3_70b_projections(rmm, H, N, T, r):
     check_projection(rmm, 4, T, H, N, r, nrows=8, ncols=256)
 
 
+# ---------------------------------------------------------------- projections sharing one input
+
+@pytest.mark.parametrize("T", [1, 16, 130, 2048])
+def test_linear_group_shares_one_kept_set(rmm, T):
+    """q, k, v of one layer (4096 -> 4096, 1024, 1024) in one grouped call."""
+    H = 4096
+    X = rmm_synth.activations(T, H, rmm_synth.seed_for(1, 90 + T % 100, 0))
+    Ws = [rmm_synth.weights(N, H, rmm_synth.seed_for(1, 91 + i, 1), std=0.02) for i, N in enumerate((4096, 1024, 1024))]
+    Wts = [rmm.rmm_transpose_weight(W.cuda()) for W in Ws]
+    k = rmm.rmm_k_for(H, 0.5)
+    idx = torch.empty(k, dtype=torch.int32, device="cuda")
+    Ys = rmm.rmm_linear_group(X.cuda(), Wts, 0.5, idx_out=idx)
+    torch.cuda.synchronize()
+    io = oracle.select(oracle.score(X), k)
+    assert np.array_equal(idx.cpu().numpy(), io)
+    rows = sample_indices(T, 12, seed=T)
+    for W, Y in zip(Ws, Ys):
+        cols = sample_indices(W.shape[0], 256, seed=W.shape[0])
+        Yo = oracle.reduced_product(X, W, io, rows=rows, cols=cols)
+        assert_close(Y.cpu()[rows][:, cols], Yo, f"group T={T} N={W.shape[0]}")
+
+
 # ---------------------------------------------------------------- product for a given kept list
 
 @pytest.mark.parametrize("T", [4, 300])
