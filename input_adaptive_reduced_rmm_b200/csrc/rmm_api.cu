@@ -41,7 +41,7 @@ bool opts_valid(const rmm_options* o) {
     if (!o) return true;
     if (o->t_gemv < 0 || o->t_gemv > kGemvMaxT) return false;
     if (o->gemv_splits < 0) return false;
-    if (o->gemm_producer < 0 || o->gemm_producer > 1) return false;
+    if (o->gemm_producer < 0 || o->gemm_producer > 2) return false;
     for (int i = 0; i < 3; ++i)
         if (o->reserved[i] != 0) return false;
     return true;
@@ -189,14 +189,6 @@ rmm_status run_product_kernels(const void* X, int T, int H, int count, const voi
         return RMM_OK;
     }
     if (o.gemm_producer == 1 && count != 1) return RMM_ERR_UNSUPPORTED;
-    CUtensorMap mx, mw;
-    memset(&mx, 0, sizeof mx);
-    memset(&mw, 0, sizeof mw);
-    const uint16_t* xt = reinterpret_cast<const uint16_t*>(ws + L.xt);
-    if (o.gemm_producer == 1) {
-        if (!row_gather_map(xt, (uint64_t)H, (uint64_t)T, (uint64_t)L.ldT, &mx)) return RMM_ERR_CUDA;
-        if (!row_gather_map(Wts[0], (uint64_t)H, (uint64_t)Ns[0], (uint64_t)Ns[0], &mw)) return RMM_ERR_CUDA;
-    }
     GemmGroup g;
     memset(&g, 0, sizeof g);
     g.count = count;
@@ -205,9 +197,22 @@ rmm_status run_product_kernels(const void* X, int T, int H, int count, const voi
         g.Y[p] = static_cast<uint16_t*>(Ys[p]);
         g.N[p] = Ns[p];
     }
-    gemm_group_tiles(g, T);
+    if (o.gemm_producer == 0) {  // default: CTA-pair tcgen05 GEMM
+        gemm_group_tiles(g, T, 1);
+        return cuda_status(launch_gemm_pair(reinterpret_cast<const uint16_t*>(ws + L.xt), L.ldT, g, idx_padded,
+                                            k, T, H, status, o.debug_timeout_test, sms, s));
+    }
+    gemm_group_tiles(g, T, 0);
+    CUtensorMap mx, mw;
+    memset(&mx, 0, sizeof mx);
+    memset(&mw, 0, sizeof mw);
+    const uint16_t* xt = reinterpret_cast<const uint16_t*>(ws + L.xt);
+    if (o.gemm_producer == 1) {
+        if (!row_gather_map(xt, (uint64_t)H, (uint64_t)T, (uint64_t)L.ldT, &mx)) return RMM_ERR_CUDA;
+        if (!row_gather_map(Wts[0], (uint64_t)H, (uint64_t)Ns[0], (uint64_t)Ns[0], &mw)) return RMM_ERR_CUDA;
+    }
     return cuda_status(launch_gemm(mx, mw, xt, L.ldT, g, idx_padded, k, T, H, status,
-                                   o.debug_timeout_test, o.gemm_producer, sms, s));
+                                   o.debug_timeout_test, o.gemm_producer == 1, sms, s));
 }
 
 rmm_status run_products(const void* X, int T, int H, int count, const void* const* Wts, const int* Ns,

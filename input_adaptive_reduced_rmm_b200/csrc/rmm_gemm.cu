@@ -367,16 +367,343 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kMmaWarp) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
+
+// ============================================================================
+// CTA-pair variant (tcgen05 cta_group::2): a cluster of two CTAs on one TPC
+// computes a 256 x 512 output tile.  CTA r of the pair stages rows
+// [128r, 128r+128) of the X^T tile and the contiguous column half
+// [256r, 256r+256) of the W^T tile (48 KB per 64-slice stage, 4 stages).  The
+// leader (r = 0) issues, per 16-slice step, two tcgen05.mma.cta_group::2
+// 256x256x16: "lo" on the first 128 columns of each CTA's half, "hi" on the
+// second 128; each reads A from both CTAs by rows and B by column halves, and
+// accumulates rows [128r, 128r+128) in CTA r's TMEM (lo in columns 0..255, hi
+// in 256..511: all of TMEM).  Per SM this gathers 5.7 KB of operands per MFLOP
+// (11.4 KB for the single-CTA 128 x 256 tile), which matters because the
+// cp.async gather rate per SM is this kernel's measured bound; a kept W^T row
+// still arrives as one 512-byte segment per warp instruction.
+//
+// TMEM column c of a CTA holds output column
+//   n0 + 256 * ((c mod 256) / 128) + 128 * (c / 256) + (c mod 128)
+// (lo/hi, then which CTA's half the MMA took the 128 columns from).
+//
+// Synchronisation across the pair:
+//   full[s]       local: the CTA's own 512 producer threads (cp.async arrive)
+//   pair_full[s]  leader only: the peer's MMA warp relays "peer stage s full"
+//                 (cluster-scope release/acquire, after a proxy fence)
+//   empty[s]      both: the leader commits to its own and the peer's barrier
+//   tfull         both: the leader commits to its own and the peer's barrier
+//   tempty        leader only: 4 local + 4 remote epilogue-warp arrivals
+// The single accumulator is not double-buffered (it fills TMEM), so a tile's
+// epilogue does not overlap the next tile's main loop.
+// An abort (bounded wait ran out) is raised in both CTAs' flags.
+namespace pair {
+
+constexpr int BM2 = 256;                 // tile rows (two CTAs x 128)
+constexpr int BN2 = 512;                 // tile columns (two CTAs x 256)
+constexpr int HALF_M = 128;              // rows staged per CTA
+constexpr int HALF_N = 256;              // columns staged per CTA
+constexpr int STAGES2 = 4;
+constexpr int A2_STAGE_BYTES = (HALF_M / 64) * CHUNK_BYTES;  // 16 KB
+constexpr int B2_STAGE_BYTES = (HALF_N / 64) * CHUNK_BYTES;  // 32 KB
+constexpr int TMEM_COLS2 = 512;
+
+struct __align__(8) Barriers2 {
+    uint64_t full[STAGES2];
+    uint64_t pair_full[STAGES2];
+    uint64_t empty[STAGES2];
+    uint64_t tfull;
+    uint64_t tempty;
+    uint64_t never;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+constexpr size_t kSmemBytes2 =
+    1024 + (size_t)STAGES2 * (A2_STAGE_BYTES + B2_STAGE_BYTES) + sizeof(Barriers2);
+
+__device__ __forceinline__ TileCoord decode_tile2(const GemmGroup& g, int t, int m_tiles) {
+    int p = 0;
+#pragma unroll
+    for (int i = 1; i < kMaxGroup; ++i)
+        if (i < g.count && t >= g.tile_start[i]) p = i;
+    const int local = t - g.tile_start[p];
+    TileCoord c;
+    c.p = p;
+    c.m0 = (local % m_tiles) * BM2;
+    c.n0 = (local / m_tiles) * BN2;
+    return c;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const uint16_t* __restrict__ Xt, int ldT, const __grid_constant__ GemmGroup group,
+                     const int32_t* __restrict__ idx, int k, int T, int H, int* status, int debug_timeout) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES2 * A2_STAGE_BYTES;
+    Barriers2* bars = reinterpret_cast<Barriers2*>(sB + STAGES2 * B2_STAGE_BYTES);
+    volatile int* abort_flag = &bars->abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0 = leader
+    const uint32_t peer = rank ^ 1u;
+    const int m_tiles = (T + BM2 - 1) / BM2;
+    const int num_tiles = group.tile_start[group.count];
+    const int nkb = (k + BK - 1) / BK;
+    const int cluster_id = blockIdx.x >> 1;
+    const int num_clusters = gridDim.x >> 1;
+    const uint32_t peer_abort = mapa_shared(smem_addr(&bars->abort_flag), peer);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES2; ++s) {
+            mbar_init(smem_addr(&bars->full[s]), kProducerThreads);
+            mbar_init(smem_addr(&bars->pair_full[s]), 1);
+            mbar_init(smem_addr(&bars->empty[s]), 1);
+        }
+        mbar_init(smem_addr(&bars->tfull), 1);
+        mbar_init(smem_addr(&bars->tempty), 2 * kEpilogueWarps);
+        mbar_init(smem_addr(&bars->never), 1);
+        bars->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc_pair(smem_addr(&bars->tmem_base), TMEM_COLS2);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
+    tc_fence_after();
+    const uint32_t tmem_base = bars->tmem_base;
+
+    if (warp < kProducerWarps) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int q0a = __ldg(idx + lane), q1a = __ldg(idx + 32 + lane);
+        int next_kb = (1 < nkb) ? 1 : 0;
+        int q0b = __ldg(idx + next_kb * BK + lane), q1b = __ldg(idx + next_kb * BK + 32 + lane);
+        next_kb = (next_kb + 1 < nkb) ? next_kb + 1 : 0;
+        uint32_t b_off[kRowsB], a_off[kRowsA];
+#pragma unroll
+        for (int i = 0; i < kRowsB; ++i) b_off[i] = swz_offset(warp + kProducerWarps * i, lane);
+#pragma unroll
+        for (int i = 0; i < kRowsA; ++i)
+            a_off[i] = swz_offset(2 * (warp + kProducerWarps * i) + (lane >> 4), lane & 15);
+        for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
+            const TileCoord tc = decode_tile2(group, tile, m_tiles);
+            const int N = group.N[tc.p];
+            const uint16_t* __restrict__ Wt = group.Wt[tc.p];
+            const int a_col = tc.m0 + HALF_M * (int)rank + (lane & 15) * 8;  // tokens
+            const int b_col = tc.n0 + HALF_N * (int)rank + lane * 8;         // output features
+            const bool a_col_ok = a_col < T;
+            const bool b_col_ok = b_col < N;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const uint32_t full = smem_addr(&bars->full[stage]);
+                if (!mbar_wait(smem_addr(&bars->empty[stage]), phase ^ 1, status, abort_flag)) {
+                    st_shared_cluster_u32(peer_abort, 1);
+                    ok = false;
+                    break;
+                }
+                const uint32_t a_stage = smem_addr(sA + stage * A2_STAGE_BYTES);
+                const uint32_t b_stage = smem_addr(sB + stage * B2_STAGE_BYTES);
+                const int v0 = q0a, v1 = q1a;
+                q0a = q0b;
+                q1a = q1b;
+                q0b = __ldg(idx + next_kb * BK + lane);
+                q1b = __ldg(idx + next_kb * BK + 32 + lane);
+                next_kb = (next_kb + 1 < nkb) ? next_kb + 1 : 0;
+                // W^T: one 512-B row segment per warp instruction
+#pragma unroll
+                for (int i = 0; i < kRowsB; ++i) {
+                    const int jr = warp + kProducerWarps * i;  // warp-uniform
+                    const int h = __shfl_sync(0xffffffffu, jr < 32 ? v0 : v1, jr & 31);
+                    const bool ok_b = b_col_ok && h < H;
+                    cp_async_16(b_stage + b_off[i], ok_b ? Wt + (size_t)h * N + b_col : Wt, ok_b ? 16u : 0u);
+                }
+                // X^T: two 256-B row segments per warp instruction
+#pragma unroll
+                for (int i = 0; i < kRowsA; ++i) {
+                    const int jr = 2 * (warp + kProducerWarps * i) + (lane >> 4);
+                    const int h0v = __shfl_sync(0xffffffffu, v0, jr & 31);
+                    const int h1v = __shfl_sync(0xffffffffu, v1, jr & 31);
+                    const int h = jr < 32 ? h0v : h1v;
+                    const bool ok_a = a_col_ok && h < H;
+                    cp_async_16(a_stage + a_off[i], ok_a ? Xt + (size_t)h * ldT + a_col : Xt, ok_a ? 16u : 0u);
+                }
+                cp_async_arrive_noinc(full);
+                if (++stage == STAGES2) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+        cp_async_wait_all();
+    } else if (warp == kMmaWarp) {
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        if (rank == 1) {
+            // ------------------------------------------------------------ relay (peer CTA)
+            if (lane == 0) {
+                const uint32_t leader_pair_full0 = mapa_shared(smem_addr(&bars->pair_full[0]), 0);
+                for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        if (!mbar_wait(smem_addr(&bars->full[stage]), phase, status, abort_flag)) {
+                            st_shared_cluster_u32(peer_abort, 1);
+                            ok = false;
+                            break;
+                        }
+                        fence_proxy_async_smem();  // the peer's cp.async data, read by the leader's MMA
+                        mbar_arrive_cluster(leader_pair_full0 + stage * (uint32_t)sizeof(uint64_t));
+                        if (++stage == STAGES2) {
+                            stage = 0;
+                            phase ^= 1;
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+        } else {
+            // ------------------------------------------------------------ MMA issuer (leader)
+            constexpr uint32_t idesc = idesc_bf16_f32_mn_mn(BM2, 256);
+            uint32_t acc_phase = 0;
+            const uint32_t empty0_local = smem_addr(&bars->empty[0]);
+            const uint32_t empty0_peer = mapa_shared(empty0_local, 1);
+            const uint32_t tfull_local = smem_addr(&bars->tfull);
+            const uint32_t tfull_peer = mapa_shared(tfull_local, 1);
+            if (debug_timeout) {
+                ok = mbar_wait(smem_addr(&bars->never), 0, status, abort_flag, kDebugWaitLimitNs);
+                if (!ok) st_shared_cluster_u32(peer_abort, 1);
+            }
+            for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
+                if (!mbar_wait_cluster(smem_addr(&bars->tempty), acc_phase ^ 1, status, abort_flag)) {
+                    st_shared_cluster_u32(peer_abort, 1);
+                    break;
+                }
+                tc_fence_after();
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(smem_addr(&bars->full[stage]), phase, status, abort_flag) ||
+                        !mbar_wait_cluster(smem_addr(&bars->pair_full[stage]), phase, status, abort_flag)) {
+                        st_shared_cluster_u32(peer_abort, 1);
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t a_base = smem_addr(sA + stage * A2_STAGE_BYTES);
+                        const uint32_t b_base = smem_addr(sB + stage * B2_STAGE_BYTES);
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint32_t accumulate = (kb | kk) != 0 ? 1u : 0u;
+                            const uint64_t adesc = smem_desc_sw128(a_base + kk * 2048, CHUNK_BYTES, 1024);
+                            const uint64_t blo = smem_desc_sw128(b_base + kk * 2048, CHUNK_BYTES, 1024);
+                            const uint64_t bhi = smem_desc_sw128(b_base + 2 * CHUNK_BYTES + kk * 2048, CHUNK_BYTES, 1024);
+                            umma_f16_pair(tmem_base, adesc, blo, idesc, accumulate);
+                            umma_f16_pair(tmem_base + 256u, adesc, bhi, idesc, accumulate);
+                        }
+                        const uint32_t eoff = stage * (uint32_t)sizeof(uint64_t);
+                        umma_commit_pair(empty0_local + eoff);
+                        umma_commit_pair(empty0_peer + eoff);
+                    }
+                    __syncwarp();
+                    if (++stage == STAGES2) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                if (lane == 0) {
+                    umma_commit_pair(tfull_local);
+                    umma_commit_pair(tfull_peer);
+                }
+                __syncwarp();
+                acc_phase ^= 1;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        uint32_t acc_phase = 0;
+        const uint32_t tempty_leader = mapa_shared(smem_addr(&bars->tempty), 0);
+        for (int tile = cluster_id; tile < num_tiles; tile += num_clusters) {
+            const TileCoord tc = decode_tile2(group, tile, m_tiles);
+            const int N = group.N[tc.p];
+            uint16_t* __restrict__ Y = group.Y[tc.p];
+            if (!mbar_wait(smem_addr(&bars->tfull), acc_phase, status, abort_flag)) {
+                st_shared_cluster_u32(peer_abort, 1);
+                break;
+            }
+            tc_fence_after();
+            const int row = tc.m0 + HALF_M * (int)rank + q * 32 + lane;
+            uint16_t* yrow = Y + (size_t)row * N;
+#pragma unroll 1
+            for (int cc = 0; cc < TMEM_COLS2 / 32; ++cc) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(cc * 32), r);
+                tmem_ld_wait();
+                const int c = cc * 32;
+                const int ncol = tc.n0 + 256 * ((c & 255) >> 7) + 128 * (c >> 8) + (c & 127);
+                if (row < T) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const int nn = ncol + v * 8;
+                        if (nn < N) {
+                            uint4 o;
+                            o.x = pack_bf16x2(__uint_as_float(r[v * 8 + 0]), __uint_as_float(r[v * 8 + 1]));
+                            o.y = pack_bf16x2(__uint_as_float(r[v * 8 + 2]), __uint_as_float(r[v * 8 + 3]));
+                            o.z = pack_bf16x2(__uint_as_float(r[v * 8 + 4]), __uint_as_float(r[v * 8 + 5]));
+                            o.w = pack_bf16x2(__uint_as_float(r[v * 8 + 6]), __uint_as_float(r[v * 8 + 7]));
+                            *reinterpret_cast<uint4*>(yrow + nn) = o;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_leader);
+            acc_phase ^= 1;
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync();  // the leader's last MMAs and the peer's last TMEM reads are done
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc_pair(tmem_base, TMEM_COLS2);
+}
+
+}  // namespace pair
+
 }  // namespace
 
 size_t gemm_smem_bytes() { return kSmemBytes; }
 
-int gemm_group_tiles(GemmGroup& g, int T) {
-    const int m_tiles = (T + BM - 1) / BM;
+int gemm_group_tiles(GemmGroup& g, int T, int pair) {
+    const int bm = pair ? pair::BM2 : BM, bn = pair ? pair::BN2 : BN;
+    const int m_tiles = (T + bm - 1) / bm;
     g.tile_start[0] = 0;
-    for (int p = 0; p < g.count; ++p) g.tile_start[p + 1] = g.tile_start[p] + m_tiles * ((g.N[p] + BN - 1) / BN);
+    for (int p = 0; p < g.count; ++p) g.tile_start[p + 1] = g.tile_start[p] + m_tiles * ((g.N[p] + bn - 1) / bn);
     for (int p = g.count + 1; p <= kMaxGroup; ++p) g.tile_start[p] = g.tile_start[g.count];
     return g.tile_start[g.count];
+}
+
+cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group, const int32_t* idx,
+                             int k, int T, int H, int* status, int debug_timeout, int num_sms,
+                             cudaStream_t stream) {
+    if (group.count < 1 || group.count > kMaxGroup) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(pair::gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)pair::kSmemBytes2);
+    if (e != cudaSuccess) return e;
+    const int tiles = group.tile_start[group.count];
+    int clusters = num_sms / 2;
+    if (clusters > tiles) clusters = tiles;
+    if (clusters < 1) clusters = 1;
+    pair::gemm_pair_kernel<<<2 * clusters, kThreads, pair::kSmemBytes2, stream>>>(Xt, ldT, group, idx, k, T, H,
+                                                                                   status, debug_timeout);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt, const uint16_t* Xt,

@@ -97,6 +97,18 @@ def test_linear_gemm_path_for_small_T(rmm, T):
     assert_close(Y, Yo, f"gemm T={T}")
 
 
+@pytest.mark.parametrize("producer", [0, 1, 2])
+@pytest.mark.parametrize("T,H,N", [(300, 384, 776), (129, 1000, 520), (513, 256, 264), (1, 640, 1024)])
+def test_gemm_producers(rmm, producer, T, H, N):
+    """CTA-pair cp.async (0, default), single-CTA TMA gather4 (1), single-CTA cp.async (2)."""
+    X = rmm_synth.activations(T, H, 300 + T)
+    W = rmm_synth.weights(N, H, 301 + T)
+    Y, idx = run_linear(rmm, X, W, 0.4, rmm.options(t_gemv=0, gemm_producer=producer))
+    Yo, io = oracle.linear(X, W, 0.4)
+    assert np.array_equal(idx, io)
+    assert_close(Y, Yo, f"producer {producer} T={T} H={H} N={N}")
+
+
 def test_linear_tie_heavy_inputs(rmm):
     X = rmm_synth.tie_heavy((40, 256), 5)
     W = rmm_synth.weights(128, 256, 6)
