@@ -318,14 +318,24 @@ def run_rmm(args, world, rank, local):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record()
     for i in range(K):
-        step(i)
+        step()
     t1.record()
     torch.cuda.synchronize()
     barrier(world)
-    clk = clocks.stop()
     ms = t0.elapsed_time(t1)
     ms_max = max_over_ranks(ms, world)
     value = job_throughput(step_flops * K, world, ms_max) / 1e12
+
+    # the same K steps again with events recorded around each product launch
+    # (the events separate the product kernel from its predecessor, so this
+    # pass is timed on its own and only its per-kernel split is used)
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(K):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
 
     # dominant kernel: the reduced GEMM launches, timed by events the library
     # records around each product launch inside the timed region

@@ -51,6 +51,8 @@ __global__ void __launch_bounds__(D)
     const int q_lo = per_query_head ? set : set * G;
     const int q_hi = per_query_head ? set + 1 : (set + 1) * G;
     const int j = threadIdx.x;
+    pdl_wait();
+    pdl_launch_dependents();
 
     uint32_t m = 0;
     for (int q = q_lo; q < q_hi; ++q) {
@@ -107,6 +109,8 @@ __global__ void __launch_bounds__(kThreads)
     const int l_end = min(L, l_begin + chunk);
     const int R = nq * tq;  // rows: r = qi * tq + ti
     const int tid = threadIdx.x;
+    pdl_wait();
+    pdl_launch_dependents();
 
     for (int i = tid; i < k; i += kThreads) sidx[i] = idx[(size_t)blockIdx.x * k + i];
     __syncthreads();
@@ -266,6 +270,8 @@ __global__ void __launch_bounds__(kThreads)
 
 __global__ void __launch_bounds__(D)
     attn_combine_kernel(const float* __restrict__ partials, int nsplit, uint16_t* __restrict__ O) {
+    pdl_wait();
+    pdl_launch_dependents();
     const size_t row = blockIdx.x;
     const float* p = partials + row * nsplit * PSTRIDE;
     float M = -INFINITY;
@@ -310,18 +316,17 @@ cudaError_t launch_attn(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V
                         int Hkv, int T, int L, int ldL, int k, int causal, float scale,
                         int per_query_head, uint16_t* O, int32_t* idx, float* partials,
                         const AttnPlan& p, cudaStream_t stream) {
-    attn_select_kernel<<<B * p.nsets, D, 0, stream>>>(Q, Hq, Hkv, T, k, per_query_head, idx);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(attn_select_kernel, dim3(B * p.nsets), dim3(D), 0, stream, Q, Hq, Hkv, T, k,
+                               per_query_head, idx);
     if (e != cudaSuccess) return e;
     const int nq = per_query_head ? 1 : Hq / Hkv;
     if (nq > RMAX) return cudaErrorInvalidValue;
     dim3 grid(B * p.nsets, p.nsplit, (T + p.tq - 1) / p.tq);
-    attn_split_kernel<<<grid, kThreads, 0, stream>>>(Q, Kt, V, Hq, Hkv, T, L, ldL, k, causal, scale,
-                                                     per_query_head, idx, partials, p.chunk, p.tq);
-    e = cudaGetLastError();
+    e = launch_pdl(attn_split_kernel, grid, dim3(kThreads), 0, stream, Q, Kt, V, Hq, Hkv, T, L, ldL, k, causal,
+                   scale, per_query_head, (const int32_t*)idx, partials, p.chunk, p.tq);
     if (e != cudaSuccess) return e;
-    attn_combine_kernel<<<B * Hq * T, D, 0, stream>>>(partials, p.nsplit, O);
-    return cudaGetLastError();
+    return launch_pdl(attn_combine_kernel, dim3(B * Hq * T), dim3(D), 0, stream, (const float*)partials, p.nsplit,
+                      O);
 }
 
 }  // namespace rmm

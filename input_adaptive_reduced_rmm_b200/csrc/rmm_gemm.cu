@@ -155,6 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = bars->tmem_base;
+    pdl_wait();  // the kept list and X^T come from the preceding kernels
+    pdl_launch_dependents();
 
     if (warp < kProducerWarps) {
         // ------------------------------------------------------------ producer
@@ -476,6 +478,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
     tc_fence_after();
     const uint32_t tmem_base = bars->tmem_base;
+    pdl_wait();  // the kept list and X^T come from the preceding kernels
+    pdl_launch_dependents();
 
     if (warp < kProducerWarps) {
         // ------------------------------------------------------------ producer (both CTAs)
@@ -701,9 +705,8 @@ cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group
     int clusters = num_sms / 2;
     if (clusters > tiles) clusters = tiles;
     if (clusters < 1) clusters = 1;
-    pair::gemm_pair_kernel<<<2 * clusters, kThreads, pair::kSmemBytes2, stream>>>(Xt, ldT, group, idx, k, T, H,
-                                                                                   status, debug_timeout);
-    return cudaGetLastError();
+    return launch_pdl(pair::gemm_pair_kernel, dim3(2 * clusters), dim3(kThreads), pair::kSmemBytes2, stream, Xt,
+                      ldT, group, idx, k, T, H, status, debug_timeout);
 }
 
 cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt, const uint16_t* Xt,
@@ -717,9 +720,8 @@ cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt, co
     if (e != cudaSuccess) return e;
     const int tiles = group.tile_start[group.count];
     const int grid = tiles < num_sms ? tiles : num_sms;
-    kern<<<grid, kThreads, kSmemBytes, stream>>>(map_xt, map_wt, Xt, ldT, group, idx, k, T, H, status,
-                                                  debug_timeout);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), kSmemBytes, stream, map_xt, map_wt, Xt, ldT, group, idx,
+                      k, T, H, status, debug_timeout);
 }
 
 }  // namespace rmm

@@ -51,6 +51,8 @@ __global__ void __launch_bounds__(kThreads)
     float* red = reinterpret_cast<float*>(sidx + rows_per_split);  // [TT][COLS]
     __shared__ int is_last;
 
+    pdl_wait();
+    pdl_launch_dependents();
     const int tid = threadIdx.x;
     const int rg = tid / TPR, ct = tid % TPR;
     const int split = blockIdx.y;
@@ -196,9 +198,8 @@ cudaError_t launch_t(const uint16_t* X, int T, int H, const uint16_t* Wt, int N,
         if (e != cudaSuccess) return e;
     }
     dim3 grid(p.col_blocks, p.splits);
-    kern<<<grid, kThreads, smem, stream>>>(X, T, H, Wt, N, idx, k, Y, partials, counters,
-                                           p.rows_per_split);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(kThreads), smem, stream, X, T, H, Wt, N, idx, k, Y, partials,
+                      counters, p.rows_per_split);
 }
 
 template <int TT>

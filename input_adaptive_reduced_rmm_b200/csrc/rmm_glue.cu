@@ -16,6 +16,7 @@ constexpr int kTile = 64;
 
 __global__ void __launch_bounds__(256)
     transpose_kernel(const uint16_t* __restrict__ W, uint16_t* __restrict__ Wt, int N, int H) {
+    pdl_wait();
     __shared__ uint16_t tile[kTile][kTile + 2];
     const int h0 = blockIdx.x * kTile, n0 = blockIdx.y * kTile;
     const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 x 4
@@ -32,6 +33,8 @@ __global__ void __launch_bounds__(256)
 
 __global__ void pad_idx_kernel(const int32_t* __restrict__ src, int k, int H,
                                int32_t* __restrict__ dst, int pad_to) {
+    pdl_wait();
+    pdl_launch_dependents();
     for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < pad_to; j += gridDim.x * blockDim.x)
         dst[j] = (j < k) ? src[j] : H;
 }
@@ -47,8 +50,8 @@ cudaError_t launch_transpose(const uint16_t* W, uint16_t* Wt, int N, int H, cuda
 cudaError_t launch_pad_idx(const int32_t* src, int k, int H, int32_t* dst, int pad_to,
                            cudaStream_t stream) {
     const int blocks = (pad_to + 255) / 256;
-    pad_idx_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, stream>>>(src, k, H, dst, pad_to);
-    return cudaGetLastError();
+    return launch_pdl(pad_idx_kernel, dim3(blocks < 1 ? 1 : blocks), dim3(256), 0, stream, src, k, H, dst,
+                      pad_to);
 }
 
 }  // namespace rmm

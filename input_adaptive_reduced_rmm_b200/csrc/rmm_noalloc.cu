@@ -51,6 +51,8 @@ rmm_status noalloc_scratch(uint8_t** out) {
 // Zero the words a call needs to start at zero (split counters, status word);
 // the scratch keeps whatever the previous call left there.
 __global__ void noalloc_clear_kernel(unsigned* words, int n) {
+    pdl_wait();
+    pdl_launch_dependents();
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) words[i] = 0;
 }
 

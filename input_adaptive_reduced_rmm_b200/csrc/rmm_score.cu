@@ -23,7 +23,7 @@ namespace rmm {
 
 namespace {
 
-constexpr int kTileT = 64;  // tokens per tile
+constexpr int kTileT = 128;  // tokens per tile
 constexpr int kTileH = 64;  // channels per strip
 constexpr int kThreads = 256;
 
@@ -35,7 +35,10 @@ __global__ void __launch_bounds__(kThreads)
     // 8 apart then fall on distinct bank groups (2-way conflicts at most).
     __shared__ __align__(16) uint16_t tile[kTileT][kTileH + 2];
     __shared__ uint16_t red[32][kTileH];
+    constexpr int kPasses = kTileT / 32;  // 16-byte loads in flight per thread
 
+    pdl_wait();
+    pdl_launch_dependents();
     const int tid = threadIdx.x;
     const int cg = tid & 7;    // 8-channel group within the strip
     const int row = tid >> 3;  // 0..31
@@ -47,22 +50,30 @@ __global__ void __launch_bounds__(kThreads)
     for (int i = 0; i < 8; ++i) mx[i] = 0;
 
     for (int t0 = blockIdx.y * kTileT; t0 < T; t0 += gridDim.y * kTileT) {
+        // issue all of this thread's loads of the tile before using any
+        uint4 q[kPasses];
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const int r = p * 32 + row;
-            const int t = t0 + r;
-            uint16_t v[8];
+        for (int p = 0; p < kPasses; ++p) {
+            const int t = t0 + p * 32 + row;
             if (kVec && t < T && hc + 8 <= H) {
-                uint4 q = ld_nc_v4(X + (size_t)t * H + hc);
-                v[0] = q.x & 0xFFFF; v[1] = q.x >> 16;
-                v[2] = q.y & 0xFFFF; v[3] = q.y >> 16;
-                v[4] = q.z & 0xFFFF; v[5] = q.z >> 16;
-                v[6] = q.w & 0xFFFF; v[7] = q.w >> 16;
+                q[p] = ld_nc_v4(X + (size_t)t * H + hc);
             } else {
+                uint16_t w[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    v[i] = (t < T && hc + i < H) ? X[(size_t)t * H + hc + i] : (uint16_t)0;
+                    w[i] = (t < T && hc + i < H) ? X[(size_t)t * H + hc + i] : (uint16_t)0;
+                q[p] = make_uint4(w[0] | ((uint32_t)w[1] << 16), w[2] | ((uint32_t)w[3] << 16),
+                                  w[4] | ((uint32_t)w[5] << 16), w[6] | ((uint32_t)w[7] << 16));
             }
+        }
+#pragma unroll
+        for (int p = 0; p < kPasses; ++p) {
+            const int r = p * 32 + row;
+            uint16_t v[8];
+            v[0] = q[p].x & 0xFFFF; v[1] = q[p].x >> 16;
+            v[2] = q[p].y & 0xFFFF; v[3] = q[p].y >> 16;
+            v[4] = q[p].z & 0xFFFF; v[5] = q[p].z >> 16;
+            v[6] = q[p].w & 0xFFFF; v[7] = q[p].w >> 16;
 #pragma unroll
             for (int i = 0; i < 8; ++i) mx[i] = max(mx[i], (uint32_t)(v[i] & 0x7FFF));
             if (kWriteXt) {
@@ -75,11 +86,11 @@ __global__ void __launch_bounds__(kThreads)
         }
         if (kWriteXt) {
             __syncthreads();
-            // transposed write-out: 8 threads per channel row, 8 tokens each
-            const int tc = tid & 7;
+            // transposed write-out: 16 threads per channel row, 8 tokens each
+            const int tc = tid & 15;
 #pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                const int hl = p * 32 + (tid >> 3);
+            for (int p = 0; p < kTileH / 16; ++p) {
+                const int hl = p * 16 + (tid >> 4);
                 const int h = h0 + hl;
                 const int tt = t0 + tc * 8;
                 if (h < H && tt < T) {
@@ -129,18 +140,9 @@ cudaError_t launch_score(const uint16_t* X, int T, int H, uint32_t* s32, uint16_
     if (ty < 1) ty = 1;
     dim3 grid(strips, ty);
     const bool vec = (H % 8 == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
-    if (Xt) {
-        if (vec)
-            score_kernel<true, true><<<grid, kThreads, 0, stream>>>(X, T, H, s32, Xt, ldT);
-        else
-            score_kernel<true, false><<<grid, kThreads, 0, stream>>>(X, T, H, s32, Xt, ldT);
-    } else {
-        if (vec)
-            score_kernel<false, true><<<grid, kThreads, 0, stream>>>(X, T, H, s32, nullptr, 0);
-        else
-            score_kernel<false, false><<<grid, kThreads, 0, stream>>>(X, T, H, s32, nullptr, 0);
-    }
-    return cudaGetLastError();
+    auto kern = Xt ? (vec ? score_kernel<true, true> : score_kernel<true, false>)
+                   : (vec ? score_kernel<false, true> : score_kernel<false, false>);
+    return launch_pdl(kern, grid, dim3(kThreads), 0, stream, X, T, H, s32, Xt, ldT);
 }
 
 }  // namespace rmm

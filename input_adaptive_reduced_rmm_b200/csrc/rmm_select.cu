@@ -86,6 +86,25 @@ __device__ __forceinline__ int warp_find_bin(const int* cnt, int nbins, int k, i
     return __shfl_sync(0xffffffffu, found, src);
 }
 
+// Histogram of 8-bit bins over the keys: bin = (key >> shift) & 255 for keys
+// with key >> 8 == match (all keys when match == ~0).  Lanes holding the same
+// bin are merged with __match_any_sync so each distinct bin costs one shared
+// atomic per warp and chunk.
+__device__ __forceinline__ void warp_histogram(const uint16_t* s, int H, int shift, uint32_t match,
+                                               int* hist) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int h0 = warp * 32; h0 < H; h0 += kThreads) {
+        const int h = h0 + lane;
+        uint32_t bin = 0xFFFFFFFFu;  // "no bin"
+        if (h < H) {
+            const uint32_t v = s[h];
+            if (match == 0xFFFFFFFFu || (v >> 8) == match) bin = (v >> shift) & 0xFFu;
+        }
+        const unsigned same = __match_any_sync(0xffffffffu, bin);
+        if (bin != 0xFFFFFFFFu && lane == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
+    }
+}
+
 __global__ void __launch_bounds__(kThreads)
     select_kernel(uint32_t* __restrict__ s32, int clear_input, int H, int k, int32_t* __restrict__ idx,
                   int pad_to, int32_t* __restrict__ idx_copy, uint32_t* __restrict__ s_out) {
@@ -95,6 +114,8 @@ __global__ void __launch_bounds__(kThreads)
     __shared__ uint32_t warp_tot[32];
     __shared__ int sh_thresh, sh_need;
 
+    pdl_wait();
+    pdl_launch_dependents();
     const int tid = threadIdx.x;
     if (tid < 256) hist_hi[tid] = 0;
     if (tid < 256) hist_fine[tid] = 0;
@@ -109,8 +130,9 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();
 
     // 2a. coarse histogram of s >> 8 (256 bins; keys are < 2^16, and < 2^15
-    //     for finite bf16 magnitudes)
-    for (int h = tid; h < H; h += kThreads) atomicAdd(&hist_hi[s[h] >> 8], 1);
+    //     for finite bf16 magnitudes).  Scores of one input crowd into a few
+    //     exponent bins, so equal bins are merged per warp first.
+    warp_histogram(s, H, 8, 0xFFFFFFFFu, hist_hi);
     __syncthreads();
     if (tid < 32) {
         int above;
@@ -124,8 +146,7 @@ __global__ void __launch_bounds__(kThreads)
     const int bhi = sh_thresh;
     const int k2 = sh_need;
     // 2b. fine histogram of the low 8 bits inside the coarse bin
-    for (int h = tid; h < H; h += kThreads)
-        if ((s[h] >> 8) == bhi) atomicAdd(&hist_fine[s[h] & 0xFF], 1);
+    warp_histogram(s, H, 0, (uint32_t)bhi, hist_fine);
     __syncthreads();
     if (tid < 32) {
         int above;
@@ -180,8 +201,8 @@ cudaError_t launch_select(uint32_t* s32, int clear_input, int H, int k, int32_t*
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    select_kernel<<<1, kThreads, smem, stream>>>(s32, clear_input, H, k, idx, pad_to, idx_copy, s_out);
-    return cudaGetLastError();
+    return launch_pdl(select_kernel, dim3(1), dim3(kThreads), smem, stream, s32, clear_input, H, k, idx,
+                      pad_to, idx_copy, s_out);
 }
 
 }  // namespace rmm
