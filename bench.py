@@ -231,50 +231,69 @@ def make_inputs(dev):
     return acts, Wts
 
 
-def time_decode_and_attention(dev, peaks):
-    """Secondary rows: the T=1 decode GEMV over the same projections, and decode attention."""
+def time_decode(dev, peaks):
+    """Secondary row: one decode step (T = 1) over the same seven projections, grouped like
+    the prefill step, at r = 0.5; L2 flushed before every timed step."""
     from input_adaptive_reduced_rmm_b200 import rmm
 
-    out = {}
-    # decode GEMV: T = 1, all seven projections, r = 0.5, weights larger than L2 in total
     acts = {s: rmm_synth.activations(1, h, 500 + s).to(dev) for s, h in ACT_H.items()}
     Wts = {n: rmm.rmm_transpose_weight(rmm_synth.weights(N, H, 600 + i, std=0.02).to(dev))
            for i, (n, H, N, _) in enumerate(PROJ)}
-    ws = {n: rmm.new_workspace(rmm.rmm_linear_workspace_bytes(1, H, N), dev) for n, H, N, _ in PROJ}
     Ys = {n: torch.empty(1, N, dtype=torch.bfloat16, device=dev) for n, H, N, _ in PROJ}
-    ev = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n, _, _, _ in PROJ}
-    opts = {n: rmm.options(product_events=ev[n]) for n, _, _, _ in PROJ}
+    ws = {c: rmm.new_workspace(rmm.rmm_linear_group_workspace_bytes(
+        1, ACT_H[s], [PROJ_BY_NAME[n][1] for n in names]), dev) for c, (s, names) in enumerate(CALLS)}
+    ev = {c: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for c in range(len(CALLS))}
+    opts_ev = {c: rmm.options(product_events=ev[c]) for c in range(len(CALLS))}
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
-    def step():
-        for n, H, N, s in PROJ:
-            rmm.rmm_linear(acts[s], Wts[n], R, Y=Ys[n], workspace=ws[n], opts=opts[n])
+    def step(with_events):
+        for c, (s, names) in enumerate(CALLS):
+            rmm.rmm_linear_group(acts[s], [Wts[n] for n in names], R, Ys=[Ys[n] for n in names],
+                                 workspace=ws[c], opts=opts_ev[c] if with_events else None)
 
-    for _ in range(3):
-        step()
+    def dense_step():
+        for n, H, N, s in PROJ:
+            torch.matmul(acts[s], Wts[n], out=Ys[n])
+
+    def timed(fn, iters=20):
+        for _ in range(3):
+            fn()
+        total = 0.0
+        for _ in range(iters):
+            flush.zero_()  # evict the weights from L2 before every timed step
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            total += e0.elapsed_time(e1)
+        return total / iters
+
+    call_ms = timed(lambda: step(False))
+    dense_ms = timed(dense_step)
     iters = 20
-    gemv_ms = {n: 0.0 for n, _, _, _ in PROJ}
-    call_ms = 0.0
+    for _ in range(3):
+        step(True)
+    kern_ms = 0.0
     for _ in range(iters):
-        flush.zero_()  # evict the weights from L2 between iterations
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        step()
-        e1.record()
+        flush.zero_()
+        step(True)
         torch.cuda.synchronize()
-        call_ms += e0.elapsed_time(e1)
-        for n in gemv_ms:
-            gemv_ms[n] += ev[n][0].elapsed_time(ev[n][1])
-    bytes_total = sum(metrics.gemv_bytes(1, H, N, metrics.k_for(H, R)) for _, H, N, _ in PROJ)
-    gemv_total_ms = sum(gemv_ms.values()) / iters
-    out["decode_gemv"] = {
-        "workload": "T=1, same 7 projections, r=0.5, L2 flushed between iterations",
-        "kernel_us_per_step": 1e3 * gemv_total_ms,
-        "achieved_gbs": bytes_total / (gemv_total_ms * 1e-3) / 1e9,
-        "frac_of_hbm": bytes_total / (gemv_total_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-        "calls_us_per_step": 1e3 * call_ms / iters,
-        "per_projection_us": {n: 1e3 * v / iters for n, v in gemv_ms.items()},
-    }
+        kern_ms += sum(ev[c][0].elapsed_time(ev[c][1]) for c in ev)
+    kern_ms /= iters
+    kept_bytes = sum(metrics.gemv_bytes(1, H, N, metrics.k_for(H, R)) for _, H, N, _ in PROJ)
+    dense_bytes = sum(N * H * 2 + H * 2 + N * 2 for _, H, N, _ in PROJ)
+    out = {"decode_gemv": {
+        "workload": "T=1, same 7 projections (q+k+v, o, gate+up, down), r=0.5, L2 flushed before each step",
+        "step_us": 1e3 * call_ms,
+        "kernel_us": 1e3 * kern_ms,
+        "kernel_gbs": kept_bytes / (kern_ms * 1e-3) / 1e9,
+        "kernel_frac_of_hbm": kept_bytes / (kern_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "step_gbs": kept_bytes / (call_ms * 1e-3) / 1e9,
+        "dense_us": 1e3 * dense_ms,
+        "dense_gbs": dense_bytes / (dense_ms * 1e-3) / 1e9,
+        "speedup_vs_dense": dense_ms / call_ms,
+    }}
     del Wts, ws, flush
     torch.cuda.empty_cache()
     return out
@@ -392,7 +411,7 @@ def run_rmm(args, world, rank, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = job_throughput(step_flops * K, world, e2e_ms) / 1e12
 
-    extra = time_decode_and_attention(dev, peaks) if not args.skip_secondary else {}
+    extra = time_decode(dev, peaks) if not args.skip_secondary else {}
 
     cpu = None
     if rank == 0 and not args.skip_cpu_baseline:
@@ -426,6 +445,44 @@ def run_rmm(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_single(args):
+    """One rmm_linear shape timed alone (profiling aid): --single T,H,N,r."""
+    from input_adaptive_reduced_rmm_b200 import rmm
+
+    T, H, N, r = args.single.split(",")
+    T, H, N, r = int(T), int(H), int(N), float(r)
+    dev = torch.device("cuda", 0)
+    X = rmm_synth.activations(T, H, 11).to(dev)
+    Wt = rmm.rmm_transpose_weight(rmm_synth.weights(N, H, 12, std=0.02).to(dev))
+    Y = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    opts = rmm.options(gemm_producer=args.gemm_producer, product_events=ev)
+    ws = rmm.new_workspace(rmm.rmm_linear_workspace_bytes(T, H, N, opts), dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        rmm.rmm_linear(X, Wt, r, Y=Y, workspace=ws, opts=opts)
+    torch.cuda.synchronize()
+    call, kern = [], []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        rmm.rmm_linear(X, Wt, r, Y=Y, workspace=ws, opts=opts)
+        e1.record()
+        torch.cuda.synchronize()
+        call.append(e0.elapsed_time(e1))
+        kern.append(ev[0].elapsed_time(ev[1]))
+    if rmm.rmm_get_status(ws) != rmm.RMM_OK:
+        raise RuntimeError("device status not OK")
+    k = metrics.k_for(H, r)
+    km = statistics.median(kern)
+    out = {"single": {"T": T, "H": H, "N": N, "r": r, "k": k, "producer": args.gemm_producer,
+                      "call_us": 1e3 * statistics.median(call), "product_us": 1e3 * km,
+                      "product_tflops": metrics.reduced_linear_flops(T, N, k) / (km * 1e-3) / 1e12,
+                      "product_gbs": metrics.gemv_bytes(T, H, N, k) / (km * 1e-3) / 1e9}}
+    print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,9 +492,14 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=24)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-secondary", action="store_true")
+    ap.add_argument("--single", default=None, help="T,H,N,r: time one rmm_linear shape alone")
+    ap.add_argument("--gemm-producer", type=int, default=0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.single:
+        run_single(args)
+        return
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":

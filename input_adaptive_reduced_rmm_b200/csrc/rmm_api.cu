@@ -11,6 +11,27 @@
 #include "rmm_internal.h"
 
 namespace rmm {
+
+cudaError_t ensure_smem_limit_fn(const void* kern, size_t bytes) {
+    if (bytes == 0) return cudaSuccess;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+    static std::mutex mu;
+    static std::unordered_map<uint64_t, size_t> done;  // (device, kernel) -> limit set
+    const uint64_t key = (reinterpret_cast<uint64_t>(kern) << 8) ^ (uint64_t)(dev & 0xFF);
+    {
+        std::lock_guard<std::mutex> g(mu);
+        auto it = done.find(key);
+        if (it != done.end() && it->second >= bytes) return cudaSuccess;
+    }
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> g(mu);
+    size_t& v = done[key];
+    if (bytes > v) v = bytes;
+    return cudaSuccess;
+}
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -52,8 +73,8 @@ bool opts_valid(const rmm_options* o) {
 struct LinearLayout {
     bool gemv;
     int ldT;           // leading dimension of X^T (GEMM path)
-    int col_blocks;    // GEMV: most column blocks of any product
-    size_t s32, idx, counters, partials, xt, total;
+    GemvGroup plan;    // GEMV path
+    size_t s32, idx, partials, xt, total;
 };
 
 // Workspace layout for `count` products of one activation matrix [T, H] with
@@ -67,14 +88,11 @@ LinearLayout linear_layout(int T, int H, const int* Ns, int count, int k, const 
     L.idx = off;
     off += align_up(((size_t)H + 2 * kGemmBK) * sizeof(int32_t), kAlign);
     if (L.gemv) {
-        size_t part = 0;
-        for (int p = 0; p < count; ++p) {
-            const GemvPlan plan = gemv_plan(T, Ns[p], k, sms, o.gemv_splits);
-            if (plan.col_blocks > L.col_blocks) L.col_blocks = plan.col_blocks;
-            if (gemv_partials_bytes(plan, T, Ns[p]) > part) part = gemv_partials_bytes(plan, T, Ns[p]);
-        }
-        L.counters = off;
-        off += align_up((size_t)L.col_blocks * sizeof(unsigned), kAlign);
+        memset(&L.plan, 0, sizeof L.plan);
+        L.plan.count = count;
+        for (int p = 0; p < count; ++p) L.plan.N[p] = Ns[p];
+        size_t part = gemv_group_plan(L.plan, T, k, o.gemv_splits, sms);
+        if (k == H) part = gemv_partials_bound(L.plan, T, H, o.gemv_splits, sms);  // size query: any k
         L.partials = off;
         off += align_up(part, kAlign);
     } else {
@@ -177,16 +195,14 @@ rmm_status run_product_kernels(const void* X, int T, int H, int count, const voi
     int* status = reinterpret_cast<int*>(ws);
     const int sms = num_sms_current();
     if (L.gemv) {
+        GemvGroup g = L.plan;
         for (int p = 0; p < count; ++p) {
-            const GemvPlan plan = gemv_plan(T, Ns[p], k, sms, o.gemv_splits);
-            cudaError_t e = launch_gemv(static_cast<const uint16_t*>(X), T, H,
-                                        static_cast<const uint16_t*>(Wts[p]), Ns[p], idx_padded, k,
-                                        static_cast<uint16_t*>(Ys[p]),
-                                        reinterpret_cast<float*>(ws + L.partials),
-                                        reinterpret_cast<unsigned*>(ws + L.counters), plan, status, s);
-            if (e != cudaSuccess) return RMM_ERR_CUDA;
+            g.Wt[p] = static_cast<const uint16_t*>(Wts[p]);
+            g.Y[p] = static_cast<uint16_t*>(Ys[p]);
         }
-        return RMM_OK;
+        (void)status;
+        return cuda_status(launch_gemv(static_cast<const uint16_t*>(X), T, H, idx_padded, k, g,
+                                       reinterpret_cast<float*>(ws + L.partials), sms, s));
     }
     if (o.gemm_producer == 1 && count != 1) return RMM_ERR_UNSUPPORTED;
     GemmGroup g;
@@ -243,11 +259,20 @@ rmm_status linear_group(const void* X, int T, int H, double r, int count, const 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint32_t* s32 = reinterpret_cast<uint32_t*>(ws + L.s32);
     int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
-    cudaError_t e = launch_score(static_cast<const uint16_t*>(X), T, H, s32,
-                                 L.gemv ? nullptr : reinterpret_cast<uint16_t*>(ws + L.xt), L.ldT, sms, s);
-    if (e != cudaSuccess) return RMM_ERR_CUDA;
     const int pad_to = (k + kGemmBK - 1) / kGemmBK * kGemmBK;
-    e = launch_select(s32, 1, H, k, idx, pad_to, idx_out, nullptr, s);
+    cudaError_t e;
+    if (L.gemv && T == 1) {
+        // one token: the select kernel reads the score straight from X
+        e = launch_select(static_cast<const uint16_t*>(X), T, nullptr, 0, H, k, idx, pad_to, idx_out, nullptr, s);
+    } else if (L.gemv) {
+        // a few tokens: the score pass spreads the fold over the GPU, no X^T
+        e = launch_score(static_cast<const uint16_t*>(X), T, H, s32, nullptr, 0, sms, s);
+        if (e == cudaSuccess) e = launch_select(nullptr, 0, s32, 1, H, k, idx, pad_to, idx_out, nullptr, s);
+    } else {
+        e = launch_score(static_cast<const uint16_t*>(X), T, H, s32, reinterpret_cast<uint16_t*>(ws + L.xt), L.ldT,
+                         sms, s);
+        if (e == cudaSuccess) e = launch_select(nullptr, 0, s32, 1, H, k, idx, pad_to, idx_out, nullptr, s);
+    }
     if (e != cudaSuccess) return RMM_ERR_CUDA;
     return run_products(X, T, H, count, Wts, Ns, Ys, idx, k, ws, L, o, s);
 }
@@ -349,13 +374,13 @@ rmm_status rmm_score(const void* X, int T, int H, uint32_t* s_out, void* workspa
     int32_t* idx = reinterpret_cast<int32_t*>(ws + off_idx);
     cudaError_t e = launch_score(static_cast<const uint16_t*>(X), T, H, s32, nullptr, 0, num_sms_current(), s);
     if (e != cudaSuccess) return RMM_ERR_CUDA;
-    return cuda_status(launch_select(s32, 1, H, H, idx, H, nullptr, s_out, s));
+    return cuda_status(launch_select(nullptr, 0, s32, 1, H, H, idx, H, nullptr, s_out, s));
 }
 
 rmm_status rmm_select(const uint32_t* sc, int H, int k, int32_t* idx_out, void* /*workspace*/,
                       size_t /*workspace_bytes*/, rmm_stream_t stream) {
     if (!sc || !idx_out || H < 1 || H > 65535 || k < 1 || k > H) return RMM_ERR_INVALID_ARG;
-    return cuda_status(launch_select(const_cast<uint32_t*>(sc), 0, H, k, idx_out, k, nullptr, nullptr,
+    return cuda_status(launch_select(nullptr, 0, const_cast<uint32_t*>(sc), 0, H, k, idx_out, k, nullptr, nullptr,
                                      static_cast<cudaStream_t>(stream)));
 }
 

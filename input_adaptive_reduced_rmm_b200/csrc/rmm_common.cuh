@@ -373,6 +373,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32_mn_mn(int M, int N) {
            | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
 
+// Host: raise a kernel's dynamic shared-memory limit to at least `bytes`,
+// once per (device, kernel, size) -- the attribute call costs host time, so
+// later launches skip it.  The limit also matters below 48 KB when the
+// kernel has static shared memory.  (Defined in rmm_api.cu.)
+cudaError_t ensure_smem_limit_fn(const void* kern, size_t bytes);
+template <typename K>
+inline cudaError_t ensure_smem_limit(K kern, size_t bytes) {
+    return ensure_smem_limit_fn(reinterpret_cast<const void*>(kern), bytes);
+}
+
 // Host: launch `kern` on `stream` as a programmatic dependent of the previous
 // kernel in the stream (its launch overlaps that kernel's tail).
 template <typename... KArgs, typename... Args>

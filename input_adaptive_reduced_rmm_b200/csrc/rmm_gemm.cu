@@ -698,8 +698,7 @@ cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group
                              int k, int T, int H, int* status, int debug_timeout, int num_sms,
                              cudaStream_t stream) {
     if (group.count < 1 || group.count > kMaxGroup) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(pair::gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)pair::kSmemBytes2);
+    cudaError_t e = ensure_smem_limit(pair::gemm_pair_kernel, pair::kSmemBytes2);
     if (e != cudaSuccess) return e;
     const int tiles = group.tile_start[group.count];
     int clusters = num_sms / 2;
@@ -716,7 +715,7 @@ cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt, co
     if (group.count < 1 || group.count > kMaxGroup || (tma_gather && group.count != 1))
         return cudaErrorInvalidValue;
     auto kern = tma_gather ? gemm_kernel<true> : gemm_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    cudaError_t e = ensure_smem_limit(kern, kSmemBytes);
     if (e != cudaSuccess) return e;
     const int tiles = group.tile_start[group.count];
     const int grid = tiles < num_sms ? tiles : num_sms;

@@ -8,13 +8,25 @@
 // reduction cuts that traffic to the k kept weight rows (k*N*2 bytes).  Each
 // kept slice h is one contiguous row of W^T (N*2 bytes).
 //
-// Grid: (column blocks of 256/512 outputs) x (splits of the kept list).  A CTA
-// stages its split's indices and the matching X values in shared memory,
-// then each thread streams 16-byte pieces of kept rows (8 outputs) with
-// non-allocating loads, accumulating T x 8 fp32 sums.  Row groups inside the
-// CTA are folded through shared memory; splits are folded deterministically
-// (fixed order 0..S-1) by the last CTA of each column block to finish, found
-// with a counter that it resets to zero afterwards.
+// Work: for the members p of a group of products sharing X (e.g. q, k, v) the
+// kept list is cut into S splits of at most 512 rows and each member's outputs
+// into column blocks of COLS (256 for T <= 4, narrower for wider T).  One CTA =
+// (member, column block) along x, split along y; x varies fastest, so the CTAs
+// running at the same moment read neighbouring 512-byte pieces of the same
+// kept rows.  S is chosen for ~6 CTAs per SM in several waves: measured on
+// B200, a streaming grid of that shape sustains ~5.5 TB/s on scattered kept
+// rows, while fewer, longer-running CTAs lose to ramp-up and ramp-down.
+//
+// A CTA stages its split's kept indices in shared memory, issues its first
+// batch of weight loads and only then gathers the X values beside them, so
+// both latencies overlap; it streams 16-byte pieces of the kept rows with
+// non-allocating loads (8 or 4 rows in flight per thread, packed fp32x2 FMAs),
+// folds its row groups (shuffles, then the warps in a fixed order) and writes
+// its fp32 partial sums -- or, with one split, Y itself.  A second launch,
+// chained by programmatic dependent launch, adds the S partials of every
+// output in split order and writes Y: no fences, counters or atomics on the
+// streaming CTAs, a deterministic result, and the fold's launch latency hidden
+// behind the product.
 #include "rmm_common.cuh"
 #include "rmm_internal.h"
 
@@ -23,6 +35,10 @@ namespace rmm {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxRowsPerItem = 512;
+constexpr int kFoldCols = 256;  // outputs of one fold CTA (32 threads x 8 columns)
+constexpr int kFoldGroups = kThreads / (kFoldCols / 8);
 
 __device__ __forceinline__ void unpack8(const uint4& w, float (&f)[8]) {
     f[0] = __uint_as_float(w.x << 16);
@@ -35,218 +51,319 @@ __device__ __forceinline__ void unpack8(const uint4& w, float (&f)[8]) {
     f[7] = __uint_as_float(w.w & 0xFFFF0000u);
 }
 
-template <int TT, int TPR>
-__global__ void __launch_bounds__(kThreads)
-    gemv_kernel(const uint16_t* __restrict__ X, int T, int H, const uint16_t* __restrict__ Wt,
-                int N, const int32_t* __restrict__ idx, int k, uint16_t* __restrict__ Y,
-                float* __restrict__ partials, unsigned* __restrict__ counters,
-                int rows_per_split) {
-    constexpr int RG = kThreads / TPR;  // row groups
-    constexpr int COLS = TPR * 8;       // outputs per CTA
+// (d0, d1) = (a * b0 + d0, a * b1 + d1), one packed fp32x2 FMA, round to nearest
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %2};\n\t"
+        "mov.b64 rb, {%3, %4};\n\t"
+        "mov.b64 rd, {%0, %1};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rd;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a), "f"(b0), "f"(b1));
+}
+
+template <int TT>
+__device__ __forceinline__ void fma_row(float (&acc)[TT][8], const uint4& w, const float* xr) {
+    float wf[8];
+    unpack8(w, wf);
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+        const float xv = xr[t];
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) fma2(acc[t][c], acc[t][c + 1], xv, wf[c], wf[c + 1]);
+    }
+}
+
+__device__ __forceinline__ void store_bf16x8(uint16_t* dst, const float* s) {
+    uint4 o;
+    o.x = pack_bf16x2(s[0], s[1]);
+    o.y = pack_bf16x2(s[2], s[3]);
+    o.z = pack_bf16x2(s[4], s[5]);
+    o.w = pack_bf16x2(s[6], s[7]);
+    *reinterpret_cast<uint4*>(dst) = o;
+}
+
+// member of a group whose prefix range holds x
+__device__ __forceinline__ int member_of(const int* start, int count, int x) {
+    int p = 0;
+#pragma unroll
+    for (int i = 1; i < kMaxGroupGemv; ++i)
+        if (i < count && x >= start[i]) p = i;
+    return p;
+}
+
+template <int TT, int COLS>
+__global__ void __launch_bounds__(kThreads, (TT <= 4) ? 3 : 1)
+    gemv_kernel(const uint16_t* __restrict__ X, int T, int H, const int32_t* __restrict__ idx, int k,
+                const __grid_constant__ GemvGroup g, float* __restrict__ partials) {
+    constexpr int TPR = COLS / 8;         // threads per kept-row piece
+    constexpr int RG = kThreads / TPR;    // row groups
     constexpr int U = (TT >= 8) ? 4 : 8;  // kept rows in flight per thread
+    constexpr int WCOLS = (COLS < 256) ? COLS : 256;  // columns held by one warp after its shuffle fold
+    constexpr int P8 = COLS / 8;
 
     extern __shared__ float smem[];
-    float* xs = smem;                                        // [rows][TT]
-    int* sidx = reinterpret_cast<int*>(xs + rows_per_split * TT);  // [rows]
-    float* red = reinterpret_cast<float*>(sidx + rows_per_split);  // [TT][COLS]
-    __shared__ int is_last;
+    float* xs = smem;                                               // [kMaxRowsPerItem][TT]
+    int* sidx = reinterpret_cast<int*>(xs + kMaxRowsPerItem * TT);  // [kMaxRowsPerItem]
+    float* fold = reinterpret_cast<float*>(sidx + kMaxRowsPerItem); // [kWarps][TT][WCOLS]
+    float* part = fold + kWarps * TT * WCOLS;                       // [TT][COLS]
 
     pdl_wait();
     pdl_launch_dependents();
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int rg = tid / TPR, ct = tid % TPR;
-    const int split = blockIdx.y;
-    const int j0 = split * rows_per_split;
-    const int nr = max(0, min(k, j0 + rows_per_split) - j0);
-    const int n = blockIdx.x * COLS + ct * 8;
+    const int p = member_of(g.item_start, g.count, blockIdx.x);
+    const int cb = blockIdx.x - g.item_start[p];
+    const int sp = blockIdx.y;
+    const int N = g.N[p];
+    const int ld = g.ld[p];
+    const int rows = g.rows_per_split[p];
+    const int j0 = sp * rows;
+    const int nr = max(0, min(k, j0 + rows) - j0);
+    const int n0 = cb * COLS;
 
-    for (int i = tid; i < nr; i += kThreads) sidx[i] = idx[j0 + i];
+    // 1. the split's kept indices
+    for (int i = tid; i < nr; i += kThreads) sidx[i] = __ldg(idx + j0 + i);
     __syncthreads();
-    for (int e = tid; e < nr * TT; e += kThreads) {
-        const int i = e / TT, t = e - (e / TT) * TT;
-        xs[e] = (t < T) ? bf16_bits_to_float(X[(size_t)t * H + sidx[i]]) : 0.0f;
+
+    // 2. the first batch of weight pieces in flight, then the X values beside them
+    const int n = n0 + ct * 8;
+    const bool col_ok = n < N;  // N % 8 == 0: the whole 16-byte piece is in range
+    const uint16_t* wcol = g.Wt[p] + (col_ok ? n : 0);
+    uint4 w[U];
+    int i = rg;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+        w[u] = (col_ok && i + u * RG < nr) ? ld_nc_v4(wcol + (size_t)sidx[i + u * RG] * ld)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+    for (int e0 = tid; e0 < nr * TT; e0 += 4 * kThreads) {
+        uint16_t v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int e = e0 + q * kThreads;
+            const int r = e / TT, t = e - (e / TT) * TT;
+            v[q] = (e < nr * TT && t < T) ? X[(size_t)t * H + sidx[r]] : (uint16_t)0;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int e = e0 + q * kThreads;
+            if (e < nr * TT) xs[e] = bf16_bits_to_float(v[q]);
+        }
     }
     __syncthreads();
 
+    // 3. stream the kept rows
     float acc[TT][8];
 #pragma unroll
     for (int t = 0; t < TT; ++t)
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[t][c] = 0.0f;
-
-    if (n < N) {
-        const uint16_t* wcol = Wt + n;
-        int i = rg;
-        for (; i + (U - 1) * RG < nr; i += U * RG) {
-            uint4 w[U];
+    for (;;) {
 #pragma unroll
-            for (int u = 0; u < U; ++u) w[u] = ld_nc_v4(wcol + (size_t)sidx[i + u * RG] * N);
+        for (int u = 0; u < U; ++u)
+            if (i + u * RG < nr) fma_row<TT>(acc, w[u], xs + (i + u * RG) * TT);
+        i += U * RG;
+        if (i >= nr) break;
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                float wf[8];
-                unpack8(w[u], wf);
-                const float* xr = xs + (i + u * RG) * TT;
-#pragma unroll
-                for (int t = 0; t < TT; ++t) {
-                    const float xv = xr[t];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) acc[t][c] = fmaf(xv, wf[c], acc[t][c]);
-                }
-            }
-        }
-        for (; i < nr; i += RG) {
-            uint4 w = ld_nc_v4(wcol + (size_t)sidx[i] * N);
-            float wf[8];
-            unpack8(w, wf);
-            const float* xr = xs + i * TT;
-#pragma unroll
-            for (int t = 0; t < TT; ++t) {
-                const float xv = xr[t];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) acc[t][c] = fmaf(xv, wf[c], acc[t][c]);
-            }
-        }
+        for (int u = 0; u < U; ++u)
+            w[u] = (col_ok && i + u * RG < nr) ? ld_nc_v4(wcol + (size_t)sidx[i + u * RG] * ld)
+                                               : make_uint4(0u, 0u, 0u, 0u);
     }
 
-    // fold the row groups into row group 0 (fixed order: deterministic)
-    for (int r = 1; r < RG; ++r) {
-        if (rg == r) {
+    // 4. fold the row groups: shuffles inside a warp, then the warps in order
 #pragma unroll
-            for (int t = 0; t < TT; ++t)
+    for (int off = TPR; off < 32; off <<= 1)
 #pragma unroll
-                for (int c = 0; c < 8; ++c) red[t * COLS + ct * 8 + c] = acc[t][c];
-        }
-        __syncthreads();
-        if (rg == 0) {
+        for (int t = 0; t < TT; ++t)
 #pragma unroll
-            for (int t = 0; t < TT; ++t)
+            for (int c = 0; c < 8; ++c) acc[t][c] += __shfl_xor_sync(0xffffffffu, acc[t][c], off);
+    if (lane * 8 < WCOLS) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) acc[t][c] += red[t * COLS + ct * 8 + c];
-        }
-        __syncthreads();
+        for (int t = 0; t < TT; ++t)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) fold[(warp * TT + t) * WCOLS + lane * 8 + c] = acc[t][c];
     }
-
-    if (gridDim.y == 1) {
-        if (rg == 0 && n < N) {
+    __syncthreads();
+    constexpr int WPR = (TPR > 32) ? TPR / 32 : 1;  // warps per row group
+    for (int o = tid; o < TT * COLS; o += kThreads) {
+        const int t = o / COLS, col = o - (o / COLS) * COLS;
+        const int wsel = col / WCOLS;
+        float s = 0.0f;
 #pragma unroll
-            for (int t = 0; t < TT; ++t) {
-                if (t < T) {
-                    uint4 o;
-                    o.x = pack_bf16x2(acc[t][0], acc[t][1]);
-                    o.y = pack_bf16x2(acc[t][2], acc[t][3]);
-                    o.z = pack_bf16x2(acc[t][4], acc[t][5]);
-                    o.w = pack_bf16x2(acc[t][6], acc[t][7]);
-                    *reinterpret_cast<uint4*>(Y + (size_t)t * N + n) = o;
-                }
-            }
+        for (int w2 = 0; w2 < kWarps; ++w2)
+            if (w2 % WPR == wsel) s += fold[(w2 * TT + t) * WCOLS + (col - wsel * WCOLS)];
+        part[o] = s;
+    }
+    __syncthreads();
+
+    // 5. Y itself with one split, else this split's partial sums
+    if (g.splits[p] == 1) {
+        uint16_t* Y = g.Y[p];
+        for (int o8 = tid; o8 < TT * P8; o8 += kThreads) {
+            const int t = o8 / P8, c8 = o8 - (o8 / P8) * P8;
+            const int nn = n0 + c8 * 8;
+            if (t < T && nn < N) store_bf16x8(Y + (size_t)t * ld + nn, part + t * COLS + c8 * 8);
         }
         return;
     }
+    float* pbase = partials + g.partial_off[p];
+    for (int o8 = tid; o8 < TT * P8; o8 += kThreads) {
+        const int t = o8 / P8, c8 = o8 - (o8 / P8) * P8;
+        const int nn = n0 + c8 * 8;
+        if (t < T && nn < N) {
+            float4* dst = reinterpret_cast<float4*>(pbase + ((size_t)sp * T + t) * N + nn);
+            const float* s = part + t * COLS + c8 * 8;
+            __stcg(dst, make_float4(s[0], s[1], s[2], s[3]));
+            __stcg(dst + 1, make_float4(s[4], s[5], s[6], s[7]));
+        }
+    }
+}
 
-    if (rg == 0 && n < N) {
+// Y[t, n..n+8) = sum over splits s (in order) of the partials.  One CTA = 256
+// columns of one member and one token; its 8 thread groups take consecutive
+// ranges of the splits (four splits' loads in flight at a time) and the range
+// sums are added in range order.
+__global__ void __launch_bounds__(kThreads)
+    gemv_fold_kernel(const __grid_constant__ GemvGroup g, int T, const float* __restrict__ partials) {
+    __shared__ float4 gs[kFoldGroups][kFoldCols / 8][2];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int tid = threadIdx.x;
+    const int p = member_of(g.fold_start, g.count, blockIdx.x);
+    const int c = tid % (kFoldCols / 8);
+    const int n = (blockIdx.x - g.fold_start[p]) * kFoldCols + c * 8;
+    const int grp = tid / (kFoldCols / 8);
+    const int t = blockIdx.y;
+    const int N = g.N[p], S = g.splits[p];
+    const bool live = n < N;
+    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (live) {
+        const float* b = partials + g.partial_off[p] + (size_t)t * N + n;
+        const size_t stride = (size_t)T * N;
+        const int s_hi = (grp + 1) * S / kFoldGroups;
+        for (int s0 = grp * S / kFoldGroups; s0 < s_hi; s0 += 4) {
+            float4 v[4][2];
 #pragma unroll
-        for (int t = 0; t < TT; ++t) {
-            if (t < T) {
-                float4* dst = reinterpret_cast<float4*>(partials + ((size_t)split * T + t) * N + n);
-                dst[0] = make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
-                dst[1] = make_float4(acc[t][4], acc[t][5], acc[t][6], acc[t][7]);
+            for (int u = 0; u < 4; ++u) {
+                if (s0 + u < s_hi) {
+                    v[u][0] = __ldcg(reinterpret_cast<const float4*>(b + (s0 + u) * stride));
+                    v[u][1] = __ldcg(reinterpret_cast<const float4*>(b + (s0 + u) * stride + 4));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (s0 + u < s_hi) {
+                    s[0] += v[u][0].x; s[1] += v[u][0].y; s[2] += v[u][0].z; s[3] += v[u][0].w;
+                    s[4] += v[u][1].x; s[5] += v[u][1].y; s[6] += v[u][1].z; s[7] += v[u][1].w;
+                }
             }
         }
     }
-    __threadfence();
+    gs[grp][c][0] = make_float4(s[0], s[1], s[2], s[3]);
+    gs[grp][c][1] = make_float4(s[4], s[5], s[6], s[7]);
     __syncthreads();
-    if (tid == 0) {
-        const unsigned prev = atomicAdd(&counters[blockIdx.x], 1u);
-        is_last = (prev == gridDim.y - 1);
-    }
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    const int S = gridDim.y;
-    constexpr int Q4 = COLS / 4;
-    for (int e = tid; e < T * Q4; e += kThreads) {
-        const int t = e / Q4, c4 = e - (e / Q4) * Q4;
-        const int nn = blockIdx.x * COLS + c4 * 4;
-        if (nn >= N) continue;
-        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp = 0; sp < S; ++sp) {
-            const float4 v =
-                __ldcg(reinterpret_cast<const float4*>(partials + ((size_t)sp * T + t) * N + nn));
-            s.x += v.x;
-            s.y += v.y;
-            s.z += v.z;
-            s.w += v.w;
+    if (grp == 0 && live) {
+        float tot[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q = 0; q < kFoldGroups; ++q) {
+            const float4 a = gs[q][c][0], d = gs[q][c][1];
+            tot[0] += a.x; tot[1] += a.y; tot[2] += a.z; tot[3] += a.w;
+            tot[4] += d.x; tot[5] += d.y; tot[6] += d.z; tot[7] += d.w;
         }
-        uint2 o;
-        o.x = pack_bf16x2(s.x, s.y);
-        o.y = pack_bf16x2(s.z, s.w);
-        *reinterpret_cast<uint2*>(Y + (size_t)t * N + nn) = o;
+        store_bf16x8(g.Y[p] + (size_t)t * g.ld[p] + n, tot);
     }
-    if (tid == 0) counters[blockIdx.x] = 0;  // leave the counter ready for the next call
-}
-
-template <int TT, int TPR>
-cudaError_t launch_t(const uint16_t* X, int T, int H, const uint16_t* Wt, int N,
-                     const int32_t* idx, int k, uint16_t* Y, float* partials, unsigned* counters,
-                     const GemvPlan& p, cudaStream_t stream) {
-    const size_t smem = (size_t)p.rows_per_split * TT * sizeof(float) +
-                        (size_t)p.rows_per_split * sizeof(int) + (size_t)TT * TPR * 8 * sizeof(float);
-    auto kern = gemv_kernel<TT, TPR>;
-    if (smem > 48 * 1024) {
-        cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    dim3 grid(p.col_blocks, p.splits);
-    return launch_pdl(kern, grid, dim3(kThreads), smem, stream, X, T, H, Wt, N, idx, k, Y, partials,
-                      counters, p.rows_per_split);
 }
 
 template <int TT>
-cudaError_t launch_tt(const uint16_t* X, int T, int H, const uint16_t* Wt, int N,
-                      const int32_t* idx, int k, uint16_t* Y, float* partials, unsigned* counters,
-                      const GemvPlan& p, cudaStream_t stream) {
-    if (p.cols_per_cta == 512)
-        return launch_t<TT, 64>(X, T, H, Wt, N, idx, k, Y, partials, counters, p, stream);
-    return launch_t<TT, 32>(X, T, H, Wt, N, idx, k, Y, partials, counters, p, stream);
+cudaError_t launch_tt(const uint16_t* X, int T, int H, const int32_t* idx, int k, const GemvGroup& g,
+                      float* partials, cudaStream_t stream) {
+    constexpr int COLS = TT <= 4 ? 256 : TT <= 8 ? 128 : 64;  // gemv_cols_for
+    if (g.cols != COLS) return cudaErrorInvalidValue;
+    const size_t smem = gemv_smem_bytes(COLS, T);
+    auto kern = gemv_kernel<TT, COLS>;
+    cudaError_t e = ensure_smem_limit(kern, smem);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(kern, dim3(g.item_start[g.count], g.splits[0]), dim3(kThreads), smem, stream, X, T, H, idx, k, g,
+                   partials);
+    if (e != cudaSuccess || g.splits[0] == 1) return e;
+    return launch_pdl(gemv_fold_kernel, dim3(g.fold_start[g.count], T), dim3(kThreads), 0, stream, g, T,
+                      static_cast<const float*>(partials));
+}
+
+// Splits before rounding to whole rows; never decreases as k grows.
+int initial_splits(const GemvGroup& g, int T, int k, int forced_splits, int num_sms) {
+    const int cols = gemv_cols_for(T);
+    int blocks = 0;
+    for (int p = 0; p < g.count; ++p) blocks += (g.N[p] + cols - 1) / cols;
+    if (blocks < 1) blocks = 1;
+    // ~6 CTAs per SM for decode sizes (several short waves), fewer for wide T
+    // where the split partials cost more; at least 32 kept rows each
+    const int target = num_sms * (T <= 4 ? 6 : 2);
+    int S = forced_splits > 0 ? forced_splits : (target + blocks - 1) / blocks;
+    const int max_by_rows = (k + 31) / 32;
+    if (forced_splits <= 0 && S > max_by_rows) S = max_by_rows;
+    const int min_splits = (k + kMaxRowsPerItem - 1) / kMaxRowsPerItem;
+    if (S < min_splits) S = min_splits;
+    if (S > k) S = k;
+    if (S > 65535) S = 65535;
+    if (S < 1) S = 1;
+    return S;
 }
 
 }  // namespace
 
-GemvPlan gemv_plan(int T, int N, int k, int num_sms, int forced_splits) {
-    GemvPlan p;
-    p.cols_per_cta = (N >= 8192) ? 512 : 256;
-    p.col_blocks = (N + p.cols_per_cta - 1) / p.cols_per_cta;
-    const int target = num_sms * (T <= 4 ? 4 : 2);
-    int splits = forced_splits > 0 ? forced_splits : (target + p.col_blocks - 1) / p.col_blocks;
-    const int max_splits = forced_splits > 0 ? k : (k / 32 > 1 ? k / 32 : 1);
-    if (splits > max_splits) splits = max_splits;
-    if (splits > 1024) splits = 1024;
-    if (splits < 1) splits = 1;
-    p.rows_per_split = (k + splits - 1) / splits;
-    p.splits = (k + p.rows_per_split - 1) / p.rows_per_split;
-    return p;
-}
+int gemv_cols_for(int T) { return T <= 4 ? 256 : T <= 8 ? 128 : 64; }
 
-size_t gemv_smem_bytes(const GemvPlan& p, int T) {
+size_t gemv_smem_bytes(int cols, int T) {
     const int TT = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : T <= 8 ? 8 : 16;
-    return (size_t)p.rows_per_split * TT * sizeof(float) + (size_t)p.rows_per_split * sizeof(int) +
-           (size_t)TT * p.cols_per_cta * sizeof(float);
+    const int wcols = cols < 256 ? cols : 256;
+    return (size_t)kMaxRowsPerItem * TT * sizeof(float) + (size_t)kMaxRowsPerItem * sizeof(int) +
+           ((size_t)kWarps * TT * wcols + (size_t)TT * cols) * sizeof(float);
 }
 
-size_t gemv_partials_bytes(const GemvPlan& p, int T, int N) {
-    return p.splits > 1 ? (size_t)p.splits * T * N * sizeof(float) : 0;
+size_t gemv_partials_bound(const GemvGroup& g, int T, int H, int forced_splits, int num_sms) {
+    const int S = initial_splits(g, T, H, forced_splits, num_sms);
+    if (S <= 1) return 0;
+    size_t n = 0;
+    for (int p = 0; p < g.count; ++p) n += (size_t)g.N[p];
+    return (size_t)S * T * n * sizeof(float);
 }
 
-cudaError_t launch_gemv(const uint16_t* X, int T, int H, const uint16_t* Wt, int N,
-                        const int32_t* idx, int k, uint16_t* Y, float* partials,
-                        unsigned* counters, const GemvPlan& p, int* /*status*/,
-                        cudaStream_t stream) {
-    if (T <= 1) return launch_tt<1>(X, T, H, Wt, N, idx, k, Y, partials, counters, p, stream);
-    if (T <= 2) return launch_tt<2>(X, T, H, Wt, N, idx, k, Y, partials, counters, p, stream);
-    if (T <= 4) return launch_tt<4>(X, T, H, Wt, N, idx, k, Y, partials, counters, p, stream);
-    if (T <= 8) return launch_tt<8>(X, T, H, Wt, N, idx, k, Y, partials, counters, p, stream);
-    return launch_tt<16>(X, T, H, Wt, N, idx, k, Y, partials, counters, p, stream);
+size_t gemv_group_plan(GemvGroup& g, int T, int k, int forced_splits, int num_sms) {
+    g.cols = gemv_cols_for(T);
+    int S = initial_splits(g, T, k, forced_splits, num_sms);
+    const int rows = (k + S - 1) / S;
+    S = (k + rows - 1) / rows;
+    size_t part = 0;
+    g.item_start[0] = 0;
+    g.fold_start[0] = 0;
+    for (int p = 0; p < g.count; ++p) {
+        if (g.ld[p] == 0) g.ld[p] = g.N[p];
+        g.rows_per_split[p] = rows;
+        g.splits[p] = S;
+        g.col_blocks[p] = (g.N[p] + g.cols - 1) / g.cols;
+        g.item_start[p + 1] = g.item_start[p] + g.col_blocks[p];
+        g.fold_start[p + 1] = g.fold_start[p] + (g.N[p] + kFoldCols - 1) / kFoldCols;
+        g.partial_off[p] = part;
+        if (S > 1) part += (size_t)S * T * g.N[p];
+    }
+    for (int p = g.count + 1; p <= kMaxGroupGemv; ++p) {
+        g.item_start[p] = g.item_start[g.count];
+        g.fold_start[p] = g.fold_start[g.count];
+    }
+    return part * sizeof(float);
+}
+
+cudaError_t launch_gemv(const uint16_t* X, int T, int H, const int32_t* idx, int k, const GemvGroup& g,
+                        float* partials, int num_sms, cudaStream_t stream) {
+    (void)num_sms;
+    if (g.count < 1 || g.count > kMaxGroupGemv) return cudaErrorInvalidValue;
+    if (T <= 1) return launch_tt<1>(X, T, H, idx, k, g, partials, stream);
+    if (T <= 2) return launch_tt<2>(X, T, H, idx, k, g, partials, stream);
+    if (T <= 4) return launch_tt<4>(X, T, H, idx, k, g, partials, stream);
+    if (T <= 8) return launch_tt<8>(X, T, H, idx, k, g, partials, stream);
+    return launch_tt<16>(X, T, H, idx, k, g, partials, stream);
 }
 
 }  // namespace rmm

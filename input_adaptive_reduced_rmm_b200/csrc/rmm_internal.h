@@ -18,34 +18,51 @@ cudaError_t launch_score(const uint16_t* X, int T, int H, uint32_t* s32, uint16_
                          int num_sms, cudaStream_t stream);
 
 // ---- select (rmm_select.cu)
-// Reads the scores s32 (u32 [H]; zeroed afterwards when clear_input != 0),
-// optionally stores them to s_out, and writes the k best indices ascending to
-// idx[0..k), then idx[k..pad_to) = H; idx_copy (if not null) receives the
-// same k indices without padding.
-cudaError_t launch_select(uint32_t* s32, int clear_input, int H, int k, int32_t* idx, int pad_to,
-                          int32_t* idx_copy, uint32_t* s_out, cudaStream_t stream);
+// Scores: max_t |X[t,h]| folded from X [T, H] when X is not null (decode-sized
+// T: score and selection in one launch), else read from s32 (u32 [H]; zeroed
+// afterwards when clear_input != 0).  Optionally stores the scores to s_out,
+// and writes the k best indices ascending to idx[0..k), then
+// idx[k..pad_to) = H; idx_copy (if not null) receives the same k indices
+// without padding.
+cudaError_t launch_select(const uint16_t* X, int T, uint32_t* s32, int clear_input, int H, int k, int32_t* idx,
+                          int pad_to, int32_t* idx_copy, uint32_t* s_out, cudaStream_t stream);
 
 // ---- split-K GEMV (rmm_gemv.cu)
-struct GemvPlan {
-    int cols_per_cta;  // 256 or 512
-    int splits;
-    int rows_per_split;
-    int col_blocks;
+constexpr int kMaxGroupGemv = 4;
+// Up to 4 decode products sharing X and the kept list, planned by
+// gemv_group_plan (fill count, Wt, Y, N first).
+struct GemvGroup {
+    const uint16_t* Wt[kMaxGroupGemv];
+    uint16_t* Y[kMaxGroupGemv];
+    int N[kMaxGroupGemv];               // output columns of the member
+    int ld[kMaxGroupGemv];              // row stride (elements) of its W^T and Y; N when 0 at planning
+    int col_blocks[kMaxGroupGemv];
+    int splits[kMaxGroupGemv];          // the same for every member
+    int rows_per_split[kMaxGroupGemv];
+    int item_start[kMaxGroupGemv + 1];  // prefix sums of col_blocks (grid x of the product)
+    int fold_start[kMaxGroupGemv + 1];  // prefix sums of 256-column blocks (grid x of the fold)
+    size_t partial_off[kMaxGroupGemv];  // float offsets of each member's split partials
+    int cols;                           // outputs per column block
+    int count;
 };
-GemvPlan gemv_plan(int T, int N, int k, int num_sms, int forced_splits);
-size_t gemv_partials_bytes(const GemvPlan& p, int T, int N);
-size_t gemv_smem_bytes(const GemvPlan& p, int T);  // dynamic shared memory of one CTA
+int gemv_cols_for(int T);
+// Fills the plan; returns the bytes of split partial sums the group needs.
+size_t gemv_group_plan(GemvGroup& g, int T, int k, int forced_splits, int num_sms);
+// Upper bound of gemv_group_plan's partial bytes over every k <= H (needs g.N, g.count).
+size_t gemv_partials_bound(const GemvGroup& g, int T, int H, int forced_splits, int num_sms);
+size_t gemv_smem_bytes(int cols, int T);  // dynamic shared memory of one CTA
 constexpr size_t kGemvMaxSmemBytes = 200 * 1024;
-cudaError_t launch_gemv(const uint16_t* X, int T, int H, const uint16_t* Wt, int N,
-                        const int32_t* idx, int k, uint16_t* Y, float* partials,
-                        unsigned* counters, const GemvPlan& plan, int* status,
-                        cudaStream_t stream);
+// The product (and, with more than one split, the fold of the split partials
+// in a second launch).  partials: the planned bytes, no initial contents.
+cudaError_t launch_gemv(const uint16_t* X, int T, int H, const int32_t* idx, int k, const GemvGroup& g,
+                        float* partials, int num_sms, cudaStream_t stream);
 
 // ---- tcgen05 GEMM (rmm_gemm.cu)
 // Up to kMaxGroup products that share the activations (X^T, T, H and the kept
 // list) and differ in the weight: one persistent launch walks the tiles of
 // all of them.
 constexpr int kMaxGroup = 4;
+static_assert(kMaxGroup == kMaxGroupGemv, "one group size for both products");
 struct GemmGroup {
     const uint16_t* Wt[kMaxGroup];
     uint16_t* Y[kMaxGroup];

@@ -7,13 +7,15 @@
 // is being recorded into a CUDA graph, where a cudaMalloc would break the
 // capture.  rmm_linear_decode_noalloc serves them: the same score -> kept set ->
 // split-K GEMV path as rmm_linear for T <= 16, but every intermediate (partial
-// score vector, the kept list, the split partial sums, the split counters) lives in
+// score vector, the kept list, the split partial sums) lives in
 // one file-scope __device__ array of fixed size that every GPU loading the
 // library holds until the process exits.  Nothing is allocated or freed.
 //
 // Host code never uses the array's name as a device address: on first use on
 // a device (with that device current) the address is obtained once with
 // cudaGetSymbolAddress, checked, cached per device, and passed to the kernels.
+#include <string.h>
+
 #include <mutex>
 
 #include "rmm_common.cuh"
@@ -48,7 +50,7 @@ rmm_status noalloc_scratch(uint8_t** out) {
     return RMM_OK;
 }
 
-// Zero the words a call needs to start at zero (split counters, status word);
+// Zero the words a call needs to start at zero (status word, score vector);
 // the scratch keeps whatever the previous call left there.
 __global__ void noalloc_clear_kernel(unsigned* words, int n) {
     pdl_wait();
@@ -78,41 +80,61 @@ extern "C" rmm_status rmm_linear_decode_noalloc(const void* X, const void* Wt, i
     rmm_status st = noalloc_scratch(&scratch);
     if (st != RMM_OK) return st;
 
-    // scratch layout: status | score vector | kept list | split counters | split partials
-    GemvPlan plan = gemv_plan(T, N, k, sms, 0);
+    // scratch layout: status | score vector | kept list | split partials
     const size_t off_s32 = kNoAllocStatusBytes;
     const size_t off_idx = off_s32 + up256((size_t)H * sizeof(uint32_t));
-    const size_t off_cnt = off_idx + up256(((size_t)H + 2 * kGemmBK) * sizeof(int32_t));
-    const size_t off_partials = off_cnt + up256((size_t)plan.col_blocks * sizeof(unsigned));
-    if (off_partials > kNoAllocScratchBytes) return RMM_ERR_UNSUPPORTED;
+    const size_t off_partials = off_idx + up256(((size_t)H + 2 * kGemmBK) * sizeof(int32_t));
+    if (off_partials >= kNoAllocScratchBytes) return RMM_ERR_UNSUPPORTED;
     const size_t room = kNoAllocScratchBytes - off_partials;
-    if (gemv_partials_bytes(plan, T, N) > room) {
-        // fewer splits so that the partial sums fit; one split needs none
-        const size_t per_split = (size_t)T * N * sizeof(float);
-        int splits = (int)(room / per_split);
-        if (splits < 2) splits = 1;
-        plan = gemv_plan(T, N, k, sms, splits);
-        if (gemv_partials_bytes(plan, T, N) > room) return RMM_ERR_UNSUPPORTED;
+    if (gemv_smem_bytes(gemv_cols_for(T), T) > kGemvMaxSmemBytes) return RMM_ERR_UNSUPPORTED;
+
+    // Plan for the output columns [c0, c0 + w): the default splits when their
+    // partial sums fit, else fewer; false when even the fewest do not fit.
+    auto plan_for = [&](GemvGroup& g, int c0, int w) {
+        memset(&g, 0, sizeof g);
+        g.count = 1;
+        g.Wt[0] = static_cast<const uint16_t*>(Wt) + c0;
+        g.Y[0] = static_cast<uint16_t*>(Y) + c0;
+        g.N[0] = w;
+        g.ld[0] = N;
+        size_t part = gemv_group_plan(g, T, k, 0, sms);
+        if (part > room) {
+            const int splits = (int)(room / ((size_t)T * w * sizeof(float)));
+            g.ld[0] = N;
+            part = gemv_group_plan(g, T, k, splits < 2 ? 1 : splits, sms);
+        }
+        return part <= room;
+    };
+    // columns per launch: all N when the partial sums fit, else halves of it
+    // (multiples of 8 columns, so every launch keeps 16-byte alignment)
+    GemvGroup g;
+    int chunk = N;
+    while (!plan_for(g, 0, chunk)) {
+        if (chunk <= 64) return RMM_ERR_UNSUPPORTED;
+        chunk = (chunk / 2 + 7) / 8 * 8;
     }
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (gemv_smem_bytes(plan, T) > kGemvMaxSmemBytes) return RMM_ERR_UNSUPPORTED;
-    // status word and score vector: the score pass folds maxima into zeros
+    // status word and score vector: they must start at zero
     noalloc_clear_kernel<<<(int)((off_idx / 4 + 255) / 256), 256, 0, s>>>(reinterpret_cast<unsigned*>(scratch),
                                                                          (int)(off_idx / 4));
-    noalloc_clear_kernel<<<(plan.col_blocks + 255) / 256, 256, 0, s>>>(
-        reinterpret_cast<unsigned*>(scratch + off_cnt), plan.col_blocks);
     if (cudaGetLastError() != cudaSuccess) return RMM_ERR_CUDA;
 
     uint32_t* s32 = reinterpret_cast<uint32_t*>(scratch + off_s32);
     int32_t* idx = reinterpret_cast<int32_t*>(scratch + off_idx);
-    if (launch_score(static_cast<const uint16_t*>(X), T, H, s32, nullptr, 0, sms, s) != cudaSuccess)
-        return RMM_ERR_CUDA;
-    if (launch_select(s32, 1, H, k, idx, k, idx_out, nullptr, s) != cudaSuccess) return RMM_ERR_CUDA;
-    if (launch_gemv(static_cast<const uint16_t*>(X), T, H, static_cast<const uint16_t*>(Wt), N, idx, k,
-                    static_cast<uint16_t*>(Y), reinterpret_cast<float*>(scratch + off_partials),
-                    reinterpret_cast<unsigned*>(scratch + off_cnt), plan,
-                    reinterpret_cast<int*>(scratch), s) != cudaSuccess)
-        return RMM_ERR_CUDA;
+    // the score vector was just cleared; the select clears it again after reading
+    cudaError_t e = (T == 1) ? launch_select(static_cast<const uint16_t*>(X), T, nullptr, 0, H, k, idx, k, idx_out,
+                                             nullptr, s)
+                             : launch_score(static_cast<const uint16_t*>(X), T, H, s32, nullptr, 0, sms, s);
+    if (e == cudaSuccess && T > 1) e = launch_select(nullptr, 0, s32, 1, H, k, idx, k, idx_out, nullptr, s);
+    if (e != cudaSuccess) return RMM_ERR_CUDA;
+    // one product per column chunk, one after another through the same partials
+    for (int c0 = 0; c0 < N; c0 += chunk) {
+        const int w = (N - c0 < chunk) ? N - c0 : chunk;
+        if (!plan_for(g, c0, w)) return RMM_ERR_UNSUPPORTED;
+        if (launch_gemv(static_cast<const uint16_t*>(X), T, H, idx, k, g,
+                        reinterpret_cast<float*>(scratch + off_partials), sms, s) != cudaSuccess)
+            return RMM_ERR_CUDA;
+    }
     return RMM_OK;
 }

@@ -6,17 +6,26 @@
 // top-k; §6.1 demo: top-k followed by a sort so the kept slices keep their
 // original order).
 //
-// One CTA of 1024 threads, scores resident in shared memory:
-//   1. read the score vector into shared memory (and clear it for the next
-//      call when it is the library's own accumulator);
-//   2. radix select on the key: a 256-bin histogram of s>>8 finds the bin of
-//      the k-th largest score, a 256-bin histogram of s&255 inside that bin
-//      finds the threshold score s*; c_gt = #{s > s*}, need = k - c_gt;
-//   3. ordered compaction: every thread owns a contiguous run of indices, one
-//      block-wide scan of packed (#gt, #eq) counts gives each run its output
-//      offset, and index h is kept iff s_h > s*, or s_h == s* and fewer than
-//      `need` equal scores precede it -- which yields the ascending list
-//      directly, with ties resolved toward the lower index.
+// One CTA of 1024 threads; keys are 16-bit (bf16 magnitude bits):
+//   1. every thread loads its strided share of the keys into registers, all
+//      loads in flight at once (from X for one token, else from the score
+//      vector, which is cleared behind the read when it is the library's own
+//      accumulator), while the CTA clears a 128 KB shared histogram;
+//   2. one shared-memory atomic per key counts it in a histogram over all
+//      2^16 key values (two 16-bit counts per word).  Exact bins: a warp's
+//      keys rarely share a value, so the atomics hardly ever serialise, even
+//      though an activation's magnitudes crowd into a few exponents;
+//   3. the threshold s* = the k-th largest key: per-warp sums of 32 ranges of
+//      2048 keys, then one warp descends from the top through the range, a
+//      32-word chunk of it and a word of that chunk; c_gt = #{s > s*} comes
+//      out of the descent and need = k - c_gt;
+//   4. ordered compaction straight from the registers: ballots count each
+//      warp's greater and equal keys per row of 1024 slices, one block-wide
+//      scan of the packed (#gt, #eq) counts gives every warp-row its output
+//      offset, and the ballots rank each key inside it.  Index h is kept iff
+//      s_h > s*, or s_h == s* and fewer than `need` equal scores precede it --
+//      which yields the ascending list directly, with ties resolved toward the
+//      lower index.
 #include "rmm_common.cuh"
 #include "rmm_internal.h"
 
@@ -26,6 +35,9 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
+constexpr int kHistWords = 32768;  // 2^16 keys, two 16-bit counts per word
+constexpr size_t kSmemBytes = kHistWords * sizeof(uint32_t);  // then the compaction's counts
+static_assert(kWarps == 32, "the descent takes one range per warp");
 
 // Inclusive block-wide sum of one value per thread (all threads participate).
 __device__ __forceinline__ uint32_t block_inclusive_scan(uint32_t v, uint32_t* warp_tot) {
@@ -52,157 +64,259 @@ __device__ __forceinline__ uint32_t block_inclusive_scan(uint32_t v, uint32_t* w
     return base + v;
 }
 
-// Within one warp: given counts cnt[b] of nbins bins, find the bin holding the
-// k-th largest element counting from the top bin down.  Returns the bin and
-// the number of elements in higher bins (via *above).
-__device__ __forceinline__ int warp_find_bin(const int* cnt, int nbins, int k, int* above) {
+__device__ __forceinline__ uint32_t warp_inclusive_scan(uint32_t v) {
     const int lane = threadIdx.x & 31;
-    const int per = nbins / 32;  // bins per lane, lane 0 owns the highest bins
-    int hi = nbins - 1 - lane * per;
-    int sum = 0;
-    for (int i = 0; i < per; ++i) sum += cnt[hi - i];
-    int incl = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
+        uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
     }
-    int run = incl - sum;  // elements in bins above this lane's run
-    int found = -1, found_above = 0;
-    if (run < k && run + sum >= k) {
-        for (int i = 0; i < per; ++i) {
-            int b = hi - i;
-            if (run + cnt[b] >= k) {
-                found = b;
-                found_above = run;
-                break;
+    return v;
+}
+
+// Keys this thread holds: key e is slice tid + e * kThreads.  E <= 16 keys are
+// held one per register, more two per register (even e low half, odd e high).
+template <int E>
+struct Keys {
+    static constexpr bool kPacked = E > 16;
+    static constexpr int R = kPacked ? E / 2 : E;
+    uint32_t v[R];
+
+    __device__ __forceinline__ uint32_t get(int e) const {
+        if (kPacked) return (e & 1) ? (v[e / 2] >> 16) : (v[e / 2] & 0xFFFFu);
+        return v[e];
+    }
+
+    // Read the keys -- the fold of X's T rows, or the score vector (cleared
+    // behind the read when asked) -- into registers; up to 16 loads are in
+    // flight per thread.  Slices past H get key 0 and are never counted.
+    // `meanwhile` runs once, after the first loads are issued and before any
+    // is used.
+    template <class F>
+    __device__ __forceinline__ void load(const uint16_t* __restrict__ X, int T, uint32_t* __restrict__ s32,
+                                         int clear_input, int H, uint32_t* __restrict__ s_out, F&& meanwhile) {
+        const int tid = threadIdx.x;
+        constexpr int B = E < 16 ? E : 16;
+#pragma unroll
+        for (int b0 = 0; b0 < E; b0 += B) {
+            uint32_t raw[B];
+#pragma unroll
+            for (int u = 0; u < B; ++u) {
+                const int h = tid + (b0 + u) * kThreads;
+                raw[u] = 0;
+                if (h < H) raw[u] = X ? (uint32_t)X[h] : s32[h];
             }
-            run += cnt[b];
+            if (b0 == 0) meanwhile();
+#pragma unroll
+            for (int u = 0; u < B; ++u) raw[u] &= X ? 0x7FFFu : 0xFFFFu;
+            if (X) {
+                for (int t = 1; t < T; ++t) {
+#pragma unroll
+                    for (int u = 0; u < B; ++u) {
+                        const int h = tid + (b0 + u) * kThreads;
+                        if (h < H) raw[u] = max(raw[u], (uint32_t)(X[(size_t)t * H + h] & 0x7FFFu));
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < B; ++u) {
+                const int e = b0 + u;
+                const int h = tid + e * kThreads;
+                if (h < H) {
+                    if (!X && clear_input) s32[h] = 0;
+                    if (s_out) s_out[h] = raw[u];
+                }
+                if (kPacked) {
+                    if (e & 1) v[e / 2] |= raw[u] << 16;
+                    else v[e / 2] = raw[u];
+                } else {
+                    v[e] = raw[u];
+                }
+            }
         }
     }
-    unsigned m = __ballot_sync(0xffffffffu, found >= 0);
-    int src = __ffs(m) - 1;
-    *above = __shfl_sync(0xffffffffu, found_above, src);
-    return __shfl_sync(0xffffffffu, found, src);
-}
+};
 
-// Histogram of 8-bit bins over the keys: bin = (key >> shift) & 255 for keys
-// with key >> 8 == match (all keys when match == ~0).  Lanes holding the same
-// bin are merged with __match_any_sync so each distinct bin costs one shared
-// atomic per warp and chunk.
-__device__ __forceinline__ void warp_histogram(const uint16_t* s, int H, int shift, uint32_t match,
-                                               int* hist) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int h0 = warp * 32; h0 < H; h0 += kThreads) {
-        const int h = h0 + lane;
-        uint32_t bin = 0xFFFFFFFFu;  // "no bin"
-        if (h < H) {
-            const uint32_t v = s[h];
-            if (match == 0xFFFFFFFFu || (v >> 8) == match) bin = (v >> shift) & 0xFFu;
-        }
-        const unsigned same = __match_any_sync(0xffffffffu, bin);
-        if (bin != 0xFFFFFFFFu && lane == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
+// Warp 0: the k-th largest key from the histogram.  hist word w counts key 2w
+// in its low half and key 2w+1 in its high half; range_tot[r] counts the keys
+// of words [1024 r, 1024 r + 1024).  Lane l looks at the (31 - l)-th piece, so
+// that lane order runs from the largest keys down; at each level the first
+// lane whose running count reaches k names the piece holding s*, and `above`
+// accumulates the keys in the pieces above it.
+__device__ __forceinline__ void descend(const uint32_t* hist, const uint32_t* range_tot, uint32_t k,
+                                        uint32_t* thr_out, uint32_t* above_out) {
+    const int lane = threadIdx.x & 31;
+    // ranges of 1024 words
+    uint32_t c = range_tot[31 - lane];
+    uint32_t incl = warp_inclusive_scan(c);
+    int L = __ffs(__ballot_sync(0xffffffffu, incl >= k)) - 1;
+    uint32_t above = __shfl_sync(0xffffffffu, incl - c, L);
+    const int r = 31 - L;
+    // chunks of 32 words inside the range (read rotated: 4-way bank conflicts at most)
+    const uint4* chunk = reinterpret_cast<const uint4*>(hist + r * 1024 + (31 - lane) * 32);
+    uint32_t w = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint4 x = chunk[(j + lane) & 7];
+        w += x.x + x.y + x.z + x.w;
     }
+    c = (w & 0xFFFFu) + (w >> 16);
+    incl = warp_inclusive_scan(c);
+    L = __ffs(__ballot_sync(0xffffffffu, above + incl >= k)) - 1;
+    above += __shfl_sync(0xffffffffu, incl - c, L);
+    const int cw = r * 1024 + (31 - L) * 32;
+    // words of the chunk
+    const uint32_t wv = hist[cw + 31 - lane];
+    c = (wv & 0xFFFFu) + (wv >> 16);
+    incl = warp_inclusive_scan(c);
+    L = __ffs(__ballot_sync(0xffffffffu, above + incl >= k)) - 1;
+    above += __shfl_sync(0xffffffffu, incl - c, L);
+    const uint32_t wsel = __shfl_sync(0xffffffffu, wv, L);
+    const uint32_t b = (uint32_t)(cw + 31 - L);
+    const uint32_t n_odd = wsel >> 16;  // count of key 2b+1, the larger of the word's two
+    if (above + n_odd >= k) {
+        *thr_out = 2 * b + 1;
+    } else {
+        above += n_odd;
+        *thr_out = 2 * b;
+    }
+    *above_out = above;
 }
 
-__global__ void __launch_bounds__(kThreads)
-    select_kernel(uint32_t* __restrict__ s32, int clear_input, int H, int k, int32_t* __restrict__ idx,
-                  int pad_to, int32_t* __restrict__ idx_copy, uint32_t* __restrict__ s_out) {
-    extern __shared__ uint16_t s[];  // H keys
-    __shared__ int hist_hi[256];
-    __shared__ int hist_fine[256];
+template <int E>  // keys per thread: H <= E * kThreads
+__global__ void __launch_bounds__(kThreads, 1)
+    select_kernel(const uint16_t* __restrict__ X, int T, uint32_t* __restrict__ s32, int clear_input, int H,
+                  int k, int32_t* __restrict__ idx, int pad_to, int32_t* __restrict__ idx_copy,
+                  uint32_t* __restrict__ s_out) {
+    extern __shared__ __align__(16) uint32_t hist[];  // kHistWords; later the H keys
+    __shared__ uint32_t range_tot[32];
     __shared__ uint32_t warp_tot[32];
-    __shared__ int sh_thresh, sh_need;
+    __shared__ uint32_t sh_thr, sh_need;
 
     pdl_wait();
     pdl_launch_dependents();
-    const int tid = threadIdx.x;
-    if (tid < 256) hist_hi[tid] = 0;
-    if (tid < 256) hist_fine[tid] = 0;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // 1. load the scores
-    for (int h = tid; h < H; h += kThreads) {
-        const uint32_t m = s32[h] & 0xFFFFu;
-        if (clear_input) s32[h] = 0;
-        s[h] = (uint16_t)m;
-        if (s_out) s_out[h] = m;
-    }
+    // 1. the keys into registers; the histogram is cleared while they arrive
+    Keys<E> keys;
+    keys.load(X, T, s32, clear_input, H, s_out, [&] {
+        uint4* h4 = reinterpret_cast<uint4*>(hist);
+#pragma unroll
+        for (int i = 0; i < kHistWords / 4 / kThreads; ++i) h4[tid + i * kThreads] = make_uint4(0u, 0u, 0u, 0u);
+    });
     __syncthreads();
 
-    // 2a. coarse histogram of s >> 8 (256 bins; keys are < 2^16, and < 2^15
-    //     for finite bf16 magnitudes).  Scores of one input crowd into a few
-    //     exponent bins, so equal bins are merged per warp first.
-    warp_histogram(s, H, 8, 0xFFFFFFFFu, hist_hi);
-    __syncthreads();
-    if (tid < 32) {
-        int above;
-        int b = warp_find_bin(hist_hi, 256, k, &above);
-        if (tid == 0) {
-            sh_thresh = b;
-            sh_need = k - above;  // elements still to take from bin b downward
+    // 2. exact histogram
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int h = tid + e * kThreads;
+        if (h < H) {
+            const uint32_t key = keys.get(e);
+            atomicAdd(&hist[key >> 1], (key & 1u) ? 0x10000u : 1u);
         }
     }
     __syncthreads();
-    const int bhi = sh_thresh;
-    const int k2 = sh_need;
-    // 2b. fine histogram of the low 8 bits inside the coarse bin
-    warp_histogram(s, H, 0, (uint32_t)bhi, hist_fine);
+
+    // 3. per-range totals (warp w: words [1024 w, 1024 w + 1024)), then the descent
+    {
+        const uint4* q = reinterpret_cast<const uint4*>(hist + warp * 1024);
+        uint32_t w = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint4 x = q[lane + 32 * j];
+            w += x.x + x.y + x.z + x.w;
+        }
+        const uint32_t c = __reduce_add_sync(0xffffffffu, (w & 0xFFFFu) + (w >> 16));
+        if (lane == 0) range_tot[warp] = c;
+    }
     __syncthreads();
-    if (tid < 32) {
-        int above;
-        int b = warp_find_bin(hist_fine, 256, k2, &above);
-        if (tid == 0) {
-            sh_thresh = (bhi << 8) | b;
-            sh_need = k2 - above;  // equal-to-threshold elements to keep
+    if (warp == 0) {
+        uint32_t thr, above;
+        descend(hist, range_tot, (uint32_t)k, &thr, &above);
+        if (lane == 0) {
+            sh_thr = thr;
+            sh_need = (uint32_t)k - above;
         }
     }
     __syncthreads();
-    const uint32_t thr = (uint32_t)sh_thresh;
-    const uint32_t need = (uint32_t)sh_need;
+    const uint32_t thr = sh_thr;
+    const uint32_t need = sh_need;
 
-    // 3. ordered compaction over contiguous runs
-    const int per = (H + kThreads - 1) / kThreads;
-    const int lo = min(H, tid * per), hi = min(H, lo + per);
-    uint32_t gt = 0, eq = 0;
-    for (int h = lo; h < hi; ++h) {
-        uint32_t v = s[h];
-        gt += (v > thr);
-        eq += (v == thr);
+    // 4. ordered compaction.  Slice h = tid + 1024 e, so index order is
+    //    (e, warp, lane).  Each warp counts its greater and equal keys of every
+    //    row e with two ballots and stores them packed (#gt << 16 | #eq, both
+    //    totals < 2^16) at cnt[e * 32 + warp]; one block-wide scan turns the
+    //    counts into exclusive prefixes in index order; the ballots again rank
+    //    each key inside its warp.
+    uint32_t* cnt = hist;  // E * 32 words, over the histogram
+    const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int h = tid + e * kThreads;
+        const uint32_t v = keys.get(e);
+        const uint32_t bg = __ballot_sync(0xffffffffu, h < H && v > thr);
+        const uint32_t be = __ballot_sync(0xffffffffu, h < H && v == thr);
+        if (lane == 0) cnt[e * 32 + warp] = ((uint32_t)__popc(bg) << 16) | (uint32_t)__popc(be);
     }
-    // pack (gt, eq) in one word: both totals are <= H <= 65535
-    uint32_t incl = block_inclusive_scan((gt << 16) | eq, warp_tot);
-    uint32_t excl = incl - ((gt << 16) | eq);
-    uint32_t gt_before = excl >> 16, eq_before = excl & 0xFFFFu;
-    for (int h = lo; h < hi; ++h) {
-        uint32_t v = s[h];
-        if (v > thr) {
-            const uint32_t pos = gt_before + min(eq_before, need);
+    __syncthreads();
+    {
+        constexpr int P = (E * 32 + kThreads - 1) / kThreads;  // entries per thread
+        uint32_t x[P], sum = 0;
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+            const int i = tid * P + p;
+            x[p] = (i < E * 32) ? cnt[i] : 0u;
+            sum += x[p];
+        }
+        uint32_t run = block_inclusive_scan(sum, warp_tot) - sum;
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+            const int i = tid * P + p;
+            if (i < E * 32) cnt[i] = run;
+            run += x[p];
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int h = tid + e * kThreads;
+        const uint32_t v = keys.get(e);
+        const bool is_gt = h < H && v > thr;
+        const bool is_eq = h < H && v == thr;
+        const uint32_t bg = __ballot_sync(0xffffffffu, is_gt);
+        const uint32_t be = __ballot_sync(0xffffffffu, is_eq);
+        const uint32_t base = cnt[e * 32 + warp];
+        const uint32_t g_rank = (base >> 16) + __popc(bg & lt_mask);
+        const uint32_t e_rank = (base & 0xFFFFu) + __popc(be & lt_mask);
+        if (is_gt || (is_eq && e_rank < need)) {
+            const uint32_t pos = g_rank + min(e_rank, need);
             idx[pos] = h;
             if (idx_copy) idx_copy[pos] = h;
-            ++gt_before;
-        } else if (v == thr) {
-            if (eq_before < need) {
-                idx[gt_before + eq_before] = h;
-                if (idx_copy) idx_copy[gt_before + eq_before] = h;
-            }
-            ++eq_before;
         }
     }
     for (int j = k + tid; j < pad_to; j += kThreads) idx[j] = H;
 }
 
+template <int E>
+cudaError_t launch_e(const uint16_t* X, int T, uint32_t* s32, int clear_input, int H, int k, int32_t* idx,
+                     int pad_to, int32_t* idx_copy, uint32_t* s_out, cudaStream_t stream) {
+    cudaError_t e = ensure_smem_limit(select_kernel<E>, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(select_kernel<E>, dim3(1), dim3(kThreads), kSmemBytes, stream, X, T, s32, clear_input, H, k,
+                      idx, pad_to, idx_copy, s_out);
+}
+
 }  // namespace
 
-cudaError_t launch_select(uint32_t* s32, int clear_input, int H, int k, int32_t* idx, int pad_to,
-                          int32_t* idx_copy, uint32_t* s_out, cudaStream_t stream) {
-    const size_t smem = ((size_t)H * sizeof(uint16_t) + 15) & ~(size_t)15;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(select_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    return launch_pdl(select_kernel, dim3(1), dim3(kThreads), smem, stream, s32, clear_input, H, k, idx,
-                      pad_to, idx_copy, s_out);
+cudaError_t launch_select(const uint16_t* X, int T, uint32_t* s32, int clear_input, int H, int k, int32_t* idx,
+                          int pad_to, int32_t* idx_copy, uint32_t* s_out, cudaStream_t stream) {
+    if (H < 1 || H > 65535 || k < 1 || k > H) return cudaErrorInvalidValue;
+    // the fewest keys per thread that cover H
+    if (H <= 4 * kThreads) return launch_e<4>(X, T, s32, clear_input, H, k, idx, pad_to, idx_copy, s_out, stream);
+    if (H <= 8 * kThreads) return launch_e<8>(X, T, s32, clear_input, H, k, idx, pad_to, idx_copy, s_out, stream);
+    if (H <= 16 * kThreads) return launch_e<16>(X, T, s32, clear_input, H, k, idx, pad_to, idx_copy, s_out, stream);
+    if (H <= 32 * kThreads) return launch_e<32>(X, T, s32, clear_input, H, k, idx, pad_to, idx_copy, s_out, stream);
+    return launch_e<64>(X, T, s32, clear_input, H, k, idx, pad_to, idx_copy, s_out, stream);
 }
 
 }  // namespace rmm
