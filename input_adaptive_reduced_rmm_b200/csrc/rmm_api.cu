@@ -99,6 +99,8 @@ LinearLayout linear_layout(int T, int H, const int* Ns, int count, int k, const 
         L.ldT = (T + 7) / 8 * 8;
         L.xt = off;
         off += align_up((size_t)H * L.ldT * sizeof(uint16_t), kAlign);
+        L.partials = off;  // fp32 partials of the split last wave (CTA-pair GEMM)
+        off += align_up(gemm_pair_partial_bytes(sms), kAlign);
     }
     L.total = off;
     return L;
@@ -216,7 +218,8 @@ rmm_status run_product_kernels(const void* X, int T, int H, int count, const voi
     if (o.gemm_producer == 0) {  // default: CTA-pair tcgen05 GEMM
         gemm_group_tiles(g, T, 1);
         return cuda_status(launch_gemm_pair(reinterpret_cast<const uint16_t*>(ws + L.xt), L.ldT, g, idx_padded,
-                                            k, T, H, status, o.debug_timeout_test, sms, s));
+                                            k, T, H, reinterpret_cast<float*>(ws + L.partials), status,
+                                            o.debug_timeout_test, sms, s));
     }
     gemm_group_tiles(g, T, 0);
     CUtensorMap mx, mw;

@@ -420,8 +420,16 @@ struct __align__(8) Barriers2 {
     int abort_flag;
 };
 
+constexpr int EPI_STAGE_BYTES = 32 * 128;  // one epilogue warp's 32 rows x 64 bf16 columns
+// Eight epilogue warps: warps w and w + 4 share TMEM lane quarter w % 4 and
+// drain the lower and upper 256 accumulator columns, halving the time the
+// MMA waits for the (single, TMEM-filling) accumulator between tiles.
+constexpr int kEpiWarps2 = 8;
+constexpr int kMmaWarp2 = kProducerWarps + kEpiWarps2;
+constexpr int kThreads2 = 32 * (kMmaWarp2 + 1);
 constexpr size_t kSmemBytes2 =
-    1024 + (size_t)STAGES2 * (A2_STAGE_BYTES + B2_STAGE_BYTES) + sizeof(Barriers2);
+    1024 + (size_t)STAGES2 * (A2_STAGE_BYTES + B2_STAGE_BYTES) + (size_t)kEpiWarps2 * EPI_STAGE_BYTES +
+    sizeof(Barriers2);
 
 __device__ __forceinline__ TileCoord decode_tile2(const GemmGroup& g, int t, int m_tiles) {
     int p = 0;
@@ -436,7 +444,32 @@ __device__ __forceinline__ TileCoord decode_tile2(const GemmGroup& g, int t, int
     return c;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// Work unit u: a whole tile (u < units_full), or one K-range of a tile of the
+// split last wave; part = the unit's slot in the fp32 partials, -1 if whole.
+struct Unit {
+    TileCoord tc;
+    int kb0, kb1, part;
+};
+
+__device__ __forceinline__ Unit decode_unit(const GemmGroup& g, int u, int m_tiles, int nkb) {
+    Unit r;
+    if (u < g.units_full) {
+        r.tc = decode_tile2(g, u, m_tiles);
+        r.kb0 = 0;
+        r.kb1 = nkb;
+        r.part = -1;
+    } else {
+        const int v = u - g.units_full;
+        const int sp = v % g.tail_splits;
+        r.tc = decode_tile2(g, g.units_full + v / g.tail_splits, m_tiles);
+        r.kb0 = sp * nkb / g.tail_splits;
+        r.kb1 = (sp + 1) * nkb / g.tail_splits;
+        r.part = v;
+    }
+    return r;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     gemm_pair_kernel(const uint16_t* __restrict__ Xt, int ldT, const __grid_constant__ GemmGroup group,
                      const int32_t* __restrict__ idx, int k, int T, int H, int* status, int debug_timeout) {
     extern __shared__ uint8_t smem_raw[];
@@ -444,7 +477,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                                ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES2 * A2_STAGE_BYTES;
-    Barriers2* bars = reinterpret_cast<Barriers2*>(sB + STAGES2 * B2_STAGE_BYTES);
+    uint8_t* sE = sB + STAGES2 * B2_STAGE_BYTES;  // epilogue staging, one block per epilogue warp
+    Barriers2* bars = reinterpret_cast<Barriers2*>(sE + kEpiWarps2 * EPI_STAGE_BYTES);
     volatile int* abort_flag = &bars->abort_flag;
 
     const int warp = threadIdx.x >> 5;
@@ -452,7 +486,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t rank = cluster_ctarank();  // 0 = leader
     const uint32_t peer = rank ^ 1u;
     const int m_tiles = (T + BM2 - 1) / BM2;
-    const int num_tiles = group.tile_start[group.count];
+    const int num_units = group.units;
     const int nkb = (k + BK - 1) / BK;
     const int cluster_id = blockIdx.x >> 1;
     const int num_clusters = gridDim.x >> 1;
@@ -465,12 +499,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(smem_addr(&bars->empty[s]), 1);
         }
         mbar_init(smem_addr(&bars->tfull), 1);
-        mbar_init(smem_addr(&bars->tempty), 2 * kEpilogueWarps);
+        mbar_init(smem_addr(&bars->tempty), 2 * kEpiWarps2);
         mbar_init(smem_addr(&bars->never), 1);
         bars->abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == kMmaWarp) {
+    if (warp == kMmaWarp2) {
         tmem_alloc_pair(smem_addr(&bars->tmem_base), TMEM_COLS2);
         tmem_relinquish_pair();
     }
@@ -486,25 +520,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        int q0a = __ldg(idx + lane), q1a = __ldg(idx + 32 + lane);
-        int next_kb = (1 < nkb) ? 1 : 0;
-        int q0b = __ldg(idx + next_kb * BK + lane), q1b = __ldg(idx + next_kb * BK + 32 + lane);
-        next_kb = (next_kb + 1 < nkb) ? next_kb + 1 : 0;
+        // kept indices of the (unit, K-block) sequence this pair walks, two
+        // K-blocks ahead of use; past the last unit any in-range block will do
+        int pu = cluster_id, pkb = 0, pkb1 = 1 << 30;
+        if (pu < num_units) {
+            const Unit x = decode_unit(group, pu, m_tiles, nkb);
+            pkb = x.kb0;
+            pkb1 = x.kb1;
+        }
+        auto advance = [&]() {
+            if (++pkb >= pkb1) {
+                pu += num_clusters;
+                pkb = 0;
+                pkb1 = 1 << 30;
+                if (pu < num_units) {
+                    const Unit x = decode_unit(group, pu, m_tiles, nkb);
+                    pkb = x.kb0;
+                    pkb1 = x.kb1;
+                }
+            }
+        };
+        auto kq = [&]() { return pu < num_units ? pkb : 0; };
+        int q0a = __ldg(idx + kq() * BK + lane), q1a = __ldg(idx + kq() * BK + 32 + lane);
+        advance();
+        int q0b = __ldg(idx + kq() * BK + lane), q1b = __ldg(idx + kq() * BK + 32 + lane);
         uint32_t b_off[kRowsB], a_off[kRowsA];
 #pragma unroll
         for (int i = 0; i < kRowsB; ++i) b_off[i] = swz_offset(warp + kProducerWarps * i, lane);
 #pragma unroll
         for (int i = 0; i < kRowsA; ++i)
             a_off[i] = swz_offset(2 * (warp + kProducerWarps * i) + (lane >> 4), lane & 15);
-        for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
-            const TileCoord tc = decode_tile2(group, tile, m_tiles);
+        for (int u = cluster_id; ok && u < num_units; u += num_clusters) {
+            const Unit ux = decode_unit(group, u, m_tiles, nkb);
+            const TileCoord tc = ux.tc;
             const int N = group.N[tc.p];
             const uint16_t* __restrict__ Wt = group.Wt[tc.p];
             const int a_col = tc.m0 + HALF_M * (int)rank + (lane & 15) * 8;  // tokens
             const int b_col = tc.n0 + HALF_N * (int)rank + lane * 8;         // output features
             const bool a_col_ok = a_col < T;
             const bool b_col_ok = b_col < N;
-            for (int kb = 0; kb < nkb; ++kb) {
+            for (int kb = ux.kb0; kb < ux.kb1; ++kb) {
                 const uint32_t full = smem_addr(&bars->full[stage]);
                 if (!mbar_wait(smem_addr(&bars->empty[stage]), phase ^ 1, status, abort_flag)) {
                     st_shared_cluster_u32(peer_abort, 1);
@@ -516,9 +571,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int v0 = q0a, v1 = q1a;
                 q0a = q0b;
                 q1a = q1b;
-                q0b = __ldg(idx + next_kb * BK + lane);
-                q1b = __ldg(idx + next_kb * BK + 32 + lane);
-                next_kb = (next_kb + 1 < nkb) ? next_kb + 1 : 0;
+                advance();
+                q0b = __ldg(idx + kq() * BK + lane);
+                q1b = __ldg(idx + kq() * BK + 32 + lane);
                 // W^T: one 512-B row segment per warp instruction
 #pragma unroll
                 for (int i = 0; i < kRowsB; ++i) {
@@ -545,7 +600,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
         }
         cp_async_wait_all();
-    } else if (warp == kMmaWarp) {
+    } else if (warp == kMmaWarp2) {
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -553,8 +608,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // ------------------------------------------------------------ relay (peer CTA)
             if (lane == 0) {
                 const uint32_t leader_pair_full0 = mapa_shared(smem_addr(&bars->pair_full[0]), 0);
-                for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
-                    for (int kb = 0; kb < nkb; ++kb) {
+                for (int u = cluster_id; ok && u < num_units; u += num_clusters) {
+                    const Unit ux = decode_unit(group, u, m_tiles, nkb);
+                    for (int kb = ux.kb0; kb < ux.kb1; ++kb) {
                         if (!mbar_wait(smem_addr(&bars->full[stage]), phase, status, abort_flag)) {
                             st_shared_cluster_u32(peer_abort, 1);
                             ok = false;
@@ -582,13 +638,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 ok = mbar_wait(smem_addr(&bars->never), 0, status, abort_flag, kDebugWaitLimitNs);
                 if (!ok) st_shared_cluster_u32(peer_abort, 1);
             }
-            for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
+            for (int u = cluster_id; ok && u < num_units; u += num_clusters) {
+                const Unit ux = decode_unit(group, u, m_tiles, nkb);
                 if (!mbar_wait_cluster(smem_addr(&bars->tempty), acc_phase ^ 1, status, abort_flag)) {
                     st_shared_cluster_u32(peer_abort, 1);
                     break;
                 }
                 tc_fence_after();
-                for (int kb = 0; kb < nkb; ++kb) {
+                for (int kb = ux.kb0; kb < ux.kb1; ++kb) {
                     if (!mbar_wait(smem_addr(&bars->full[stage]), phase, status, abort_flag) ||
                         !mbar_wait_cluster(smem_addr(&bars->pair_full[stage]), phase, status, abort_flag)) {
                         st_shared_cluster_u32(peer_abort, 1);
@@ -602,7 +659,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         const uint32_t b_base = smem_addr(sB + stage * B2_STAGE_BYTES);
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk) {
-                            const uint32_t accumulate = (kb | kk) != 0 ? 1u : 0u;
+                            const uint32_t accumulate = (kb != ux.kb0 || kk != 0) ? 1u : 0u;
                             const uint64_t adesc = smem_desc_sw128(a_base + kk * 2048, CHUNK_BYTES, 1024);
                             const uint64_t blo = smem_desc_sw128(b_base + kk * 2048, CHUNK_BYTES, 1024);
                             const uint64_t bhi = smem_desc_sw128(b_base + 2 * CHUNK_BYTES + kk * 2048, CHUNK_BYTES, 1024);
@@ -630,11 +687,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
-        const int q = warp & 3;
+        const int q = warp & 3;                            // TMEM lane quarter
+        const int e = warp - kProducerWarps;               // 0..7
+        const int c64_begin = (e / 4) * (TMEM_COLS2 / 128);  // this warp's half of the columns
         uint32_t acc_phase = 0;
         const uint32_t tempty_leader = mapa_shared(smem_addr(&bars->tempty), 0);
-        for (int tile = cluster_id; tile < num_tiles; tile += num_clusters) {
-            const TileCoord tc = decode_tile2(group, tile, m_tiles);
+        for (int u = cluster_id; u < num_units; u += num_clusters) {
+            const Unit ux = decode_unit(group, u, m_tiles, nkb);
+            const TileCoord tc = ux.tc;
             const int N = group.N[tc.p];
             uint16_t* __restrict__ Y = group.Y[tc.p];
             if (!mbar_wait(smem_addr(&bars->tfull), acc_phase, status, abort_flag)) {
@@ -642,27 +702,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const int row = tc.m0 + HALF_M * (int)rank + q * 32 + lane;
-            uint16_t* yrow = Y + (size_t)row * N;
+            const int rbase = tc.m0 + HALF_M * (int)rank + q * 32;  // first row of this warp
+            const uint32_t stg = smem_addr(sE + e * EPI_STAGE_BYTES);
+            // 64 TMEM columns at a time: the 64 output columns they hold are contiguous
 #pragma unroll 1
-            for (int cc = 0; cc < TMEM_COLS2 / 32; ++cc) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(cc * 32), r);
-                tmem_ld_wait();
-                const int c = cc * 32;
-                const int ncol = tc.n0 + 256 * ((c & 255) >> 7) + 128 * (c >> 8) + (c & 127);
-                if (row < T) {
+            for (int c64 = c64_begin; c64 < c64_begin + TMEM_COLS2 / 128; ++c64) {
+                const int c = c64 * 64;
+                const int lcol = 256 * ((c & 255) >> 7) + 128 * (c >> 8) + (c & 127);  // column inside the tile
+                if (ux.part < 0) __syncwarp();  // the previous block's reads of the staging area are done
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        const int nn = ncol + v * 8;
-                        if (nn < N) {
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(c + 32 * h), r);
+                    tmem_ld_wait();
+                    if (ux.part >= 0) {
+                        // a K-range of a split tile: fp32 partials in the lanes' order, one
+                        // 512-byte store per instruction: [cta][warp][32-col chunk][v][lane][4]
+                        float4* dst = reinterpret_cast<float4*>(group.partials + (size_t)ux.part * BM2 * BN2) +
+                                      ((((int)rank * kEpilogueWarps + q) * (TMEM_COLS2 / 32) + 2 * c64 + h) * 8) * 32 +
+                                      lane;
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            __stcg(dst + v * 32,
+                                   make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                               __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
+                    } else {
+                        // bf16 row pieces into shared memory, 16-byte chunks XOR-swizzled by row
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int ch = 4 * h + j;
                             uint4 o;
-                            o.x = pack_bf16x2(__uint_as_float(r[v * 8 + 0]), __uint_as_float(r[v * 8 + 1]));
-                            o.y = pack_bf16x2(__uint_as_float(r[v * 8 + 2]), __uint_as_float(r[v * 8 + 3]));
-                            o.z = pack_bf16x2(__uint_as_float(r[v * 8 + 4]), __uint_as_float(r[v * 8 + 5]));
-                            o.w = pack_bf16x2(__uint_as_float(r[v * 8 + 6]), __uint_as_float(r[v * 8 + 7]));
-                            *reinterpret_cast<uint4*>(yrow + nn) = o;
+                            o.x = pack_bf16x2(__uint_as_float(r[j * 8 + 0]), __uint_as_float(r[j * 8 + 1]));
+                            o.y = pack_bf16x2(__uint_as_float(r[j * 8 + 2]), __uint_as_float(r[j * 8 + 3]));
+                            o.z = pack_bf16x2(__uint_as_float(r[j * 8 + 4]), __uint_as_float(r[j * 8 + 5]));
+                            o.w = pack_bf16x2(__uint_as_float(r[j * 8 + 6]), __uint_as_float(r[j * 8 + 7]));
+                            st_shared_v4(stg + lane * 128 + ((ch ^ (lane & 7)) << 4), o);
                         }
+                    }
+                }
+                if (ux.part < 0) {
+                    // then 4 full 128-byte row segments per store instruction
+                    __syncwarp();
+#pragma unroll
+                    for (int it = 0; it < 8; ++it) {
+                        const int rr = it * 4 + (lane >> 3), ch = lane & 7;
+                        const uint4 o = ld_shared_v4(stg + rr * 128 + ((ch ^ (rr & 7)) << 4));
+                        const int row = rbase + rr, col = tc.n0 + lcol + ch * 8;
+                        if (row < T && col < N) *reinterpret_cast<uint4*>(Y + (size_t)row * N + col) = o;
                     }
                 }
             }
@@ -676,7 +762,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fence_before();
     cluster_sync();  // the leader's last MMAs and the peer's last TMEM reads are done
     tc_fence_after();
-    if (warp == kMmaWarp) tmem_dealloc_pair(tmem_base, TMEM_COLS2);
+    if (warp == kMmaWarp2) tmem_dealloc_pair(tmem_base, TMEM_COLS2);
+}
+
+// Y = the sum, in split order, of the fp32 partials of each split tile.  The
+// epilogue left them in its lanes' order, [cta][warp][32-column chunk][v][lane]
+// float4s; here warp w of a CTA takes one (cta, warp, chunk, column octet) and
+// lane l the row that epilogue lane l held, so every load is 512 contiguous
+// bytes.  64 CTAs of 8 warps cover one 256 x 512 tile.
+__global__ void __launch_bounds__(256)
+    gemm_fold_kernel(const __grid_constant__ GemmGroup group, int T) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int m_tiles = (T + BM2 - 1) / BM2;
+    const int lane = threadIdx.x & 31;
+    const int tail = blockIdx.x / 64;
+    const int item = (blockIdx.x % 64) * 8 + (threadIdx.x >> 5);  // 0..511
+    const int vp = item % 4, cc = (item / 4) % (TMEM_COLS2 / 32), qw = (item / 64) % kEpilogueWarps;
+    const int rk = item / (4 * (TMEM_COLS2 / 32) * kEpilogueWarps);
+    const int lrow = rk * HALF_M + qw * 32 + lane;
+    const int c = cc * 32 + vp * 8;  // TMEM column of the octet
+    const int lcol = 256 * ((c & 255) >> 7) + 128 * (c >> 8) + (c & 127);
+    const TileCoord tc = decode_tile2(group, group.units_full + tail, m_tiles);
+    const int row = tc.m0 + lrow, col = tc.n0 + lcol;
+    const int N = group.N[tc.p];
+    if (row >= T || col >= N) return;
+    const int S = group.tail_splits;
+    const size_t off = ((size_t)((rk * kEpilogueWarps + qw) * (TMEM_COLS2 / 32) + cc) * 8 + 2 * vp) * 32 + lane;
+    const float4* src = reinterpret_cast<const float4*>(group.partials + (size_t)tail * S * BM2 * BN2) + off;
+    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s0 = 0; s0 < S; s0 += 4) {
+        float4 v[4][2];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (s0 + u < S) {
+                const float4* q = src + (size_t)(s0 + u) * (BM2 * BN2 / 4);
+                v[u][0] = __ldcg(q);
+                v[u][1] = __ldcg(q + 32);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (s0 + u < S) {
+                a[0] += v[u][0].x; a[1] += v[u][0].y; a[2] += v[u][0].z; a[3] += v[u][0].w;
+                a[4] += v[u][1].x; a[5] += v[u][1].y; a[6] += v[u][1].z; a[7] += v[u][1].w;
+            }
+        }
+    }
+    uint4 o;
+    o.x = pack_bf16x2(a[0], a[1]);
+    o.y = pack_bf16x2(a[2], a[3]);
+    o.z = pack_bf16x2(a[4], a[5]);
+    o.w = pack_bf16x2(a[6], a[7]);
+    *reinterpret_cast<uint4*>(group.Y[tc.p] + (size_t)row * N + col) = o;
 }
 
 }  // namespace pair
@@ -691,21 +829,49 @@ int gemm_group_tiles(GemmGroup& g, int T, int pair) {
     g.tile_start[0] = 0;
     for (int p = 0; p < g.count; ++p) g.tile_start[p + 1] = g.tile_start[p] + m_tiles * ((g.N[p] + bn - 1) / bn);
     for (int p = g.count + 1; p <= kMaxGroup; ++p) g.tile_start[p] = g.tile_start[g.count];
+    g.units_full = g.units = g.tile_start[g.count];
+    g.tail_splits = 1;
+    g.partials = nullptr;
     return g.tile_start[g.count];
 }
 
+size_t gemm_pair_partial_bytes(int num_sms) {
+    const int pairs = num_sms / 2 > 0 ? num_sms / 2 : 1;
+    return (size_t)pairs * pair::BM2 * pair::BN2 * sizeof(float);
+}
+
+// Whole tiles fill every full wave over the pairs; the R tiles of the last,
+// partial wave are each cut into s = pairs / R K-ranges (at most one K-block
+// each), so that wave takes about 1/s of a tile's time instead of a whole one.
 cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group, const int32_t* idx,
-                             int k, int T, int H, int* status, int debug_timeout, int num_sms,
+                             int k, int T, int H, float* partials, int* status, int debug_timeout, int num_sms,
                              cudaStream_t stream) {
     if (group.count < 1 || group.count > kMaxGroup) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem_limit(pair::gemm_pair_kernel, pair::kSmemBytes2);
     if (e != cudaSuccess) return e;
     const int tiles = group.tile_start[group.count];
-    int clusters = num_sms / 2;
-    if (clusters > tiles) clusters = tiles;
+    const int nkb = (k + BK - 1) / BK;
+    const int pairs = num_sms / 2 > 0 ? num_sms / 2 : 1;
+    GemmGroup g = group;
+    g.units_full = g.units = tiles;
+    g.tail_splits = 1;
+    g.partials = partials;
+    const int R = tiles % pairs;
+    if (partials && R > 0) {
+        int s = pairs / R;
+        if (s > nkb) s = nkb;
+        if (s > 1) {
+            g.units_full = tiles - R;
+            g.tail_splits = s;
+            g.units = g.units_full + R * s;
+        }
+    }
+    int clusters = pairs < g.units ? pairs : g.units;
     if (clusters < 1) clusters = 1;
-    return launch_pdl(pair::gemm_pair_kernel, dim3(2 * clusters), dim3(kThreads), pair::kSmemBytes2, stream, Xt,
-                      ldT, group, idx, k, T, H, status, debug_timeout);
+    e = launch_pdl(pair::gemm_pair_kernel, dim3(2 * clusters), dim3(pair::kThreads2), pair::kSmemBytes2, stream, Xt, ldT,
+                   g, idx, k, T, H, status, debug_timeout);
+    if (e != cudaSuccess || g.tail_splits == 1) return e;
+    return launch_pdl(pair::gemm_fold_kernel, dim3(R * (pair::BM2 / 4)), dim3(256), 0, stream, g, T);
 }
 
 cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt, const uint16_t* Xt,

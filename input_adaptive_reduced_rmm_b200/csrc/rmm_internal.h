@@ -69,14 +69,22 @@ struct GemmGroup {
     int N[kMaxGroup];
     int tile_start[kMaxGroup + 1];  // prefix sums of the products' tile counts
     int count;
+    // Work units of the CTA-pair kernel (set by launch_gemm_pair): tiles
+    // [0, units_full) whole, the remaining tiles each cut into tail_splits
+    // K-ranges whose fp32 partials go to `partials` and are folded afterwards.
+    int units_full, tail_splits, units;
+    float* partials;
 };
 // Fills tile_start for the given T and tile shape (pair != 0: the 256 x 256
 // CTA-pair tile, else 128 x 256); returns the total tile count.
 int gemm_group_tiles(GemmGroup& g, int T, int pair);
 // CTA-pair (tcgen05 cta_group::2) GEMM, cp.async producer; tiles from gemm_group_tiles(g, T, 1).
+// partials: gemm_pair_partial_bytes(num_sms) of scratch for the split last
+// wave (null: no split).
 cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group, const int32_t* idx,
-                             int k, int T, int H, int* status, int debug_timeout, int num_sms,
+                             int k, int T, int H, float* partials, int* status, int debug_timeout, int num_sms,
                              cudaStream_t stream);
+size_t gemm_pair_partial_bytes(int num_sms);
 // map_xt / map_wt are used only by the TMA tile::gather4 producer
 // (tma_gather != 0), which handles a group of one.
 cudaError_t launch_gemm(const CUtensorMap& map_xt, const CUtensorMap& map_wt, const uint16_t* Xt,
