@@ -80,7 +80,7 @@ def _load():
     lib.oracle_linear.argtypes = [_u16p, _u16p, L, L, L, D, P, L, P, L, _f64p, _i32p]
     lib.oracle_linear.restype = I
     lib.oracle_attention.argtypes = [_u16p, _u16p, _u16p, L, L, L, L, L, L, L, I, D, I, P, L,
-                                     _f64p, _i32p]
+                                     _f64p, _i32p, P]
     lib.oracle_attention.restype = I
     lib.oracle_rmsnorm.argtypes = [_u16p, L, L, D, _f64p]
     lib.oracle_rmsnorm.restype = I
@@ -174,8 +174,9 @@ def linear(X, W, r: float, rows=None, cols=None):
 
 
 def attention(Q, K, V, k: int, causal: bool = True, scale: float | None = None,
-              per_query_head: bool = False, t_rows=None):
-    """Reduced attention.  Q [B,Hq,T,d], K/V [B,Hkv,L,d] (bf16).
+              per_query_head: bool = False, t_rows=None, idx_in=None):
+    """Reduced attention.  Q [B,Hq,T,d], K/V [B,Hkv,L,d] (bf16).  idx_in (int32
+    [B,Hkv|Hq,k]) supplies the kept sets instead of selecting them from Q.
 
     Returns (O fp64 [B,Hq,nrows,d], idx int32 [B,Hkv|Hq,k]).
     """
@@ -189,8 +190,12 @@ def attention(Q, K, V, k: int, causal: bool = True, scale: float | None = None,
     O = np.zeros((B, Hq, nrows, d), dtype=np.float64)
     nsets = Hq if per_query_head else Hkv
     idx = np.zeros((B, nsets, int(k)), dtype=np.int32)
+    given = None
+    if idx_in is not None:
+        given = np.ascontiguousarray(np.asarray(idx_in, dtype=np.int32).reshape(B, nsets, int(k)))
     _check(_load().oracle_attention(q, kk, v, B, Hq, Hkv, T, L, d, int(k), int(bool(causal)),
-                                    float(scale), int(bool(per_query_head)), rp, nr, O, idx),
+                                    float(scale), int(bool(per_query_head)), rp, nr, O, idx,
+                                    None if given is None else given.ctypes.data_as(ctypes.c_void_p)),
            "oracle_attention")
     return O, idx
 

@@ -230,11 +230,14 @@ int oracle_linear(const uint16_t* X, const uint16_t* W, long T, long H, long N, 
  * masked out.  Softmax in fp64 (max-subtracted), O = sum_l p_l V[b,g,l,:].
  * idx_out: [B, Hkv, k] (or [B, Hq, k] per query head), may be NULL.
  * t_rows (NULL: all T) lists the query rows to compute; the kept set always
- * uses all T rows. */
+ * uses all T rows.  idx_in (NULL: select as above) supplies the kept sets
+ * instead, laid out like idx_out -- for a layer oracle that follows the index
+ * sets another implementation chose, so that a near-tie in an upstream input
+ * cannot make the two compute different products. */
 int oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, long B, long Hq,
                      long Hkv, long T, long L, long d, long k, int causal, double scale,
                      int per_query_head, const int64_t* t_rows, long nrows, double* O,
-                     int32_t* idx_out) {
+                     int32_t* idx_out, const int32_t* idx_in) {
     if (!Q || !K || !V || !O || B < 1 || Hq < 1 || Hkv < 1 || T < 1 || L < T || d < 1 || k < 1 ||
         k > d || Hq % Hkv != 0)
         return ORACLE_ERR_ARG;
@@ -259,16 +262,24 @@ int oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, lo
             long q_lo = per_query_head ? set : set * G;
             long q_hi = per_query_head ? set + 1 : (set + 1) * G;
             long g = per_query_head ? set / G : set;
-            /* score over the set's stacked query rows */
-            for (long j = 0; j < d; ++j) s[j] = 0;
-            for (long q = q_lo; q < q_hi; ++q)
-                for (long t = 0; t < T; ++t)
-                    for (long j = 0; j < d; ++j) {
-                        uint16_t m = bf16_magnitude_key(Q[((b * Hq + q) * T + t) * d + j]);
-                        if (m > s[j]) s[j] = m;
-                    }
-            rc = oracle_select(s, d, k, S);
-            if (rc) break;
+            if (idx_in) {
+                /* the given kept set */
+                memcpy(S, idx_in + (b * nsets + set) * k, sizeof(int32_t) * (size_t)k);
+                for (long j = 0; j < k; ++j)
+                    if (S[j] < 0 || S[j] >= d) rc = ORACLE_ERR_ARG;
+                if (rc) break;
+            } else {
+                /* score over the set's stacked query rows */
+                for (long j = 0; j < d; ++j) s[j] = 0;
+                for (long q = q_lo; q < q_hi; ++q)
+                    for (long t = 0; t < T; ++t)
+                        for (long j = 0; j < d; ++j) {
+                            uint16_t m = bf16_magnitude_key(Q[((b * Hq + q) * T + t) * d + j]);
+                            if (m > s[j]) s[j] = m;
+                        }
+                rc = oracle_select(s, d, k, S);
+                if (rc) break;
+            }
             if (idx_out) memcpy(idx_out + (b * nsets + set) * k, S, sizeof(int32_t) * (size_t)k);
             const uint16_t* Kg = K + (b * Hkv + g) * L * d;
             const uint16_t* Vg = V + (b * Hkv + g) * L * d;

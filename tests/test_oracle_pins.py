@@ -250,6 +250,31 @@ def test_attention_equals_library_attention_on_masked_q(T, L, causal, per_head):
             assert np.max(np.abs(O[b, h] - ref)) <= 1e-12
 
 
+def test_attention_given_sets_are_followed():
+    """With kept sets supplied (not the top-k of Q), the oracle equals library
+    attention on Q masked to those dimensions; supplying its own selection
+    reproduces its own result."""
+    B, Hq, Hkv, T, L, d, k = 1, 4, 2, 3, 13, 16, 5
+    Q = rmm_synth.normal((B, Hq, T, d), seed=71)
+    K = rmm_synth.normal((B, Hkv, L, d), seed=72)
+    V = rmm_synth.normal((B, Hkv, L, d), seed=73)
+    scale = 1.0 / math.sqrt(d)
+    rng = np.random.default_rng(74)
+    given = np.stack([np.sort(rng.choice(d, k, replace=False)) for _ in range(Hkv)]).astype(np.int32)[None]
+    O, idx = oracle.attention(Q, K, V, k, causal=True, scale=scale, idx_in=given)
+    assert np.array_equal(idx, given)
+    q, Kf, Vf = f64(Q), f64(K), f64(V)
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        qm = np.zeros_like(q[0, h])
+        qm[:, given[0, g]] = q[0, h][:, given[0, g]]
+        ref = numpy_attention(qm, Kf[0, g], Vf[0, g], scale, True)
+        assert np.max(np.abs(O[0, h] - ref)) <= 1e-12
+    O_own, idx_own = oracle.attention(Q, K, V, k, causal=True, scale=scale)
+    O_again, _ = oracle.attention(Q, K, V, k, causal=True, scale=scale, idx_in=idx_own)
+    assert np.array_equal(O_own, O_again)
+
+
 def test_attention_full_head_dim_is_standard_attention():
     B, Hq, Hkv, T, L, d = 1, 4, 1, 3, 11, 8
     Q = rmm_synth.normal((B, Hq, T, d), seed=61)
