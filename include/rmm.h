@@ -211,6 +211,44 @@ rmm_status rmm_attn_qk(const void* Q, const void* Kt, const void* V, int B, int 
 rmm_status rmm_linear_decode_noalloc(const void* X, const void* Wt, int T, int H, int N, double r,
                                      void* Y, int32_t* idx_out, rmm_stream_t stream);
 
+/* ---------------------------------------------------------------- decoder-layer glue
+ *
+ * The memory-bound ops that sit between the reduced products of one decoder
+ * layer: RMSNorm in place of LayerNorm, a residual stream through every block
+ * and a gated SwiGLU MLP ('Numerical Linear Algebra for LLMs' paper digest,
+ * ai-feeds.com, section 'Method: key modules').  All tensors are bf16
+ * row-major device buffers owned by the caller, 16-byte aligned; arithmetic
+ * inside an op is fp32, every output is rounded to bf16 (round to nearest
+ * even).  Calls are asynchronous on `stream`; argument errors are returned
+ * before anything is launched. */
+
+/* Hsum = X + R and Y = RMSNorm(Hsum) * weight for each of the T rows of H:
+ *   Hsum[t,h] = bf16(X[t,h] + R[t,h])        (R NULL: Hsum = X)
+ *   Y[t,h]    = bf16(Hsum[t,h] / sqrt(mean_h Hsum[t,h]^2 + eps) * weight[h])
+ * weight NULL means 1; Hsum or Y may be NULL to skip that output (not both).
+ * Requires H % 8 == 0 and 8 <= H <= 16384.  Y may alias X. */
+rmm_status rmm_add_rmsnorm(const void* X, const void* R, int T, int H, float eps, const void* weight,
+                           void* Hsum, void* Y, rmm_stream_t stream);
+
+/* Out[i] = bf16(silu(G[i]) * U[i]), silu(z) = z / (1 + exp(-z)), for n
+ * elements (n % 8 == 0). */
+rmm_status rmm_swiglu(const void* G, const void* U, int64_t n, void* Out, rmm_stream_t stream);
+
+/* The q/k/v projections of T tokens (token-major, as rmm_linear_group writes
+ * them) into the attention layouts of rmm_attn_qk (batch 1), appending the new
+ * keys and values to the caches at positions L0 .. L0+T-1:
+ *   Yq [T, Hq*d] -> Q  [Hq, T, d]
+ *   Yk [T, Hkv*d] -> Kt [Hkv, d, ldL]  (Kt[g, j, L0+t] = Yk[t, g*d+j])
+ *   Yv [T, Hkv*d] -> V  [Hkv, ldL, d]  (V[g, L0+t, :] = Yv[t, g*d : g*d+d])
+ * Requires d == 128 and L0 + T <= ldL; cache positions outside the append are
+ * not touched. */
+rmm_status rmm_qkv_heads(const void* Yq, const void* Yk, const void* Yv, int T, int Hq, int Hkv, int d,
+                         void* Q, void* Kt, void* V, int ldL, int L0, rmm_stream_t stream);
+
+/* Attention output back to token-major rows for the o projection:
+ * A[t, h*d + j] = O[h, t, j] for O [Hq, T, d] (batch 1), d == 128. */
+rmm_status rmm_heads_to_tokens(const void* O, int Hq, int T, int d, void* A, rmm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -452,4 +452,43 @@ rmm_status rmm_attn_qk(const void* Q, const void* Kt, const void* V, int B, int 
                                    static_cast<cudaStream_t>(stream)));
 }
 
+rmm_status rmm_add_rmsnorm(const void* X, const void* R, int T, int H, float eps, const void* weight, void* Hsum,
+                           void* Y, rmm_stream_t stream) {
+    if (!X || (!Hsum && !Y) || T < 1 || H < 8 || H % 8 != 0 || H > 16384 || !(eps >= 0.0f)) return RMM_ERR_INVALID_ARG;
+    if (!aligned16(X) || (R && !aligned16(R)) || (weight && !aligned16(weight)) || (Hsum && !aligned16(Hsum)) ||
+        (Y && !aligned16(Y)))
+        return RMM_ERR_INVALID_ARG;
+    return cuda_status(launch_add_rmsnorm(static_cast<const uint16_t*>(X), static_cast<const uint16_t*>(R), T, H, eps,
+                                          static_cast<const uint16_t*>(weight), static_cast<uint16_t*>(Hsum),
+                                          static_cast<uint16_t*>(Y), static_cast<cudaStream_t>(stream)));
+}
+
+rmm_status rmm_swiglu(const void* G, const void* U, int64_t n, void* Out, rmm_stream_t stream) {
+    if (!G || !U || !Out || n < 8 || n % 8 != 0) return RMM_ERR_INVALID_ARG;
+    if (!aligned16(G) || !aligned16(U) || !aligned16(Out)) return RMM_ERR_INVALID_ARG;
+    return cuda_status(launch_swiglu(static_cast<const uint16_t*>(G), static_cast<const uint16_t*>(U), (size_t)n,
+                                     static_cast<uint16_t*>(Out), num_sms_current(),
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+rmm_status rmm_qkv_heads(const void* Yq, const void* Yk, const void* Yv, int T, int Hq, int Hkv, int d, void* Q,
+                         void* Kt, void* V, int ldL, int L0, rmm_stream_t stream) {
+    if (!Yq || !Yk || !Yv || !Q || !Kt || !V || T < 1 || Hq < 1 || Hkv < 1 || L0 < 0 || L0 + T > ldL)
+        return RMM_ERR_INVALID_ARG;
+    if (d != 128) return RMM_ERR_UNSUPPORTED;
+    if (!aligned16(Yq) || !aligned16(Yk) || !aligned16(Yv) || !aligned16(Q) || !aligned16(V)) return RMM_ERR_INVALID_ARG;
+    return cuda_status(launch_qkv_heads(static_cast<const uint16_t*>(Yq), static_cast<const uint16_t*>(Yk),
+                                        static_cast<const uint16_t*>(Yv), T, Hq, Hkv, static_cast<uint16_t*>(Q),
+                                        static_cast<uint16_t*>(Kt), static_cast<uint16_t*>(V), ldL, L0,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+rmm_status rmm_heads_to_tokens(const void* O, int Hq, int T, int d, void* A, rmm_stream_t stream) {
+    if (!O || !A || Hq < 1 || T < 1) return RMM_ERR_INVALID_ARG;
+    if (d != 128) return RMM_ERR_UNSUPPORTED;
+    if (!aligned16(O) || !aligned16(A)) return RMM_ERR_INVALID_ARG;
+    return cuda_status(launch_heads_to_tokens(static_cast<const uint16_t*>(O), Hq, T, static_cast<uint16_t*>(A),
+                                              num_sms_current(), static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -841,8 +841,9 @@ size_t gemm_pair_partial_bytes(int num_sms) {
 }
 
 // Whole tiles fill every full wave over the pairs; the R tiles of the last,
-// partial wave are each cut into s = pairs / R K-ranges (at most one K-block
-// each), so that wave takes about 1/s of a tile's time instead of a whole one.
+// partial wave are each cut into s = min(pairs / R, 8) K-ranges (at least one
+// K-block each), so that wave takes about 1/s of a tile's time instead of a
+// whole one.
 cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group, const int32_t* idx,
                              int k, int T, int H, float* partials, int* status, int debug_timeout, int num_sms,
                              cudaStream_t stream) {
@@ -858,7 +859,10 @@ cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group
     g.partials = partials;
     const int R = tiles % pairs;
     if (partials && R > 0) {
+        // at most 8 ranges: beyond that the fold's reads of the partials cost
+        // more than the shorter tail saves
         int s = pairs / R;
+        if (s > 8) s = 8;
         if (s > nkb) s = nkb;
         if (s > 1) {
             g.units_full = tiles - R;

@@ -57,6 +57,15 @@ constexpr size_t kGemvMaxSmemBytes = 200 * 1024;
 cudaError_t launch_gemv(const uint16_t* X, int T, int H, const int32_t* idx, int k, const GemvGroup& g,
                         float* partials, int num_sms, cudaStream_t stream);
 
+// ---- decoder-layer glue (rmm_layer.cu); bf16 in and out, B = 1, d = 128
+cudaError_t launch_add_rmsnorm(const uint16_t* X, const uint16_t* R, int T, int H, float eps, const uint16_t* Wn,
+                               uint16_t* Hsum, uint16_t* Y, cudaStream_t stream);
+cudaError_t launch_swiglu(const uint16_t* G, const uint16_t* U, size_t n, uint16_t* Out, int num_sms,
+                          cudaStream_t stream);
+cudaError_t launch_qkv_heads(const uint16_t* Yq, const uint16_t* Yk, const uint16_t* Yv, int T, int Hq, int Hkv,
+                             uint16_t* Q, uint16_t* Kt, uint16_t* V, int ldL, int L0, cudaStream_t stream);
+cudaError_t launch_heads_to_tokens(const uint16_t* O, int Hq, int T, uint16_t* A, int num_sms, cudaStream_t stream);
+
 // ---- tcgen05 GEMM (rmm_gemm.cu)
 // Up to kMaxGroup products that share the activations (X^T, T, H and the kept
 // list) and differ in the weight: one persistent launch walks the tiles of

@@ -29,6 +29,7 @@ EXPORTED = (
     "rmm_transpose_weight", "rmm_linear_workspace_bytes", "rmm_linear", "rmm_score",
     "rmm_select", "rmm_gemm_reduced", "rmm_attn_workspace_bytes", "rmm_attn_qk",
     "rmm_linear_decode_noalloc", "rmm_linear_group", "rmm_linear_group_workspace_bytes",
+    "rmm_add_rmsnorm", "rmm_swiglu", "rmm_qkv_heads", "rmm_heads_to_tokens",
 )
 
 
@@ -97,6 +98,10 @@ def lib() -> ctypes.CDLL:
         "rmm_linear_decode_noalloc": (I, [P, P, I, I, I, D, P, P, P]),
         "rmm_linear_group_workspace_bytes": (Z, [I, I, I, P, OP]),
         "rmm_linear_group": (I, [P, I, I, D, I, P, P, P, P, P, Z, P, OP]),
+        "rmm_add_rmsnorm": (I, [P, P, I, I, F, P, P, P, P]),
+        "rmm_swiglu": (I, [P, P, ctypes.c_int64, P, P]),
+        "rmm_qkv_heads": (I, [P, P, P, I, I, I, I, P, P, P, I, I, P]),
+        "rmm_heads_to_tokens": (I, [P, I, I, I, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -304,3 +309,53 @@ def rmm_linear_decode_noalloc(X: torch.Tensor, Wt: torch.Tensor, r: float, Y: to
     _check(lib().rmm_linear_decode_noalloc(_ptr(X), _ptr(Wt), T, H, N, float(r), _ptr(Y), _ptr(idx_out),
                                            _stream(stream)), "rmm_linear_decode_noalloc")
     return Y
+
+
+# ---------------------------------------------------------------- decoder-layer glue
+
+def rmm_add_rmsnorm(X: torch.Tensor, R: torch.Tensor | None = None, eps: float = 1e-5,
+                    weight: torch.Tensor | None = None, Hsum: torch.Tensor | None = None,
+                    Y: torch.Tensor | None = None, want_y: bool = True, stream=None):
+    """Hsum = bf16(X + R); Y = bf16(RMSNorm(Hsum) * weight).  Returns (Hsum, Y); an output
+    not asked for (Hsum None and R None, or want_y False) comes back as None."""
+    _bf16_cuda(X, "X")
+    T, H = X.shape
+    if R is not None:
+        _bf16_cuda(R, "R")
+        if Hsum is None:
+            Hsum = torch.empty_like(X)
+    if want_y and Y is None:
+        Y = torch.empty_like(X)
+    _check(lib().rmm_add_rmsnorm(_ptr(X), _ptr(R), T, H, float(eps), _ptr(weight), _ptr(Hsum), _ptr(Y),
+                                 _stream(stream)), "rmm_add_rmsnorm")
+    return Hsum, Y
+
+
+def rmm_swiglu(G: torch.Tensor, U: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out = bf16(silu(G) * U), elementwise."""
+    _bf16_cuda(G, "G")
+    _bf16_cuda(U, "U")
+    if out is None:
+        out = torch.empty_like(G)
+    _check(lib().rmm_swiglu(_ptr(G), _ptr(U), G.numel(), _ptr(out), _stream(stream)), "rmm_swiglu")
+    return out
+
+
+def rmm_qkv_heads(Yq: torch.Tensor, Yk: torch.Tensor, Yv: torch.Tensor, Q: torch.Tensor, Kt: torch.Tensor,
+                  V: torch.Tensor, L0: int, stream=None) -> torch.Tensor:
+    """Token-major q/k/v -> Q [Hq,T,d] and the caches Kt [Hkv,d,ldL], V [Hkv,ldL,d] at L0 (batch 1)."""
+    T = Yq.shape[0]
+    Hq, _, d = Q.shape
+    Hkv, _, ldL = Kt.shape
+    _check(lib().rmm_qkv_heads(_ptr(Yq), _ptr(Yk), _ptr(Yv), T, Hq, Hkv, d, _ptr(Q), _ptr(Kt), _ptr(V), ldL,
+                               int(L0), _stream(stream)), "rmm_qkv_heads")
+    return Q
+
+
+def rmm_heads_to_tokens(O: torch.Tensor, A: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """O [Hq, T, d] -> A [T, Hq*d]."""
+    Hq, T, d = O.shape
+    if A is None:
+        A = torch.empty(T, Hq * d, dtype=torch.bfloat16, device=O.device)
+    _check(lib().rmm_heads_to_tokens(_ptr(O), Hq, T, d, _ptr(A), _stream(stream)), "rmm_heads_to_tokens")
+    return A
