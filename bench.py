@@ -313,6 +313,114 @@ def time_decode(dev, peaks):
     return out
 
 
+def launches_per_step(dev) -> int:
+    """Our kernels launched by one step: per call the score pass, the select, the CTA-pair
+    GEMM, and the fold of the split last wave when the call's tiles leave a partial wave
+    that the GEMM splits (more than one K-range per tile)."""
+    pairs = torch.cuda.get_device_properties(dev).multi_processor_count // 2
+    n = 0
+    for s, names in CALLS:
+        H = ACT_H[s]
+        nkb = -(-metrics.k_for(H, R) // 64)
+        tiles = sum(-(-T_PREFILL // 256) * -(-PROJ_BY_NAME[m][1] // 512) for m in names)
+        rem = tiles % pairs
+        split = min(pairs // rem, 8, nkb) if rem else 1
+        n += 3 + (1 if split > 1 else 0)
+    return n
+
+
+def time_layer(dev, hweights):
+    """Secondary row: one Llama-3-8B decoder layer (hidden 4096, 32 query / 8 KV heads,
+    MLP 14336, B = 1): prefill of T = 2048 tokens, then 128 decode steps against the
+    growing KV cache, r = 0.5; against the same layer with dense products (cuBLAS) and
+    dense attention (SDPA).  Prefill per op with CUDA events (L2 flushed before each
+    run) from a captured graph with timing events as graph nodes; decode as CUDA-graph
+    replays, one graph per cache position, timed end to end."""
+    from input_adaptive_reduced_rmm_b200.layer import DecoderLayer, DenseLayer, LayerDims
+
+    dims = LayerDims()
+    Tp, steps = T_PREFILL, 128
+    W = {n: hweights[n] for n in ("q", "k", "v", "o", "gate", "up", "down")}
+    layers = {"rmm": DecoderLayer(dims, W, Tp + steps, R, dev), "dense": DenseLayer(dims, W, Tp + steps, dev)}
+    xp = rmm_synth.activations(Tp, dims.H, 700).to(dev)
+    xd = rmm_synth.activations(steps, dims.H, 701).to(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    out = {}
+    for name, layer in layers.items():
+        # prefill: captured once (timing events as graph nodes), replayed after an L2 flush
+        layer.reset()
+        layer.forward(xp)
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        ev = []
+        gp = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            layer.reset()
+            with torch.cuda.graph(gp, stream=side):
+                layer.forward(xp, events=ev)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        runs, totals = [], []
+        for i in range(6):
+            flush.zero_()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record()
+            gp.replay()
+            t1.record()
+            torch.cuda.synchronize()
+            if i:
+                runs.append({n: e0.elapsed_time(e1) for n, e0, e1 in ev})
+                totals.append(t0.elapsed_time(t1))
+        del gp
+        per_op = {n: 1e3 * statistics.median(r[n] for r in runs) for n in runs[0]}
+        prefill_us = 1e3 * statistics.median(totals)
+        # decode: warm the T = 1 buffers eagerly, then capture one graph per position
+        layer.reset()
+        layer.forward(xp)
+        layer.forward(xd[0:1])
+        torch.cuda.synchronize()
+        layer.pos = Tp
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        graphs = []
+        with torch.cuda.stream(side):
+            for t in range(steps):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=side):
+                    layer.forward(xd[t:t + 1])
+                graphs.append(g)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(3):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for g in graphs:
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        del graphs
+        out[name] = {"prefill_us": prefill_us, "prefill_per_op_us": per_op,
+                     "decode_128_steps_us": 1e3 * statistics.median(times),
+                     "decode_step_us": 1e3 * statistics.median(times) / steps}
+    del layers, flush
+    torch.cuda.empty_cache()
+    r_, d_ = out["rmm"], out["dense"]
+    return {"layer": {
+        "workload": "Llama-3-8B decoder layer (RMSNorm, q/k/v, reduced attention over the head dim, o, "
+                    "residual, RMSNorm, gate/up, SwiGLU, down, residual), B=1, prefill T=2048 then 128 "
+                    "decode steps, r=0.5; dense = cuBLAS products + SDPA attention, same glue kernels",
+        "rmm": r_, "dense": d_,
+        "prefill_speedup_vs_dense": d_["prefill_us"] / r_["prefill_us"],
+        "decode_speedup_vs_dense": d_["decode_128_steps_us"] / r_["decode_128_steps_us"],
+        "total_us": r_["prefill_us"] + r_["decode_128_steps_us"],
+        "dense_total_us": d_["prefill_us"] + d_["decode_128_steps_us"],
+    }}
+
+
 def run_rmm(args, world, rank, local):
     from input_adaptive_reduced_rmm_b200 import rmm
 
@@ -425,7 +533,10 @@ def run_rmm(args, world, rank, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = job_throughput(step_flops * K, world, e2e_ms) / 1e12
 
-    extra = time_decode(dev, peaks) if not args.skip_secondary else {}
+    extra = {}
+    if not args.skip_secondary:
+        extra.update(time_decode(dev, peaks))
+        extra.update(time_layer(dev, host_inputs()[1]))
 
     cpu = None
     if rank == 0 and not args.skip_cpu_baseline:
@@ -451,7 +562,7 @@ def run_rmm(args, world, rank, local):
                   "effective_tflops_at_reduced_flops": step_flops / (dense_ms * 1e-3) / 1e12},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "cpu_baseline": cpu,
-        "gpu_launches": 3 * len(CALLS) * K,
+        "gpu_launches": launches_per_step(dev) * K,
         "clocks": clk,
         "per_call": per_call,
     }

@@ -213,12 +213,16 @@ class _NullCtx:
 
 
 class _EventCtx:
+    """Timing events around one op; recorded as graph nodes when the call is being
+    captured (external events), so a replayed graph reports per-op device time."""
+
     def __init__(self, events, name):
         self.events, self.name = events, name
 
     def __enter__(self):
-        self.e0 = torch.cuda.Event(enable_timing=True)
-        self.e1 = torch.cuda.Event(enable_timing=True)
+        ext = torch.cuda.is_current_stream_capturing()
+        self.e0 = torch.cuda.Event(enable_timing=True, external=ext)
+        self.e1 = torch.cuda.Event(enable_timing=True, external=ext)
         self.e0.record()
         return self
 
