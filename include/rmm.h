@@ -71,11 +71,18 @@ typedef struct rmm_options {
      * limit, on a barrier that nothing signals; the call then reports
      * RMM_ERR_TIMEOUT through rmm_get_status() and leaves Y unspecified. */
     int debug_timeout_test;
-    /* Operand producer of the reduced GEMM: 0 (default) = four warps gather
-     * the kept rows with 16-byte cp.async into the swizzled layout; 1 = TMA
-     * tile::gather4 (one instruction per four kept rows x 64 columns). */
+    /* Operand producer of the reduced GEMM: 0 (default) = the CTA-pair
+     * kernel, sixteen warps per CTA gathering the kept rows with 16-byte
+     * cp.async into the swizzled layout; 1 = single-CTA kernel with TMA
+     * tile::gather4 (one instruction per four kept rows x 64 columns);
+     * 2 = single-CTA kernel with the cp.async producer. */
     int gemm_producer;
-    int reserved[3]; /* must be zero */
+    /* Attention kernel for the product: 0 (default) = tensor cores (tcgen05)
+     * for query chunks of 16 or more tokens, the CUDA-core split pass for
+     * shorter ones (decode); 1 = always the split pass; 2 = always the tensor
+     * cores. */
+    int attn_path;
+    int reserved[2]; /* must be zero */
     /* Optional pair of cudaEvent_t handles (NULL: none) recorded on the
      * stream immediately before and after the reduced-product kernel (GEMV or
      * GEMM) of rmm_linear / rmm_gemm_reduced, so that a caller can time that

@@ -54,7 +54,7 @@ int num_sms_current() {
 }
 
 const rmm_options& opts_or_default(const rmm_options* o) {
-    static const rmm_options d = {16, 0, 0, 0, 0, {0, 0, 0}, nullptr, nullptr};
+    static const rmm_options d = {16, 0, 0, 0, 0, 0, {0, 0}, nullptr, nullptr};
     return o ? *o : d;
 }
 
@@ -63,7 +63,8 @@ bool opts_valid(const rmm_options* o) {
     if (o->t_gemv < 0 || o->t_gemv > kGemvMaxT) return false;
     if (o->gemv_splits < 0) return false;
     if (o->gemm_producer < 0 || o->gemm_producer > 2) return false;
-    for (int i = 0; i < 3; ++i)
+    if (o->attn_path < 0 || o->attn_path > 2) return false;
+    for (int i = 0; i < 2; ++i)
         if (o->reserved[i] != 0) return false;
     return true;
 }
@@ -420,7 +421,7 @@ size_t rmm_attn_workspace_bytes(int B, int Hq, int Hkv, int T, int L, int d,
         return 0;
     const rmm_options& o = opts_or_default(options);
     const AttnPlan p = attn_plan(B, Hq, Hkv, T, L, o.attn_per_query_head, num_sms_current());
-    return kStatusBytes + align_up((size_t)B * p.nsets * d * sizeof(int32_t), kAlign) +
+    return kStatusBytes + 2 * align_up((size_t)B * p.nsets * d * sizeof(int32_t), kAlign) +
            align_up(attn_partials_bytes(p, B, Hq, T), kAlign);
 }
 
@@ -439,17 +440,19 @@ rmm_status rmm_attn_qk(const void* Q, const void* Kt, const void* V, int B, int 
     const rmm_options& o = opts_or_default(options);
     if (!o.attn_per_query_head && Hq / Hkv > 8) return RMM_ERR_UNSUPPORTED;
     const AttnPlan p = attn_plan(B, Hq, Hkv, T, L, o.attn_per_query_head, num_sms_current());
+    // workspace: status | kept sets | per-set score vectors (zero between calls) | split partials
     const size_t idx_bytes = align_up((size_t)B * p.nsets * d * sizeof(int32_t), kAlign);
-    const size_t need = kStatusBytes + idx_bytes + align_up(attn_partials_bytes(p, B, Hq, T), kAlign);
+    const size_t need = kStatusBytes + 2 * idx_bytes + align_up(attn_partials_bytes(p, B, Hq, T), kAlign);
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return RMM_ERR_WORKSPACE;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + kStatusBytes);
-    float* partials = reinterpret_cast<float*>(ws + kStatusBytes + idx_bytes);
+    uint32_t* sc = reinterpret_cast<uint32_t*>(ws + kStatusBytes + idx_bytes);
+    float* partials = reinterpret_cast<float*>(ws + kStatusBytes + 2 * idx_bytes);
     return cuda_status(launch_attn(static_cast<const uint16_t*>(Q), static_cast<const uint16_t*>(Kt),
                                    static_cast<const uint16_t*>(V), B, Hq, Hkv, T, L, ldL, k,
                                    causal ? 1 : 0, scale, o.attn_per_query_head,
-                                   static_cast<uint16_t*>(O), idx, partials, p,
-                                   static_cast<cudaStream_t>(stream)));
+                                   static_cast<uint16_t*>(O), idx, partials, sc, reinterpret_cast<int*>(ws),
+                                   o.attn_path, p, static_cast<cudaStream_t>(stream)));
 }
 
 rmm_status rmm_add_rmsnorm(const void* X, const void* R, int T, int H, float eps, const void* weight, void* Hsum,

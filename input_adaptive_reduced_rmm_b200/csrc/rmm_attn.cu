@@ -14,14 +14,19 @@
 // k of the d rows, and V is read in full.
 //
 // Kernels:
-//   attn_select_kernel  one CTA per kept set: column max over the set's query
-//                       rows, then an exact rank-based top-k of the d scores
+//   attn_score_kernel   column max of |Q| over a set's query rows, many CTAs,
+//                       atomicMax into a per-set score vector (long chunks)
+//   attn_select_kernel  one CTA per kept set: the scores (or, for short
+//                       chunks, the column max itself), then an exact
+//                       rank-based top-k of the d scores
 //   attn_split_kernel   one CTA per (set, split of L, block of query tokens):
 //                       logits for a 1024-key sub-block (each thread 4 keys,
 //                       8-byte loads of kept K^T rows), online softmax in fp32,
 //                       P.V with 16-byte loads of V rows; writes the split's
 //                       running max, sum and unnormalised output
 //   attn_combine_kernel merges the splits (flash-decoding style) into bf16 O.
+// Prefill chunks of 16 or more tokens run on the tensor cores instead
+// (rmm_attn_tc.cu); the split pass serves decode.
 #include <math.h>
 
 #include "rmm_common.cuh"
@@ -39,9 +44,56 @@ constexpr int PSTRIDE = D + 2;  // floats per split partial: m, l, O[d]
 
 // ---------------------------------------------------------------- selection
 
+// Column max of |Q| over a set's stacked query rows (its heads x T tokens),
+// spread over many CTAs: CTA (set of batch b, chunk of 64 rows); 16-byte loads,
+// 16 row lanes x 16 dim chunks; folded into sc[set][d] with atomicMax (sc
+// starts at zero: the select kernel clears it after reading).
+__global__ void __launch_bounds__(256)
+    attn_score_kernel(const uint16_t* __restrict__ Q, int Hq, int Hkv, int T, int per_query_head,
+                      uint32_t* __restrict__ sc) {
+    __shared__ uint32_t red[16][D];
+    const int nsets = per_query_head ? Hq : Hkv;
+    const int set = blockIdx.x % nsets;
+    const int b = blockIdx.x / nsets;
+    const int nq = per_query_head ? 1 : Hq / Hkv;
+    const int q_lo = per_query_head ? set : set * nq;
+    const int nrows = nq * T;
+    const int c16 = threadIdx.x & 15, rl = threadIdx.x >> 4;
+    pdl_wait();
+    pdl_launch_dependents();
+    uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const int r0 = blockIdx.y * 64;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = r0 + rl + 16 * i;
+        if (r < nrows) {
+            const int q = q_lo + r / T, t = r % T;
+            const uint4 v = ld_nc_v4(Q + (((size_t)b * Hq + q) * T + t) * D + c16 * 8);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                m[2 * e] = max(m[2 * e], w[e] & 0x7FFFu);
+                m[2 * e + 1] = max(m[2 * e + 1], (w[e] >> 16) & 0x7FFFu);
+            }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[rl][c16 * 8 + e] = m[e];
+    __syncthreads();
+    if (threadIdx.x < D) {
+        uint32_t mm = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mm = max(mm, red[i][threadIdx.x]);
+        if (mm > 0) atomicMax(sc + (size_t)blockIdx.x * D + threadIdx.x, mm);
+    }
+}
+
+// One CTA per kept set: the scores (from sc, cleared after reading, or, with
+// sc null, folded here from Q for short chunks), then an exact rank-based
+// top-k of the d scores under (score desc, index asc), ascending.
 __global__ void __launch_bounds__(D)
     attn_select_kernel(const uint16_t* __restrict__ Q, int Hq, int Hkv, int T, int k,
-                       int per_query_head, int32_t* __restrict__ idx) {
+                       int per_query_head, uint32_t* __restrict__ sc, int32_t* __restrict__ idx) {
     __shared__ uint32_t sv[D];
     __shared__ int warp_cnt[D / 32];
     const int nsets = per_query_head ? Hq : Hkv;
@@ -55,9 +107,14 @@ __global__ void __launch_bounds__(D)
     pdl_launch_dependents();
 
     uint32_t m = 0;
-    for (int q = q_lo; q < q_hi; ++q) {
-        const uint16_t* row = Q + ((size_t)(b * Hq + q) * T) * D + j;
-        for (int t = 0; t < T; ++t) m = max(m, (uint32_t)(row[(size_t)t * D] & 0x7FFF));
+    if (sc) {
+        m = sc[(size_t)blockIdx.x * D + j];
+        sc[(size_t)blockIdx.x * D + j] = 0;
+    } else {
+        for (int q = q_lo; q < q_hi; ++q) {
+            const uint16_t* row = Q + ((size_t)(b * Hq + q) * T) * D + j;
+            for (int t = 0; t < T; ++t) m = max(m, (uint32_t)(row[(size_t)t * D] & 0x7FFF));
+        }
     }
     sv[j] = m;
     __syncthreads();
@@ -314,12 +371,24 @@ size_t attn_partials_bytes(const AttnPlan& p, int B, int Hq, int T) {
 
 cudaError_t launch_attn(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq,
                         int Hkv, int T, int L, int ldL, int k, int causal, float scale,
-                        int per_query_head, uint16_t* O, int32_t* idx, float* partials,
-                        const AttnPlan& p, cudaStream_t stream) {
-    cudaError_t e = launch_pdl(attn_select_kernel, dim3(B * p.nsets), dim3(D), 0, stream, Q, Hq, Hkv, T, k,
-                               per_query_head, idx);
-    if (e != cudaSuccess) return e;
+                        int per_query_head, uint16_t* O, int32_t* idx, float* partials, uint32_t* sc,
+                        int* status, int path, const AttnPlan& p, cudaStream_t stream) {
     const int nq = per_query_head ? 1 : Hq / Hkv;
+    // the kept sets: the column max over many CTAs when the chunk is long
+    cudaError_t e;
+    const bool wide = nq * T >= 64;
+    if (wide) {
+        e = launch_pdl(attn_score_kernel, dim3(B * p.nsets, (nq * T + 63) / 64), dim3(256), 0, stream, Q, Hq, Hkv, T,
+                       per_query_head, sc);
+        if (e != cudaSuccess) return e;
+    }
+    e = launch_pdl(attn_select_kernel, dim3(B * p.nsets), dim3(D), 0, stream, Q, Hq, Hkv, T, k, per_query_head,
+                   wide ? sc : (uint32_t*)nullptr, idx);
+    if (e != cudaSuccess) return e;
+    const bool tc = path == 2 || (path == 0 && attn_tc_supported(T, k));
+    if (tc)
+        return launch_attn_tc(Q, Kt, V, B, Hq, Hkv, T, L, ldL, k, causal, scale, per_query_head, idx, O, status,
+                              stream);
     if (nq > RMAX) return cudaErrorInvalidValue;
     dim3 grid(B * p.nsets, p.nsplit, (T + p.tq - 1) / p.tq);
     e = launch_pdl(attn_split_kernel, grid, dim3(kThreads), 0, stream, Q, Kt, V, Hq, Hkv, T, L, ldL, k, causal,

@@ -1,0 +1,439 @@
+// rmm_attn_tc.cu -- the prefill chunk of the reduced attention on the tensor
+// cores (tcgen05, accumulators in TMEM).
+//
+// For one (batch b, query head h) and 128 query rows t0 .. t0+127, with the
+// head's kept set S (k of the d = 128 head dims, padded to kp = roundup(k, 16)
+// with dims whose query values are zero):
+//   S_j = Q[:, S] K_j[:, S]^T    over key blocks j of 128 keys   (M=128, N=128, K=kp)
+//   O  += P_j V_j                P_j = exp(S_j - m) in bf16      (M=128, N=128, K=128)
+// with a causal mask (query t sits at key position L - T + t) and an fp32
+// online softmax.  The reduction along the head dimension and the full
+// softmax.V follow the cf-1.com post on input-adaptive matrix-product
+// reduction, §3.3 (reduce inside a head) and the paper abstract (attention
+// products reduced along their contraction dimension).
+//
+// Operands in shared memory, 128-byte swizzled: the gathered query tile and
+// the key block are MN-major (a kept dim is one row of 128 tokens / keys --
+// the d-major key cache makes each kept dim of a key block one contiguous
+// 256-byte segment); V blocks are MN-major (a key is one row of d values);
+// P is written by the softmax threads as a K-major operand (each thread owns
+// one query row).  TMEM holds two S buffers (columns 0-127, 128-255) and O
+// (256-383).
+//
+// Warp roles (256 threads):
+//   0-3  softmax: thread i owns query row t0 + i (TMEM lane i); reads S_j,
+//        masks, keeps a running reference max m and sum l; P_j to shared
+//        memory.  O is rescaled in TMEM only when a row's block max exceeds m
+//        by more than 2^8 (the reference max is then raised), so P stays below
+//        256 and most blocks need no rescale.  At the end O / l goes to HBM.
+//   4    MMA: one thread issues S_{j+1} before P_j V_j so the tensor pipe
+//        overlaps the softmax; tcgen05.commit releases buffers.
+//   5-7  producers: the query tile once (kept dims gathered), then per key
+//        block the kp kept rows of K^T and 128 rows of V with 16-byte
+//        cp.async (zero-filled past the valid keys), two stages.
+// Every wait is bounded: on expiry the kernel records RMM_ERR_TIMEOUT, every
+// role leaves its loop, in-flight tensor-core work drains, TMEM is freed.
+#include <math.h>
+
+#include "rmm_common.cuh"
+#include "rmm_internal.h"
+
+namespace rmm {
+
+namespace {
+
+constexpr int D = 128;
+constexpr int BQ = 128;   // query rows per CTA (= TMEM lanes)
+constexpr int BKV = 128;  // keys per block
+constexpr int KV_STAGES = 2;
+constexpr int kSoftmaxThreads = 128;
+constexpr int kMmaWarp = 4;
+constexpr int kProdWarps = 3;  // 8 warps in all: two per SM sub-partition, so a thread may hold 255 registers
+constexpr int kProdThreads = 32 * kProdWarps;
+constexpr int kThreadsTc = 32 * (4 + 1 + kProdWarps);
+constexpr int V_CHUNK = BKV * 128;     // 64 dims x 128 key rows (bytes)
+constexpr int V_BYTES = 2 * V_CHUNK;   // 32 KB
+constexpr int P_ATOM = BQ * 128;       // 128 rows x 64 keys (bytes)
+constexpr int P_BYTES = 2 * P_ATOM;    // 32 KB
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_S0 = 0, TM_O = 256;
+constexpr float kRescaleLog2 = 8.0f;   // rescale O when a block max exceeds the reference by 2^8
+
+struct __align__(8) Bars {
+    uint64_t q_full;
+    uint64_t kv_full[KV_STAGES];
+    uint64_t kv_empty[KV_STAGES];
+    uint64_t s_full[2];
+    uint64_t s_empty[2];
+    uint64_t p_full;
+    uint64_t p_empty;
+    uint64_t o_full;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+// 2^x with the hardware approximation (ex2.approx.ftz: ~2 ulp; -inf gives 0);
+// P is rounded to bf16 right after, so its error is far below that rounding.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Byte offset of 16-byte chunk c16 (along M/N) of row j (along K) in the
+// 128-byte-swizzled MN-major layout whose 64-element groups are `chunk` apart.
+__device__ __forceinline__ uint32_t swz(int j, int c16, int chunk) {
+    return (uint32_t)((c16 >> 3) * chunk + j * 128 + (((c16 & 7) ^ (j & 7)) << 4));
+}
+
+// Softmax pass 1 for one row of a key block: the max of the raw logits
+// (scale > 0) in 8 independent chains, 64 TMEM columns per round trip.
+// kMask: keys past the cache end or (causal) past the row's position count as -inf.
+template <bool kMask>
+__device__ __forceinline__ float row_max(uint32_t srow, int kb0, int L, int causal, int pos) {
+    float mx[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[2][32];
+        tmem_ld_32x32b_x32(srow + hh * 64, r[0]);
+        tmem_ld_32x32b_x32(srow + hh * 64 + 32, r[1]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                float x = __uint_as_float(r[q][c]);
+                if (kMask) {
+                    const int key = kb0 + hh * 64 + q * 32 + c;
+                    if (!(key < L && (!causal || key <= pos))) x = -INFINITY;
+                }
+                mx[c & 7] = fmaxf(mx[c & 7], x);
+            }
+    }
+    return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+}
+
+// Softmax pass 2: p = 2^(s * scale_log2 - m) (one FMA and one hardware exp2;
+// masked logits give 0), the row sum, and P (bf16) written as the K-major A
+// operand: row i at prow, keys in two 64-key atoms, 16-byte chunks
+// XOR-swizzled by row.
+template <bool kMask>
+__device__ __forceinline__ float row_exp(uint32_t srow, int kb0, int L, int causal, int pos, float scale_log2,
+                                         float neg_m, uint32_t prow, int i) {
+    float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[2][32];
+        tmem_ld_32x32b_x32(srow + hh * 64, r[0]);
+        tmem_ld_32x32b_x32(srow + hh * 64 + 32, r[1]);
+        tmem_ld_wait();
+        float pv[64];
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                float p = fast_exp2(fmaf(__uint_as_float(r[q][c]), scale_log2, neg_m));
+                if (kMask) {
+                    const int key = kb0 + hh * 64 + q * 32 + c;
+                    if (!(key < L && (!causal || key <= pos))) p = 0.0f;
+                }
+                pv[q * 32 + c] = p;
+                sm[c & 7] += p;
+            }
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+            const uint4 w = make_uint4(pack_bf16x2(pv[c8 * 8 + 0], pv[c8 * 8 + 1]),
+                                       pack_bf16x2(pv[c8 * 8 + 2], pv[c8 * 8 + 3]),
+                                       pack_bf16x2(pv[c8 * 8 + 4], pv[c8 * 8 + 5]),
+                                       pack_bf16x2(pv[c8 * 8 + 6], pv[c8 * 8 + 7]));
+            st_shared_v4(prow + hh * P_ATOM + ((c8 ^ (i & 7)) << 4), w);
+        }
+    }
+    return ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+}
+
+__global__ void __launch_bounds__(kThreadsTc, 1)
+    attn_tc_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ Kt, const uint16_t* __restrict__ V,
+                   int Hq, int Hkv, int T, int L, int ldL, int k, int kp, int causal, float scale_log2,
+                   int per_query_head, const int32_t* __restrict__ idx, uint16_t* __restrict__ O, int* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const int QK_BYTES = kp * 256;  // a gathered query tile or key block
+    uint8_t* sP = smem;                                   // 32 KB (1024-aligned)
+    uint8_t* sV = sP + P_BYTES;                           // KV_STAGES x 32 KB
+    uint8_t* sQ = sV + KV_STAGES * V_BYTES;               // kp x 256
+    uint8_t* sK = sQ + QK_BYTES;                          // KV_STAGES x kp x 256
+    int* sidx = reinterpret_cast<int*>(sK + KV_STAGES * QK_BYTES);  // kp kept dims
+    Bars* bars = reinterpret_cast<Bars*>(sidx + D);
+    volatile int* abort_flag = &bars->abort_flag;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_tiles = (T + BQ - 1) / BQ;
+    const int tile = n_tiles - 1 - (int)blockIdx.x;  // the longest (latest) tiles first
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int G = Hq / Hkv;
+    const int g = h / G;
+    const int nsets = per_query_head ? Hq : Hkv;
+    const int set = per_query_head ? h : g;
+    const int t0 = tile * BQ;
+    // key blocks this tile needs
+    int last_key = L - 1;
+    if (causal) last_key = min(last_key, L - T + min(t0 + BQ - 1, T - 1));
+    const int nkb = last_key / BKV + 1;
+
+    if (tid == 0) {
+        mbar_init(smem_addr(&bars->q_full), kProdThreads);
+        for (int s = 0; s < KV_STAGES; ++s) {
+            mbar_init(smem_addr(&bars->kv_full[s]), kProdThreads);
+            mbar_init(smem_addr(&bars->kv_empty[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_addr(&bars->s_full[s]), 1);
+            mbar_init(smem_addr(&bars->s_empty[s]), kSoftmaxThreads);
+        }
+        mbar_init(smem_addr(&bars->p_full), kSoftmaxThreads);
+        mbar_init(smem_addr(&bars->p_empty), 1);
+        mbar_init(smem_addr(&bars->o_full), 1);
+        mbar_init(smem_addr(&bars->drain), 1);
+        bars->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_addr(&bars->tmem_base), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    pdl_wait();  // Q, the caches and the kept sets come from the preceding kernels
+    pdl_launch_dependents();
+
+    if (warp > kMmaWarp) {
+        // ------------------------------------------------------------ producers
+        const int pt = tid - 32 * (kMmaWarp + 1);
+        const int32_t* S = idx + ((size_t)b * nsets + set) * k;
+        for (int j = pt; j < kp; j += kProdThreads) sidx[j] = j < k ? __ldg(S + j) : -1;
+        asm volatile("bar.sync 1, %0;" ::"r"(kProdThreads));
+        // the query tile: 128 tokens x 128 dims staged row-major in the (not yet
+        // used) P buffer with coalesced 16-byte copies, then the kp kept dims
+        // gathered from there into the MN-major operand, 8 tokens per chunk
+        const uint16_t* Qh = Q + ((size_t)b * Hq + h) * T * D;
+        const uint32_t qstage = smem_addr(sP);
+        for (int it = pt; it < BQ * 16; it += kProdThreads) {
+            const int tr = it >> 4, c16 = it & 15;
+            const bool ok = t0 + tr < T;
+            cp_async_16(qstage + tr * 256 + c16 * 16, ok ? Qh + (size_t)(t0 + tr) * D + c16 * 8 : Qh, ok ? 16u : 0u);
+        }
+        cp_async_wait_all();
+        asm volatile("bar.sync 1, %0;" ::"r"(kProdThreads));
+        const uint16_t* qs = reinterpret_cast<const uint16_t*>(sP);
+        for (int it = pt; it < kp * 16; it += kProdThreads) {
+            const int jr = it >> 4, c16 = it & 15;
+            const int dim = sidx[jr];
+            uint16_t v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = dim >= 0 ? qs[(c16 * 8 + e) * D + dim] : (uint16_t)0;
+            const uint4 w = make_uint4(v[0] | ((uint32_t)v[1] << 16), v[2] | ((uint32_t)v[3] << 16),
+                                       v[4] | ((uint32_t)v[5] << 16), v[6] | ((uint32_t)v[7] << 16));
+            st_shared_v4(smem_addr(sQ) + swz(jr, c16, kp * 128), w);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(smem_addr(&bars->q_full));
+        const uint16_t* Kg = Kt + ((size_t)b * Hkv + g) * D * ldL;
+        const uint16_t* Vg = V + ((size_t)b * Hkv + g) * ldL * D;
+        for (int j = 0; j < nkb; ++j) {
+            const int s = j % KV_STAGES;
+            const uint32_t ph = (uint32_t)(j / KV_STAGES) & 1u;
+            if (!mbar_wait(smem_addr(&bars->kv_empty[s]), ph ^ 1u, status, abort_flag)) break;
+            const int kb0 = j * BKV;
+            const uint32_t kst = smem_addr(sK + s * QK_BYTES), vst = smem_addr(sV + s * V_BYTES);
+            for (int it = pt; it < kp * 16; it += kProdThreads) {
+                const int jr = it >> 4, c16 = it & 15;
+                const int key = kb0 + c16 * 8;
+                const int dim = sidx[jr];
+                const bool ok = dim >= 0 && key < ldL;
+                cp_async_16(kst + swz(jr, c16, kp * 128), ok ? Kg + (size_t)dim * ldL + key : Kg, ok ? 16u : 0u);
+            }
+            for (int it = pt; it < BKV * 16; it += kProdThreads) {
+                const int kr = it >> 4, c16 = it & 15;
+                const int key = kb0 + kr;
+                const bool ok = key < L;  // V past the valid keys reads as zero (P is 0 there)
+                cp_async_16(vst + swz(kr, c16, V_CHUNK), ok ? Vg + (size_t)key * D + c16 * 8 : Vg, ok ? 16u : 0u);
+            }
+            cp_async_arrive_noinc(smem_addr(&bars->kv_full[s]));
+        }
+        cp_async_wait_all();
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        bool ok = __all_sync(0xffffffffu, mbar_wait(smem_addr(&bars->q_full), 0, status, abort_flag));
+        const uint32_t idesc_s = idesc_bf16_f32(BQ, BKV, 1, 1);  // Q_S and K_S both MN-major
+        const uint32_t idesc_pv = idesc_bf16_f32(BQ, D, 0, 1);   // P K-major, V MN-major
+        const uint32_t qbase = smem_addr(sQ);
+        fence_proxy_async_smem();
+        tc_fence_after();
+        for (int j = 0; ok && j <= nkb; ++j) {
+            if (j < nkb) {
+                const int s = j % KV_STAGES, sb = j & 1;
+                bool got = mbar_wait(smem_addr(&bars->kv_full[s]), (uint32_t)(j / KV_STAGES) & 1u, status, abort_flag);
+                got = got && mbar_wait(smem_addr(&bars->s_empty[sb]), ((uint32_t)(j >> 1) & 1u) ^ 1u, status, abort_flag);
+                if (!__all_sync(0xffffffffu, got)) {  // the warp leaves together
+                    ok = false;
+                    break;
+                }
+                fence_proxy_async_smem();  // the producers' cp.async data, read by the tensor cores
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t kbase = smem_addr(sK + s * QK_BYTES);
+                    for (int kk = 0; kk < kp / 16; ++kk)
+                        umma_f16(tmem + TM_S0 + sb * BKV, smem_desc_sw128(qbase + kk * 2048, kp * 128, 1024),
+                                 smem_desc_sw128(kbase + kk * 2048, kp * 128, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                    umma_commit(smem_addr(&bars->s_full[sb]));
+                }
+                __syncwarp();
+            }
+            if (j >= 1) {
+                const int jp = j - 1, sp = jp % KV_STAGES;
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars->p_full), (uint32_t)jp & 1u, status, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                fence_proxy_async_smem();  // P written by the softmax threads
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t pbase = smem_addr(sP), vbase = smem_addr(sV + sp * V_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BKV / 16; ++kk)
+                        umma_f16(tmem + TM_O, smem_desc_sw128(pbase + (kk >> 2) * P_ATOM + (kk & 3) * 32, 16, 1024),
+                                 smem_desc_sw128(vbase + kk * 2048, V_CHUNK, 1024), idesc_pv,
+                                 (jp > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(smem_addr(&bars->p_empty));
+                    umma_commit(smem_addr(&bars->kv_empty[sp]));
+                }
+                __syncwarp();
+            }
+        }
+        if (lane == 0) {
+            if (ok) umma_commit(smem_addr(&bars->o_full));
+            umma_commit(smem_addr(&bars->drain));  // everything issued so far has completed
+        }
+        __syncwarp();
+        // wait for the issued MMAs even after an abort (they finish on their own) so
+        // that TMEM is never freed under them; only the time limit ends this wait
+        volatile int no_abort = 0;
+        mbar_wait(smem_addr(&bars->drain), 0, status, &no_abort, kWaitLimitNs);
+    } else {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int i = tid;  // query row inside the tile = TMEM lane
+        const int t = t0 + i;
+        const int pos = L - T + t;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        float m_use = -INFINITY, l_sum = 0.0f;
+        bool ok = true;
+        for (int j = 0; j < nkb; ++j) {
+            const int sb = j & 1;
+            // waits and branches around tcgen05.ld/st (.sync.aligned: the whole warp,
+            // converged) are decided warp-wide
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(smem_addr(&bars->s_full[sb]), (uint32_t)(j >> 1) & 1u, status, abort_flag))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int kb0 = j * BKV;
+            // mask only where the warp's rows cross the diagonal or the cache end
+            const bool full =
+                __all_sync(0xffffffffu, kb0 + BKV - 1 < L && (!causal || kb0 + BKV - 1 <= pos));
+            const uint32_t srow = tmem + lane_base + TM_S0 + sb * BKV;
+            const float m_blk = (full ? row_max<false>(srow, kb0, L, causal, pos)
+                                      : row_max<true>(srow, kb0, L, causal, pos)) * scale_log2;
+            const bool resc = m_blk > m_use + kRescaleLog2;
+            const float m_new = resc ? m_blk : m_use;
+            const float alpha = resc ? exp2f(m_use - m_new) : 1.0f;  // exp2(-inf) = 0 on the first block
+            const float neg_m = (m_new == -INFINITY) ? 0.0f : -m_new;
+            // P_{j-1} V_{j-1} has finished: O is final for the earlier blocks and P is free
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(smem_addr(&bars->p_empty), ((uint32_t)j & 1u) ^ 1u, status, abort_flag))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (j > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t o[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + TM_O + q * 32, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                    tmem_st_32x32b_x32(tmem + lane_base + TM_O + q * 32, o);
+                }
+                tmem_st_wait();
+            }
+            m_use = m_new;
+            const uint32_t prow = smem_addr(sP) + i * 128;
+            const float rs = full ? row_exp<false>(srow, kb0, L, causal, pos, scale_log2, neg_m, prow, i)
+                                  : row_exp<true>(srow, kb0, L, causal, pos, scale_log2, neg_m, prow, i);
+            tc_fence_before();
+            mbar_arrive(smem_addr(&bars->s_empty[sb]));  // S_j fully read
+            l_sum = l_sum * alpha + rs;
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(smem_addr(&bars->p_full));
+        }
+        if (ok && __all_sync(0xffffffffu, mbar_wait(smem_addr(&bars->o_full), 0, status, abort_flag))) {
+            tc_fence_after();
+            const float inv = 1.0f / l_sum;
+            uint16_t* orow = O + (((size_t)b * Hq + h) * T + (t < T ? t : 0)) * D;
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t o[32];
+                tmem_ld_32x32b_x32(tmem + lane_base + TM_O + q * 32, o);
+                tmem_ld_wait();
+                if (t < T) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const uint4 w = make_uint4(
+                            pack_bf16x2(__uint_as_float(o[v * 8 + 0]) * inv, __uint_as_float(o[v * 8 + 1]) * inv),
+                            pack_bf16x2(__uint_as_float(o[v * 8 + 2]) * inv, __uint_as_float(o[v * 8 + 3]) * inv),
+                            pack_bf16x2(__uint_as_float(o[v * 8 + 4]) * inv, __uint_as_float(o[v * 8 + 5]) * inv),
+                            pack_bf16x2(__uint_as_float(o[v * 8 + 6]) * inv, __uint_as_float(o[v * 8 + 7]) * inv));
+                        *reinterpret_cast<uint4*>(orow + q * 32 + v * 8) = w;
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+size_t attn_tc_smem_bytes(int kp) {
+    return 1024 + P_BYTES + (size_t)KV_STAGES * V_BYTES + (size_t)(1 + KV_STAGES) * kp * 256 + D * sizeof(int) +
+           sizeof(Bars);
+}
+
+}  // namespace
+
+bool attn_tc_supported(int T, int k) { return T >= kAttnTcMinT && k >= 1 && k <= D; }
+
+cudaError_t launch_attn_tc(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq, int Hkv, int T,
+                           int L, int ldL, int k, int causal, float scale, int per_query_head, const int32_t* idx,
+                           uint16_t* O, int* status, cudaStream_t stream) {
+    const int kp = (k + 15) / 16 * 16;
+    const size_t smem = attn_tc_smem_bytes(kp);
+    cudaError_t e = ensure_smem_limit(attn_tc_kernel, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((T + BQ - 1) / BQ, Hq, B);
+    return launch_pdl(attn_tc_kernel, grid, dim3(kThreadsTc), smem, stream, Q, Kt, V, Hq, Hkv, T, L, ldL, k, kp,
+                      causal, scale * 1.4426950408889634f, per_query_head, idx, O, status);
+}
+
+}  // namespace rmm

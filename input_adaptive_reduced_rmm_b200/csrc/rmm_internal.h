@@ -57,6 +57,14 @@ constexpr size_t kGemvMaxSmemBytes = 200 * 1024;
 cudaError_t launch_gemv(const uint16_t* X, int T, int H, const int32_t* idx, int k, const GemvGroup& g,
                         float* partials, int num_sms, cudaStream_t stream);
 
+// ---- tensor-core prefill attention (rmm_attn_tc.cu): query chunks of at
+// least kAttnTcMinT tokens, kept sets from the attention select kernel
+constexpr int kAttnTcMinT = 16;
+bool attn_tc_supported(int T, int k);
+cudaError_t launch_attn_tc(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq, int Hkv, int T,
+                           int L, int ldL, int k, int causal, float scale, int per_query_head, const int32_t* idx,
+                           uint16_t* O, int* status, cudaStream_t stream);
+
 // ---- decoder-layer glue (rmm_layer.cu); bf16 in and out, B = 1, d = 128
 cudaError_t launch_add_rmsnorm(const uint16_t* X, const uint16_t* R, int T, int H, float eps, const uint16_t* Wn,
                                uint16_t* Hsum, uint16_t* Y, cudaStream_t stream);
@@ -111,10 +119,13 @@ struct AttnPlan {
 };
 AttnPlan attn_plan(int B, int Hq, int Hkv, int T, int L, int per_query_head, int num_sms);
 size_t attn_partials_bytes(const AttnPlan& p, int B, int Hq, int T);
+// path: 0 auto (tensor cores for chunks of kAttnTcMinT+ tokens), 1 the
+// CUDA-core split pass, 2 tensor cores.  sc: u32 [B * nsets * d] of zeros
+// (left at zero); status: the workspace status word.
 cudaError_t launch_attn(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq,
                         int Hkv, int T, int L, int ldL, int k, int causal, float scale,
-                        int per_query_head, uint16_t* O, int32_t* idx, float* partials,
-                        const AttnPlan& plan, cudaStream_t stream);
+                        int per_query_head, uint16_t* O, int32_t* idx, float* partials, uint32_t* sc,
+                        int* status, int path, const AttnPlan& plan, cudaStream_t stream);
 
 // ---- glue (rmm_glue.cu)
 cudaError_t launch_transpose(const uint16_t* W, uint16_t* Wt, int N, int H, cudaStream_t stream);

@@ -46,17 +46,20 @@ class rmm_options(ctypes.Structure):
         ("gemv_splits", ctypes.c_int),
         ("debug_timeout_test", ctypes.c_int),
         ("gemm_producer", ctypes.c_int),
-        ("reserved", ctypes.c_int * 3),
+        ("attn_path", ctypes.c_int),
+        ("reserved", ctypes.c_int * 2),
         ("product_event_begin", ctypes.c_void_p),
         ("product_event_end", ctypes.c_void_p),
     ]
 
 
 def options(t_gemv: int = 16, attn_per_query_head: bool = False, gemv_splits: int = 0,
-            debug_timeout_test: bool = False, gemm_producer: int = 0, product_events=None) -> rmm_options:
-    """An rmm_options struct; product_events = (begin, end) torch.cuda.Event pair (enable_timing)."""
+            debug_timeout_test: bool = False, gemm_producer: int = 0, attn_path: int = 0,
+            product_events=None) -> rmm_options:
+    """An rmm_options struct; product_events = (begin, end) torch.cuda.Event pair (enable_timing);
+    attn_path 0 = auto, 1 = CUDA-core split pass, 2 = tensor cores."""
     o = rmm_options(int(t_gemv), int(bool(attn_per_query_head)), int(gemv_splits),
-                    int(bool(debug_timeout_test)), int(gemm_producer), (ctypes.c_int * 3)(0, 0, 0),
+                    int(bool(debug_timeout_test)), int(gemm_producer), int(attn_path), (ctypes.c_int * 2)(0, 0),
                     None, None)
     if product_events is not None:
         b, e = product_events

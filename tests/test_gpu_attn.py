@@ -119,6 +119,30 @@ def test_attention_llama3_70b(rmm, T):
     check_large(rmm, 4, 1, 64, 8, T, 65536, 0.5, nrows=2)
 
 
+@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("B,T,L,r,causal,per_head", [
+    (1, 16, 16, 0.5, True, False),      # one ragged query tile, one key block
+    (2, 130, 300, 0.3, True, False),    # k = 39 (padded to 48 on the tensor cores), two query tiles
+    (1, 200, 200, 0.25, False, False),  # non-causal, ragged tile
+    (1, 129, 700, 1.0, True, True),     # all dims, per-query-head sets, chunk at the end of the cache
+    (1, 256, 1000, 0.5, True, False),   # key blocks past the diagonal and a ragged last key block
+])
+def test_attention_both_paths(rmm, path, B, T, L, r, causal, per_head):
+    """The tensor-core prefill kernel (path 2) and the CUDA-core split pass (path 1)
+    against the oracle on the same inputs."""
+    Hq, Hkv = 8, 2
+    seed = rmm_synth.seed_for(7, T, 5)
+    Q = rmm_synth.normal((B, Hq, T, D), seed)
+    K = rmm_synth.normal((B, Hkv, L, D), seed + 1)
+    V = rmm_synth.normal((B, Hkv, L, D), seed + 2)
+    opts = rmm.options(attn_per_query_head=per_head, attn_path=path)
+    O, idx, k = run_attn(rmm, Q, K, V, r, causal, per_head=per_head, opts=opts)
+    rows = sample_indices(T, 24, seed=T)
+    Oo, io = oracle.attention(Q, K, V, k, causal=causal, per_query_head=per_head, t_rows=rows)
+    assert np.array_equal(idx, io)
+    assert_close(O[:, :, rows], Oo, f"path={path} B={B} T={T} L={L} r={r} causal={causal}")
+
+
 def test_attention_rejects_bad_head_dim(rmm):
     L = rmm.lib()
     Q = torch.zeros(1, 2, 1, 64, dtype=torch.bfloat16, device="cuda")
