@@ -20,17 +20,19 @@
 // one query row).  TMEM holds two S buffers (columns 0-127, 128-255) and O
 // (256-383).
 //
-// Warp roles (256 threads):
-//   0-3  softmax: thread i owns query row t0 + i (TMEM lane i); reads S_j,
+// Warp roles (384 threads):
+//   0-7  softmax: warps q and q+4 own query rows 32q .. 32q+31 (their TMEM
+//        lanes), one row per thread, and split the 128 columns; reads S_j,
 //        masks, keeps a running reference max m and sum l; P_j to shared
 //        memory.  O is rescaled in TMEM only when a row's block max exceeds m
 //        by more than 2^8 (the reference max is then raised), so P stays below
 //        256 and most blocks need no rescale.  At the end O / l goes to HBM.
-//   4    MMA: one thread issues S_{j+1} before P_j V_j so the tensor pipe
-//        overlaps the softmax; tcgen05.commit releases buffers.
-//   5-7  producers: the query tile once (kept dims gathered), then per key
+//   8    MMA: one thread keeps two S blocks ahead of the softmax and issues
+//        P_j V_j as soon as P_j is written; tcgen05.commit releases buffers.
+//   9-11 producers: the query tile once (kept dims gathered), then per key
 //        block the kp kept rows of K^T and 128 rows of V with 16-byte
-//        cp.async (zero-filled past the valid keys), two stages.
+//        cp.async (zero-filled past the valid keys), three stages (two when
+//        128 kept dims leave no room).
 // Every wait is bounded: on expiry the kernel records RMM_ERR_TIMEOUT, every
 // role leaves its loop, in-flight tensor-core work drains, TMEM is freed.
 #include <math.h>
@@ -45,12 +47,13 @@ namespace {
 constexpr int D = 128;
 constexpr int BQ = 128;   // query rows per CTA (= TMEM lanes)
 constexpr int BKV = 128;  // keys per block
-constexpr int KV_STAGES = 2;
-constexpr int kSoftmaxThreads = 128;
-constexpr int kMmaWarp = 4;
-constexpr int kProdWarps = 3;  // 8 warps in all: two per SM sub-partition, so a thread may hold 255 registers
+constexpr int KV_STAGES_MAX = 3;  // key/value stages: 3 when they fit (kp <= 96), else 2
+constexpr int kSoftmaxWarps = 8;  // two per TMEM lane quarter, each on 64 of the 128 columns
+constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+constexpr int kMmaWarp = kSoftmaxWarps;
+constexpr int kProdWarps = 3;
 constexpr int kProdThreads = 32 * kProdWarps;
-constexpr int kThreadsTc = 32 * (4 + 1 + kProdWarps);
+constexpr int kThreadsTc = 32 * (kSoftmaxWarps + 1 + kProdWarps);  // 12 warps: three per SM sub-partition
 constexpr int V_CHUNK = BKV * 128;     // 64 dims x 128 key rows (bytes)
 constexpr int V_BYTES = 2 * V_CHUNK;   // 32 KB
 constexpr int P_ATOM = BQ * 128;       // 128 rows x 64 keys (bytes)
@@ -61,14 +64,15 @@ constexpr float kRescaleLog2 = 8.0f;   // rescale O when a block max exceeds the
 
 struct __align__(8) Bars {
     uint64_t q_full;
-    uint64_t kv_full[KV_STAGES];
-    uint64_t kv_empty[KV_STAGES];
+    uint64_t kv_full[KV_STAGES_MAX];
+    uint64_t kv_empty[KV_STAGES_MAX];
     uint64_t s_full[2];
     uint64_t s_empty[2];
     uint64_t p_full;
     uint64_t p_empty;
     uint64_t o_full;
     uint64_t drain;
+    uint64_t pair[4];  // per TMEM lane quarter: the two softmax warps on those rows meet here
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -87,70 +91,61 @@ __device__ __forceinline__ uint32_t swz(int j, int c16, int chunk) {
     return (uint32_t)((c16 >> 3) * chunk + j * 128 + (((c16 & 7) ^ (j & 7)) << 4));
 }
 
-// Softmax pass 1 for one row of a key block: the max of the raw logits
-// (scale > 0) in 8 independent chains, 64 TMEM columns per round trip.
-// kMask: keys past the cache end or (causal) past the row's position count as -inf.
+// Softmax pass 1 for one row and 64 columns (col0 .. col0+63) of a key block:
+// the max of the raw logits (scale > 0) in 8 independent chains.  kMask: keys
+// past the cache end or (causal) past the row's position count as -inf.
 template <bool kMask>
-__device__ __forceinline__ float row_max(uint32_t srow, int kb0, int L, int causal, int pos) {
+__device__ __forceinline__ float row_max64(uint32_t scol, int key0, int L, int causal, int pos) {
+    uint32_t r[2][32];
+    tmem_ld_32x32b_x32(scol, r[0]);
+    tmem_ld_32x32b_x32(scol + 32, r[1]);
+    tmem_ld_wait();
     float mx[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        uint32_t r[2][32];
-        tmem_ld_32x32b_x32(srow + hh * 64, r[0]);
-        tmem_ld_32x32b_x32(srow + hh * 64 + 32, r[1]);
-        tmem_ld_wait();
+    for (int q = 0; q < 2; ++q)
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                float x = __uint_as_float(r[q][c]);
-                if (kMask) {
-                    const int key = kb0 + hh * 64 + q * 32 + c;
-                    if (!(key < L && (!causal || key <= pos))) x = -INFINITY;
-                }
-                mx[c & 7] = fmaxf(mx[c & 7], x);
+        for (int c = 0; c < 32; ++c) {
+            float x = __uint_as_float(r[q][c]);
+            if (kMask) {
+                const int key = key0 + q * 32 + c;
+                if (!(key < L && (!causal || key <= pos))) x = -INFINITY;
             }
-    }
+            mx[c & 7] = fmaxf(mx[c & 7], x);
+        }
     return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
 }
 
-// Softmax pass 2: p = 2^(s * scale_log2 - m) (one FMA and one hardware exp2;
-// masked logits give 0), the row sum, and P (bf16) written as the K-major A
-// operand: row i at prow, keys in two 64-key atoms, 16-byte chunks
+// Softmax pass 2 for the same 64 columns: p = 2^(s * scale_log2 - m) (one FMA
+// and one hardware exp2; masked logits give 0), their sum, and P (bf16) as
+// one 64-key atom of the K-major A operand: row i at prow, 16-byte chunks
 // XOR-swizzled by row.
 template <bool kMask>
-__device__ __forceinline__ float row_exp(uint32_t srow, int kb0, int L, int causal, int pos, float scale_log2,
-                                         float neg_m, uint32_t prow, int i) {
+__device__ __forceinline__ float row_exp64(uint32_t scol, int key0, int L, int causal, int pos, float scale_log2,
+                                           float neg_m, uint32_t prow, int i) {
+    uint32_t r[2][32];
+    tmem_ld_32x32b_x32(scol, r[0]);
+    tmem_ld_32x32b_x32(scol + 32, r[1]);
+    tmem_ld_wait();
     float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        uint32_t r[2][32];
-        tmem_ld_32x32b_x32(srow + hh * 64, r[0]);
-        tmem_ld_32x32b_x32(srow + hh * 64 + 32, r[1]);
-        tmem_ld_wait();
-        float pv[64];
+    for (int c8 = 0; c8 < 8; ++c8) {
+        float p[8];
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                float p = fast_exp2(fmaf(__uint_as_float(r[q][c]), scale_log2, neg_m));
-                if (kMask) {
-                    const int key = kb0 + hh * 64 + q * 32 + c;
-                    if (!(key < L && (!causal || key <= pos))) p = 0.0f;
-                }
-                pv[q * 32 + c] = p;
-                sm[c & 7] += p;
+        for (int e = 0; e < 8; ++e) {
+            const int c = c8 * 8 + e;
+            float v = fast_exp2(fmaf(__uint_as_float(r[c >> 5][c & 31]), scale_log2, neg_m));
+            if (kMask) {
+                const int key = key0 + c;
+                if (!(key < L && (!causal || key <= pos))) v = 0.0f;
             }
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-            const uint4 w = make_uint4(pack_bf16x2(pv[c8 * 8 + 0], pv[c8 * 8 + 1]),
-                                       pack_bf16x2(pv[c8 * 8 + 2], pv[c8 * 8 + 3]),
-                                       pack_bf16x2(pv[c8 * 8 + 4], pv[c8 * 8 + 5]),
-                                       pack_bf16x2(pv[c8 * 8 + 6], pv[c8 * 8 + 7]));
-            st_shared_v4(prow + hh * P_ATOM + ((c8 ^ (i & 7)) << 4), w);
+            p[e] = v;
+            sm[e] += v;
         }
+        const uint4 w = make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
+                                   pack_bf16x2(p[6], p[7]));
+        st_shared_v4(prow + ((c8 ^ (i & 7)) << 4), w);
     }
     return ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
 }
@@ -163,13 +158,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     const int QK_BYTES = kp * 256;  // a gathered query tile or key block
+    const int ks = kp <= 96 ? 3 : 2;   // key/value stages
     uint8_t* sP = smem;                                   // 32 KB (1024-aligned)
-    uint8_t* sV = sP + P_BYTES;                           // KV_STAGES x 32 KB
-    uint8_t* sQ = sV + KV_STAGES * V_BYTES;               // kp x 256
-    uint8_t* sK = sQ + QK_BYTES;                          // KV_STAGES x kp x 256
-    int* sidx = reinterpret_cast<int*>(sK + KV_STAGES * QK_BYTES);  // kp kept dims
+    uint8_t* sV = sP + P_BYTES;                           // ks x 32 KB
+    uint8_t* sQ = sV + ks * V_BYTES;                      // kp x 256
+    uint8_t* sK = sQ + QK_BYTES;                          // ks x kp x 256
+    int* sidx = reinterpret_cast<int*>(sK + ks * QK_BYTES);  // kp kept dims
     Bars* bars = reinterpret_cast<Bars*>(sidx + D);
     volatile int* abort_flag = &bars->abort_flag;
+    __shared__ float red_max[2][2][BQ];  // [block parity][half][row]: the halves' row maxima
+    __shared__ float red_sum[2][BQ];     // [half][row]: the halves' row sums at the end
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_tiles = (T + BQ - 1) / BQ;
@@ -187,7 +185,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 
     if (tid == 0) {
         mbar_init(smem_addr(&bars->q_full), kProdThreads);
-        for (int s = 0; s < KV_STAGES; ++s) {
+        for (int s = 0; s < ks; ++s) {
             mbar_init(smem_addr(&bars->kv_full[s]), kProdThreads);
             mbar_init(smem_addr(&bars->kv_empty[s]), 1);
         }
@@ -199,6 +197,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         mbar_init(smem_addr(&bars->p_empty), 1);
         mbar_init(smem_addr(&bars->o_full), 1);
         mbar_init(smem_addr(&bars->drain), 1);
+        for (int q = 0; q < 4; ++q) mbar_init(smem_addr(&bars->pair[q]), 64);
         bars->abort_flag = 0;
         fence_mbar_init();
     }
@@ -247,8 +246,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         const uint16_t* Kg = Kt + ((size_t)b * Hkv + g) * D * ldL;
         const uint16_t* Vg = V + ((size_t)b * Hkv + g) * ldL * D;
         for (int j = 0; j < nkb; ++j) {
-            const int s = j % KV_STAGES;
-            const uint32_t ph = (uint32_t)(j / KV_STAGES) & 1u;
+            const int s = j % ks;
+            const uint32_t ph = (uint32_t)(j / ks) & 1u;
             if (!mbar_wait(smem_addr(&bars->kv_empty[s]), ph ^ 1u, status, abort_flag)) break;
             const int kb0 = j * BKV;
             const uint32_t kst = smem_addr(sK + s * QK_BYTES), vst = smem_addr(sV + s * V_BYTES);
@@ -276,46 +275,48 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         const uint32_t qbase = smem_addr(sQ);
         fence_proxy_async_smem();
         tc_fence_after();
-        for (int j = 0; ok && j <= nkb; ++j) {
-            if (j < nkb) {
-                const int s = j % KV_STAGES, sb = j & 1;
-                bool got = mbar_wait(smem_addr(&bars->kv_full[s]), (uint32_t)(j / KV_STAGES) & 1u, status, abort_flag);
-                got = got && mbar_wait(smem_addr(&bars->s_empty[sb]), ((uint32_t)(j >> 1) & 1u) ^ 1u, status, abort_flag);
-                if (!__all_sync(0xffffffffu, got)) {  // the warp leaves together
-                    ok = false;
-                    break;
-                }
-                fence_proxy_async_smem();  // the producers' cp.async data, read by the tensor cores
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t kbase = smem_addr(sK + s * QK_BYTES);
-                    for (int kk = 0; kk < kp / 16; ++kk)
-                        umma_f16(tmem + TM_S0 + sb * BKV, smem_desc_sw128(qbase + kk * 2048, kp * 128, 1024),
-                                 smem_desc_sw128(kbase + kk * 2048, kp * 128, 1024), idesc_s, kk > 0 ? 1u : 0u);
-                    umma_commit(smem_addr(&bars->s_full[sb]));
-                }
-                __syncwarp();
+        // S_j into TMEM buffer j & 1, once block j has landed and the softmax has
+        // read S_{j-2} from that buffer
+        auto issue_s = [&](int j) -> bool {
+            const int s = j % ks, sb = j & 1;
+            bool got = mbar_wait(smem_addr(&bars->kv_full[s]), (uint32_t)(j / ks) & 1u, status, abort_flag);
+            got = got && mbar_wait(smem_addr(&bars->s_empty[sb]), ((uint32_t)(j >> 1) & 1u) ^ 1u, status, abort_flag);
+            if (!__all_sync(0xffffffffu, got)) return false;  // the warp leaves together
+            fence_proxy_async_smem();  // the producers' cp.async data, read by the tensor cores
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t kbase = smem_addr(sK + s * QK_BYTES);
+                for (int kk = 0; kk < kp / 16; ++kk)
+                    umma_f16(tmem + TM_S0 + sb * BKV, smem_desc_sw128(qbase + kk * 2048, kp * 128, 1024),
+                             smem_desc_sw128(kbase + kk * 2048, kp * 128, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                umma_commit(smem_addr(&bars->s_full[sb]));
             }
-            if (j >= 1) {
-                const int jp = j - 1, sp = jp % KV_STAGES;
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars->p_full), (uint32_t)jp & 1u, status, abort_flag))) {
-                    ok = false;
-                    break;
-                }
-                fence_proxy_async_smem();  // P written by the softmax threads
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t pbase = smem_addr(sP), vbase = smem_addr(sV + sp * V_BYTES);
+            __syncwarp();
+            return true;
+        };
+        // two S blocks ahead; then, per block, P_j V_j as soon as P_j is written and
+        // S_{j+2} after it, so a late key block never holds back a ready P.V
+        if (ok && nkb > 0) ok = issue_s(0);
+        if (ok && nkb > 1) ok = issue_s(1);
+        for (int j = 0; ok && j < nkb; ++j) {
+            const int sp = j % ks;
+            if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars->p_full), (uint32_t)j & 1u, status, abort_flag))) {
+                ok = false;
+                break;
+            }
+            fence_proxy_async_smem();  // P written by the softmax threads
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t pbase = smem_addr(sP), vbase = smem_addr(sV + sp * V_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < BKV / 16; ++kk)
-                        umma_f16(tmem + TM_O, smem_desc_sw128(pbase + (kk >> 2) * P_ATOM + (kk & 3) * 32, 16, 1024),
-                                 smem_desc_sw128(vbase + kk * 2048, V_CHUNK, 1024), idesc_pv,
-                                 (jp > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(smem_addr(&bars->p_empty));
-                    umma_commit(smem_addr(&bars->kv_empty[sp]));
-                }
-                __syncwarp();
+                for (int kk = 0; kk < BKV / 16; ++kk)
+                    umma_f16(tmem + TM_O, smem_desc_sw128(pbase + (kk >> 2) * P_ATOM + (kk & 3) * 32, 16, 1024),
+                             smem_desc_sw128(vbase + kk * 2048, V_CHUNK, 1024), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(smem_addr(&bars->p_empty));
+                umma_commit(smem_addr(&bars->kv_empty[sp]));
             }
+            __syncwarp();
+            if (j + 2 < nkb) ok = issue_s(j + 2);
         }
         if (lane == 0) {
             if (ok) umma_commit(smem_addr(&bars->o_full));
@@ -328,11 +329,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         mbar_wait(smem_addr(&bars->drain), 0, status, &no_abort, kWaitLimitNs);
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        const int i = tid;  // query row inside the tile = TMEM lane
+        // warps q and q + 4 share TMEM lanes 32q .. 32q+31 (query rows) and take
+        // columns 0-63 and 64-127 of S, of P (one atom each) and of O; the row max
+        // is combined through shared memory with one barrier per pair and block,
+        // the row sums are kept per half and added at the end
+        const int quarter = warp & 3, half = warp >> 2;
+        const int i = quarter * 32 + lane;  // query row inside the tile = TMEM lane
         const int t = t0 + i;
         const int pos = L - T + t;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        float m_use = -INFINITY, l_sum = 0.0f;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t pair_mb = smem_addr(&bars->pair[quarter]);  // the two warps on these rows
+        int pair_phase = 0;
+        float m_use = -INFINITY, l_half = 0.0f;
         bool ok = true;
         for (int j = 0; j < nkb; ++j) {
             const int sb = j & 1;
@@ -344,13 +352,20 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 break;
             }
             tc_fence_after();
-            const int kb0 = j * BKV;
+            const int key0 = j * BKV + half * 64;
             // mask only where the warp's rows cross the diagonal or the cache end
-            const bool full =
-                __all_sync(0xffffffffu, kb0 + BKV - 1 < L && (!causal || kb0 + BKV - 1 <= pos));
-            const uint32_t srow = tmem + lane_base + TM_S0 + sb * BKV;
-            const float m_blk = (full ? row_max<false>(srow, kb0, L, causal, pos)
-                                      : row_max<true>(srow, kb0, L, causal, pos)) * scale_log2;
+            const bool full = __all_sync(0xffffffffu, key0 + 63 < L && (!causal || key0 + 63 <= pos));
+            const uint32_t scol = tmem + lane_base + TM_S0 + sb * BKV + half * 64;
+            const float m_mine = full ? row_max64<false>(scol, key0, L, causal, pos)
+                                      : row_max64<true>(scol, key0, L, causal, pos);
+            red_max[j & 1][half][i] = m_mine;
+            // meet the partner warp (bounded, like every wait here)
+            mbar_arrive(pair_mb);
+            if (!__all_sync(0xffffffffu, mbar_wait(pair_mb, (uint32_t)(pair_phase++) & 1u, status, abort_flag))) {
+                ok = false;
+                break;
+            }
+            const float m_blk = fmaxf(m_mine, red_max[j & 1][half ^ 1][i]) * scale_log2;
             const bool resc = m_blk > m_use + kRescaleLog2;
             const float m_new = resc ? m_blk : m_use;
             const float alpha = resc ? exp2f(m_use - m_new) : 1.0f;  // exp2(-inf) = 0 on the first block
@@ -364,35 +379,41 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             tc_fence_after();
             if (j > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 2; ++q) {
                     uint32_t o[32];
-                    tmem_ld_32x32b_x32(tmem + lane_base + TM_O + q * 32, o);
+                    const uint32_t oc = tmem + lane_base + TM_O + half * 64 + q * 32;
+                    tmem_ld_32x32b_x32(oc, o);
                     tmem_ld_wait();
 #pragma unroll
                     for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                    tmem_st_32x32b_x32(tmem + lane_base + TM_O + q * 32, o);
+                    tmem_st_32x32b_x32(oc, o);
                 }
                 tmem_st_wait();
             }
             m_use = m_new;
-            const uint32_t prow = smem_addr(sP) + i * 128;
-            const float rs = full ? row_exp<false>(srow, kb0, L, causal, pos, scale_log2, neg_m, prow, i)
-                                  : row_exp<true>(srow, kb0, L, causal, pos, scale_log2, neg_m, prow, i);
+            const uint32_t prow = smem_addr(sP) + half * P_ATOM + i * 128;
+            const float rs = full ? row_exp64<false>(scol, key0, L, causal, pos, scale_log2, neg_m, prow, i)
+                                  : row_exp64<true>(scol, key0, L, causal, pos, scale_log2, neg_m, prow, i);
             tc_fence_before();
             mbar_arrive(smem_addr(&bars->s_empty[sb]));  // S_j fully read
-            l_sum = l_sum * alpha + rs;
+            l_half = l_half * alpha + rs;
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(smem_addr(&bars->p_full));
         }
-        if (ok && __all_sync(0xffffffffu, mbar_wait(smem_addr(&bars->o_full), 0, status, abort_flag))) {
+        const bool done = ok && __all_sync(0xffffffffu, mbar_wait(smem_addr(&bars->o_full), 0, status, abort_flag));
+        // the two halves' row sums
+        red_sum[half][i] = l_half;
+        mbar_arrive(pair_mb);
+        const bool met = __all_sync(0xffffffffu, mbar_wait(pair_mb, (uint32_t)pair_phase & 1u, status, abort_flag));
+        if (done && met) {
             tc_fence_after();
-            const float inv = 1.0f / l_sum;
-            uint16_t* orow = O + (((size_t)b * Hq + h) * T + (t < T ? t : 0)) * D;
+            const float inv = 1.0f / (red_sum[0][i] + red_sum[1][i]);
+            uint16_t* orow = O + (((size_t)b * Hq + h) * T + (t < T ? t : 0)) * D + half * 64;
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
                 uint32_t o[32];
-                tmem_ld_32x32b_x32(tmem + lane_base + TM_O + q * 32, o);
+                tmem_ld_32x32b_x32(tmem + lane_base + TM_O + half * 64 + q * 32, o);
                 tmem_ld_wait();
                 if (t < T) {
 #pragma unroll
@@ -416,8 +437,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 }
 
 size_t attn_tc_smem_bytes(int kp) {
-    return 1024 + P_BYTES + (size_t)KV_STAGES * V_BYTES + (size_t)(1 + KV_STAGES) * kp * 256 + D * sizeof(int) +
-           sizeof(Bars);
+    const int ks = kp <= 96 ? 3 : 2;
+    return 1024 + P_BYTES + (size_t)ks * V_BYTES + (size_t)(1 + ks) * kp * 256 + D * sizeof(int) + sizeof(Bars);
 }
 
 }  // namespace
