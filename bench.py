@@ -40,6 +40,10 @@ from input_adaptive_reduced_rmm_b200 import metrics  # noqa: E402
 
 T_PREFILL = 2048
 R = 0.5
+# DRAM bytes (read + write) of one step's four GEMM launches from one ncu capture of
+# this kernel (profiles/gemm_pair_step_traffic_llama3_8b_T2048_r0.5.md); set to None
+# whenever the GEMM kernel changes until it is captured again.
+STEP_GEMM_DRAM_BYTES = 363_977_216
 PROJ = [  # (name, H, N, activation stream)
     ("q", 4096, 4096, 0), ("k", 4096, 1024, 0), ("v", 4096, 1024, 0), ("o", 4096, 4096, 1),
     ("gate", 4096, 14336, 2), ("up", 4096, 14336, 2), ("down", 14336, 4096, 3),
@@ -554,8 +558,9 @@ def run_rmm(args, world, rank, local):
                    "calls_per_step": "q+k+v grouped, o, gate+up grouped, down",
                    "l2": "inputs larger than L2 (0.55 GB of weights and activations per step)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
-                     "kernel": "gemm_kernel (tcgen05 reduced GEMM), the 4 launches of a step",
+                     "frac": achieved / peak, "traffic": STEP_GEMM_DRAM_BYTES,
+                     "traffic_unit": "bytes (ncu dram read + write) over the step's 4 GEMM launches",
+                     "kernel": "gemm_pair_kernel (tcgen05 cta_group::2 reduced GEMM), the 4 launches of a step",
                      "peak_source": f"{peaks['source']} bf16 burst"},
         "speedup_vs_dense": dense_ms / (ms_max / K),
         "dense": {"ms_per_step": dense_ms, "tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
