@@ -130,26 +130,29 @@ EncodeTiledFn encode_fn() {
 
 struct MapKey {
     const void* ptr;
-    uint64_t rows, cols, ld;
+    uint64_t rows, cols, ld, box_rows;
     bool operator==(const MapKey& o) const {
-        return ptr == o.ptr && rows == o.rows && cols == o.cols && ld == o.ld;
+        return ptr == o.ptr && rows == o.rows && cols == o.cols && ld == o.ld && box_rows == o.box_rows;
     }
 };
 struct MapKeyHash {
     size_t operator()(const MapKey& k) const {
         size_t h = std::hash<const void*>()(k.ptr);
-        h ^= std::hash<uint64_t>()(k.rows * 1000003ull + k.cols * 7919ull + k.ld) + 0x9e3779b9 + (h << 6) + (h >> 2);
+        h ^= std::hash<uint64_t>()(k.rows * 1000003ull + k.cols * 7919ull + k.ld * 31ull + k.box_rows) + 0x9e3779b9 +
+             (h << 6) + (h >> 2);
         return h;
     }
 };
 
-// A row-gather map over a bf16 matrix [rows, cols] (leading dimension ld
-// elements): box = 1 row x 64 columns, 128-byte swizzle, out-of-range
-// elements read as zero.  Cached by (pointer, shape).
-bool row_gather_map(const void* base, uint64_t rows, uint64_t cols, uint64_t ld, CUtensorMap* out) {
+// A tiled map over a bf16 matrix [rows, cols] (leading dimension ld elements):
+// box = box_rows rows x 64 columns (128 bytes), 128-byte swizzle; loads read
+// zeros and stores skip elements outside the matrix.  Cached by (pointer,
+// shape, box).  box_rows 1 is the row-gather map of the TMA producer; 32 the
+// output tile of one GEMM epilogue warp.
+bool tiled_map(const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows, CUtensorMap* out) {
     static std::mutex mu;
     static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
-    const MapKey key{base, rows, cols, ld};
+    const MapKey key{base, rows, cols, ld, box_rows};
     {
         std::lock_guard<std::mutex> g(mu);
         auto it = cache.find(key);
@@ -164,7 +167,7 @@ bool row_gather_map(const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
     memset(&m, 0, sizeof m);
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {ld * sizeof(uint16_t)};
-    const cuuint32_t box[2] = {64, 1};
+    const cuuint32_t box[2] = {64, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -178,6 +181,10 @@ bool row_gather_map(const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
 }
 
 rmm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RMM_OK : RMM_ERR_CUDA; }
+
+bool row_gather_map(const void* base, uint64_t rows, uint64_t cols, uint64_t ld, CUtensorMap* out) {
+    return tiled_map(base, rows, cols, ld, 1, out);
+}
 
 bool group_args_ok(const void* X, int T, int H, int count, const void* const* Wts, const int* Ns,
                    void* const* Ys) {
@@ -218,7 +225,11 @@ rmm_status run_product_kernels(const void* X, int T, int H, int count, const voi
     }
     if (o.gemm_producer == 0) {  // default: CTA-pair tcgen05 GEMM
         gemm_group_tiles(g, T, 1);
-        return cuda_status(launch_gemm_pair(reinterpret_cast<const uint16_t*>(ws + L.xt), L.ldT, g, idx_padded,
+        GemmOutMaps ym;
+        memset(&ym, 0, sizeof ym);
+        for (int p = 0; p < count; ++p)
+            if (!tiled_map(Ys[p], (uint64_t)T, (uint64_t)Ns[p], (uint64_t)Ns[p], 32, &ym.m[p])) return RMM_ERR_CUDA;
+        return cuda_status(launch_gemm_pair(reinterpret_cast<const uint16_t*>(ws + L.xt), L.ldT, g, ym, idx_padded,
                                             k, T, H, reinterpret_cast<float*>(ws + L.partials), status,
                                             o.debug_timeout_test, sms, s));
     }

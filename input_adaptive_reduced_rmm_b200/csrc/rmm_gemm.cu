@@ -471,7 +471,8 @@ __device__ __forceinline__ Unit decode_unit(const GemmGroup& g, int u, int m_til
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     gemm_pair_kernel(const uint16_t* __restrict__ Xt, int ldT, const __grid_constant__ GemmGroup group,
-                     const int32_t* __restrict__ idx, int k, int T, int H, int* status, int debug_timeout) {
+                     const __grid_constant__ GemmOutMaps ymaps, const int32_t* __restrict__ idx, int k, int T,
+                     int H, int* status, int debug_timeout) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -709,7 +710,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
             for (int c64 = c64_begin; c64 < c64_begin + TMEM_COLS2 / 128; ++c64) {
                 const int c = c64 * 64;
                 const int lcol = 256 * ((c & 255) >> 7) + 128 * (c >> 8) + (c & 127);  // column inside the tile
-                if (ux.part < 0) __syncwarp();  // the previous block's reads of the staging area are done
+                if (ux.part < 0) {
+                    // the previous block's TMA store has finished reading the staging area
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+                }
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     uint32_t r[32];
@@ -741,14 +746,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
                     }
                 }
                 if (ux.part < 0) {
-                    // then 4 full 128-byte row segments per store instruction
+                    // the staged 32 x 64 block goes out as one TMA tile store (rows past
+                    // T and columns past N are clipped by the map)
+                    fence_proxy_async_smem();
                     __syncwarp();
-#pragma unroll
-                    for (int it = 0; it < 8; ++it) {
-                        const int rr = it * 4 + (lane >> 3), ch = lane & 7;
-                        const uint4 o = ld_shared_v4(stg + rr * 128 + ((ch ^ (rr & 7)) << 4));
-                        const int row = rbase + rr, col = tc.n0 + lcol + ch * 8;
-                        if (row < T && col < N) *reinterpret_cast<uint4*>(Y + (size_t)row * N + col) = o;
+                    if (lane == 0) {
+                        tma_store_2d(&ymaps.m[tc.p], stg, tc.n0 + lcol, rbase);
+                        bulk_commit();
                     }
                 }
             }
@@ -757,6 +761,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
             if (lane == 0) mbar_arrive_cluster(tempty_leader);
             acc_phase ^= 1;
         }
+        if (lane == 0) bulk_wait_all();  // this warp's tile stores have completed
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -844,9 +850,9 @@ size_t gemm_pair_partial_bytes(int num_sms) {
 // partial wave are each cut into s = min(pairs / R, 8) K-ranges (at least one
 // K-block each), so that wave takes about 1/s of a tile's time instead of a
 // whole one.
-cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group, const int32_t* idx,
-                             int k, int T, int H, float* partials, int* status, int debug_timeout, int num_sms,
-                             cudaStream_t stream) {
+cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group, const GemmOutMaps& ymaps,
+                             const int32_t* idx, int k, int T, int H, float* partials, int* status,
+                             int debug_timeout, int num_sms, cudaStream_t stream) {
     if (group.count < 1 || group.count > kMaxGroup) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem_limit(pair::gemm_pair_kernel, pair::kSmemBytes2);
     if (e != cudaSuccess) return e;
@@ -873,7 +879,7 @@ cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group
     int clusters = pairs < g.units ? pairs : g.units;
     if (clusters < 1) clusters = 1;
     e = launch_pdl(pair::gemm_pair_kernel, dim3(2 * clusters), dim3(pair::kThreads2), pair::kSmemBytes2, stream, Xt, ldT,
-                   g, idx, k, T, H, status, debug_timeout);
+                   g, ymaps, idx, k, T, H, status, debug_timeout);
     if (e != cudaSuccess || g.tail_splits == 1) return e;
     return launch_pdl(pair::gemm_fold_kernel, dim3(R * (pair::BM2 / 4)), dim3(256), 0, stream, g, T);
 }

@@ -98,9 +98,14 @@ int gemm_group_tiles(GemmGroup& g, int T, int pair);
 // CTA-pair (tcgen05 cta_group::2) GEMM, cp.async producer; tiles from gemm_group_tiles(g, T, 1).
 // partials: gemm_pair_partial_bytes(num_sms) of scratch for the split last
 // wave (null: no split).
-cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group, const int32_t* idx,
-                             int k, int T, int H, float* partials, int* status, int debug_timeout, int num_sms,
-                             cudaStream_t stream);
+// Output tensor maps of the group's products (Y [T, N] bf16, box 32 rows x 64
+// columns, 128-byte swizzle): the epilogue stores its tiles with TMA.
+struct __align__(64) GemmOutMaps {
+    CUtensorMap m[kMaxGroup];
+};
+cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group, const GemmOutMaps& ymaps,
+                             const int32_t* idx, int k, int T, int H, float* partials, int* status,
+                             int debug_timeout, int num_sms, cudaStream_t stream);
 size_t gemm_pair_partial_bytes(int num_sms);
 // map_xt / map_wt are used only by the TMA tile::gather4 producer
 // (tma_gather != 0), which handles a group of one.
