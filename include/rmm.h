@@ -86,7 +86,8 @@ typedef struct rmm_options {
     /* Optional pair of cudaEvent_t handles (NULL: none) recorded on the
      * stream immediately before and after the reduced-product kernel (GEMV or
      * GEMM) of rmm_linear / rmm_gemm_reduced, so that a caller can time that
-     * kernel alone inside a longer sequence of calls. */
+     * kernel alone inside a longer sequence of calls.  During CUDA-graph
+     * capture they are recorded as external event nodes of the graph. */
     void* product_event_begin;
     void* product_event_end;
 } rmm_options;

@@ -246,15 +246,23 @@ rmm_status run_product_kernels(const void* X, int T, int H, int count, const voi
                                    o.debug_timeout_test, o.gemm_producer == 1, sms, s));
 }
 
+// Records a caller's timing event; while the stream is being captured into a
+// CUDA graph the record becomes an event node of the graph (so a replay times
+// the product kernels too).
+cudaError_t record_product_event(void* ev, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return cudaErrorUnknown;
+    return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev), s,
+                                    cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal
+                                                                        : cudaEventRecordDefault);
+}
+
 rmm_status run_products(const void* X, int T, int H, int count, const void* const* Wts, const int* Ns,
                         void* const* Ys, const int32_t* idx_padded, int k, uint8_t* ws,
                         const LinearLayout& L, const rmm_options& o, cudaStream_t s) {
-    if (o.product_event_begin &&
-        cudaEventRecord(static_cast<cudaEvent_t>(o.product_event_begin), s) != cudaSuccess)
-        return RMM_ERR_CUDA;
+    if (o.product_event_begin && record_product_event(o.product_event_begin, s) != cudaSuccess) return RMM_ERR_CUDA;
     rmm_status st = run_product_kernels(X, T, H, count, Wts, Ns, Ys, idx_padded, k, ws, L, o, s);
-    if (st == RMM_OK && o.product_event_end &&
-        cudaEventRecord(static_cast<cudaEvent_t>(o.product_event_end), s) != cudaSuccess)
+    if (st == RMM_OK && o.product_event_end && record_product_event(o.product_event_end, s) != cudaSuccess)
         return RMM_ERR_CUDA;
     return st;
 }

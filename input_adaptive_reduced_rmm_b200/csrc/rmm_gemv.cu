@@ -13,14 +13,15 @@
 // into column blocks of COLS (256 for T <= 4, narrower for wider T).  One CTA =
 // (member, column block) along x, split along y; x varies fastest, so the CTAs
 // running at the same moment read neighbouring 512-byte pieces of the same
-// kept rows.  S is chosen for ~6 CTAs per SM in several waves: measured on
-// B200, a streaming grid of that shape sustains ~5.5 TB/s on scattered kept
-// rows, while fewer, longer-running CTAs lose to ramp-up and ramp-down.
+// kept rows.  S gives a grid of ~6 CTAs per SM (~12 above 100 MB of kept
+// weights) in several waves: measured on B200, such grids sustain 5.4-5.8
+// TB/s on scattered kept rows, while fewer, longer-running CTAs lose to
+// ramp-up and ramp-down and shorter ones to their set-up.
 //
 // A CTA stages its split's kept indices in shared memory, issues its first
 // batch of weight loads and only then gathers the X values beside them, so
 // both latencies overlap; it streams 16-byte pieces of the kept rows with
-// non-allocating loads (8 or 4 rows in flight per thread, packed fp32x2 FMAs),
+// non-allocating loads (16, 8 or 4 rows in flight per thread, packed fp32x2 FMAs),
 // folds its row groups (shuffles, then the warps in a fixed order) and writes
 // its fp32 partial sums -- or, with one split, Y itself.  A second launch,
 // chained by programmatic dependent launch, adds the S partials of every
@@ -93,13 +94,12 @@ __device__ __forceinline__ int member_of(const int* start, int count, int x) {
     return p;
 }
 
-template <int TT, int COLS>
+template <int TT, int COLS, int U>
 __global__ void __launch_bounds__(kThreads, (TT <= 4) ? 3 : 1)
     gemv_kernel(const uint16_t* __restrict__ X, int T, int H, const int32_t* __restrict__ idx, int k,
                 const __grid_constant__ GemvGroup g, float* __restrict__ partials) {
     constexpr int TPR = COLS / 8;         // threads per kept-row piece
     constexpr int RG = kThreads / TPR;    // row groups
-    constexpr int U = (TT >= 8) ? 4 : 8;  // kept rows in flight per thread
     constexpr int WCOLS = (COLS < 256) ? COLS : 256;  // columns held by one warp after its shuffle fold
     constexpr int P8 = COLS / 8;
 
@@ -281,7 +281,10 @@ cudaError_t launch_tt(const uint16_t* X, int T, int H, const int32_t* idx, int k
     constexpr int COLS = TT <= 4 ? 256 : TT <= 8 ? 128 : 64;  // gemv_cols_for
     if (g.cols != COLS) return cudaErrorInvalidValue;
     const size_t smem = gemv_smem_bytes(COLS, T);
-    auto kern = gemv_kernel<TT, COLS>;
+    // kept rows in flight per thread: 16 for long splits of one or two tokens
+    constexpr int U_SHORT = TT >= 8 ? 4 : 8;
+    constexpr int U_LONG = TT <= 2 ? 16 : U_SHORT;
+    auto kern = g.rows_per_split[0] >= 192 ? gemv_kernel<TT, COLS, U_LONG> : gemv_kernel<TT, COLS, U_SHORT>;
     cudaError_t e = ensure_smem_limit(kern, smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3(g.item_start[g.count], g.splits[0]), dim3(kThreads), smem, stream, X, T, H, idx, k, g,
@@ -291,15 +294,24 @@ cudaError_t launch_tt(const uint16_t* X, int T, int H, const int32_t* idx, int k
                       static_cast<const float*>(partials));
 }
 
-// Splits before rounding to whole rows; never decreases as k grows.
+// Splits before rounding to whole rows; never decreases as k grows.  Measured
+// on B200 (one token, graph replays, kept rows scattered): a grid of ~6 CTAs
+// per SM streams best up to ~100 MB of kept weights (4096 -> 14336 at r=0.5:
+// 896 CTAs of 128 rows, 14.0 us) and ~12 per SM above (8192 -> 28672: 1792
+// CTAs of 256 rows, 40.7 us, 5.8 TB/s); fewer, longer CTAs lose to ramp-up and
+// ramp-down, more, shorter ones to their set-up.  At least 32 rows per split.
 int initial_splits(const GemvGroup& g, int T, int k, int forced_splits, int num_sms) {
     const int cols = gemv_cols_for(T);
     int blocks = 0;
-    for (int p = 0; p < g.count; ++p) blocks += (g.N[p] + cols - 1) / cols;
+    size_t n_total = 0;
+    for (int p = 0; p < g.count; ++p) {
+        blocks += (g.N[p] + cols - 1) / cols;
+        n_total += (size_t)g.N[p];
+    }
     if (blocks < 1) blocks = 1;
-    // ~6 CTAs per SM for decode sizes (several short waves), fewer for wide T
-    // where the split partials cost more; at least 32 kept rows each
-    const int target = num_sms * (T <= 4 ? 6 : 2);
+    const size_t kept_bytes = (size_t)k * n_total * 2;
+    const int per_sm = T <= 4 ? (kept_bytes > (size_t)100 << 20 ? 12 : 6) : 2;
+    const int target = num_sms * per_sm;
     int S = forced_splits > 0 ? forced_splits : (target + blocks - 1) / blocks;
     const int max_by_rows = (k + 31) / 32;
     if (forced_splits <= 0 && S > max_by_rows) S = max_by_rows;
