@@ -85,6 +85,26 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// 2^x on the FMA pipe, for x <= 8 (P's range): round-to-nearest range
+// reduction x = n + f, |f| <= 1/2, by adding 1.5 * 2^23 (the integer n lands
+// in the low mantissa bits); 2^f = e^(f ln 2) by its Taylor expansion to
+// degree 4 (remainder < 6e-5 relative for |f ln 2| <= 0.35, well below the
+// bf16 rounding of P); n is added to the exponent bits.  x below -126 is
+// clamped (2^-126 is zero for P's purposes).  Half of each row's
+// exponentials run here instead of on the special-function unit, whose
+// throughput otherwise bounds the softmax.
+__device__ __forceinline__ float poly_exp2(float x) {
+    x = fmaxf(x, -126.0f);
+    const float t = x + 12582912.0f;
+    const float f = x - (t - 12582912.0f);
+    float p = fmaf(f, 0.0096181291076285f, 0.0555041086648216f);
+    p = fmaf(p, f, 0.2402265069591007f);
+    p = fmaf(p, f, 0.6931471805599453f);
+    p = fmaf(p, f, 1.0f);
+    const int n = __float_as_int(t) - 0x4B400000;
+    return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
 // Byte offset of 16-byte chunk c16 (along M/N) of row j (along K) in the
 // 128-byte-swizzled MN-major layout whose 64-element groups are `chunk` apart.
 __device__ __forceinline__ uint32_t swz(int j, int c16, int chunk) {
@@ -135,7 +155,8 @@ __device__ __forceinline__ float row_exp64(uint32_t scol, int key0, int L, int c
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const int c = c8 * 8 + e;
-            float v = fast_exp2(fmaf(__uint_as_float(r[c >> 5][c & 31]), scale_log2, neg_m));
+            const float x = fmaf(__uint_as_float(r[c >> 5][c & 31]), scale_log2, neg_m);
+            float v = (e & 1) ? poly_exp2(x) : fast_exp2(x);
             if (kMask) {
                 const int key = key0 + c;
                 if (!(key < L && (!causal || key <= pos))) v = 0.0f;
