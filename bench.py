@@ -631,6 +631,40 @@ def run_single(args):
     print(json.dumps(out), flush=True)
 
 
+def run_single_attn(args):
+    """One rmm_attn_qk call timed alone (profiling aid): --single-attn B,Hq,Hkv,T,L,r (causal,
+    d = 128, queries at the last T positions of a cache of L keys)."""
+    from input_adaptive_reduced_rmm_b200 import rmm
+
+    B, Hq, Hkv, T, L, r = args.single_attn.split(",")
+    B, Hq, Hkv, T, L, r = int(B), int(Hq), int(Hkv), int(T), int(L), float(r)
+    dev = torch.device("cuda", 0)
+    D = 128
+    Q = rmm_synth.normal((B, Hq, T, D), 21).to(dev)
+    Kt = rmm_synth.normal((B, Hkv, D, L), 22).to(dev)
+    V = rmm_synth.normal((B, Hkv, L, D), 23).to(dev)
+    O = torch.empty_like(Q)
+    ws = rmm.new_workspace(rmm.rmm_attn_workspace_bytes(B, Hq, Hkv, T, L, D), dev)
+    for _ in range(args.warmup):
+        rmm.rmm_attn_qk(Q, Kt, V, L, r, O=O, workspace=ws)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        rmm.rmm_attn_qk(Q, Kt, V, L, r, O=O, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    if rmm.rmm_get_status(ws) != rmm.RMM_OK:
+        raise RuntimeError("device status not OK")
+    k = metrics.k_for(D, r)
+    ms = statistics.median(ts)
+    flops = metrics.attn_flops(B, Hq, T, L, D, k, causal=True)
+    print(json.dumps({"single_attn": {"B": B, "Hq": Hq, "Hkv": Hkv, "T": T, "L": L, "r": r, "k": k,
+                                      "call_us": 1e3 * ms, "tflops": flops / (ms * 1e-3) / 1e12}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -641,10 +675,14 @@ def main():
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-secondary", action="store_true")
     ap.add_argument("--single", default=None, help="T,H,N,r: time one rmm_linear shape alone")
+    ap.add_argument("--single-attn", default=None, help="B,Hq,Hkv,T,L,r: time one rmm_attn_qk call alone")
     ap.add_argument("--gemm-producer", type=int, default=0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.single_attn:
+        run_single_attn(args)
+        return
     if args.single:
         run_single(args)
         return
