@@ -82,6 +82,8 @@ def _load():
     lib.oracle_attention.argtypes = [_u16p, _u16p, _u16p, L, L, L, L, L, L, L, I, D, I, P, L,
                                      _f64p, _i32p, P]
     lib.oracle_attention.restype = I
+    lib.oracle_block_select.argtypes = [_u16p, L, L, L, _i32p]
+    lib.oracle_block_select.restype = I
     lib.oracle_rmsnorm.argtypes = [_u16p, L, L, D, _f64p]
     lib.oracle_rmsnorm.restype = I
     lib.oracle_swiglu.argtypes = [_u16p, _u16p, L, _f64p]
@@ -171,6 +173,27 @@ def linear(X, W, r: float, rows=None, cols=None):
     idx = np.zeros(k, dtype=np.int32)
     _check(_load().oracle_linear(x, w, T, H, N, float(r), rp, nr, cp, nc, Y, idx), "oracle_linear")
     return Y, idx
+
+
+def block_select(s, block: int, kb: int) -> np.ndarray:
+    """The kb best blocks of `block` consecutive slices (block score = max of its
+    slices' scores), ascending block indices."""
+    sv = np.ascontiguousarray(np.asarray(s, dtype=np.uint16))
+    H = sv.size
+    out = np.zeros(int(kb), dtype=np.int32)
+    _check(_load().oracle_block_select(sv, H, int(block), int(kb), out), "oracle_block_select")
+    return out
+
+
+def linear_blocks(X, W, r: float, block: int = 64, rows=None, cols=None):
+    """The reduced linear map with a block-granular kept set: kb = ceil(r * H / block)
+    blocks; the product over their slices.  Returns (Y fp64, kept blocks)."""
+    x = _bits(X)
+    H = x.shape[1]
+    kb = k_for(H // block, r)
+    blocks = block_select(score(X), block, kb)
+    idx = (blocks[:, None] * block + np.arange(block, dtype=np.int32)[None, :]).reshape(-1)
+    return reduced_product(X, W, idx, rows=rows, cols=cols), blocks
 
 
 def attention(Q, K, V, k: int, causal: bool = True, scale: float | None = None,

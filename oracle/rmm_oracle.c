@@ -192,6 +192,33 @@ int oracle_reduced_product(const uint16_t* X, const uint16_t* W, long T, long H,
     return 0;
 }
 
+/* ---- block-granular kept sets (§5.2, §6.1 demo) ------------------------ */
+
+/* The kept set chosen per block of `block` consecutive contraction slices
+ * (the demo keeps 64-wide blocks of the down projection's input, scored from
+ * the current activation, top-k of the block scores, sorted).  Block j covers
+ * slices [j*block, (j+1)*block); its score is the largest of its slices'
+ * scores s (max keeps the score exact and independent of any summation
+ * order, as the per-slice score is).  The kb best blocks under (score desc,
+ * block index asc) are written to blocks in ascending order.  H must be a
+ * multiple of block. */
+int oracle_block_select(const uint16_t* s, long H, long block, long kb, int32_t* blocks) {
+    if (!s || !blocks || block < 1 || H < block || H % block != 0) return ORACLE_ERR_ARG;
+    long nb = H / block;
+    if (kb < 1 || kb > nb) return ORACLE_ERR_ARG;
+    uint16_t* bs = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)nb);
+    if (!bs) return ORACLE_ERR_NOMEM;
+    for (long j = 0; j < nb; ++j) {
+        uint16_t m = 0;
+        for (long i = 0; i < block; ++i)
+            if (s[j * block + i] > m) m = s[j * block + i];
+        bs[j] = m;
+    }
+    int rc = oracle_select(bs, nb, kb, blocks);
+    free(bs);
+    return rc;
+}
+
 /* The whole reduced linear map: k = ceil(r*H); score; select; gather and
  * product.  idx_out (k entries, may be NULL) receives the kept set. */
 int oracle_linear(const uint16_t* X, const uint16_t* W, long T, long H, long N, double r,

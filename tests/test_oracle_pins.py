@@ -325,3 +325,60 @@ def test_row_and_column_subsets():
     Ys, idx2 = oracle.linear(X, W, 0.3, rows=rows, cols=cols)
     assert idx.tolist() == idx2.tolist()
     assert np.array_equal(Ys, Y[np.ix_(rows, cols)])
+
+
+# ---------------------------------------------------------------- block-granular kept sets
+
+def test_block_select_with_unit_blocks_is_the_slice_select():
+    s = rmm_synth.tie_heavy((97,), 81).view(torch.int16).numpy().view(np.uint16) & 0x7FFF
+    for k in (1, 13, 50, 97):
+        assert oracle.block_select(s, 1, k).tolist() == oracle.select(s, k).tolist()
+
+
+@pytest.mark.parametrize("block,nb", [(4, 6), (3, 7)])
+def test_block_select_brute_force(block, nb):
+    """The kept blocks are the unique subset of size kb in which every kept block beats
+    every dropped one under (block max desc, block index asc) -- checked over all subsets."""
+    rng = np.random.default_rng(82 + block)
+    s = rng.integers(0, 6, size=block * nb).astype(np.uint16)  # few values: many ties
+    bmax = s.reshape(nb, block).max(axis=1).astype(np.int64)
+    for kb in range(1, nb + 1):
+        got = oracle.block_select(s, block, kb).tolist()
+        valid = []
+        for sub in itertools.combinations(range(nb), kb):
+            kept, dropped = set(sub), set(range(nb)) - set(sub)
+            if all((bmax[a] > bmax[d]) or (bmax[a] == bmax[d] and a < d) for a in kept for d in dropped):
+                valid.append(list(sub))
+        assert valid == [got]
+
+
+def test_block_select_nested_over_kb():
+    s = rmm_synth.activations(9, 640, 83)
+    sc = oracle.score(s)
+    prev = set()
+    for kb in range(1, 11):
+        cur = set(oracle.block_select(sc, 64, kb).tolist())
+        assert prev <= cur and len(cur) == kb
+        prev = cur
+
+
+def test_linear_blocks_full_ratio_is_the_dense_product():
+    X = rmm_synth.activations(5, 256, 84)
+    W = rmm_synth.weights(40, 256, 85)
+    Y, blocks = oracle.linear_blocks(X, W, 1.0, block=64)
+    assert blocks.tolist() == [0, 1, 2, 3]
+    assert np.allclose(Y, f64(X) @ f64(W).T, rtol=0, atol=1e-12)
+
+
+def test_linear_blocks_keeps_the_outlier_block_and_splits_the_product():
+    """A single large value makes its block the best one; kept plus dropped blocks
+    sum to the dense product."""
+    T, H, N = 3, 512, 24
+    X = (rmm_synth.normal((T, H), 86) * 0.01).to(torch.bfloat16)
+    X[1, 5 * 64 + 17] = 40.0
+    W = rmm_synth.weights(N, H, 87)
+    Y, blocks = oracle.linear_blocks(X, W, 1 / 8, block=64)
+    assert blocks.tolist() == [5]
+    dropped = np.array([j for j in range(H) if j // 64 != 5], dtype=np.int32)
+    Yd = oracle.reduced_product(X, W, dropped)
+    assert np.allclose(Y + Yd, f64(X) @ f64(W).T, rtol=0, atol=1e-12)
