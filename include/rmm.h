@@ -82,7 +82,15 @@ typedef struct rmm_options {
      * shorter ones (decode); 1 = always the split pass; 2 = always the tensor
      * cores. */
     int attn_path;
-    int reserved[2]; /* must be zero */
+    /* Granularity of the kept set of rmm_linear / rmm_linear_group: 0
+     * (default) = single contraction slices; 16, 32, 64, 128 or 256 = blocks
+     * of that many consecutive slices (H a multiple of it, at most 1024
+     * blocks), as in the FFN demo of the cf-1.com post (§6.1, 64-wide blocks).
+     * A block scores the largest of its slices' scores; kb = ceil(r * H /
+     * block_size) blocks are kept under (score desc, block index asc); idx_out
+     * then receives their k = kb * block_size slices, ascending. */
+    int block_size;
+    int reserved[1]; /* must be zero */
     /* Optional pair of cudaEvent_t handles (NULL: none) recorded on the
      * stream immediately before and after the reduced-product kernel (GEMV or
      * GEMM) of rmm_linear / rmm_gemm_reduced, so that a caller can time that

@@ -54,7 +54,7 @@ int num_sms_current() {
 }
 
 const rmm_options& opts_or_default(const rmm_options* o) {
-    static const rmm_options d = {16, 0, 0, 0, 0, 0, {0, 0}, nullptr, nullptr};
+    static const rmm_options d = {16, 0, 0, 0, 0, 0, 0, {0}, nullptr, nullptr};
     return o ? *o : d;
 }
 
@@ -64,8 +64,8 @@ bool opts_valid(const rmm_options* o) {
     if (o->gemv_splits < 0) return false;
     if (o->gemm_producer < 0 || o->gemm_producer > 2) return false;
     if (o->attn_path < 0 || o->attn_path > 2) return false;
-    for (int i = 0; i < 2; ++i)
-        if (o->reserved[i] != 0) return false;
+    if (o->block_size < 0) return false;
+    if (o->reserved[0] != 0) return false;
     return true;
 }
 
@@ -272,9 +272,13 @@ rmm_status linear_group(const void* X, int T, int H, double r, int count, const 
                         const int* Ns, void* const* Ys, int32_t* idx_out, void* workspace,
                         size_t workspace_bytes, rmm_stream_t stream, const rmm_options* options) {
     if (!group_args_ok(X, T, H, count, Wts, Ns, Ys) || !opts_valid(options)) return RMM_ERR_INVALID_ARG;
-    const int k = rmm_k_for(H, r);
-    if (k < 1) return RMM_ERR_INVALID_ARG;
     const rmm_options& o = opts_or_default(options);
+    const int bsz = o.block_size;
+    if (!block_size_ok(H, bsz)) return RMM_ERR_UNSUPPORTED;
+    // kept slices: ceil(r*H), or ceil(r*H/block) whole blocks
+    const int kb = bsz ? rmm_k_for(H / bsz, r) : 0;
+    const int k = bsz ? (kb < 1 ? -1 : kb * bsz) : rmm_k_for(H, r);
+    if (k < 1) return RMM_ERR_INVALID_ARG;
     const int sms = num_sms_current();
     const LinearLayout L = linear_layout(T, H, Ns, count, k, o, sms);
     if (!workspace || workspace_bytes < L.total || !aligned16(workspace)) return RMM_ERR_WORKSPACE;
@@ -284,7 +288,13 @@ rmm_status linear_group(const void* X, int T, int H, double r, int count, const 
     int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
     const int pad_to = (k + kGemmBK - 1) / kGemmBK * kGemmBK;
     cudaError_t e;
-    if (L.gemv && T == 1) {
+    if (bsz) {
+        // block-granular: the score pass (with X^T on the GEMM path), then the blocks
+        e = launch_score(static_cast<const uint16_t*>(X), T, H, s32,
+                         L.gemv ? nullptr : reinterpret_cast<uint16_t*>(ws + L.xt), L.ldT, sms, s);
+        if (e == cudaSuccess) e = launch_block_select(s32, H, bsz, kb, idx, idx_out, nullptr, s);
+        if (e == cudaSuccess && pad_to > k) e = launch_pad_idx(idx, k, H, idx, pad_to, s);
+    } else if (L.gemv && T == 1) {
         // one token: the select kernel reads the score straight from X
         e = launch_select(static_cast<const uint16_t*>(X), T, nullptr, 0, H, k, idx, pad_to, idx_out, nullptr, s);
     } else if (L.gemv) {

@@ -27,6 +27,15 @@ cudaError_t launch_score(const uint16_t* X, int T, int H, uint32_t* s32, uint16_
 cudaError_t launch_select(const uint16_t* X, int T, uint32_t* s32, int clear_input, int H, int k, int32_t* idx,
                           int pad_to, int32_t* idx_copy, uint32_t* s_out, cudaStream_t stream);
 
+// ---- block-granular kept sets (rmm_blocks.cu)
+// block 0 (single slices) or 16..256 dividing H with at most 1024 blocks
+bool block_size_ok(int H, int block);
+// From the score vector s32 (u32 [H], zeroed afterwards): the kb best blocks of
+// `block` slices (block score = max of its slices), their kb * block slices
+// ascending to idx (and idx_copy if not null), the blocks to blocks_out if not null.
+cudaError_t launch_block_select(uint32_t* s32, int H, int block, int kb, int32_t* idx, int32_t* idx_copy,
+                                int32_t* blocks_out, cudaStream_t stream);
+
 // ---- split-K GEMV (rmm_gemv.cu)
 constexpr int kMaxGroupGemv = 4;
 // Up to 4 decode products sharing X and the kept list, planned by
