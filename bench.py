@@ -604,7 +604,7 @@ def run_single(args):
     Wt = rmm.rmm_transpose_weight(rmm_synth.weights(N, H, 12, std=0.02).to(dev))
     Y = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
     ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-    opts = rmm.options(gemm_producer=args.gemm_producer, product_events=ev)
+    opts = rmm.options(gemm_producer=args.gemm_producer, block_size=args.block_size, product_events=ev)
     ws = rmm.new_workspace(rmm.rmm_linear_workspace_bytes(T, H, N, opts), dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
@@ -622,9 +622,10 @@ def run_single(args):
         kern.append(ev[0].elapsed_time(ev[1]))
     if rmm.rmm_get_status(ws) != rmm.RMM_OK:
         raise RuntimeError("device status not OK")
-    k = metrics.k_for(H, r)
+    bs = args.block_size
+    k = metrics.k_for(H // bs, r) * bs if bs else metrics.k_for(H, r)
     km = statistics.median(kern)
-    out = {"single": {"T": T, "H": H, "N": N, "r": r, "k": k, "producer": args.gemm_producer,
+    out = {"single": {"T": T, "H": H, "N": N, "r": r, "k": k, "producer": args.gemm_producer, "block_size": bs,
                       "call_us": 1e3 * statistics.median(call), "product_us": 1e3 * km,
                       "product_tflops": metrics.reduced_linear_flops(T, N, k) / (km * 1e-3) / 1e12,
                       "product_gbs": metrics.gemv_bytes(T, H, N, k) / (km * 1e-3) / 1e9}}
@@ -677,6 +678,7 @@ def main():
     ap.add_argument("--single", default=None, help="T,H,N,r: time one rmm_linear shape alone")
     ap.add_argument("--single-attn", default=None, help="B,Hq,Hkv,T,L,r: time one rmm_attn_qk call alone")
     ap.add_argument("--gemm-producer", type=int, default=0)
+    ap.add_argument("--block-size", type=int, default=0, help="with --single: block-granular kept sets")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -229,8 +229,20 @@ rmm_status run_product_kernels(const void* X, int T, int H, int count, const voi
         memset(&ym, 0, sizeof ym);
         for (int p = 0; p < count; ++p)
             if (!tiled_map(Ys[p], (uint64_t)T, (uint64_t)Ns[p], (uint64_t)Ns[p], 32, &ym.m[p])) return RMM_ERR_CUDA;
-        return cuda_status(launch_gemm_pair(reinterpret_cast<const uint16_t*>(ws + L.xt), L.ldT, g, ym, idx_padded,
-                                            k, T, H, reinterpret_cast<float*>(ws + L.partials), status,
+        const uint16_t* xt = reinterpret_cast<const uint16_t*>(ws + L.xt);
+        // block-granular sets in runs of 64 slices: every K-block is 64 contiguous
+        // rows, loaded by TMA tile copies
+        GemmInMaps im;
+        const bool tma_rows = o.block_size > 0 && o.block_size % kGemmBK == 0;
+        if (tma_rows) {
+            memset(&im, 0, sizeof im);
+            if (!tiled_map(xt, (uint64_t)H, (uint64_t)T, (uint64_t)L.ldT, kGemmBK, &im.xt)) return RMM_ERR_CUDA;
+            for (int p = 0; p < count; ++p)
+                if (!tiled_map(Wts[p], (uint64_t)H, (uint64_t)Ns[p], (uint64_t)Ns[p], kGemmBK, &im.wt[p]))
+                    return RMM_ERR_CUDA;
+        }
+        return cuda_status(launch_gemm_pair(xt, L.ldT, g, ym, tma_rows ? &im : nullptr, idx_padded, k, T, H,
+                                            reinterpret_cast<float*>(ws + L.partials), status,
                                             o.debug_timeout_test, sms, s));
     }
     gemm_group_tiles(g, T, 0);

@@ -469,10 +469,15 @@ __device__ __forceinline__ Unit decode_unit(const GemmGroup& g, int u, int m_til
     return r;
 }
 
+// kTmaRows: every 64-slice K-block of the kept list is 64 contiguous slices
+// (block-granular kept sets whose block is a multiple of 64), so one thread
+// loads each stage with six TMA tile loads (two 64-token boxes of X^T, four
+// 64-column boxes of W^T, 64 rows each) instead of the cp.async gather.
+template <bool kTmaRows>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     gemm_pair_kernel(const uint16_t* __restrict__ Xt, int ldT, const __grid_constant__ GemmGroup group,
-                     const __grid_constant__ GemmOutMaps ymaps, const int32_t* __restrict__ idx, int k, int T,
-                     int H, int* status, int debug_timeout) {
+                     const __grid_constant__ GemmOutMaps ymaps, const __grid_constant__ GemmInMaps imaps,
+                     const int32_t* __restrict__ idx, int k, int T, int H, int* status, int debug_timeout) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -495,7 +500,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES2; ++s) {
-            mbar_init(smem_addr(&bars->full[s]), kProducerThreads);
+            mbar_init(smem_addr(&bars->full[s]), kTmaRows ? 1 : kProducerThreads);
             mbar_init(smem_addr(&bars->pair_full[s]), 1);
             mbar_init(smem_addr(&bars->empty[s]), 1);
         }
@@ -516,7 +521,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     pdl_wait();  // the kept list and X^T come from the preceding kernels
     pdl_launch_dependents();
 
-    if (warp < kProducerWarps) {
+    if (kTmaRows && warp < kProducerWarps) {
+        // ------------------------------------------------------------ TMA producer (both CTAs)
+        if (warp == 0 && lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_phase[STAGES2];
+            bool issued[STAGES2];
+            for (int s = 0; s < STAGES2; ++s) issued[s] = false;
+            bool ok = true;
+            for (int u = cluster_id; ok && u < num_units; u += num_clusters) {
+                const Unit ux = decode_unit(group, u, m_tiles, nkb);
+                const TileCoord tc = ux.tc;
+                const int a_col = tc.m0 + HALF_M * (int)rank;
+                const int b_col = tc.n0 + HALF_N * (int)rank;
+                int row_next = __ldg(idx + ux.kb0 * BK);  // first slice of the K-block: its 64 rows are contiguous
+                for (int kb = ux.kb0; kb < ux.kb1; ++kb) {
+                    const int row = row_next;
+                    if (kb + 1 < ux.kb1) row_next = __ldg(idx + (kb + 1) * BK);
+                    const uint32_t full = smem_addr(&bars->full[stage]);
+                    if (!mbar_wait(smem_addr(&bars->empty[stage]), phase ^ 1, status, abort_flag)) {
+                        st_shared_cluster_u32(peer_abort, 1);
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(full, A2_STAGE_BYTES + B2_STAGE_BYTES);
+                    const uint32_t a_stage = smem_addr(sA + stage * A2_STAGE_BYTES);
+                    const uint32_t b_stage = smem_addr(sB + stage * B2_STAGE_BYTES);
+#pragma unroll
+                    for (int i = 0; i < HALF_M / 64; ++i)
+                        tma_load_2d(a_stage + i * CHUNK_BYTES, &imaps.xt, full, a_col + 64 * i, row);
+#pragma unroll
+                    for (int i = 0; i < HALF_N / 64; ++i)
+                        tma_load_2d(b_stage + i * CHUNK_BYTES, &imaps.wt[tc.p], full, b_col + 64 * i, row);
+                    issued[stage] = true;
+                    issued_phase[stage] = phase;
+                    if (++stage == STAGES2) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            // no copy may still be landing in shared memory when the CTA leaves
+            volatile int no_abort = 0;
+            for (int s = 0; s < STAGES2; ++s)
+                if (issued[s]) mbar_wait(smem_addr(&bars->full[s]), issued_phase[s], status, &no_abort);
+        }
+    } else if (warp < kProducerWarps) {
         // ------------------------------------------------------------ producer (both CTAs)
         int stage = 0;
         uint32_t phase = 0;
@@ -851,11 +902,17 @@ size_t gemm_pair_partial_bytes(int num_sms) {
 // K-block each), so that wave takes about 1/s of a tile's time instead of a
 // whole one.
 cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group, const GemmOutMaps& ymaps,
-                             const int32_t* idx, int k, int T, int H, float* partials, int* status,
-                             int debug_timeout, int num_sms, cudaStream_t stream) {
+                             const GemmInMaps* imaps, const int32_t* idx, int k, int T, int H, float* partials,
+                             int* status, int debug_timeout, int num_sms, cudaStream_t stream) {
     if (group.count < 1 || group.count > kMaxGroup) return cudaErrorInvalidValue;
-    cudaError_t e = ensure_smem_limit(pair::gemm_pair_kernel, pair::kSmemBytes2);
+    auto kern = imaps ? pair::gemm_pair_kernel<true> : pair::gemm_pair_kernel<false>;
+    cudaError_t e = ensure_smem_limit(kern, pair::kSmemBytes2);
     if (e != cudaSuccess) return e;
+    GemmInMaps no_maps;
+    if (!imaps) {
+        memset(&no_maps, 0, sizeof no_maps);
+        imaps = &no_maps;
+    }
     const int tiles = group.tile_start[group.count];
     const int nkb = (k + BK - 1) / BK;
     const int pairs = num_sms / 2 > 0 ? num_sms / 2 : 1;
@@ -878,8 +935,8 @@ cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group
     }
     int clusters = pairs < g.units ? pairs : g.units;
     if (clusters < 1) clusters = 1;
-    e = launch_pdl(pair::gemm_pair_kernel, dim3(2 * clusters), dim3(pair::kThreads2), pair::kSmemBytes2, stream, Xt, ldT,
-                   g, ymaps, idx, k, T, H, status, debug_timeout);
+    e = launch_pdl(kern, dim3(2 * clusters), dim3(pair::kThreads2), pair::kSmemBytes2, stream, Xt, ldT, g, ymaps,
+                   *imaps, idx, k, T, H, status, debug_timeout);
     if (e != cudaSuccess || g.tail_splits == 1) return e;
     return launch_pdl(pair::gemm_fold_kernel, dim3(R * (pair::BM2 / 4)), dim3(256), 0, stream, g, T);
 }

@@ -112,9 +112,17 @@ int gemm_group_tiles(GemmGroup& g, int T, int pair);
 struct __align__(64) GemmOutMaps {
     CUtensorMap m[kMaxGroup];
 };
+// Input tensor maps for kept lists made of whole 64-slice runs (block-granular
+// sets): X^T [H, T] and each member's W^T [H, N], box 64 rows x 64 columns,
+// 128-byte swizzle.  With them the GEMM loads its stages by TMA tile copies.
+struct __align__(64) GemmInMaps {
+    CUtensorMap xt;
+    CUtensorMap wt[kMaxGroup];
+};
+// imaps null: the cp.async gather producer (any kept list).
 cudaError_t launch_gemm_pair(const uint16_t* Xt, int ldT, const GemmGroup& group, const GemmOutMaps& ymaps,
-                             const int32_t* idx, int k, int T, int H, float* partials, int* status,
-                             int debug_timeout, int num_sms, cudaStream_t stream);
+                             const GemmInMaps* imaps, const int32_t* idx, int k, int T, int H, float* partials,
+                             int* status, int debug_timeout, int num_sms, cudaStream_t stream);
 size_t gemm_pair_partial_bytes(int num_sms);
 // map_xt / map_wt are used only by the TMA tile::gather4 producer
 // (tma_gather != 0), which handles a group of one.
