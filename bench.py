@@ -335,6 +335,54 @@ def time_decode(dev, peaks):
     return out
 
 
+def time_blocks(dev, acts, Wts, Ys, dense_ms, steps, warmup, block=64):
+    """Secondary row: the same prefill step with block-granular kept sets (blocks of
+    `block` consecutive slices scored by their largest slice score; with 64-slice runs
+    the GEMM stages its operands by TMA tile copies)."""
+    from input_adaptive_reduced_rmm_b200 import rmm
+
+    ks = {n: metrics.k_for(H // block, R) * block for n, H, _, _ in PROJ}
+    flops = sum(metrics.reduced_linear_flops(T_PREFILL, N, ks[n]) for n, _, N, _ in PROJ)
+    evs = {c: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)] for c in range(len(CALLS))}
+    opts = {c: [rmm.options(block_size=block, product_events=evs[c][i]) for i in range(steps)]
+            for c in range(len(CALLS))}
+    plain = rmm.options(block_size=block)
+    ws = {c: rmm.new_workspace(rmm.rmm_linear_group_workspace_bytes(
+        T_PREFILL, ACT_H[s], [PROJ_BY_NAME[n][1] for n in names], plain), dev) for c, (s, names) in enumerate(CALLS)}
+
+    def step(i=None):
+        for c, (s, names) in enumerate(CALLS):
+            rmm.rmm_linear_group(acts[s], [Wts[n] for n in names], R, Ys=[Ys[n] for n in names],
+                                 workspace=ws[c], opts=plain if i is None else opts[c][i])
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    for i in range(steps):
+        step(i)
+    torch.cuda.synchronize()
+    for c in ws:
+        if rmm.rmm_get_status(ws[c]) != rmm.RMM_OK:
+            raise RuntimeError("device status not OK (block-granular step)")
+    gemm_ms = sum(b.elapsed_time(e) for c in evs for b, e in evs[c]) / steps
+    return {"blocks": {
+        "workload": f"the prefill step (T={T_PREFILL}, r={R}) with {block}-slice block-granular kept sets",
+        "ms_per_step": ms,
+        "tflops": flops / (ms * 1e-3) / 1e12,
+        "gemm_us": 1e3 * gemm_ms,
+        "gemm_tflops": flops / (gemm_ms * 1e-3) / 1e12,
+        "speedup_vs_dense": dense_ms / ms,
+    }}
+
+
 def launches_per_step(dev) -> int:
     """Our kernels launched by one step: per call the score pass, the select, the CTA-pair
     GEMM, and the fold of the split last wave when the call's tiles leave a partial wave
@@ -557,6 +605,7 @@ def run_rmm(args, world, rank, local):
 
     extra = {}
     if not args.skip_secondary:
+        extra.update(time_blocks(dev, acts, Wts, Ys, dense_ms, K, W))
         extra.update(time_decode(dev, peaks))
         extra.update(time_layer(dev, host_inputs()[1]))
 

@@ -29,12 +29,12 @@ def expand(blocks, block):
     return (np.asarray(blocks)[:, None] * block + np.arange(block)[None, :]).reshape(-1)
 
 
-def run_blocks(rmm, X, W, r, block, t_gemv=16):
+def run_blocks(rmm, X, W, r, block, t_gemv=16, producer=0):
     T, H = X.shape
     N = W.shape[0]
     Wt = rmm.rmm_transpose_weight(W.cuda())
     kb = oracle.k_for(H // block, r)
-    opts = rmm.options(block_size=block, t_gemv=t_gemv)
+    opts = rmm.options(block_size=block, t_gemv=t_gemv, gemm_producer=producer)
     idx = torch.full((kb * block,), -1, dtype=torch.int32, device="cuda")
     ws = rmm.new_workspace(rmm.rmm_linear_workspace_bytes(T, H, N, opts))
     Y = rmm.rmm_linear(X.cuda(), Wt, r, idx_out=idx, workspace=ws, opts=opts)
@@ -84,6 +84,20 @@ def test_blocks_llama3_8b_prefill_sampled(rmm):
     Yo, blocks = oracle.linear_blocks(X, W, r, block=block, rows=rows)
     assert idx.tolist() == expand(blocks, block).tolist()
     assert_close(Y[rows], Yo, "llama3-8b prefill blocks")
+
+
+@pytest.mark.parametrize("producer", [0, 2])
+@pytest.mark.parametrize("T,H,N,block", [(700, 1024, 1800, 64), (300, 2048, 776, 128), (2048, 512, 3000, 256)])
+def test_blocks_tma_tiles(rmm, producer, T, H, N, block):
+    """Blocks of 64 slices or more: the CTA-pair GEMM (0) loads whole 64-row runs by TMA
+    tile copies; the single-CTA cp.async GEMM (2) gathers them row by row.  Ragged M and N
+    edges, split last wave."""
+    X = rmm_synth.activations(T, H, rmm_synth.seed_for(9, T, 3))
+    W = rmm_synth.weights(N, H, rmm_synth.seed_for(9, T, 4), std=0.02)
+    Y, idx, kb = run_blocks(rmm, X, W, 0.5, block, producer=producer)
+    Yo, blocks = oracle.linear_blocks(X, W, 0.5, block=block)
+    assert idx.tolist() == expand(blocks, block).tolist()
+    assert_close(Y, Yo, f"T={T} H={H} N={N} block={block} producer={producer}")
 
 
 def test_blocks_group_shares_one_set(rmm):

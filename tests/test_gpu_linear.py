@@ -109,6 +109,19 @@ def test_gemm_producers(rmm, producer, T, H, N):
     assert_close(Y, Yo, f"producer {producer} T={T} H={H} N={N}")
 
 
+@pytest.mark.parametrize("producer", [0, 2])
+@pytest.mark.parametrize("T,H,N,r", [(1000, 1024, 5000, 0.4), (2304, 512, 4608, 0.5)])
+def test_gemm_pair_many_tiles(rmm, producer, T, H, N, r):
+    """Several tiles per CTA (the accumulator reused tile after tile), a ragged last M
+    tile and N tile, and a split last wave."""
+    X = rmm_synth.activations(T, H, 310 + T)
+    W = rmm_synth.weights(N, H, 311 + T)
+    Y, idx = run_linear(rmm, X, W, r, rmm.options(gemm_producer=producer))
+    Yo, io = oracle.linear(X, W, r)
+    assert np.array_equal(idx, io)
+    assert_close(Y, Yo, f"producer {producer} T={T} H={H} N={N}")
+
+
 def test_linear_tie_heavy_inputs(rmm):
     X = rmm_synth.tie_heavy((40, 256), 5)
     W = rmm_synth.weights(128, 256, 6)
