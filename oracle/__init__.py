@@ -45,6 +45,7 @@ ERR_NOMEM = -3
 _u16p = np.ctypeslib.ndpointer(dtype=np.uint16, flags="C_CONTIGUOUS")
 _i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
 _f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+_f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
 
 
 def build(force: bool = False) -> str:
@@ -82,6 +83,15 @@ def _load():
     lib.oracle_attention.argtypes = [_u16p, _u16p, _u16p, L, L, L, L, L, L, L, I, D, I, P, L,
                                      _f64p, _i32p, P]
     lib.oracle_attention.restype = I
+    lib.oracle_ctx_block_means.argtypes = [_u16p, L, L, L, L, L, _f32p]
+    lib.oracle_ctx_block_means.restype = I
+    lib.oracle_ctx_block_scores.argtypes = [_u16p, _f32p, L, L, L, L, L, L, I, _f32p]
+    lib.oracle_ctx_block_scores.restype = I
+    lib.oracle_ctx_select.argtypes = [_f32p, L, L, _i32p]
+    lib.oracle_ctx_select.restype = I
+    lib.oracle_attention_ctx.argtypes = [_u16p, _u16p, _u16p, L, L, L, L, L, L, L, I, D, I, L, L, P, L,
+                                         _f64p, _i32p, _i32p, P, P]
+    lib.oracle_attention_ctx.restype = I
     lib.oracle_block_select.argtypes = [_u16p, L, L, L, _i32p]
     lib.oracle_block_select.restype = I
     lib.oracle_rmsnorm.argtypes = [_u16p, L, L, D, _f64p]
@@ -221,6 +231,71 @@ def attention(Q, K, V, k: int, causal: bool = True, scale: float | None = None,
                                     None if given is None else given.ctypes.data_as(ctypes.c_void_p)),
            "oracle_attention")
     return O, idx
+
+
+def ctx_block_means(K, bc: int) -> np.ndarray:
+    """Mean key of each block of bc consecutive positions.  K [B,Hkv,L,d] (bf16).
+    Returns float32 [B,Hkv,ceil(L/bc),d] (float sums over l ascending, then / n)."""
+    kk = _bits(K)
+    B, Hkv, L, d = kk.shape
+    nblk = -(-L // int(bc))
+    out = np.zeros((B, Hkv, nblk, d), dtype=np.float32)
+    _check(_load().oracle_ctx_block_means(kk, B, Hkv, L, d, int(bc), out), "oracle_ctx_block_means")
+    return out
+
+
+def ctx_block_scores(Q, means, Hkv: int, per_query_head: bool = False) -> np.ndarray:
+    """Block scores: for each kept set, the largest fmaf-chain dot of its query rows with
+    each block mean.  Q [B,Hq,T,d] (bf16), means float32 [B,Hkv,nblk,d].
+    Returns float32 [B,nsets,nblk]."""
+    q = _bits(Q)
+    B, Hq, T, d = q.shape
+    m = np.ascontiguousarray(means, dtype=np.float32)
+    nblk = m.shape[2]
+    nsets = Hq if per_query_head else Hkv
+    out = np.zeros((B, nsets, nblk), dtype=np.float32)
+    _check(_load().oracle_ctx_block_scores(q, m, B, Hq, Hkv, T, nblk, d, int(bool(per_query_head)), out),
+           "oracle_ctx_block_scores")
+    return out
+
+
+def ctx_select(scores, kc: int) -> np.ndarray:
+    """The kc best blocks of one score row under (score desc, index asc), ascending."""
+    sc = np.ascontiguousarray(np.asarray(scores, dtype=np.float32).reshape(-1))
+    out = np.zeros(int(kc), dtype=np.int32)
+    _check(_load().oracle_ctx_select(sc, sc.size, int(kc), out), "oracle_ctx_select")
+    return out
+
+
+def attention_ctx(Q, K, V, k: int, bc: int, kc: int, causal: bool = True, scale: float | None = None,
+                  per_query_head: bool = False, t_rows=None, idx_in=None, blocks_in=None):
+    """Reduced attention over the kept head dimensions and the kept context blocks.
+    Q [B,Hq,T,d], K/V [B,Hkv,L,d] (bf16); bc keys per block, kc blocks kept per set.
+
+    Returns (O fp64 [B,Hq,nrows,d], idx int32 [B,nsets,k], blocks int32 [B,nsets,kc]).
+    """
+    q, kk, v = _bits(Q), _bits(K), _bits(V)
+    B, Hq, T, d = q.shape
+    _, Hkv, L, _ = kk.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rp, nr, _keep = _rows(t_rows)
+    nrows = nr if t_rows is not None else T
+    O = np.zeros((B, Hq, nrows, d), dtype=np.float64)
+    nsets = Hq if per_query_head else Hkv
+    idx = np.zeros((B, nsets, int(k)), dtype=np.int32)
+    blocks = np.zeros((B, nsets, int(kc)), dtype=np.int32)
+    gi = gb = None
+    if idx_in is not None:
+        gi = np.ascontiguousarray(np.asarray(idx_in, dtype=np.int32).reshape(B, nsets, int(k)))
+    if blocks_in is not None:
+        gb = np.ascontiguousarray(np.asarray(blocks_in, dtype=np.int32).reshape(B, nsets, int(kc)))
+    _check(_load().oracle_attention_ctx(
+        q, kk, v, B, Hq, Hkv, T, L, d, int(k), int(bool(causal)), float(scale), int(bool(per_query_head)),
+        int(bc), int(kc), rp, nr, O, idx, blocks,
+        None if gi is None else gi.ctypes.data_as(ctypes.c_void_p),
+        None if gb is None else gb.ctypes.data_as(ctypes.c_void_p)), "oracle_attention_ctx")
+    return O, idx, blocks
 
 
 def rmsnorm(x, eps: float = 1e-5) -> np.ndarray:

@@ -6,8 +6,9 @@
  * CPU-baseline / reference legs of bench.py use it.  It shares no code,
  * header, table or helper with the CUDA library.
  *
- * Plain, single-threaded, obviously-correct C.  All floating-point arithmetic
- * is done in fp64 (inputs are bf16 bit patterns, widened exactly).
+ * Plain, single-threaded, obviously-correct C.  Floating-point arithmetic is
+ * done in fp64 (inputs are bf16 bit patterns, widened exactly), except the
+ * context-block score, which decides an integer set (see below).
  *
  * What it computes, and where it comes from:
  *
@@ -35,6 +36,11 @@
  *   Attention: the same reduction applied to Q K^T along the head dimension
  *   (cf-1.com post §3.3: reduce inside a head, never drop whole heads), then
  *   an unreduced softmax(.) V.
+ *
+ *   Context-block attention (cf-1.com post §3.1): keys cut into blocks, a
+ *   cheap per-block score, Q K^T on the kept blocks only.  Its kept-block
+ *   decision is computed in single precision in a fixed order (stated at
+ *   oracle_ctx_block_means); everything else stays fp64.
  *
  *   Decoder-layer glue: RMSNorm and SwiGLU as in Numerical Linear Algebra for
  *   Large Language Models (ai-feeds 2610.04631), Transformer component list.
@@ -261,10 +267,13 @@ int oracle_linear(const uint16_t* X, const uint16_t* W, long T, long H, long N, 
  * instead, laid out like idx_out -- for a layer oracle that follows the index
  * sets another implementation chose, so that a near-tie in an upstream input
  * cannot make the two compute different products. */
-int oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, long B, long Hq,
-                     long Hkv, long T, long L, long d, long k, int causal, double scale,
-                     int per_query_head, const int64_t* t_rows, long nrows, double* O,
-                     int32_t* idx_out, const int32_t* idx_in) {
+/* The attention of one call.  key_keep (NULL: every key) is a 0/1 mask
+ * [B][nsets][L]: the keys a set's query rows may attend to (the context-block
+ * reduction below); a row that may attend to no key gets a zero output. */
+static int attention_core(const uint16_t* Q, const uint16_t* K, const uint16_t* V, long B, long Hq,
+                          long Hkv, long T, long L, long d, long k, int causal, double scale,
+                          int per_query_head, const int64_t* t_rows, long nrows, double* O,
+                          int32_t* idx_out, const int32_t* idx_in, const uint8_t* key_keep) {
     if (!Q || !K || !V || !O || B < 1 || Hq < 1 || Hkv < 1 || T < 1 || L < T || d < 1 || k < 1 ||
         k > d || Hq % Hkv != 0)
         return ORACLE_ERR_ARG;
@@ -318,9 +327,11 @@ int oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, lo
                         break;
                     }
                     const uint16_t* qv = Q + ((b * Hq + q) * T + t) * d;
+                    const uint8_t* kk = key_keep ? key_keep + (b * nsets + set) * L : NULL;
                     long last = causal ? (L - T + t) : (L - 1);
                     double mx = -INFINITY;
                     for (long l = 0; l <= last; ++l) {
+                        if (kk && !kk[l]) continue;
                         double acc = 0.0;
                         for (long j = 0; j < k; ++j)
                             acc += bf16_to_double(qv[S[j]]) * bf16_to_double(Kg[l * d + S[j]]);
@@ -329,14 +340,16 @@ int oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, lo
                     }
                     double den = 0.0;
                     for (long l = 0; l <= last; ++l) {
+                        if (kk && !kk[l]) continue;
                         logit[l] = exp(logit[l] - mx);
                         den += logit[l];
                     }
                     double* o = O + ((b * Hq + q) * nrows + r) * d;
                     for (long c = 0; c < d; ++c) {
                         double acc = 0.0;
-                        for (long l = 0; l <= last; ++l) acc += logit[l] * bf16_to_double(Vg[l * d + c]);
-                        o[c] = acc / den;
+                        for (long l = 0; l <= last; ++l)
+                            if (!kk || kk[l]) acc += logit[l] * bf16_to_double(Vg[l * d + c]);
+                        o[c] = den > 0.0 ? acc / den : 0.0;
                     }
                 }
             }
@@ -348,7 +361,171 @@ int oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, lo
     return rc;
 }
 
-/* ---- decoder-layer glue --------------------------------------------------- */
+int oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, long B, long Hq,
+                     long Hkv, long T, long L, long d, long k, int causal, double scale,
+                     int per_query_head, const int64_t* t_rows, long nrows, double* O,
+                     int32_t* idx_out, const int32_t* idx_in) {
+    return attention_core(Q, K, V, B, Hq, Hkv, T, L, d, k, causal, scale, per_query_head, t_rows, nrows, O,
+                          idx_out, idx_in, NULL);
+}
+
+/* ---- context-block reduction of Q K^T (sequence direction) ----------------
+ *
+ * Input-adaptive matrix-product reduction for LLM inference (cf-1.com post),
+ * §3.1: during generation the keys are cut into blocks of consecutive
+ * positions, a cheap score tells which blocks may draw real attention, and
+ * the full Q K^T runs on the kept blocks only; §7: the gain grows with the
+ * context.  The pages fix neither the cheap score nor the kept count; the
+ * readings taken here:
+ *   - block j holds the positions [j*bc, min(L, (j+1)*bc));
+ *   - its summary is its mean key  mean_j[c] = (sum over its l of K[l,c]) / n_j;
+ *   - its score for a kept set (a KV head's stacked query rows, or one query
+ *     head's rows) is the largest dot product of one of the set's query rows
+ *     with mean_j;
+ *   - kc = ceil(r_ctx * nblk) blocks are kept under (score desc, index asc),
+ *     listed in ascending order;
+ *   - keys of dropped blocks take no part in the softmax.
+ * Summary and score decide which blocks are kept, so they are computed in
+ * single precision in one fixed order, the precision and order in which the
+ * GPU path takes the same decision:
+ *   sum  : float additions over l ascending, starting from 0;
+ *   mean : sum / (float)n_j (correctly rounded division);
+ *   dot  : fmaf chain over c ascending, starting from 0. */
+
+static float bf16_to_float(uint16_t b) { return (float)bf16_to_double(b); }
+
+/* means [B][Hkv][nblk][d], nblk = ceil(L / bc); K [B][Hkv][L][d]. */
+int oracle_ctx_block_means(const uint16_t* K, long B, long Hkv, long L, long d, long bc, float* means) {
+    if (!K || !means || B < 1 || Hkv < 1 || L < 1 || d < 1 || bc < 1) return ORACLE_ERR_ARG;
+    if (!all_finite(K, B * Hkv * L * d)) return ORACLE_ERR_NONFINITE;
+    long nblk = (L + bc - 1) / bc;
+    for (long b = 0; b < B; ++b)
+        for (long g = 0; g < Hkv; ++g) {
+            const uint16_t* Kg = K + (b * Hkv + g) * L * d;
+            for (long j = 0; j < nblk; ++j) {
+                long l0 = j * bc, l1 = l0 + bc < L ? l0 + bc : L;
+                for (long c = 0; c < d; ++c) {
+                    float sum = 0.0f;
+                    for (long l = l0; l < l1; ++l) sum += bf16_to_float(Kg[l * d + c]);
+                    means[((b * Hkv + g) * nblk + j) * d + c] = sum / (float)(l1 - l0);
+                }
+            }
+        }
+    return 0;
+}
+
+/* scores [B][nsets][nblk] from Q [B][Hq][T][d] and the block means. */
+int oracle_ctx_block_scores(const uint16_t* Q, const float* means, long B, long Hq, long Hkv, long T,
+                            long nblk, long d, int per_query_head, float* scores) {
+    if (!Q || !means || !scores || B < 1 || Hq < 1 || Hkv < 1 || T < 1 || nblk < 1 || d < 1 ||
+        Hq % Hkv != 0)
+        return ORACLE_ERR_ARG;
+    if (!all_finite(Q, B * Hq * T * d)) return ORACLE_ERR_NONFINITE;
+    long G = Hq / Hkv;
+    long nsets = per_query_head ? Hq : Hkv;
+    for (long b = 0; b < B; ++b)
+        for (long set = 0; set < nsets; ++set) {
+            long q_lo = per_query_head ? set : set * G;
+            long q_hi = per_query_head ? set + 1 : (set + 1) * G;
+            long g = per_query_head ? set / G : set;
+            for (long j = 0; j < nblk; ++j) {
+                const float* m = means + ((b * Hkv + g) * nblk + j) * d;
+                float best = -INFINITY;
+                for (long q = q_lo; q < q_hi; ++q)
+                    for (long t = 0; t < T; ++t) {
+                        const uint16_t* qv = Q + ((b * Hq + q) * T + t) * d;
+                        float acc = 0.0f;
+                        for (long c = 0; c < d; ++c) acc = fmaf(bf16_to_float(qv[c]), m[c], acc);
+                        if (acc > best) best = acc;
+                    }
+                scores[(b * nsets + set) * nblk + j] = best;
+            }
+        }
+    return 0;
+}
+
+typedef struct {
+    float score;
+    int32_t index;
+} fkeyed;
+
+static int fbetter_first(const void* a, const void* b) {
+    const fkeyed* x = (const fkeyed*)a;
+    const fkeyed* y = (const fkeyed*)b;
+    if (x->score != y->score) return x->score > y->score ? -1 : 1;
+    return x->index < y->index ? -1 : (x->index > y->index ? 1 : 0);
+}
+
+/* The kc best of nblk block scores under (score desc, index asc), ascending. */
+int oracle_ctx_select(const float* scores, long nblk, long kc, int32_t* blocks) {
+    if (!scores || !blocks || nblk < 1 || kc < 1 || kc > nblk) return ORACLE_ERR_ARG;
+    fkeyed* all = (fkeyed*)malloc(sizeof(fkeyed) * (size_t)nblk);
+    if (!all) return ORACLE_ERR_NOMEM;
+    for (long j = 0; j < nblk; ++j) {
+        if (isnan(scores[j])) {
+            free(all);
+            return ORACLE_ERR_NONFINITE;
+        }
+        all[j].score = scores[j];
+        all[j].index = (int32_t)j;
+    }
+    qsort(all, (size_t)nblk, sizeof(fkeyed), fbetter_first);
+    for (long j = 0; j < kc; ++j) blocks[j] = all[j].index;
+    free(all);
+    qsort(blocks, (size_t)kc, sizeof(int32_t), ascending_int);
+    return 0;
+}
+
+/* Attention with both reductions: the kept head dimensions (k of d, as in
+ * oracle_attention) and the kept context blocks (kc of ceil(L/bc) blocks of
+ * bc keys).  blocks_in ([B][nsets][kc], NULL: select them as above) and
+ * idx_in ([B][nsets][k], NULL: select from Q) supply given sets; blocks_out
+ * and idx_out (may be NULL) receive the sets used. */
+int oracle_attention_ctx(const uint16_t* Q, const uint16_t* K, const uint16_t* V, long B, long Hq,
+                         long Hkv, long T, long L, long d, long k, int causal, double scale,
+                         int per_query_head, long bc, long kc, const int64_t* t_rows, long nrows,
+                         double* O, int32_t* idx_out, int32_t* blocks_out, const int32_t* idx_in,
+                         const int32_t* blocks_in) {
+    if (!Q || !K || !V || !O || B < 1 || Hq < 1 || Hkv < 1 || T < 1 || L < T || d < 1 || bc < 1 ||
+        Hq % Hkv != 0)
+        return ORACLE_ERR_ARG;
+    long nblk = (L + bc - 1) / bc;
+    if (kc < 1 || kc > nblk) return ORACLE_ERR_ARG;
+    long nsets = per_query_head ? Hq : Hkv;
+    int32_t* blocks = (int32_t*)malloc(sizeof(int32_t) * (size_t)(B * nsets * kc));
+    uint8_t* keep = (uint8_t*)calloc((size_t)(B * nsets * L), 1);
+    float* means = NULL;
+    float* scores = NULL;
+    int rc = (blocks && keep) ? 0 : ORACLE_ERR_NOMEM;
+    if (rc == 0 && blocks_in) {
+        memcpy(blocks, blocks_in, sizeof(int32_t) * (size_t)(B * nsets * kc));
+        for (long i = 0; i < B * nsets * kc; ++i)
+            if (blocks[i] < 0 || blocks[i] >= nblk) rc = ORACLE_ERR_ARG;
+    } else if (rc == 0) {
+        means = (float*)malloc(sizeof(float) * (size_t)(B * Hkv * nblk * d));
+        scores = (float*)malloc(sizeof(float) * (size_t)(B * nsets * nblk));
+        if (!means || !scores) rc = ORACLE_ERR_NOMEM;
+        if (rc == 0) rc = oracle_ctx_block_means(K, B, Hkv, L, d, bc, means);
+        if (rc == 0) rc = oracle_ctx_block_scores(Q, means, B, Hq, Hkv, T, nblk, d, per_query_head, scores);
+        for (long i = 0; rc == 0 && i < B * nsets; ++i)
+            rc = oracle_ctx_select(scores + i * nblk, nblk, kc, blocks + i * kc);
+    }
+    for (long i = 0; rc == 0 && i < B * nsets; ++i)
+        for (long j = 0; j < kc; ++j) {
+            long l0 = (long)blocks[i * kc + j] * bc, l1 = l0 + bc < L ? l0 + bc : L;
+            for (long l = l0; l < l1; ++l) keep[i * L + l] = 1;
+        }
+    if (rc == 0 && blocks_out) memcpy(blocks_out, blocks, sizeof(int32_t) * (size_t)(B * nsets * kc));
+    if (rc == 0)
+        rc = attention_core(Q, K, V, B, Hq, Hkv, T, L, d, k, causal, scale, per_query_head, t_rows, nrows, O,
+                            idx_out, idx_in, keep);
+    free(blocks);
+    free(keep);
+    free(means);
+    free(scores);
+    return rc;
+}
+
 
 /* y[t,:] = x[t,:] / sqrt(mean_h x[t,h]^2 + eps)  (norm weight 1). */
 int oracle_rmsnorm(const uint16_t* x, long T, long H, double eps, double* y) {

@@ -382,3 +382,156 @@ def test_linear_blocks_keeps_the_outlier_block_and_splits_the_product():
     dropped = np.array([j for j in range(H) if j // 64 != 5], dtype=np.int32)
     Yd = oracle.reduced_product(X, W, dropped)
     assert np.allclose(Y + Yd, f64(X) @ f64(W).T, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- context blocks
+# cf-1.com post §3.1: keys cut into blocks of consecutive positions, a cheap
+# per-block score (here: the best dot product of a query row with the block's
+# mean key), Q K^T on the kept blocks only.
+
+
+def small_ints(shape, lo, hi, seed):
+    g = np.random.default_rng(seed)
+    return torch.tensor(g.integers(lo, hi + 1, size=shape), dtype=torch.bfloat16)
+
+
+def test_ctx_block_means_exact_on_integers_and_ragged_block():
+    """Integer keys: every float sum is exact; blocks of 64 divide by a power of two, and the
+    ragged last block (3 keys) holds one repeated value, so every mean is exact."""
+    B, Hkv, L, d, bc = 2, 3, 131, 16, 64
+    K = small_ints((B, Hkv, L, d), -8, 8, 81)
+    K[:, :, 128:] = K[:, :, 128:129]  # the last block: three copies of one key
+    m = oracle.ctx_block_means(K, bc)
+    Ki = K.to(torch.int64).numpy()
+    assert m.shape == (B, Hkv, 3, d)
+    assert np.array_equal(m[:, :, 0], Ki[:, :, 0:64].sum(axis=2) / 64)
+    assert np.array_equal(m[:, :, 1], Ki[:, :, 64:128].sum(axis=2) / 64)
+    assert np.array_equal(m[:, :, 2], Ki[:, :, 128])
+
+
+def test_ctx_block_means_close_to_fp64_mean():
+    K = rmm_synth.normal((1, 2, 200, 32), seed=82)
+    m = oracle.ctx_block_means(K, 48)
+    Kf = f64(K)
+    for j in range(5):
+        ref = Kf[:, :, 48 * j:min(200, 48 * (j + 1))].mean(axis=2)
+        assert np.max(np.abs(m[:, :, j] - ref)) <= 1e-5
+
+
+@pytest.mark.parametrize("per_head", [False, True])
+def test_ctx_block_scores_exact_on_integers(per_head):
+    """Integer queries and integer block means (constant keys per block): every fmaf is
+    exact, so the score is the integer max over the set's query rows of the dot product."""
+    B, Hq, Hkv, T, L, d, bc = 1, 4, 2, 3, 256, 16, 64
+    Q = small_ints((B, Hq, T, d), -4, 4, 83)
+    Kb = small_ints((B, Hkv, L // bc, 1, d), -8, 8, 84)
+    K = Kb.expand(B, Hkv, L // bc, bc, d).reshape(B, Hkv, L, d).contiguous()
+    m = oracle.ctx_block_means(K, bc)
+    sc = oracle.ctx_block_scores(Q, m, Hkv, per_query_head=per_head)
+    Qi, Mi = Q.to(torch.int64).numpy(), Kb.to(torch.int64).numpy()[:, :, :, 0]
+    G = Hq // Hkv
+    for s in range(Hq if per_head else Hkv):
+        heads = [s] if per_head else list(range(s * G, (s + 1) * G))
+        g = s // G if per_head else s
+        dots = np.einsum("htd,jd->htj", Qi[0, heads], Mi[0, g])
+        assert np.array_equal(sc[0, s], dots.max(axis=(0, 1)))
+
+
+def test_ctx_block_scores_close_to_fp64():
+    Q = rmm_synth.normal((1, 4, 2, 64), seed=85)
+    K = rmm_synth.normal((1, 1, 320, 64), seed=86)
+    m = oracle.ctx_block_means(K, 64)
+    sc = oracle.ctx_block_scores(Q, m, 1)
+    ref = np.einsum("htd,jd->htj", f64(Q)[0], m[0, 0].astype(np.float64)).max(axis=(0, 1))
+    assert np.max(np.abs(sc[0, 0] - ref)) <= 1e-4
+
+
+@pytest.mark.parametrize("nblk", [1, 4, 7, 10])
+def test_ctx_select_brute_force(nblk):
+    """Over every kc-subset: the kept set is the unique one whose every member beats every
+    dropped block under (score desc, index asc); tie-heavy scores, signed zeros included."""
+    g = np.random.default_rng(87 + nblk)
+    for trial in range(6):
+        sc = g.integers(-2, 3, size=nblk).astype(np.float32)
+        sc[sc == 0] = np.where(g.random(int((sc == 0).sum())) < 0.5, -0.0, 0.0)
+        for kc in range(1, nblk + 1):
+            got = oracle.ctx_select(sc, kc).tolist()
+            valid = []
+            for S in itertools.combinations(range(nblk), kc):
+                out = [j for j in range(nblk) if j not in S]
+                if all(sc[i] > sc[j] or (sc[i] == sc[j] and i < j) for i in S for j in out):
+                    valid.append(list(S))
+            assert valid == [got]
+
+
+def test_ctx_all_blocks_is_the_head_dim_reduction():
+    B, Hq, Hkv, T, L, d = 1, 4, 2, 2, 150, 32
+    Q = rmm_synth.normal((B, Hq, T, d), seed=88)
+    K = rmm_synth.normal((B, Hkv, L, d), seed=89)
+    V = rmm_synth.normal((B, Hkv, L, d), seed=90)
+    O, idx, blocks = oracle.attention_ctx(Q, K, V, 16, 64, 3, causal=True)
+    Oa, ia = oracle.attention(Q, K, V, 16, causal=True)
+    assert np.array_equal(O, Oa) and np.array_equal(idx, ia)
+    assert blocks.tolist() == [[[0, 1, 2], [0, 1, 2]]]
+
+
+@pytest.mark.parametrize("T,causal", [(1, True), (3, True), (2, False)])
+def test_ctx_given_blocks_equal_library_attention_on_gathered_keys(T, causal):
+    """Attention over the kept blocks equals library softmax attention over a cache that
+    holds only those blocks' keys and values (causal mask by original position), with Q
+    masked to the kept head dimensions."""
+    B, Hq, Hkv, L, d, k, bc = 1, 4, 2, 200, 16, 8, 32
+    Q = rmm_synth.normal((B, Hq, T, d), seed=91)
+    K = rmm_synth.normal((B, Hkv, L, d), seed=92)
+    V = rmm_synth.normal((B, Hkv, L, d), seed=93)
+    nblk = -(-L // bc)
+    given = np.array([[[1, 4, 6], [0, 5, 6]]], dtype=np.int32)  # block 6 is the ragged one (8 keys)
+    scale = 1.0 / math.sqrt(d)
+    O, idx, blocks = oracle.attention_ctx(Q, K, V, k, bc, 3, causal=causal, scale=scale, blocks_in=given)
+    assert np.array_equal(blocks, given) and nblk == 7
+    q, Kf, Vf = f64(Q), f64(K), f64(V)
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        pos = np.concatenate([np.arange(j * bc, min(L, (j + 1) * bc)) for j in given[0, g]])
+        qm = np.zeros_like(q[0, h])
+        qm[:, idx[0, g]] = q[0, h][:, idx[0, g]]
+        logits = scale * (qm @ Kf[0, g, pos].T)
+        if causal:
+            last = L - T + np.arange(T)
+            logits = np.where(pos[None, :] <= last[:, None], logits, -np.inf)
+        p = np.exp(logits - logits.max(axis=1, keepdims=True))
+        ref = (p / p.sum(axis=1, keepdims=True)) @ Vf[0, g, pos]
+        assert np.max(np.abs(O[0, h] - ref)) <= 1e-12
+
+
+def test_ctx_dropped_blocks_do_not_matter():
+    """With the kept blocks fixed, keys and values inside dropped blocks leave O unchanged;
+    values there never enter the score, so changing them keeps the selection too."""
+    B, Hq, Hkv, T, L, d = 1, 2, 1, 1, 256, 32
+    Q = rmm_synth.normal((B, Hq, T, d), seed=94)
+    K = rmm_synth.normal((B, Hkv, L, d), seed=95)
+    V = rmm_synth.normal((B, Hkv, L, d), seed=96)
+    O, idx, blocks = oracle.attention_ctx(Q, K, V, 16, 64, 2)
+    drop = [j for j in range(4) if j not in blocks[0, 0]]
+    V2 = V.clone()
+    K2 = K.clone()
+    for j in drop:
+        V2[:, :, 64 * j:64 * (j + 1)] = rmm_synth.normal((1, 1, 64, d), seed=97 + j)
+        K2[:, :, 64 * j:64 * (j + 1)] = rmm_synth.normal((1, 1, 64, d), seed=197 + j)
+    O_v, _, b_v = oracle.attention_ctx(Q, K, V2, 16, 64, 2)
+    assert np.array_equal(b_v, blocks) and np.array_equal(O_v, O)
+    O_k, _, _ = oracle.attention_ctx(Q, K2, V2, 16, 64, 2, idx_in=idx, blocks_in=blocks)
+    assert np.array_equal(O_k, O)
+
+
+def test_ctx_dominant_block_is_kept_and_unseen_rows_are_zero():
+    B, Hq, Hkv, T, L, d = 1, 1, 1, 3, 130, 16
+    Q = rmm_synth.normal((B, Hq, T, d), seed=98)
+    K = rmm_synth.normal((B, Hkv, L, d), seed=99) * 0.01
+    K[0, 0, 64:128] = (Q[0, 0, 0] * 4).to(torch.bfloat16)  # block 1 points along a query row
+    V = rmm_synth.normal((B, Hkv, L, d), seed=100)
+    _, _, blocks = oracle.attention_ctx(Q, K, V, d, 64, 1, causal=False)
+    assert blocks.tolist() == [[[1]]]
+    # only the ragged block 2 (positions 128, 129) kept: the query at position 127 sees none
+    O, _, _ = oracle.attention_ctx(Q, K, V, d, 64, 1, causal=True, blocks_in=[[[2]]])
+    assert np.all(O[0, 0, 0] == 0.0) and np.any(O[0, 0, 1] != 0.0)
