@@ -204,6 +204,51 @@ rmm_status rmm_attn_qk(const void* Q, const void* Kt, const void* V, int B, int 
                        int32_t* idx_out, void* workspace, size_t workspace_bytes,
                        rmm_stream_t stream, const rmm_options* options);
 
+/* ---------------------------------------------------------------- context blocks
+ *
+ * Reduction of Q K^T along the sequence (cf-1.com post §3.1: in generation,
+ * cut the cached keys into blocks, score the blocks cheaply, run the full
+ * Q K^T only on the blocks that may draw attention; §7: the gain grows with
+ * the context).  Block j holds positions [j*block, min(L, (j+1)*block)),
+ * block in {32, 64, 128, 256}; its summary is its mean key; a kept set's
+ * score for block j is the largest dot product of one of the set's query
+ * rows with that mean; the kc = ceil(r_ctx * nblk) best blocks are kept
+ * (ties to the lower block index); dropped keys take no part in the softmax.
+ * Mean and score are computed in single precision in a fixed order (float
+ * sums over l ascending, one correctly rounded division, an fmaf chain over
+ * the d dims ascending) so the kept blocks are reproducible exactly. */
+
+/* means[b][g][j][c] = (sum over l in block j of Kt[b][g][c][l]) / n_j, fp32,
+ * for the blocks j in [blk_begin, blk_end) (other blocks untouched: refresh
+ * the block that receives a new key after each append).
+ *   Kt    bf16 [B, Hkv, d, ldL], the first L positions valid
+ *   means fp32 [B, Hkv, ceil(ldL / block), d] (caller-owned)
+ * Requirements: d == 128, 1 <= L <= ldL, ldL % 8 == 0, 0 <= blk_begin <
+ * blk_end <= ceil(L / block), 16-byte aligned pointers. */
+rmm_status rmm_ctx_block_means(const void* Kt, int B, int Hkv, int d, int L, int ldL, int block, int blk_begin,
+                               int blk_end, float* means, rmm_stream_t stream);
+
+/* Workspace bytes needed by rmm_attn_ctx for these sizes. */
+size_t rmm_attn_ctx_workspace_bytes(int B, int Hq, int Hkv, int T, int L, int d, int block, double r_ctx,
+                                    const rmm_options* options);
+
+/* Reduced attention with both reductions: the kept head dimensions of
+ * rmm_attn_qk (k = ceil(r*d) per set) and the kept context blocks (kc =
+ * ceil(r_ctx * ceil(L/block)) per set), then softmax over the kept keys and
+ * O = P . V over the full d.  A query row that may attend to no kept key
+ * (possible only with causal chunks) gets O = 0.  Same layouts, scale and
+ * causal rule as rmm_attn_qk; means as written by rmm_ctx_block_means for
+ * every block below ceil(L / block).
+ *   idx_out    int32 [B, nsets, k] or NULL (kept head dimensions, ascending)
+ *   blocks_out int32 [B, nsets, kc] or NULL (kept blocks, ascending)
+ * nsets = Hkv, or Hq with options.attn_per_query_head.  Runs the CUDA-core
+ * split pass: T <= 16 (decode and short chunks), ceil(L/block) <= 2048,
+ * Hq / Hkv <= 8 for per-KV-head sets; RMM_ERR_UNSUPPORTED otherwise. */
+rmm_status rmm_attn_ctx(const void* Q, const void* Kt, const void* V, const float* means, int B, int Hq, int Hkv,
+                        int T, int L, int ldL, int d, double r, double r_ctx, int block, int causal, float scale,
+                        void* O, int32_t* idx_out, int32_t* blocks_out, void* workspace, size_t workspace_bytes,
+                        rmm_stream_t stream, const rmm_options* options);
+
 /* The decode-sized reduced linear map without a workspace.  The pages have
  * no counterpart to this entry point; it exists for callers that cannot give
  * the library device memory of its own: a plugin whose host framework owns

@@ -496,6 +496,90 @@ rmm_status rmm_attn_qk(const void* Q, const void* Kt, const void* V, int B, int 
                                    o.attn_path, p, static_cast<cudaStream_t>(stream)));
 }
 
+// ---------------------------------------------------------------- context blocks
+
+rmm_status rmm_ctx_block_means(const void* Kt, int B, int Hkv, int d, int L, int ldL, int block, int blk_begin,
+                               int blk_end, float* means, rmm_stream_t stream) {
+    if (!Kt || !means || B < 1 || Hkv < 1 || L < 1 || ldL < L || ldL % 8 != 0 || !ctx_block_ok(block))
+        return RMM_ERR_INVALID_ARG;
+    if (!aligned16(Kt) || !aligned16(means)) return RMM_ERR_INVALID_ARG;
+    if (blk_begin < 0 || blk_end <= blk_begin || blk_end > (L + block - 1) / block) return RMM_ERR_INVALID_ARG;
+    if (d != 128) return RMM_ERR_UNSUPPORTED;
+    return cuda_status(launch_ctx_means(static_cast<const uint16_t*>(Kt), B, Hkv, L, ldL, block, blk_begin, blk_end,
+                                        means, static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+
+// workspace of rmm_attn_ctx: status | idx | dims scores (zero between calls) |
+// block keys | kept blocks | split partials
+struct CtxLayout {
+    size_t idx, sc, keys, blocks, partials, total;
+};
+
+CtxLayout ctx_layout(int B, int Hq, int T, int d, int nblk, int kc, const AttnPlan& p) {
+    CtxLayout c;
+    size_t off = kStatusBytes;
+    c.idx = off;
+    off += align_up((size_t)B * p.nsets * d * sizeof(int32_t), kAlign);
+    c.sc = off;
+    off += align_up((size_t)B * p.nsets * d * sizeof(uint32_t), kAlign);
+    c.keys = off;
+    off += align_up((size_t)B * p.nsets * nblk * sizeof(uint32_t), kAlign);
+    c.blocks = off;
+    off += align_up((size_t)B * p.nsets * kc * sizeof(int32_t), kAlign);
+    c.partials = off;
+    off += align_up(attn_partials_bytes(p, B, Hq, T), kAlign);
+    c.total = off;
+    return c;
+}
+
+}  // namespace
+
+size_t rmm_attn_ctx_workspace_bytes(int B, int Hq, int Hkv, int T, int L, int d, int block, double r_ctx,
+                                    const rmm_options* options) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || L < T || d != 128 || Hq % Hkv != 0 || !ctx_block_ok(block) ||
+        !opts_valid(options))
+        return 0;
+    const int nblk = (L + block - 1) / block;
+    const int kc = rmm_k_for(nblk, r_ctx);
+    if (kc < 1) return 0;
+    const rmm_options& o = opts_or_default(options);
+    const AttnPlan p = attn_plan(B, Hq, Hkv, T, kc * block, o.attn_per_query_head, num_sms_current());
+    return ctx_layout(B, Hq, T, d, nblk, kc, p).total;
+}
+
+rmm_status rmm_attn_ctx(const void* Q, const void* Kt, const void* V, const float* means, int B, int Hq, int Hkv,
+                        int T, int L, int ldL, int d, double r, double r_ctx, int block, int causal, float scale,
+                        void* O, int32_t* idx_out, int32_t* blocks_out, void* workspace, size_t workspace_bytes,
+                        rmm_stream_t stream, const rmm_options* options) {
+    if (!Q || !Kt || !V || !means || !O || B < 1 || Hq < 1 || Hkv < 1 || T < 1 || L < T || ldL < L ||
+        ldL % 8 != 0 || Hq % Hkv != 0 || !ctx_block_ok(block) || !opts_valid(options))
+        return RMM_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(Kt) || !aligned16(V) || !aligned16(O) || !aligned16(means))
+        return RMM_ERR_INVALID_ARG;
+    if (!(scale > 0.0f) || !isfinite(scale)) return RMM_ERR_INVALID_ARG;
+    if (d != 128) return RMM_ERR_UNSUPPORTED;
+    const int k = rmm_k_for(d, r);
+    const int nblk = (L + block - 1) / block;
+    const int kc = rmm_k_for(nblk, r_ctx);
+    if (k < 1 || kc < 1) return RMM_ERR_INVALID_ARG;
+    const rmm_options& o = opts_or_default(options);
+    if (T > kCtxMaxT || nblk > kCtxMaxBlocks || (!o.attn_per_query_head && Hq / Hkv > 8))
+        return RMM_ERR_UNSUPPORTED;
+    const AttnPlan p = attn_plan(B, Hq, Hkv, T, kc * block, o.attn_per_query_head, num_sms_current());
+    const CtxLayout c = ctx_layout(B, Hq, T, d, nblk, kc, p);
+    if (!workspace || workspace_bytes < c.total || !aligned16(workspace)) return RMM_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + c.idx);
+    int32_t* blocks = blocks_out ? blocks_out : reinterpret_cast<int32_t*>(ws + c.blocks);
+    return cuda_status(launch_attn_ctx(
+        static_cast<const uint16_t*>(Q), static_cast<const uint16_t*>(Kt), static_cast<const uint16_t*>(V), means, B,
+        Hq, Hkv, T, L, ldL, k, block, kc, causal ? 1 : 0, scale, o.attn_per_query_head, static_cast<uint16_t*>(O),
+        idx, reinterpret_cast<uint32_t*>(ws + c.sc), reinterpret_cast<uint32_t*>(ws + c.keys), blocks,
+        reinterpret_cast<float*>(ws + c.partials), p, static_cast<cudaStream_t>(stream)));
+}
+
 rmm_status rmm_add_rmsnorm(const void* X, const void* R, int T, int H, float eps, const void* weight, void* Hsum,
                            void* Y, rmm_stream_t stream) {
     if (!X || (!Hsum && !Y) || T < 1 || H < 8 || H % 8 != 0 || H > 16384 || !(eps >= 0.0f)) return RMM_ERR_INVALID_ARG;

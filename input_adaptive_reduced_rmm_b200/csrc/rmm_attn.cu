@@ -39,7 +39,7 @@ namespace {
 constexpr int D = 128;        // head dimension handled by this build
 constexpr int kThreads = 256;
 constexpr int SB = 1024;      // keys per sub-block
-constexpr int RMAX = 8;       // query rows per CTA
+constexpr int RMAX = 8;       // query rows per CTA (at most)
 constexpr int PSTRIDE = D + 2;  // floats per split partial: m, l, O[d]
 
 // ---------------------------------------------------------------- selection
@@ -136,21 +136,30 @@ __global__ void __launch_bounds__(D)
 
 // ---------------------------------------------------------------- split pass
 
-__global__ void __launch_bounds__(kThreads)
+// kCtx: the keys are the kept context blocks only.  The split then runs over
+// Lv = kc * 2^bc_shift virtual positions: position v is key
+// blocks[set][v >> bc_shift] * 2^bc_shift + (v mod 2^bc_shift) of the cache, and
+// positions at or past L (the ragged last block) are masked.  Without kCtx,
+// Lv = L and position v is key v.
+// kRows (4 or 8): query rows per CTA; 4 when a set has at most 4 rows per
+// call (decode with up to 4 query heads per KV head), halving the registers.
+template <bool kCtx, int kRows>
+__global__ void __launch_bounds__(kThreads, kRows == 4 ? 2 : 1)
     attn_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ Kt,
                       const uint16_t* __restrict__ V, int Hq, int Hkv, int T, int L, int ldL, int k,
                       int causal, float scale, int per_query_head, const int32_t* __restrict__ idx,
-                      float* __restrict__ partials, int chunk, int tq) {
-    __shared__ float qs[RMAX][D];      // scaled kept query values
+                      float* __restrict__ partials, int chunk, int tq, int Lv,
+                      const int32_t* __restrict__ blocks, int bc_shift, int kc) {
+    __shared__ float qs[kRows][D];      // scaled kept query values
     __shared__ int sidx[D];
     // One buffer, two uses: logits/probabilities of the current sub-block
-    // [RMAX][SB] inside the key loop, the cross-warp fold of P.V [8][RMAX][D]
+    // [kRows][SB] inside the key loop, the cross-warp fold of P.V [8][kRows][D]
     // after it (both 32 KB).
-    __shared__ float buf[RMAX * SB];
+    __shared__ float buf[kRows * SB];
     float (*lg)[SB] = reinterpret_cast<float (*)[SB]>(buf);
-    float (*red)[RMAX][D] = reinterpret_cast<float (*)[RMAX][D]>(buf);
-    static_assert(8 * RMAX * D <= RMAX * SB, "fold buffer must fit in the logits buffer");
-    __shared__ float m_run[RMAX], l_run[RMAX], alpha[RMAX];
+    float (*red)[kRows][D] = reinterpret_cast<float (*)[kRows][D]>(buf);
+    static_assert(8 * kRows * D <= kRows * SB, "fold buffer must fit in the logits buffer");
+    __shared__ float m_run[kRows], l_run[kRows], alpha[kRows];
 
     const int nsets = per_query_head ? Hq : Hkv;
     const int set = blockIdx.x % nsets;
@@ -163,7 +172,14 @@ __global__ void __launch_bounds__(kThreads)
     const int nsplit = gridDim.y;
     const int t0 = blockIdx.z * tq;
     const int l_begin = split * chunk;
-    const int l_end = min(L, l_begin + chunk);
+    const int l_end = min(Lv, l_begin + chunk);
+    const int32_t* __restrict__ set_blocks = kCtx ? blocks + (size_t)blockIdx.x * kc : nullptr;
+    const int bc_mask = (1 << bc_shift) - 1;
+    // cache position of virtual position v (4-aligned v gives a 4-aligned position)
+    auto key_pos = [&](int v) -> int {
+        if constexpr (kCtx) return (__ldg(set_blocks + (v >> bc_shift)) << bc_shift) + (v & bc_mask);
+        return v;
+    };
     const int R = nq * tq;  // rows: r = qi * tq + ti
     const int tid = threadIdx.x;
     pdl_wait();
@@ -171,7 +187,7 @@ __global__ void __launch_bounds__(kThreads)
 
     for (int i = tid; i < k; i += kThreads) sidx[i] = idx[(size_t)blockIdx.x * k + i];
     __syncthreads();
-    for (int e = tid; e < RMAX * D; e += kThreads) {
+    for (int e = tid; e < kRows * D; e += kThreads) {
         const int r = e / D, jj = e % D;
         float v = 0.0f;
         if (r < R && jj < k) {
@@ -180,16 +196,16 @@ __global__ void __launch_bounds__(kThreads)
         }
         qs[r][jj] = v;
     }
-    if (tid < RMAX) {
+    if (tid < kRows) {
         m_run[tid] = -INFINITY;
         l_run[tid] = 0.0f;
     }
     __syncthreads();
 
     // last key each row may see
-    int last[RMAX];
+    int last[kRows];
 #pragma unroll
-    for (int r = 0; r < RMAX; ++r) {
+    for (int r = 0; r < kRows; ++r) {
         const int ti = (r < R) ? r % tq : 0;
         const int t = t0 + ti;
         last[r] = (r < R && t < T) ? (causal ? (L - T + t) : (L - 1)) : -1;
@@ -200,47 +216,56 @@ __global__ void __launch_bounds__(kThreads)
 
     // P.V mapping: 16 column groups of 8 dims x 16 key groups
     const int cgp = tid & 15, kg = tid >> 4;
-    float acc[RMAX][8];
+    float acc[kRows][8];
 #pragma unroll
-    for (int r = 0; r < RMAX; ++r)
+    for (int r = 0; r < kRows; ++r)
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[r][c] = 0.0f;
 
     for (int l0 = l_begin; l0 < l_end; l0 += SB) {
         // ---- logits: thread owns keys l0 + 4*tid .. +3
         const int l = l0 + tid * 4;
-        float s4[RMAX][4];
+        const int lp = l < l_end ? key_pos(l) : L;  // cache position of the thread's first key
+        float s4[kRows][4];
 #pragma unroll
-        for (int r = 0; r < RMAX; ++r)
+        for (int r = 0; r < kRows; ++r)
 #pragma unroll
             for (int c = 0; c < 4; ++c) s4[r][c] = 0.0f;
-        if (l < l_end) {
-            for (int jj = 0; jj < k; ++jj) {
-                const uint2 kv = ld_nc_v2(kbase + (size_t)sidx[jj] * ldL + l);
-                const float k0 = __uint_as_float(kv.x << 16), k1 = __uint_as_float(kv.x & 0xFFFF0000u);
-                const float k2 = __uint_as_float(kv.y << 16), k3 = __uint_as_float(kv.y & 0xFFFF0000u);
+        if (lp < L) {  // lp + 3 < roundup(L, 4) <= ldL: the 8-byte load stays in the row
+            // kUnrollK kept rows per step: their loads are all in flight before the FMAs
+            constexpr int kUnrollK = kRows == 4 ? 16 : 8;
+            for (int jj0 = 0; jj0 < k; jj0 += kUnrollK) {
+                uint2 kv[kUnrollK];
 #pragma unroll
-                for (int r = 0; r < RMAX; ++r) {
-                    const float qv = qs[r][jj];
-                    s4[r][0] = fmaf(qv, k0, s4[r][0]);
-                    s4[r][1] = fmaf(qv, k1, s4[r][1]);
-                    s4[r][2] = fmaf(qv, k2, s4[r][2]);
-                    s4[r][3] = fmaf(qv, k3, s4[r][3]);
+                for (int u = 0; u < kUnrollK; ++u)
+                    kv[u] = jj0 + u < k ? ld_nc_v2(kbase + (size_t)sidx[jj0 + u] * ldL + lp) : make_uint2(0u, 0u);
+#pragma unroll
+                for (int u = 0; u < kUnrollK; ++u) {
+                    const float k0 = __uint_as_float(kv[u].x << 16), k1 = __uint_as_float(kv[u].x & 0xFFFF0000u);
+                    const float k2 = __uint_as_float(kv[u].y << 16), k3 = __uint_as_float(kv[u].y & 0xFFFF0000u);
+#pragma unroll
+                    for (int r = 0; r < kRows; ++r) {
+                        const float qv = qs[r][jj0 + u];  // zero past k
+                        s4[r][0] = fmaf(qv, k0, s4[r][0]);
+                        s4[r][1] = fmaf(qv, k1, s4[r][1]);
+                        s4[r][2] = fmaf(qv, k2, s4[r][2]);
+                        s4[r][3] = fmaf(qv, k3, s4[r][3]);
+                    }
                 }
             }
         }
 #pragma unroll
-        for (int r = 0; r < RMAX; ++r)
+        for (int r = 0; r < kRows; ++r)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const int lc = l + c;
-                lg[r][tid * 4 + c] = (lc < l_end && lc <= last[r]) ? s4[r][c] : -INFINITY;
+                const int lc = lp + c;
+                lg[r][tid * 4 + c] = (l + c < l_end && lc < L && lc <= last[r]) ? s4[r][c] : -INFINITY;
             }
         __syncthreads();
 
         // ---- online softmax, one warp per row
         const int warp = tid >> 5, lane = tid & 31;
-        for (int r = warp; r < RMAX; r += kThreads / 32) {
+        for (int r = warp; r < kRows; r += kThreads / 32) {
             float mx = -INFINITY;
             for (int i = lane; i < SB; i += 32) mx = fmaxf(mx, lg[r][i]);
 #pragma unroll
@@ -270,24 +295,38 @@ __global__ void __launch_bounds__(kThreads)
 
         // ---- P.V
 #pragma unroll
-        for (int r = 0; r < RMAX; ++r) {
+        for (int r = 0; r < kRows; ++r) {
             const float a = alpha[r];
 #pragma unroll
             for (int c = 0; c < 8; ++c) acc[r][c] *= a;
         }
         const int nkeys = min(SB, l_end - l0);
-        for (int i = kg; i < nkeys; i += 16) {
-            const uint4 v = ld_nc_v4(vbase + (size_t)(l0 + i) * D + cgp * 8);
-            float vf[8];
-            vf[0] = __uint_as_float(v.x << 16); vf[1] = __uint_as_float(v.x & 0xFFFF0000u);
-            vf[2] = __uint_as_float(v.y << 16); vf[3] = __uint_as_float(v.y & 0xFFFF0000u);
-            vf[4] = __uint_as_float(v.z << 16); vf[5] = __uint_as_float(v.z & 0xFFFF0000u);
-            vf[6] = __uint_as_float(v.w << 16); vf[7] = __uint_as_float(v.w & 0xFFFF0000u);
+        // kUnrollV V rows per step, their loads in flight together
+        constexpr int kUnrollV = 4;
+        for (int i0 = kg; i0 < nkeys; i0 += 16 * kUnrollV) {
+            uint4 v[kUnrollV];
 #pragma unroll
-            for (int r = 0; r < RMAX; ++r) {
-                const float p = lg[r][i];
+            for (int u = 0; u < kUnrollV; ++u) {
+                const int i = i0 + 16 * u;
+                const int lv = i < nkeys ? key_pos(l0 + i) : L;
+                // a masked key (probability 0) past the cache's end is not loaded
+                v[u] = lv < L ? ld_nc_v4(vbase + (size_t)lv * D + cgp * 8) : make_uint4(0u, 0u, 0u, 0u);
+            }
 #pragma unroll
-                for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(p, vf[c], acc[r][c]);
+            for (int u = 0; u < kUnrollV; ++u) {
+                const int i = i0 + 16 * u;
+                if (i >= nkeys) break;
+                float vf[8];
+                vf[0] = __uint_as_float(v[u].x << 16); vf[1] = __uint_as_float(v[u].x & 0xFFFF0000u);
+                vf[2] = __uint_as_float(v[u].y << 16); vf[3] = __uint_as_float(v[u].y & 0xFFFF0000u);
+                vf[4] = __uint_as_float(v[u].z << 16); vf[5] = __uint_as_float(v[u].z & 0xFFFF0000u);
+                vf[6] = __uint_as_float(v[u].w << 16); vf[7] = __uint_as_float(v[u].w & 0xFFFF0000u);
+#pragma unroll
+                for (int r = 0; r < kRows; ++r) {
+                    const float p = lg[r][i];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(p, vf[c], acc[r][c]);
+                }
             }
         }
         __syncthreads();  // lg is rewritten by the next sub-block
@@ -295,13 +334,13 @@ __global__ void __launch_bounds__(kThreads)
 
     // fold the 16 key groups: pairs within a warp by shuffle, then 8 warps via smem
 #pragma unroll
-    for (int r = 0; r < RMAX; ++r)
+    for (int r = 0; r < kRows; ++r)
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[r][c] += __shfl_xor_sync(0xffffffffu, acc[r][c], 16);
     const int warp = tid >> 5, lane = tid & 31;
     if (lane < 16) {
 #pragma unroll
-        for (int r = 0; r < RMAX; ++r)
+        for (int r = 0; r < kRows; ++r)
 #pragma unroll
             for (int c = 0; c < 8; ++c) red[warp][r][cgp * 8 + c] = acc[r][c];
     }
@@ -341,7 +380,8 @@ __global__ void __launch_bounds__(D)
         den += w * p[s * PSTRIDE + 1];
         num += w * p[s * PSTRIDE + 2 + threadIdx.x];
     }
-    O[row * D + threadIdx.x] = float_to_bf16_bits(num / den);
+    // a row that saw no key (only with kept context blocks) is zero
+    O[row * D + threadIdx.x] = float_to_bf16_bits(den > 0.0f ? num / den : 0.0f);
 }
 
 }  // namespace
@@ -350,7 +390,8 @@ AttnPlan attn_plan(int B, int Hq, int Hkv, int T, int L, int per_query_head, int
     AttnPlan p;
     p.nsets = per_query_head ? Hq : Hkv;
     const int nq = per_query_head ? 1 : Hq / Hkv;
-    p.tq = RMAX / nq;
+    p.rows = (nq <= 4 && nq * T <= 4) ? 4 : RMAX;
+    p.tq = p.rows / nq;
     if (p.tq < 1) p.tq = 1;
     if (p.tq > T) p.tq = T;
     const long long base = (long long)B * p.nsets * ((T + p.tq - 1) / p.tq);
@@ -369,21 +410,42 @@ size_t attn_partials_bytes(const AttnPlan& p, int B, int Hq, int T) {
     return (size_t)B * Hq * T * p.nsplit * PSTRIDE * sizeof(float);
 }
 
-cudaError_t launch_attn(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq,
-                        int Hkv, int T, int L, int ldL, int k, int causal, float scale,
-                        int per_query_head, uint16_t* O, int32_t* idx, float* partials, uint32_t* sc,
-                        int* status, int path, const AttnPlan& p, cudaStream_t stream) {
+cudaError_t launch_attn_dims(const uint16_t* Q, int B, int Hq, int Hkv, int T, int k, int per_query_head, int nsets,
+                             int32_t* idx, uint32_t* sc, cudaStream_t stream) {
     const int nq = per_query_head ? 1 : Hq / Hkv;
     // the kept sets: the column max over many CTAs when the chunk is long
     cudaError_t e;
     const bool wide = nq * T >= 64;
     if (wide) {
-        e = launch_pdl(attn_score_kernel, dim3(B * p.nsets, (nq * T + 63) / 64), dim3(256), 0, stream, Q, Hq, Hkv, T,
+        e = launch_pdl(attn_score_kernel, dim3(B * nsets, (nq * T + 63) / 64), dim3(256), 0, stream, Q, Hq, Hkv, T,
                        per_query_head, sc);
         if (e != cudaSuccess) return e;
     }
-    e = launch_pdl(attn_select_kernel, dim3(B * p.nsets), dim3(D), 0, stream, Q, Hq, Hkv, T, k, per_query_head,
-                   wide ? sc : (uint32_t*)nullptr, idx);
+    return launch_pdl(attn_select_kernel, dim3(B * nsets), dim3(D), 0, stream, Q, Hq, Hkv, T, k, per_query_head,
+                      wide ? sc : (uint32_t*)nullptr, idx);
+}
+
+cudaError_t launch_attn_split_ctx(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq, int Hkv,
+                                  int T, int L, int ldL, int k, int causal, float scale, int per_query_head,
+                                  uint16_t* O, const int32_t* idx, const int32_t* blocks, int bc_shift, int kc,
+                                  float* partials, const AttnPlan& p, cudaStream_t stream) {
+    const int nq = per_query_head ? 1 : Hq / Hkv;
+    if (nq > RMAX) return cudaErrorInvalidValue;
+    dim3 grid(B * p.nsets, p.nsplit, (T + p.tq - 1) / p.tq);
+    cudaError_t e = launch_pdl(p.rows == 4 ? attn_split_kernel<true, 4> : attn_split_kernel<true, RMAX>, grid,
+                               dim3(kThreads), 0, stream, Q, Kt, V, Hq, Hkv, T, L, ldL, k, causal, scale,
+                               per_query_head, idx, partials, p.chunk, p.tq, kc << bc_shift, blocks, bc_shift, kc);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(attn_combine_kernel, dim3(B * Hq * T), dim3(D), 0, stream, (const float*)partials, p.nsplit,
+                      O);
+}
+
+cudaError_t launch_attn(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq,
+                        int Hkv, int T, int L, int ldL, int k, int causal, float scale,
+                        int per_query_head, uint16_t* O, int32_t* idx, float* partials, uint32_t* sc,
+                        int* status, int path, const AttnPlan& p, cudaStream_t stream) {
+    const int nq = per_query_head ? 1 : Hq / Hkv;
+    cudaError_t e = launch_attn_dims(Q, B, Hq, Hkv, T, k, per_query_head, p.nsets, idx, sc, stream);
     if (e != cudaSuccess) return e;
     const bool tc = path == 2 || (path == 0 && attn_tc_supported(T, k));
     if (tc)
@@ -391,8 +453,9 @@ cudaError_t launch_attn(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V
                               stream);
     if (nq > RMAX) return cudaErrorInvalidValue;
     dim3 grid(B * p.nsets, p.nsplit, (T + p.tq - 1) / p.tq);
-    e = launch_pdl(attn_split_kernel, grid, dim3(kThreads), 0, stream, Q, Kt, V, Hq, Hkv, T, L, ldL, k, causal,
-                   scale, per_query_head, (const int32_t*)idx, partials, p.chunk, p.tq);
+    e = launch_pdl(p.rows == 4 ? attn_split_kernel<false, 4> : attn_split_kernel<false, RMAX>, grid, dim3(kThreads), 0,
+                   stream, Q, Kt, V, Hq, Hkv, T, L, ldL, k, causal, scale, per_query_head, (const int32_t*)idx,
+                   partials, p.chunk, p.tq, L, (const int32_t*)nullptr, 0, 0);
     if (e != cudaSuccess) return e;
     return launch_pdl(attn_combine_kernel, dim3(B * Hq * T), dim3(D), 0, stream, (const float*)partials, p.nsplit,
                       O);

@@ -1,0 +1,215 @@
+// rmm_ctx.cu -- context-block reduction of Q K^T (the sequence direction).
+//
+// Input-adaptive matrix-product reduction for LLM inference (cf-1.com post),
+// §3.1: in generation the cached keys are cut into blocks of consecutive
+// positions, a cheap score tells which blocks may draw real attention, and
+// the full Q K^T (and softmax . V) runs on the kept blocks only; §7: the gain
+// grows with the context.  Readings of what the post leaves open:
+//   block j       positions [j*bc, min(L, (j+1)*bc)), bc in {32, 64, 128, 256}
+//   summary       the block's mean key  mean_j[c] = (sum_l K[l,c]) / n_j, kept
+//                 beside the cache (fp32 [B, Hkv, ceil(ldL/bc), d]) and
+//                 refreshed for the blocks that change as keys are appended
+//   score         for a kept set (a KV head's stacked query rows, or one
+//                 query head's rows): the largest dot product of one of its
+//                 query rows with mean_j
+//   kept blocks   kc = ceil(r_ctx * nblk) best under (score desc, index asc),
+//                 ascending; keys of dropped blocks take no part in the
+//                 softmax
+// Summary and score decide an integer set, so they are computed in single
+// precision in one fixed order: float additions over l ascending from 0,
+// then one correctly rounded division by n_j; the dot product as an fmaf
+// chain over c ascending from 0.
+//
+// Kernels:
+//   ctx_means_kernel   one CTA per (block, KV head), thread c sums row c of
+//                      the d-major K^T cache over the block (16-byte loads)
+//   ctx_score_kernel   one thread per (set, block): the set's query rows
+//                      staged in shared memory 16 at a time, four fmaf chains
+//                      in flight; the best dot written as an order-preserving
+//                      32-bit key (-0 and +0 share a key)
+//   ctx_select_kernel  one CTA per set: bitonic sort of (key desc, block asc)
+//                      over up to 2048 blocks, then the kept blocks listed in
+//                      ascending order by one block-wide scan
+// The attention itself is the split pass of rmm_attn.cu over the kept blocks.
+#include <math.h>
+
+#include "rmm_common.cuh"
+#include "rmm_internal.h"
+
+namespace rmm {
+
+namespace {
+
+constexpr int D = 128;
+constexpr int kSelThreads = 1024;
+
+__global__ void __launch_bounds__(D)
+    ctx_means_kernel(const uint16_t* __restrict__ Kt, int L, int ldL, int bc, int blk_begin, int nblk_stride,
+                     float* __restrict__ means) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int j = blk_begin + blockIdx.x;
+    const int bg = blockIdx.y;  // b * Hkv + g
+    const int c = threadIdx.x;
+    const int l0 = j * bc, l1 = min(L, l0 + bc);
+    const uint16_t* row = Kt + ((size_t)bg * D + c) * ldL;
+    float sum = 0.0f;
+    int l = l0;
+    for (; l + 8 <= l1; l += 8) {  // l0 is a multiple of 32 and ldL of 8: 16-byte aligned
+        const uint4 v = ld_nc_v4(row + l);
+        sum += __uint_as_float(v.x << 16);
+        sum += __uint_as_float(v.x & 0xFFFF0000u);
+        sum += __uint_as_float(v.y << 16);
+        sum += __uint_as_float(v.y & 0xFFFF0000u);
+        sum += __uint_as_float(v.z << 16);
+        sum += __uint_as_float(v.z & 0xFFFF0000u);
+        sum += __uint_as_float(v.w << 16);
+        sum += __uint_as_float(v.w & 0xFFFF0000u);
+    }
+    for (; l < l1; ++l) sum += bf16_bits_to_float(row[l]);
+    means[((size_t)bg * nblk_stride + j) * D + c] = __fdiv_rn(sum, (float)(l1 - l0));
+}
+
+// Order-preserving key of a finite float: larger float, larger key; -0 -> +0.
+__device__ __forceinline__ uint32_t float_key(float f) {
+    if (f == 0.0f) f = 0.0f;
+    const uint32_t b = __float_as_uint(f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__global__ void __launch_bounds__(128)
+    ctx_score_kernel(const uint16_t* __restrict__ Q, const float* __restrict__ means, int Hq, int Hkv, int T,
+                     int nblk, int nblk_stride, int per_query_head, uint32_t* __restrict__ keys) {
+    __shared__ float qs[16][D];
+    const int nsets = per_query_head ? Hq : Hkv;
+    const int set = blockIdx.y % nsets;
+    const int b = blockIdx.y / nsets;
+    const int G = Hq / Hkv;
+    const int g = per_query_head ? set / G : set;
+    const int q_lo = per_query_head ? set : set * G;
+    const int nq = per_query_head ? 1 : G;
+    const int R = nq * T;
+    const int j = blockIdx.x * 128 + threadIdx.x;
+    const bool valid = j < nblk;
+    const float4* m4 = reinterpret_cast<const float4*>(means + ((size_t)(b * Hkv + g) * nblk_stride + (valid ? j : 0)) * D);
+    pdl_wait();
+    pdl_launch_dependents();
+    float best = -INFINITY;
+    for (int r0 = 0; r0 < R; r0 += 16) {
+        __syncthreads();
+        for (int e = threadIdx.x; e < 16 * D; e += 128) {
+            const int rr = e / D, c = e % D, r = r0 + rr;
+            float v = 0.0f;
+            if (r < R) v = bf16_bits_to_float(Q[(((size_t)b * Hq + q_lo + r / T) * T + r % T) * D + c]);
+            qs[rr][c] = v;
+        }
+        __syncthreads();
+        const int nr = min(16, R - r0);
+        if (valid) {
+            for (int rr = 0; rr < nr; rr += 4) {
+                float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+                for (int c4 = 0; c4 < D / 4; ++c4) {
+                    const float4 mv = __ldg(m4 + c4);
+                    const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int c = 4 * c4 + u;
+                        a0 = fmaf(qs[rr][c], mm[u], a0);
+                        a1 = fmaf(qs[rr + 1][c], mm[u], a1);
+                        a2 = fmaf(qs[rr + 2][c], mm[u], a2);
+                        a3 = fmaf(qs[rr + 3][c], mm[u], a3);
+                    }
+                }
+                if (a0 > best) best = a0;
+                if (rr + 1 < nr && a1 > best) best = a1;
+                if (rr + 2 < nr && a2 > best) best = a2;
+                if (rr + 3 < nr && a3 > best) best = a3;
+            }
+        }
+    }
+    if (valid) keys[(size_t)blockIdx.y * nblk + j] = float_key(best);
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+    ctx_select_kernel(const uint32_t* __restrict__ keys, int nblk, int P, int kc, int32_t* __restrict__ blocks) {
+    extern __shared__ uint64_t v[];  // P entries
+    __shared__ uint8_t flag[2 * kSelThreads];
+    __shared__ int warp_sum[kSelThreads / 32];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int tid = threadIdx.x;
+    const uint32_t* key = keys + (size_t)blockIdx.x * nblk;
+    // ascending order of (~key, block) = (score desc, block asc)
+    for (int i = tid; i < P; i += kSelThreads)
+        v[i] = i < nblk ? ((uint64_t)(~key[i]) << 32) | (uint32_t)i : ~0ull;
+    for (int i = tid; i < 2 * kSelThreads; i += kSelThreads) flag[i] = 0;
+    __syncthreads();
+    for (int k2 = 2; k2 <= P; k2 <<= 1)
+        for (int jj = k2 >> 1; jj > 0; jj >>= 1) {
+            for (int i = tid; i < P; i += kSelThreads) {
+                const int ixj = i ^ jj;
+                if (ixj > i) {
+                    const uint64_t a = v[i], c = v[ixj];
+                    if ((a > c) == ((i & k2) == 0)) {
+                        v[i] = c;
+                        v[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    for (int i = tid; i < kc; i += kSelThreads) flag[(uint32_t)v[i]] = 1;
+    __syncthreads();
+    // thread t owns blocks 2t and 2t+1: exclusive scan of the kept counts
+    const int cnt = flag[2 * tid] + flag[2 * tid + 1];
+    const int lane = tid & 31, warp = tid >> 5;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    int pos = incl - cnt;
+    for (int w = 0; w < warp; ++w) pos += warp_sum[w];
+    int32_t* out = blocks + (size_t)blockIdx.x * kc;
+    if (flag[2 * tid]) out[pos++] = 2 * tid;
+    if (flag[2 * tid + 1]) out[pos] = 2 * tid + 1;
+}
+
+}  // namespace
+
+bool ctx_block_ok(int bc) { return bc == 32 || bc == 64 || bc == 128 || bc == 256; }
+
+cudaError_t launch_ctx_means(const uint16_t* Kt, int B, int Hkv, int L, int ldL, int bc, int blk_begin, int blk_end,
+                             float* means, cudaStream_t stream) {
+    const int nblk_stride = (ldL + bc - 1) / bc;
+    return launch_pdl(ctx_means_kernel, dim3(blk_end - blk_begin, B * Hkv), dim3(D), 0, stream, Kt, L, ldL, bc,
+                      blk_begin, nblk_stride, means);
+}
+
+cudaError_t launch_attn_ctx(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, const float* means, int B,
+                            int Hq, int Hkv, int T, int L, int ldL, int k, int bc, int kc, int causal, float scale,
+                            int per_query_head, uint16_t* O, int32_t* idx, uint32_t* sc, uint32_t* keys,
+                            int32_t* blocks, float* partials, const AttnPlan& p, cudaStream_t stream) {
+    const int nblk = (L + bc - 1) / bc;
+    const int nblk_stride = (ldL + bc - 1) / bc;
+    int P = 2;
+    while (P < nblk) P <<= 1;
+    if (P > 2 * kSelThreads) return cudaErrorInvalidValue;
+    int bc_shift = 0;
+    while ((1 << bc_shift) < bc) ++bc_shift;
+    cudaError_t e = launch_attn_dims(Q, B, Hq, Hkv, T, k, per_query_head, p.nsets, idx, sc, stream);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(ctx_score_kernel, dim3((nblk + 127) / 128, B * p.nsets), dim3(128), 0, stream, Q, means, Hq, Hkv,
+                   T, nblk, nblk_stride, per_query_head, keys);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(ctx_select_kernel, dim3(B * p.nsets), dim3(kSelThreads), (size_t)P * sizeof(uint64_t), stream,
+                   (const uint32_t*)keys, nblk, P, kc, blocks);
+    if (e != cudaSuccess) return e;
+    return launch_attn_split_ctx(Q, Kt, V, B, Hq, Hkv, T, L, ldL, k, causal, scale, per_query_head, O, idx, blocks,
+                                 bc_shift, kc, partials, p, stream);
+}
+
+}  // namespace rmm

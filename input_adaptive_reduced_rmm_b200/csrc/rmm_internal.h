@@ -138,6 +138,7 @@ struct AttnPlan {
     int nsplit;   // splits over L
     int tq;       // query tokens per CTA
     int nsets;    // kept sets per batch (Hkv or Hq)
+    int rows;     // query rows per CTA of the split pass (4 or 8)
 };
 AttnPlan attn_plan(int B, int Hq, int Hkv, int T, int L, int per_query_head, int num_sms);
 size_t attn_partials_bytes(const AttnPlan& p, int B, int Hq, int T);
@@ -148,6 +149,29 @@ cudaError_t launch_attn(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V
                         int Hkv, int T, int L, int ldL, int k, int causal, float scale,
                         int per_query_head, uint16_t* O, int32_t* idx, float* partials, uint32_t* sc,
                         int* status, int path, const AttnPlan& plan, cudaStream_t stream);
+// The kept head dimensions alone (score + select), as launch_attn runs them.
+cudaError_t launch_attn_dims(const uint16_t* Q, int B, int Hq, int Hkv, int T, int k, int per_query_head, int nsets,
+                             int32_t* idx, uint32_t* sc, cudaStream_t stream);
+// The split pass + combine over kept context blocks (kc blocks of 2^bc_shift
+// keys per set, blocks [B * nsets * kc]); plan made for kc << bc_shift keys.
+cudaError_t launch_attn_split_ctx(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq, int Hkv,
+                                  int T, int L, int ldL, int k, int causal, float scale, int per_query_head,
+                                  uint16_t* O, const int32_t* idx, const int32_t* blocks, int bc_shift, int kc,
+                                  float* partials, const AttnPlan& p, cudaStream_t stream);
+
+// ---- context-block reduction (rmm_ctx.cu)
+constexpr int kCtxMaxBlocks = 2048;  // blocks per cache the select kernel sorts
+constexpr int kCtxMaxT = 16;         // query tokens per call (decode and short chunks)
+bool ctx_block_ok(int bc);
+// Block means of blocks [blk_begin, blk_end): means fp32 [B, Hkv, ceil(ldL/bc), d].
+cudaError_t launch_ctx_means(const uint16_t* Kt, int B, int Hkv, int L, int ldL, int bc, int blk_begin, int blk_end,
+                             float* means, cudaStream_t stream);
+// Dims select, block scores, block select, then the split pass over the kept
+// blocks.  keys: u32 [B * nsets * nblk]; blocks: int32 [B * nsets * kc].
+cudaError_t launch_attn_ctx(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, const float* means, int B,
+                            int Hq, int Hkv, int T, int L, int ldL, int k, int bc, int kc, int causal, float scale,
+                            int per_query_head, uint16_t* O, int32_t* idx, uint32_t* sc, uint32_t* keys,
+                            int32_t* blocks, float* partials, const AttnPlan& p, cudaStream_t stream);
 
 // ---- glue (rmm_glue.cu)
 cudaError_t launch_transpose(const uint16_t* W, uint16_t* Wt, int N, int H, cudaStream_t stream);

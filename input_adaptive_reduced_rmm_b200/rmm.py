@@ -30,6 +30,7 @@ EXPORTED = (
     "rmm_select", "rmm_gemm_reduced", "rmm_attn_workspace_bytes", "rmm_attn_qk",
     "rmm_linear_decode_noalloc", "rmm_linear_group", "rmm_linear_group_workspace_bytes",
     "rmm_add_rmsnorm", "rmm_swiglu", "rmm_qkv_heads", "rmm_heads_to_tokens",
+    "rmm_ctx_block_means", "rmm_attn_ctx_workspace_bytes", "rmm_attn_ctx",
 )
 
 
@@ -107,6 +108,9 @@ def lib() -> ctypes.CDLL:
         "rmm_swiglu": (I, [P, P, ctypes.c_int64, P, P]),
         "rmm_qkv_heads": (I, [P, P, P, I, I, I, I, P, P, P, I, I, P]),
         "rmm_heads_to_tokens": (I, [P, I, I, I, P, P]),
+        "rmm_ctx_block_means": (I, [P, I, I, I, I, I, I, I, I, P, P]),
+        "rmm_attn_ctx_workspace_bytes": (Z, [I, I, I, I, I, I, I, D, OP]),
+        "rmm_attn_ctx": (I, [P, P, P, P, I, I, I, I, I, I, I, D, D, I, I, F, P, P, P, P, Z, P, OP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -299,6 +303,65 @@ def rmm_attn_qk(Q: torch.Tensor, Kt: torch.Tensor, V: torch.Tensor, L: int, r: f
     _check(lib().rmm_attn_qk(_ptr(Q), _ptr(Kt), _ptr(V), B, Hq, Hkv, T, int(L), ldL, d, float(r),
                              int(bool(causal)), float(scale), _ptr(O), _ptr(idx_out), _ptr(workspace),
                              workspace.numel(), _stream(stream), _opt(opts)), "rmm_attn_qk")
+    return O
+
+
+def ctx_num_blocks(L: int, block: int) -> int:
+    return -(-int(L) // int(block))
+
+
+def new_ctx_means(Kt: torch.Tensor, block: int) -> torch.Tensor:
+    """A zeroed block-mean buffer for the key cache Kt [B,Hkv,d,ldL]: fp32 [B,Hkv,ceil(ldL/block),d]."""
+    B, Hkv, d, ldL = Kt.shape
+    return torch.zeros(B, Hkv, ctx_num_blocks(ldL, block), d, dtype=torch.float32, device=Kt.device)
+
+
+def rmm_ctx_block_means(Kt: torch.Tensor, L: int, block: int, means: torch.Tensor | None = None,
+                        blk_begin: int = 0, blk_end: int | None = None, stream=None) -> torch.Tensor:
+    """Mean key of the context blocks [blk_begin, blk_end) of the first L cache positions
+    (all of them by default), written into means (fp32 [B,Hkv,ceil(ldL/block),d])."""
+    _bf16_cuda(Kt, "Kt")
+    B, Hkv, d, ldL = Kt.shape
+    if means is None:
+        means = new_ctx_means(Kt, block)
+    if means.dtype != torch.float32 or not means.is_cuda or not means.is_contiguous():
+        raise ValueError("means must be a contiguous fp32 CUDA tensor")
+    if blk_end is None:
+        blk_end = ctx_num_blocks(L, block)
+    _check(lib().rmm_ctx_block_means(_ptr(Kt), B, Hkv, d, int(L), ldL, int(block), int(blk_begin), int(blk_end),
+                                     _ptr(means), _stream(stream)), "rmm_ctx_block_means")
+    return means
+
+
+def rmm_attn_ctx_workspace_bytes(B: int, Hq: int, Hkv: int, T: int, L: int, block: int, r_ctx: float,
+                                 d: int = 128, opts: rmm_options | None = None) -> int:
+    return int(lib().rmm_attn_ctx_workspace_bytes(B, Hq, Hkv, T, L, d, block, float(r_ctx), _opt(opts)))
+
+
+def rmm_attn_ctx(Q: torch.Tensor, Kt: torch.Tensor, V: torch.Tensor, means: torch.Tensor, L: int, r: float,
+                 r_ctx: float, block: int, causal: bool = True, scale: float | None = None,
+                 O: torch.Tensor | None = None, idx_out: torch.Tensor | None = None,
+                 blocks_out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                 opts: rmm_options | None = None, stream=None) -> torch.Tensor:
+    """Reduced attention over the kept head dimensions and the kept context blocks."""
+    for t, n in ((Q, "Q"), (Kt, "Kt"), (V, "V")):
+        _bf16_cuda(t, n)
+    B, Hq, T, d = Q.shape
+    _, Hkv, d2, ldL = Kt.shape
+    if d2 != d or V.shape != (B, Hkv, ldL, d):
+        raise ValueError("Q, Kt, V shapes disagree")
+    if means.dtype != torch.float32 or not means.is_cuda or not means.is_contiguous():
+        raise ValueError("means must be a contiguous fp32 CUDA tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(Q)
+    if workspace is None:
+        workspace = new_workspace(rmm_attn_ctx_workspace_bytes(B, Hq, Hkv, T, L, block, r_ctx, d, opts), Q.device)
+    _check(lib().rmm_attn_ctx(_ptr(Q), _ptr(Kt), _ptr(V), _ptr(means), B, Hq, Hkv, T, int(L), ldL, d, float(r),
+                              float(r_ctx), int(block), int(bool(causal)), float(scale), _ptr(O), _ptr(idx_out),
+                              _ptr(blocks_out), _ptr(workspace), workspace.numel(), _stream(stream), _opt(opts)),
+           "rmm_attn_ctx")
     return O
 
 
