@@ -88,50 +88,67 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// One CTA per kept set: the scores (from sc, cleared after reading, or, with
-// sc null, folded here from Q for short chunks), then an exact rank-based
-// top-k of the d scores under (score desc, index asc), ascending.
+// The kept head dimensions of set (b, set), computed by the CTA's first D
+// threads (thread j = dimension j; the others only pass the barriers): the
+// scores from sc (cleared after reading) or, with sc null, the column max of
+// |Q| over the set's rows, then an exact rank-based top-k under (score desc,
+// index asc), written in ascending order to out (shared or global).
+__device__ __forceinline__ void select_dims_cta(const uint16_t* __restrict__ Q, int Hq, int Hkv, int T, int k,
+                                                int per_query_head, int b, int set, uint32_t* __restrict__ sc,
+                                                uint32_t* sv, int* warp_cnt, int32_t* out) {
+    const int G = Hq / Hkv;
+    const int q_lo = per_query_head ? set : set * G;
+    const int nrows = (per_query_head ? 1 : G) * T;
+    const int j = threadIdx.x;
+    uint32_t m = 0;
+    if (j < D) {
+        const int nsets = per_query_head ? Hq : Hkv;
+        const size_t so = ((size_t)b * nsets + set) * D + j;
+        if (sc) {
+            m = sc[so];
+            sc[so] = 0;
+        } else {
+#pragma unroll 8
+            for (int r = 0; r < nrows; ++r)  // rows q_lo + r / T, token r % T: all loads independent
+                m = max(m, (uint32_t)(Q[(((size_t)b * Hq + q_lo + r / T) * T + r % T) * D + j] & 0x7FFF));
+        }
+        sv[j] = m;
+    }
+    __syncthreads();
+    bool keep = false;
+    if (j < D) {
+        // rank under (score desc, index asc): number of entries that beat j
+        int rank = 0;
+#pragma unroll 16
+        for (int i = 0; i < D; ++i) {
+            const uint32_t v = sv[i];
+            rank += (v > m) || (v == m && i < j);
+        }
+        keep = rank < k;
+    }
+    const unsigned ball = __ballot_sync(0xffffffffu, keep);
+    const int lane = j & 31, w = j >> 5;
+    if (j < D && lane == 0) warp_cnt[w] = __popc(ball);
+    __syncthreads();
+    if (j < D) {
+        int pos = __popc(ball & ((1u << lane) - 1u));
+        for (int i = 0; i < w; ++i) pos += warp_cnt[i];
+        if (keep) out[pos] = j;
+    }
+}
+
+// One CTA per kept set (long chunks; short decode chunks select inside the
+// split pass instead).
 __global__ void __launch_bounds__(D)
     attn_select_kernel(const uint16_t* __restrict__ Q, int Hq, int Hkv, int T, int k,
                        int per_query_head, uint32_t* __restrict__ sc, int32_t* __restrict__ idx) {
     __shared__ uint32_t sv[D];
     __shared__ int warp_cnt[D / 32];
     const int nsets = per_query_head ? Hq : Hkv;
-    const int set = blockIdx.x % nsets;
-    const int b = blockIdx.x / nsets;
-    const int G = Hq / Hkv;
-    const int q_lo = per_query_head ? set : set * G;
-    const int q_hi = per_query_head ? set + 1 : (set + 1) * G;
-    const int j = threadIdx.x;
     pdl_wait();
     pdl_launch_dependents();
-
-    uint32_t m = 0;
-    if (sc) {
-        m = sc[(size_t)blockIdx.x * D + j];
-        sc[(size_t)blockIdx.x * D + j] = 0;
-    } else {
-        for (int q = q_lo; q < q_hi; ++q) {
-            const uint16_t* row = Q + ((size_t)(b * Hq + q) * T) * D + j;
-            for (int t = 0; t < T; ++t) m = max(m, (uint32_t)(row[(size_t)t * D] & 0x7FFF));
-        }
-    }
-    sv[j] = m;
-    __syncthreads();
-    // rank under (score desc, index asc): number of entries that beat j
-    int rank = 0;
-    for (int i = 0; i < D; ++i) {
-        const uint32_t v = sv[i];
-        rank += (v > m) || (v == m && i < j);
-    }
-    const bool keep = rank < k;
-    const unsigned ball = __ballot_sync(0xffffffffu, keep);
-    const int lane = j & 31, w = j >> 5;
-    if (lane == 0) warp_cnt[w] = __popc(ball);
-    __syncthreads();
-    int pos = __popc(ball & ((1u << lane) - 1u));
-    for (int i = 0; i < w; ++i) pos += warp_cnt[i];
-    if (keep) idx[(size_t)blockIdx.x * k + pos] = j;
+    select_dims_cta(Q, Hq, Hkv, T, k, per_query_head, blockIdx.x / nsets, blockIdx.x % nsets, sc, sv, warp_cnt,
+                    idx + (size_t)blockIdx.x * k);
 }
 
 // ---------------------------------------------------------------- split pass
@@ -147,7 +164,7 @@ template <bool kCtx, int kRows>
 __global__ void __launch_bounds__(kThreads, kRows == 4 ? 2 : 1)
     attn_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ Kt,
                       const uint16_t* __restrict__ V, int Hq, int Hkv, int T, int L, int ldL, int k,
-                      int causal, float scale, int per_query_head, const int32_t* __restrict__ idx,
+                      int causal, float scale, int per_query_head, int32_t* __restrict__ idx, int select_here,
                       float* __restrict__ partials, int chunk, int tq, int Lv,
                       const int32_t* __restrict__ blocks, int bc_shift, int kc) {
     __shared__ float qs[kRows][D];      // scaled kept query values
@@ -185,8 +202,20 @@ __global__ void __launch_bounds__(kThreads, kRows == 4 ? 2 : 1)
     pdl_wait();
     pdl_launch_dependents();
 
-    for (int i = tid; i < k; i += kThreads) sidx[i] = idx[(size_t)blockIdx.x * k + i];
-    __syncthreads();
+    if (select_here) {
+        // short decode chunk: every CTA of the set ranks the d dims itself (a
+        // few hundred instructions), the first one also writes the kept list
+        __shared__ uint32_t sv[D];
+        __shared__ int warp_cnt[kThreads / 32];
+        select_dims_cta(Q, Hq, Hkv, T, k, per_query_head, b, set, nullptr, sv, warp_cnt, sidx);
+        __syncthreads();
+        if (split == 0 && blockIdx.z == 0)
+            for (int i = tid; i < k; i += kThreads) idx[(size_t)blockIdx.x * k + i] = sidx[i];
+    } else {
+        for (int i = tid; i < k; i += kThreads) sidx[i] = idx[(size_t)blockIdx.x * k + i];
+        __syncthreads();
+    }
+#pragma unroll
     for (int e = tid; e < kRows * D; e += kThreads) {
         const int r = e / D, jj = e % D;
         float v = 0.0f;
@@ -233,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, kRows == 4 ? 2 : 1)
             for (int c = 0; c < 4; ++c) s4[r][c] = 0.0f;
         if (lp < L) {  // lp + 3 < roundup(L, 4) <= ldL: the 8-byte load stays in the row
             // kUnrollK kept rows per step: their loads are all in flight before the FMAs
-            constexpr int kUnrollK = kRows == 4 ? 16 : 8;
+            constexpr int kUnrollK = 8;
             for (int jj0 = 0; jj0 < k; jj0 += kUnrollK) {
                 uint2 kv[kUnrollK];
 #pragma unroll
@@ -302,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, kRows == 4 ? 2 : 1)
         }
         const int nkeys = min(SB, l_end - l0);
         // kUnrollV V rows per step, their loads in flight together
-        constexpr int kUnrollV = 4;
+        constexpr int kUnrollV = kRows == 4 ? 8 : 4;
         for (int i0 = kg; i0 < nkeys; i0 += 16 * kUnrollV) {
             uint4 v[kUnrollV];
 #pragma unroll
@@ -364,24 +393,47 @@ __global__ void __launch_bounds__(kThreads, kRows == 4 ? 2 : 1)
 
 // ---------------------------------------------------------------- combine
 
+constexpr int kMaxSplits = 1024;
+
+// One CTA per output row: the splits' maxima and sums are read once into
+// shared memory (all loads in flight together), then thread c adds the
+// weighted column c of every split with eight loads in flight.
 __global__ void __launch_bounds__(D)
     attn_combine_kernel(const float* __restrict__ partials, int nsplit, uint16_t* __restrict__ O) {
+    __shared__ float sm[kMaxSplits], sl[kMaxSplits];
+    __shared__ float red[D / 32];
     pdl_wait();
     pdl_launch_dependents();
     const size_t row = blockIdx.x;
+    const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
     const float* p = partials + row * nsplit * PSTRIDE;
-    float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, p[s * PSTRIDE]);
+    float mx = -INFINITY;
+    for (int s = c; s < nsplit; s += D) {
+        const float2 ml = *reinterpret_cast<const float2*>(p + (size_t)s * PSTRIDE);
+        sm[s] = ml.x;
+        sl[s] = ml.y;
+        mx = fmaxf(mx, ml.x);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    float M = red[0];
+#pragma unroll
+    for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w]);
+    __syncthreads();
+    // weights: exp(m_s - M), zero for a split that saw no key
+    for (int s = c; s < nsplit; s += D) sm[s] = (sm[s] == -INFINITY) ? 0.0f : __expf(sm[s] - M);
+    __syncthreads();
     float num = 0.0f, den = 0.0f;
+#pragma unroll 8
     for (int s = 0; s < nsplit; ++s) {
-        const float m = p[s * PSTRIDE];
-        if (m == -INFINITY) continue;
-        const float w = __expf(m - M);
-        den += w * p[s * PSTRIDE + 1];
-        num += w * p[s * PSTRIDE + 2 + threadIdx.x];
+        const float w = sm[s];
+        den = fmaf(w, sl[s], den);
+        num = fmaf(w, p[(size_t)s * PSTRIDE + 2 + c], num);
     }
     // a row that saw no key (only with kept context blocks) is zero
-    O[row * D + threadIdx.x] = float_to_bf16_bits(den > 0.0f ? num / den : 0.0f);
+    O[row * D + c] = float_to_bf16_bits(den > 0.0f ? num / den : 0.0f);
 }
 
 }  // namespace
@@ -410,12 +462,17 @@ size_t attn_partials_bytes(const AttnPlan& p, int B, int Hq, int T) {
     return (size_t)B * Hq * T * p.nsplit * PSTRIDE * sizeof(float);
 }
 
+bool attn_dims_in_split(int Hq, int Hkv, int T, int per_query_head) {
+    const int nq = per_query_head ? 1 : Hq / Hkv;
+    return nq * T < 64;
+}
+
 cudaError_t launch_attn_dims(const uint16_t* Q, int B, int Hq, int Hkv, int T, int k, int per_query_head, int nsets,
                              int32_t* idx, uint32_t* sc, cudaStream_t stream) {
-    const int nq = per_query_head ? 1 : Hq / Hkv;
     // the kept sets: the column max over many CTAs when the chunk is long
+    const int nq = per_query_head ? 1 : Hq / Hkv;
     cudaError_t e;
-    const bool wide = nq * T >= 64;
+    const bool wide = !attn_dims_in_split(Hq, Hkv, T, per_query_head);
     if (wide) {
         e = launch_pdl(attn_score_kernel, dim3(B * nsets, (nq * T + 63) / 64), dim3(256), 0, stream, Q, Hq, Hkv, T,
                        per_query_head, sc);
@@ -427,14 +484,15 @@ cudaError_t launch_attn_dims(const uint16_t* Q, int B, int Hq, int Hkv, int T, i
 
 cudaError_t launch_attn_split_ctx(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq, int Hkv,
                                   int T, int L, int ldL, int k, int causal, float scale, int per_query_head,
-                                  uint16_t* O, const int32_t* idx, const int32_t* blocks, int bc_shift, int kc,
-                                  float* partials, const AttnPlan& p, cudaStream_t stream) {
+                                  uint16_t* O, int32_t* idx, int select_here, const int32_t* blocks, int bc_shift,
+                                  int kc, float* partials, const AttnPlan& p, cudaStream_t stream) {
     const int nq = per_query_head ? 1 : Hq / Hkv;
-    if (nq > RMAX) return cudaErrorInvalidValue;
+    if (nq > RMAX || p.nsplit > kMaxSplits) return cudaErrorInvalidValue;
     dim3 grid(B * p.nsets, p.nsplit, (T + p.tq - 1) / p.tq);
     cudaError_t e = launch_pdl(p.rows == 4 ? attn_split_kernel<true, 4> : attn_split_kernel<true, RMAX>, grid,
                                dim3(kThreads), 0, stream, Q, Kt, V, Hq, Hkv, T, L, ldL, k, causal, scale,
-                               per_query_head, idx, partials, p.chunk, p.tq, kc << bc_shift, blocks, bc_shift, kc);
+                               per_query_head, idx, select_here, partials, p.chunk, p.tq, kc << bc_shift, blocks,
+                               bc_shift, kc);
     if (e != cudaSuccess) return e;
     return launch_pdl(attn_combine_kernel, dim3(B * Hq * T), dim3(D), 0, stream, (const float*)partials, p.nsplit,
                       O);
@@ -445,16 +503,19 @@ cudaError_t launch_attn(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V
                         int per_query_head, uint16_t* O, int32_t* idx, float* partials, uint32_t* sc,
                         int* status, int path, const AttnPlan& p, cudaStream_t stream) {
     const int nq = per_query_head ? 1 : Hq / Hkv;
-    cudaError_t e = launch_attn_dims(Q, B, Hq, Hkv, T, k, per_query_head, p.nsets, idx, sc, stream);
-    if (e != cudaSuccess) return e;
     const bool tc = path == 2 || (path == 0 && attn_tc_supported(T, k));
+    // short decode chunks select their dims inside the split pass
+    const bool select_here = !tc && attn_dims_in_split(Hq, Hkv, T, per_query_head);
+    cudaError_t e = cudaSuccess;
+    if (!select_here) e = launch_attn_dims(Q, B, Hq, Hkv, T, k, per_query_head, p.nsets, idx, sc, stream);
+    if (e != cudaSuccess) return e;
     if (tc)
         return launch_attn_tc(Q, Kt, V, B, Hq, Hkv, T, L, ldL, k, causal, scale, per_query_head, idx, O, status,
                               stream);
-    if (nq > RMAX) return cudaErrorInvalidValue;
+    if (nq > RMAX || p.nsplit > kMaxSplits) return cudaErrorInvalidValue;
     dim3 grid(B * p.nsets, p.nsplit, (T + p.tq - 1) / p.tq);
     e = launch_pdl(p.rows == 4 ? attn_split_kernel<false, 4> : attn_split_kernel<false, RMAX>, grid, dim3(kThreads), 0,
-                   stream, Q, Kt, V, Hq, Hkv, T, L, ldL, k, causal, scale, per_query_head, (const int32_t*)idx,
+                   stream, Q, Kt, V, Hq, Hkv, T, L, ldL, k, causal, scale, per_query_head, idx, (int)select_here,
                    partials, p.chunk, p.tq, L, (const int32_t*)nullptr, 0, 0);
     if (e != cudaSuccess) return e;
     return launch_pdl(attn_combine_kernel, dim3(B * Hq * T), dim3(D), 0, stream, (const float*)partials, p.nsplit,

@@ -97,17 +97,30 @@ __global__ void __launch_bounds__(128)
     float best = -INFINITY;
     for (int r0 = 0; r0 < R; r0 += 16) {
         __syncthreads();
-        for (int e = threadIdx.x; e < 16 * D; e += 128) {
-            const int rr = e / D, c = e % D, r = r0 + rr;
-            float v = 0.0f;
-            if (r < R) v = bf16_bits_to_float(Q[(((size_t)b * Hq + q_lo + r / T) * T + r % T) * D + c]);
-            qs[rr][c] = v;
+        // 16 rows x 128 dims: two 16-byte pieces per thread, both loads in flight
+        uint4 piece[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int e = threadIdx.x + 128 * u, rr = e / 16, r = r0 + rr;
+            piece[u] = r < R ? ld_nc_v4(Q + (((size_t)b * Hq + q_lo + r / T) * T + r % T) * D + (e % 16) * 8)
+                             : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int e = threadIdx.x + 128 * u, rr = e / 16, c = (e % 16) * 8;
+            const uint32_t w[4] = {piece[u].x, piece[u].y, piece[u].z, piece[u].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                qs[rr][c + 2 * h] = __uint_as_float(w[h] << 16);
+                qs[rr][c + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+            }
         }
         __syncthreads();
         const int nr = min(16, R - r0);
         if (valid) {
             for (int rr = 0; rr < nr; rr += 4) {
                 float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+#pragma unroll 8
                 for (int c4 = 0; c4 < D / 4; ++c4) {
                     const float4 mv = __ldg(m4 + c4);
                     const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
@@ -200,7 +213,9 @@ cudaError_t launch_attn_ctx(const uint16_t* Q, const uint16_t* Kt, const uint16_
     if (P > 2 * kSelThreads) return cudaErrorInvalidValue;
     int bc_shift = 0;
     while ((1 << bc_shift) < bc) ++bc_shift;
-    cudaError_t e = launch_attn_dims(Q, B, Hq, Hkv, T, k, per_query_head, p.nsets, idx, sc, stream);
+    const bool select_here = attn_dims_in_split(Hq, Hkv, T, per_query_head);
+    cudaError_t e = cudaSuccess;
+    if (!select_here) e = launch_attn_dims(Q, B, Hq, Hkv, T, k, per_query_head, p.nsets, idx, sc, stream);
     if (e != cudaSuccess) return e;
     e = launch_pdl(ctx_score_kernel, dim3((nblk + 127) / 128, B * p.nsets), dim3(128), 0, stream, Q, means, Hq, Hkv,
                    T, nblk, nblk_stride, per_query_head, keys);
@@ -208,8 +223,8 @@ cudaError_t launch_attn_ctx(const uint16_t* Q, const uint16_t* Kt, const uint16_
     e = launch_pdl(ctx_select_kernel, dim3(B * p.nsets), dim3(kSelThreads), (size_t)P * sizeof(uint64_t), stream,
                    (const uint32_t*)keys, nblk, P, kc, blocks);
     if (e != cudaSuccess) return e;
-    return launch_attn_split_ctx(Q, Kt, V, B, Hq, Hkv, T, L, ldL, k, causal, scale, per_query_head, O, idx, blocks,
-                                 bc_shift, kc, partials, p, stream);
+    return launch_attn_split_ctx(Q, Kt, V, B, Hq, Hkv, T, L, ldL, k, causal, scale, per_query_head, O, idx,
+                                 (int)select_here, blocks, bc_shift, kc, partials, p, stream);
 }
 
 }  // namespace rmm

@@ -149,6 +149,9 @@ cudaError_t launch_attn(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V
                         int Hkv, int T, int L, int ldL, int k, int causal, float scale,
                         int per_query_head, uint16_t* O, int32_t* idx, float* partials, uint32_t* sc,
                         int* status, int path, const AttnPlan& plan, cudaStream_t stream);
+// True when the split pass selects the kept head dimensions itself (short
+// decode chunks: a set's rows number fewer than 64).
+bool attn_dims_in_split(int Hq, int Hkv, int T, int per_query_head);
 // The kept head dimensions alone (score + select), as launch_attn runs them.
 cudaError_t launch_attn_dims(const uint16_t* Q, int B, int Hq, int Hkv, int T, int k, int per_query_head, int nsets,
                              int32_t* idx, uint32_t* sc, cudaStream_t stream);
@@ -156,8 +159,8 @@ cudaError_t launch_attn_dims(const uint16_t* Q, int B, int Hq, int Hkv, int T, i
 // keys per set, blocks [B * nsets * kc]); plan made for kc << bc_shift keys.
 cudaError_t launch_attn_split_ctx(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq, int Hkv,
                                   int T, int L, int ldL, int k, int causal, float scale, int per_query_head,
-                                  uint16_t* O, const int32_t* idx, const int32_t* blocks, int bc_shift, int kc,
-                                  float* partials, const AttnPlan& p, cudaStream_t stream);
+                                  uint16_t* O, int32_t* idx, int select_here, const int32_t* blocks, int bc_shift,
+                                  int kc, float* partials, const AttnPlan& p, cudaStream_t stream);
 
 // ---- context-block reduction (rmm_ctx.cu)
 constexpr int kCtxMaxBlocks = 2048;  // blocks per cache the select kernel sorts

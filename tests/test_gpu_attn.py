@@ -55,7 +55,7 @@ def run_attn(rmm, Q, K, V, r, causal=True, per_head=False, opts=None):
     return O.cpu(), idx.cpu().numpy(), k
 
 
-@pytest.mark.parametrize("T,L", [(1, 37), (1, 1000), (5, 5), (5, 300), (33, 2100), (64, 64)])
+@pytest.mark.parametrize("T,L", [(1, 37), (1, 1000), (2, 4100), (5, 5), (5, 300), (33, 2100), (64, 64)])
 @pytest.mark.parametrize("r", [0.25, 0.5, 1.0])
 @pytest.mark.parametrize("causal", [True, False])
 def test_attention_small(rmm, T, L, r, causal):
