@@ -383,6 +383,66 @@ def time_blocks(dev, acts, Wts, Ys, dense_ms, steps, warmup, block=64):
     }}
 
 
+def time_attn_decode(dev, peaks, L=32768, block=64):
+    """Secondary row: one long-context decode attention call (B = 1, 32 query / 8 KV heads,
+    d = 128, T = 1, r = 0.5): the head-dim reduction, the same plus context blocks of 64 keys
+    (r_ctx = 0.5, 0.25), and dense SDPA on the same cache.  The cache (134 MB of K and V)
+    exceeds L2; L2 is flushed before each call anyway."""
+    from input_adaptive_reduced_rmm_b200 import rmm
+
+    B, Hq, Hkv, T, d, r = 1, 32, 8, 1, 128, 0.5
+    Q = rmm_synth.normal((B, Hq, T, d), 701).to(dev)
+    Kt = rmm_synth.normal((B, Hkv, d, L), 702).to(dev)
+    V = rmm_synth.normal((B, Hkv, L, d), 703).to(dev)
+    K = Kt.transpose(-1, -2).contiguous()
+    O = torch.empty_like(Q)
+    means = rmm.rmm_ctx_block_means(Kt, L, block)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def timed(fn, iters=30):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(iters):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts) * 1e3
+
+    k = rmm.rmm_k_for(d, r)
+    ws = rmm.new_workspace(rmm.rmm_attn_workspace_bytes(B, Hq, Hkv, T, L, d), dev)
+    red_us = timed(lambda: rmm.rmm_attn_qk(Q, Kt, V, L, r, O=O, workspace=ws))
+    red_bytes = Hkv * L * 2 * (k + d)
+    out = {"workload": f"decode attention, B=1, Hq=32, Hkv=8, d=128, L={L}, T=1, r=0.5; context blocks of {block}",
+           "reduced_us": red_us, "reduced_gbs": red_bytes / (red_us * 1e-6) / 1e9,
+           "reduced_frac_of_hbm": red_bytes / (red_us * 1e-6) / 1e9 / peaks["hbm_gbs"]}
+    nblk = rmm.ctx_num_blocks(L, block)
+    for rc in (0.5, 0.25):
+        kc = rmm.rmm_k_for(nblk, rc)
+        wsc = rmm.new_workspace(rmm.rmm_attn_ctx_workspace_bytes(B, Hq, Hkv, T, L, block, rc), dev)
+        us = timed(lambda: rmm.rmm_attn_ctx(Q, Kt, V, means, L, r, rc, block, O=O, workspace=wsc))
+        if rmm.rmm_get_status(wsc) != rmm.RMM_OK:
+            raise RuntimeError("device status not OK (context-block attention)")
+        cbytes = Hkv * kc * block * 2 * (k + d) + Hkv * nblk * d * 4
+        out[f"ctx_rc{rc}_us"] = us
+        out[f"ctx_rc{rc}_gbs"] = cbytes / (us * 1e-6) / 1e9
+    sdpa_us = timed(lambda: torch.nn.functional.scaled_dot_product_attention(Q, K, V, enable_gqa=True))
+    out["dense_sdpa_us"] = sdpa_us
+    out["dense_sdpa_gbs"] = Hkv * L * 2 * 2 * d / (sdpa_us * 1e-6) / 1e9
+    out["speedup_reduced_vs_dense"] = sdpa_us / red_us
+    out["speedup_ctx_rc0.25_vs_dense"] = sdpa_us / out["ctx_rc0.25_us"]
+    if rmm.rmm_get_status(ws) != rmm.RMM_OK:
+        raise RuntimeError("device status not OK (decode attention)")
+    del Q, Kt, V, K, O, means, flush
+    torch.cuda.empty_cache()
+    return {"attn_decode": out}
+
+
 def launches_per_step(dev) -> int:
     """Our kernels launched by one step: per call the score pass, the select, the CTA-pair
     GEMM, and the fold of the split last wave when the call's tiles leave a partial wave
@@ -607,6 +667,7 @@ def run_rmm(args, world, rank, local):
     if not args.skip_secondary:
         extra.update(time_blocks(dev, acts, Wts, Ys, dense_ms, K, W))
         extra.update(time_decode(dev, peaks))
+        extra.update(time_attn_decode(dev, peaks))
         extra.update(time_layer(dev, host_inputs()[1]))
 
     cpu = None

@@ -394,21 +394,25 @@ __global__ void __launch_bounds__(kThreads, kRows == 4 ? 2 : 1)
 // ---------------------------------------------------------------- combine
 
 constexpr int kMaxSplits = 1024;
+constexpr int kCombineGroups = 4;  // split groups per row, D threads each
 
 // One CTA per output row: the splits' maxima and sums are read once into
-// shared memory (all loads in flight together), then thread c adds the
-// weighted column c of every split with eight loads in flight.
-__global__ void __launch_bounds__(D)
+// shared memory (all loads in flight together); then thread (group g, column
+// c) adds the weighted column c of the splits s = g (mod 4), eight loads in
+// flight, and the four groups are added in a fixed order.
+__global__ void __launch_bounds__(kCombineGroups * D)
     attn_combine_kernel(const float* __restrict__ partials, int nsplit, uint16_t* __restrict__ O) {
     __shared__ float sm[kMaxSplits], sl[kMaxSplits];
-    __shared__ float red[D / 32];
+    __shared__ float red[kCombineGroups * D / 32];
+    __shared__ float part_num[kCombineGroups][D], part_den[kCombineGroups][D];
     pdl_wait();
     pdl_launch_dependents();
     const size_t row = blockIdx.x;
-    const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int c = tid % D, grp = tid / D;
     const float* p = partials + row * nsplit * PSTRIDE;
     float mx = -INFINITY;
-    for (int s = c; s < nsplit; s += D) {
+    for (int s = tid; s < nsplit; s += kCombineGroups * D) {
         const float2 ml = *reinterpret_cast<const float2*>(p + (size_t)s * PSTRIDE);
         sm[s] = ml.x;
         sl[s] = ml.y;
@@ -420,20 +424,31 @@ __global__ void __launch_bounds__(D)
     __syncthreads();
     float M = red[0];
 #pragma unroll
-    for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w]);
-    __syncthreads();
+    for (int w = 1; w < kCombineGroups * D / 32; ++w) M = fmaxf(M, red[w]);
     // weights: exp(m_s - M), zero for a split that saw no key
-    for (int s = c; s < nsplit; s += D) sm[s] = (sm[s] == -INFINITY) ? 0.0f : __expf(sm[s] - M);
+    for (int s = tid; s < nsplit; s += kCombineGroups * D)
+        sm[s] = (sm[s] == -INFINITY) ? 0.0f : __expf(sm[s] - M);
     __syncthreads();
     float num = 0.0f, den = 0.0f;
 #pragma unroll 8
-    for (int s = 0; s < nsplit; ++s) {
+    for (int s = grp; s < nsplit; s += kCombineGroups) {
         const float w = sm[s];
         den = fmaf(w, sl[s], den);
         num = fmaf(w, p[(size_t)s * PSTRIDE + 2 + c], num);
     }
-    // a row that saw no key (only with kept context blocks) is zero
-    O[row * D + c] = float_to_bf16_bits(den > 0.0f ? num / den : 0.0f);
+    part_num[grp][c] = num;
+    part_den[grp][c] = den;
+    __syncthreads();
+    if (grp == 0) {
+        float n = part_num[0][c], d = part_den[0][c];
+#pragma unroll
+        for (int g = 1; g < kCombineGroups; ++g) {
+            n += part_num[g][c];
+            d += part_den[g][c];
+        }
+        // a row that saw no key (only with kept context blocks) is zero
+        O[row * D + c] = float_to_bf16_bits(d > 0.0f ? n / d : 0.0f);
+    }
 }
 
 }  // namespace
@@ -494,7 +509,7 @@ cudaError_t launch_attn_split_ctx(const uint16_t* Q, const uint16_t* Kt, const u
                                per_query_head, idx, select_here, partials, p.chunk, p.tq, kc << bc_shift, blocks,
                                bc_shift, kc);
     if (e != cudaSuccess) return e;
-    return launch_pdl(attn_combine_kernel, dim3(B * Hq * T), dim3(D), 0, stream, (const float*)partials, p.nsplit,
+    return launch_pdl(attn_combine_kernel, dim3(B * Hq * T), dim3(kCombineGroups * D), 0, stream, (const float*)partials, p.nsplit,
                       O);
 }
 
@@ -518,7 +533,7 @@ cudaError_t launch_attn(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V
                    stream, Q, Kt, V, Hq, Hkv, T, L, ldL, k, causal, scale, per_query_head, idx, (int)select_here,
                    partials, p.chunk, p.tq, L, (const int32_t*)nullptr, 0, 0);
     if (e != cudaSuccess) return e;
-    return launch_pdl(attn_combine_kernel, dim3(B * Hq * T), dim3(D), 0, stream, (const float*)partials, p.nsplit,
+    return launch_pdl(attn_combine_kernel, dim3(B * Hq * T), dim3(kCombineGroups * D), 0, stream, (const float*)partials, p.nsplit,
                       O);
 }
 
