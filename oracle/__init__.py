@@ -92,6 +92,8 @@ def _load():
     lib.oracle_attention_ctx.argtypes = [_u16p, _u16p, _u16p, L, L, L, L, L, L, L, I, D, I, L, L, P, L,
                                          _f64p, _i32p, _i32p, P, P]
     lib.oracle_attention_ctx.restype = I
+    lib.oracle_block_select_mean.argtypes = [_u16p, L, L, L, L, _i32p]
+    lib.oracle_block_select_mean.restype = I
     lib.oracle_block_select.argtypes = [_u16p, L, L, L, _i32p]
     lib.oracle_block_select.restype = I
     lib.oracle_rmsnorm.argtypes = [_u16p, L, L, D, _f64p]
@@ -195,13 +197,30 @@ def block_select(s, block: int, kb: int) -> np.ndarray:
     return out
 
 
-def linear_blocks(X, W, r: float, block: int = 64, rows=None, cols=None):
+def block_select_mean(X, block: int, kb: int) -> np.ndarray:
+    """The kb best blocks of `block` consecutive slices scored by their mean |X| (single
+    precision: tokens ascending, then the block's slices ascending, then / (T*block)),
+    ascending block indices."""
+    x = _bits(X)
+    T, H = x.shape
+    out = np.zeros(int(kb), dtype=np.int32)
+    _check(_load().oracle_block_select_mean(x, T, H, int(block), int(kb), out), "oracle_block_select_mean")
+    return out
+
+
+def linear_blocks(X, W, r: float, block: int = 64, rows=None, cols=None, block_score: str = "max"):
     """The reduced linear map with a block-granular kept set: kb = ceil(r * H / block)
-    blocks; the product over their slices.  Returns (Y fp64, kept blocks)."""
+    blocks scored by the max of their slices' scores ("max") or by their mean |X|
+    ("mean"); the product over their slices.  Returns (Y fp64, kept blocks)."""
     x = _bits(X)
     H = x.shape[1]
     kb = k_for(H // block, r)
-    blocks = block_select(score(X), block, kb)
+    if block_score == "mean":
+        blocks = block_select_mean(X, block, kb)
+    elif block_score == "max":
+        blocks = block_select(score(X), block, kb)
+    else:
+        raise ValueError(block_score)
     idx = (blocks[:, None] * block + np.arange(block, dtype=np.int32)[None, :]).reshape(-1)
     return reduced_product(X, W, idx, rows=rows, cols=cols), blocks
 

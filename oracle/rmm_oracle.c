@@ -60,6 +60,8 @@
 
 /* ---- bf16 helpers -------------------------------------------------------- */
 
+int oracle_ctx_select(const float* scores, long nblk, long kc, int32_t* blocks);
+
 static double bf16_to_double(uint16_t b) {
     uint32_t u = ((uint32_t)b) << 16;
     float f;
@@ -221,6 +223,33 @@ int oracle_block_select(const uint16_t* s, long H, long block, long kb, int32_t*
         bs[j] = m;
     }
     int rc = oracle_select(bs, nb, kb, blocks);
+    free(bs);
+    return rc;
+}
+
+/* Block-granular kept set scored by the mean magnitude of the block, the
+ * score of the FFN demo in the cf-1.com post (§5.1: a block's importance is
+ * its mean absolute activation; §6.1: blocks of 64 of the FFN intermediate
+ * dimension, top blocks by that mean, sorted).  The score decides an integer
+ * set, so it is computed in single precision in one stated order: the sum
+ * runs over the tokens t ascending and, within a token, over the block's
+ * slices ascending (float additions from 0), then one correctly rounded
+ * division by T*block.  The kb best blocks under (score desc, block index
+ * asc) are written to blocks in ascending order. */
+int oracle_block_select_mean(const uint16_t* X, long T, long H, long block, long kb, int32_t* blocks) {
+    if (!X || !blocks || T < 1 || block < 1 || H < block || H % block != 0) return ORACLE_ERR_ARG;
+    long nb = H / block;
+    if (kb < 1 || kb > nb) return ORACLE_ERR_ARG;
+    if (!all_finite(X, T * H)) return ORACLE_ERR_NONFINITE;
+    float* bs = (float*)malloc(sizeof(float) * (size_t)nb);
+    if (!bs) return ORACLE_ERR_NOMEM;
+    for (long j = 0; j < nb; ++j) {
+        float sum = 0.0f;
+        for (long t = 0; t < T; ++t)
+            for (long i = 0; i < block; ++i) sum += fabsf((float)bf16_to_double(X[t * H + j * block + i]));
+        bs[j] = sum / (float)(T * block);
+    }
+    int rc = oracle_ctx_select(bs, nb, kb, blocks);
     free(bs);
     return rc;
 }

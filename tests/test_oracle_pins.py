@@ -535,3 +535,53 @@ def test_ctx_dominant_block_is_kept_and_unseen_rows_are_zero():
     # only the ragged block 2 (positions 128, 129) kept: the query at position 127 sees none
     O, _, _ = oracle.attention_ctx(Q, K, V, d, 64, 1, causal=True, blocks_in=[[[2]]])
     assert np.all(O[0, 0, 0] == 0.0) and np.any(O[0, 0, 1] != 0.0)
+
+
+# ---------------------------------------------------------------- mean-magnitude blocks
+# cf-1.com post §5.1 / §6.1: a block's importance is its mean absolute activation.
+
+
+def test_block_mean_exact_on_integers():
+    """Small-integer activations: every float sum and the division by a power of two
+    are exact, so the kept blocks are the integer ranking (ties to the lower block)."""
+    for T in (1, 4):
+        X = small_ints((T, 512), -6, 6, 111 + T)
+        Xi = np.abs(X.to(torch.int64).numpy())
+        sums = Xi.reshape(T, 8, 64).sum(axis=(0, 2))
+        for kb in (1, 3, 8):
+            order = sorted(range(8), key=lambda j: (-sums[j], j))
+            assert oracle.block_select_mean(X, 64, kb).tolist() == sorted(order[:kb])
+
+
+def test_block_mean_unit_blocks_at_one_token_is_the_slice_select():
+    """block = 1, T = 1: the mean magnitude of a slice is |x|, whose order is the order
+    of the per-slice max score."""
+    X = rmm_synth.activations(1, 300, 112)
+    for k in (1, 37, 150, 300):
+        assert oracle.block_select_mean(X, 1, k).tolist() == oracle.select(oracle.score(X), k).tolist()
+
+
+@pytest.mark.parametrize("nb", [3, 6, 9])
+def test_block_mean_brute_force(nb):
+    """Every kb-subset of blocks: the kept set is the unique one whose members all beat
+    every dropped block under (mean desc, index asc), the means taken in fp64 (distinct
+    enough here that fp32 rounding cannot reorder them)."""
+    X = rmm_synth.activations(3, 16 * nb, 113 + nb)
+    m = np.abs(f64(X)).reshape(3, nb, 16).mean(axis=(0, 2))
+    for kb in range(1, nb + 1):
+        got = oracle.block_select_mean(X, 16, kb).tolist()
+        valid = [list(S) for S in itertools.combinations(range(nb), kb)
+                 if all(m[i] > m[j] or (m[i] == m[j] and i < j) for i in S for j in range(nb) if j not in S)]
+        assert valid == [got]
+
+
+def test_block_mean_linear_full_ratio_is_dense_and_keeps_the_loud_block():
+    X = rmm_synth.activations(2, 256, 114)
+    W = rmm_synth.weights(64, 256, 115)
+    Y1, b1 = oracle.linear_blocks(X, W, 1.0, block=64, block_score="mean")
+    assert b1.tolist() == [0, 1, 2, 3]
+    assert np.max(np.abs(Y1 - f64(X) @ f64(W).T)) <= 1e-12 * max(1.0, np.abs(Y1).max())
+    X2 = X.clone()
+    X2[:, 128:192] = (X2[:, 128:192].float() * 50).to(torch.bfloat16)  # block 2 is loud
+    _, b2 = oracle.linear_blocks(X2, W, 0.25, block=64, block_score="mean")
+    assert b2.tolist() == [2]
