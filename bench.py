@@ -443,6 +443,63 @@ def time_attn_decode(dev, peaks, L=32768, block=64):
     return {"attn_decode": out}
 
 
+def time_ffn_demo(dev):
+    """Secondary row: the cf-1.com post's FFN demo (H = 1024, M = 4096, one token):
+    gate/up in full, SwiGLU, the down projection reduced to the 64-neuron blocks of
+    largest mean |h| at keep 0.5 -- against the dense FFN (cuBLAS products, the same
+    SwiGLU kernel).  Both captured as CUDA graphs, L2 flushed before each replay; the
+    output's mean |y_reduced - y_full| is the quantity the demo prints."""
+    from input_adaptive_reduced_rmm_b200.ffn_demo import FfnBlockReduce
+
+    H, M, T = 1024, 4096, 1
+    W_gate = rmm_synth.weights(M, H, 801, std=0.02).to(dev)
+    W_up = rmm_synth.weights(M, H, 802, std=0.02).to(dev)
+    W_down = rmm_synth.weights(H, M, 803, std=0.02).to(dev)
+    x = rmm_synth.normal((T, H), 804).to(dev)
+    f = FfnBlockReduce(W_gate, W_up, W_down, block=64, keep=0.5)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def graph_time(fn, iters=30):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            out = fn()
+        ts = []
+        for _ in range(iters):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        del g
+        return statistics.median(ts) * 1e3, out
+
+    red_us, _ = graph_time(lambda: f.forward(x)[0])
+    dense_us, _ = graph_time(lambda: f.forward_dense(x))
+    y_red = f.forward(x)[0].float()
+    y_full = f.forward_dense(x).float()
+    torch.cuda.synchronize()
+    out = {"ffn_demo": {
+        "workload": "FFN of the post's demo: x [1, 1024], gate/up 4096x1024 full, SwiGLU, down 1024x4096 "
+                    "reduced to mean-|h| blocks of 64 at keep 0.5",
+        "reduced_us": red_us, "dense_us": dense_us, "speedup_vs_dense": dense_us / red_us,
+        "down_proj_flops_fraction": f.kb * 64 / M,
+        "mean_abs_diff_vs_full": float((y_red - y_full).abs().mean()),
+        "mean_abs_full": float(y_full.abs().mean()),
+    }}
+    del f, W_gate, W_up, W_down, flush
+    torch.cuda.empty_cache()
+    return out
+
+
 def launches_per_step(dev) -> int:
     """Our kernels launched by one step: per call the score pass, the select, the CTA-pair
     GEMM, and the fold of the split last wave when the call's tiles leave a partial wave
@@ -668,6 +725,7 @@ def run_rmm(args, world, rank, local):
         extra.update(time_blocks(dev, acts, Wts, Ys, dense_ms, K, W))
         extra.update(time_decode(dev, peaks))
         extra.update(time_attn_decode(dev, peaks))
+        extra.update(time_ffn_demo(dev))
         extra.update(time_layer(dev, host_inputs()[1]))
 
     cpu = None

@@ -90,7 +90,13 @@ typedef struct rmm_options {
      * block_size) blocks are kept under (score desc, block index asc); idx_out
      * then receives their k = kb * block_size slices, ascending. */
     int block_size;
-    int reserved[1]; /* must be zero */
+    /* Block score with block_size > 0: 0 (default) = the largest of the
+     * block's slice scores; 1 = the block's mean magnitude over all T tokens,
+     * the score of the FFN demo (cf-1.com post §5.1, §6.1), computed in single
+     * precision in one order (tokens ascending, within a token the block's
+     * slices ascending, then one correctly rounded division by T*block_size).
+     * 1 requires T <= 16 (RMM_ERR_UNSUPPORTED otherwise). */
+    int block_score;
     /* Optional pair of cudaEvent_t handles (NULL: none) recorded on the
      * stream immediately before and after the reduced-product kernel (GEMV or
      * GEMM) of rmm_linear / rmm_gemm_reduced, so that a caller can time that

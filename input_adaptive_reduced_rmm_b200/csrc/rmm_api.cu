@@ -54,7 +54,7 @@ int num_sms_current() {
 }
 
 const rmm_options& opts_or_default(const rmm_options* o) {
-    static const rmm_options d = {16, 0, 0, 0, 0, 0, 0, {0}, nullptr, nullptr};
+    static const rmm_options d = {16, 0, 0, 0, 0, 0, 0, 0, nullptr, nullptr};
     return o ? *o : d;
 }
 
@@ -65,7 +65,7 @@ bool opts_valid(const rmm_options* o) {
     if (o->gemm_producer < 0 || o->gemm_producer > 2) return false;
     if (o->attn_path < 0 || o->attn_path > 2) return false;
     if (o->block_size < 0) return false;
-    if (o->reserved[0] != 0) return false;
+    if (o->block_score < 0 || o->block_score > 1 || (o->block_score == 1 && o->block_size == 0)) return false;
     return true;
 }
 
@@ -287,6 +287,8 @@ rmm_status linear_group(const void* X, int T, int H, double r, int count, const 
     const rmm_options& o = opts_or_default(options);
     const int bsz = o.block_size;
     if (!block_size_ok(H, bsz)) return RMM_ERR_UNSUPPORTED;
+    const bool mean_blocks = bsz > 0 && o.block_score == 1;
+    if (mean_blocks && T > kGemvMaxT) return RMM_ERR_UNSUPPORTED;
     // kept slices: ceil(r*H), or ceil(r*H/block) whole blocks
     const int kb = bsz ? rmm_k_for(H / bsz, r) : 0;
     const int k = bsz ? (kb < 1 ? -1 : kb * bsz) : rmm_k_for(H, r);
@@ -301,11 +303,20 @@ rmm_status linear_group(const void* X, int T, int H, double r, int count, const 
     const int pad_to = (k + kGemmBK - 1) / kGemmBK * kGemmBK;
     cudaError_t e;
     if (bsz) {
-        // block-granular: the score pass (with X^T on the GEMM path), then the blocks
-        e = launch_score(static_cast<const uint16_t*>(X), T, H, s32,
-                         L.gemv ? nullptr : reinterpret_cast<uint16_t*>(ws + L.xt), L.ldT, sms, s);
-        if (e == cudaSuccess) e = launch_block_select(s32, H, bsz, kb, idx, idx_out, nullptr, s);
+        // block-granular: the score pass (with X^T on the GEMM path; not needed
+        // for mean-magnitude blocks on the GEMV path), then the blocks
+        e = cudaSuccess;
+        if (!mean_blocks || !L.gemv)
+            e = launch_score(static_cast<const uint16_t*>(X), T, H, s32,
+                             L.gemv ? nullptr : reinterpret_cast<uint16_t*>(ws + L.xt), L.ldT, sms, s);
+        if (e == cudaSuccess)
+            e = launch_block_select(s32, mean_blocks ? static_cast<const uint16_t*>(X) : nullptr, T, H, bsz, kb, idx,
+                                    idx_out, nullptr, s);
         if (e == cudaSuccess && pad_to > k) e = launch_pad_idx(idx, k, H, idx, pad_to, s);
+    } else if (L.gemv && k == H) {
+        // every slice kept (ratio 1): the kept list is 0..H-1 whatever the
+        // scores, so neither score nor select runs
+        e = launch_pad_idx(nullptr, k, H, idx, pad_to, s, idx_out);
     } else if (L.gemv && T == 1) {
         // one token: the select kernel reads the score straight from X
         e = launch_select(static_cast<const uint16_t*>(X), T, nullptr, 0, H, k, idx, pad_to, idx_out, nullptr, s);

@@ -25,9 +25,12 @@ namespace {
 
 constexpr int kThreads = 1024;
 
+// X non-null: mean-magnitude blocks (T <= 16 tokens of X [T, H]); the block
+// score is then the bit pattern of a non-negative float, which orders like
+// the float.  s32 is cleared either way (the score pass may have filled it).
 __global__ void __launch_bounds__(kThreads)
-    block_select_kernel(uint32_t* __restrict__ s32, int H, int block, int kb, int32_t* __restrict__ idx,
-                        int32_t* __restrict__ idx_copy, int32_t* __restrict__ blocks_out) {
+    block_select_kernel(uint32_t* __restrict__ s32, const uint16_t* __restrict__ X, int T, int H, int block, int kb,
+                        int32_t* __restrict__ idx, int32_t* __restrict__ idx_copy, int32_t* __restrict__ blocks_out) {
     __shared__ uint32_t bs[kThreads];
     __shared__ int warp_cnt[kThreads / 32];
     pdl_wait();
@@ -36,10 +39,30 @@ __global__ void __launch_bounds__(kThreads)
     const int nb = H / block;
     uint32_t m = 0;
     if (j < nb) {
-        for (int i = 0; i < block; ++i) {
-            const int h = j * block + i;
-            m = max(m, s32[h] & 0xFFFFu);
-            s32[h] = 0;
+        if (X) {
+            // sum over tokens ascending, within a token the block's slices
+            // ascending (16-byte loads of 8 slices, added in order)
+            float sum = 0.0f;
+            for (int t = 0; t < T; ++t) {
+                const uint16_t* row = X + (size_t)t * H + (size_t)j * block;
+                for (int i = 0; i < block; i += 8) {
+                    const uint4 v = ld_nc_v4(row + i);
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        sum += __uint_as_float((w[u] << 16) & 0x7FFF0000u);
+                        sum += __uint_as_float(w[u] & 0x7FFF0000u);
+                    }
+                }
+            }
+            m = __float_as_uint(__fdiv_rn(sum, (float)(T * block)));
+            for (int i = 0; i < block; ++i) s32[j * block + i] = 0;
+        } else {
+            for (int i = 0; i < block; ++i) {
+                const int h = j * block + i;
+                m = max(m, s32[h] & 0xFFFFu);
+                s32[h] = 0;
+            }
         }
     }
     bs[j] = m;
@@ -74,10 +97,10 @@ bool block_size_ok(int H, int block) {
     return H % block == 0 && H / block <= kThreads;
 }
 
-cudaError_t launch_block_select(uint32_t* s32, int H, int block, int kb, int32_t* idx, int32_t* idx_copy,
-                                int32_t* blocks_out, cudaStream_t stream) {
+cudaError_t launch_block_select(uint32_t* s32, const uint16_t* X, int T, int H, int block, int kb, int32_t* idx,
+                                int32_t* idx_copy, int32_t* blocks_out, cudaStream_t stream) {
     if (!block_size_ok(H, block) || block == 0 || kb < 1 || kb > H / block) return cudaErrorInvalidValue;
-    return launch_pdl(block_select_kernel, dim3(1), dim3(kThreads), 0, stream, s32, H, block, kb, idx, idx_copy,
+    return launch_pdl(block_select_kernel, dim3(1), dim3(kThreads), 0, stream, s32, X, T, H, block, kb, idx, idx_copy,
                       blocks_out);
 }
 

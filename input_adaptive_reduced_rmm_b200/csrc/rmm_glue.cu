@@ -4,7 +4,9 @@
 //                     contraction slice h of the weight is one contiguous row
 //                     (the product streams or gathers whole kept rows).
 //   pad_idx_kernel    copies a caller's kept list and pads it with the
-//                     out-of-range index H to a multiple of the GEMM K-block.
+//                     out-of-range index H to a multiple of the GEMM K-block;
+//                     with no list given, the identity list 0..k-1 (keep
+//                     ratio 1: every slice kept), optionally copied out.
 #include "rmm_common.cuh"
 #include "rmm_internal.h"
 
@@ -32,11 +34,14 @@ __global__ void __launch_bounds__(256)
 }
 
 __global__ void pad_idx_kernel(const int32_t* __restrict__ src, int k, int H,
-                               int32_t* __restrict__ dst, int pad_to) {
+                               int32_t* __restrict__ dst, int pad_to, int32_t* __restrict__ dst_copy) {
     pdl_wait();
     pdl_launch_dependents();
-    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < pad_to; j += gridDim.x * blockDim.x)
-        dst[j] = (j < k) ? src[j] : H;
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < pad_to; j += gridDim.x * blockDim.x) {
+        const int32_t v = (j < k) ? (src ? src[j] : j) : H;
+        dst[j] = v;
+        if (dst_copy && j < k) dst_copy[j] = v;
+    }
 }
 
 }  // namespace
@@ -47,11 +52,11 @@ cudaError_t launch_transpose(const uint16_t* W, uint16_t* Wt, int N, int H, cuda
     return cudaGetLastError();
 }
 
-cudaError_t launch_pad_idx(const int32_t* src, int k, int H, int32_t* dst, int pad_to,
-                           cudaStream_t stream) {
+cudaError_t launch_pad_idx(const int32_t* src, int k, int H, int32_t* dst, int pad_to, cudaStream_t stream,
+                           int32_t* dst_copy) {
     const int blocks = (pad_to + 255) / 256;
     return launch_pdl(pad_idx_kernel, dim3(blocks < 1 ? 1 : blocks), dim3(256), 0, stream, src, k, H, dst,
-                      pad_to);
+                      pad_to, dst_copy);
 }
 
 }  // namespace rmm

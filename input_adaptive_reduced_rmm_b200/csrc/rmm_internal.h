@@ -30,11 +30,12 @@ cudaError_t launch_select(const uint16_t* X, int T, uint32_t* s32, int clear_inp
 // ---- block-granular kept sets (rmm_blocks.cu)
 // block 0 (single slices) or 16..256 dividing H with at most 1024 blocks
 bool block_size_ok(int H, int block);
-// From the score vector s32 (u32 [H], zeroed afterwards): the kb best blocks of
-// `block` slices (block score = max of its slices), their kb * block slices
-// ascending to idx (and idx_copy if not null), the blocks to blocks_out if not null.
-cudaError_t launch_block_select(uint32_t* s32, int H, int block, int kb, int32_t* idx, int32_t* idx_copy,
-                                int32_t* blocks_out, cudaStream_t stream);
+// The kb best blocks of `block` slices -- block score = max of its slices'
+// scores from s32 (u32 [H]), or, with X [T, H] given (T <= 16), the block's
+// mean magnitude -- their kb * block slices ascending to idx (and idx_copy if
+// not null), the blocks to blocks_out if not null; s32 is zeroed afterwards.
+cudaError_t launch_block_select(uint32_t* s32, const uint16_t* X, int T, int H, int block, int kb, int32_t* idx,
+                                int32_t* idx_copy, int32_t* blocks_out, cudaStream_t stream);
 
 // ---- split-K GEMV (rmm_gemv.cu)
 constexpr int kMaxGroupGemv = 4;
@@ -178,7 +179,9 @@ cudaError_t launch_attn_ctx(const uint16_t* Q, const uint16_t* Kt, const uint16_
 
 // ---- glue (rmm_glue.cu)
 cudaError_t launch_transpose(const uint16_t* W, uint16_t* Wt, int N, int H, cudaStream_t stream);
-cudaError_t launch_pad_idx(const int32_t* src, int k, int H, int32_t* dst, int pad_to,
-                           cudaStream_t stream);
+// src null: the identity list 0..k-1 (every slice kept); dst_copy (if not
+// null) receives the first k entries.
+cudaError_t launch_pad_idx(const int32_t* src, int k, int H, int32_t* dst, int pad_to, cudaStream_t stream,
+                           int32_t* dst_copy = nullptr);
 
 }  // namespace rmm

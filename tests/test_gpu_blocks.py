@@ -127,3 +127,61 @@ def test_blocks_reject_bad_sizes(rmm):
         rc = L.rmm_linear(rmm._ptr(X), rmm._ptr(Wt), 2, 1000, 64, 0.5, rmm._ptr(Y), None, rmm._ptr(ws),
                           ws.numel(), rmm._stream(None), rmm.ctypes.byref(opts))
         assert rc == rmm.RMM_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------- mean-magnitude blocks
+
+def run_mean_blocks(rmm, X, W, r, block, t_gemv=16):
+    T, H = X.shape
+    N = W.shape[0]
+    Wt = rmm.rmm_transpose_weight(W.cuda())
+    kb = oracle.k_for(H // block, r)
+    opts = rmm.options(block_size=block, block_score=1, t_gemv=t_gemv)
+    idx = torch.full((kb * block,), -1, dtype=torch.int32, device="cuda")
+    ws = rmm.new_workspace(rmm.rmm_linear_workspace_bytes(T, H, N, opts))
+    Y = rmm.rmm_linear(X.cuda(), Wt, r, idx_out=idx, workspace=ws, opts=opts)
+    torch.cuda.synchronize()
+    assert rmm.rmm_get_status(ws) == rmm.RMM_OK
+    return Y.cpu(), idx.cpu().numpy(), ws
+
+
+@pytest.mark.parametrize("T,H,N,r,block,t_gemv", [
+    (1, 4096, 1024, 0.5, 64, 16),    # the FFN demo's down projection
+    (1, 512, 264, 0.3, 16, 16),
+    (7, 1024, 520, 0.5, 128, 16),
+    (16, 2048, 1024, 0.25, 256, 16),
+    (5, 1024, 1032, 0.5, 64, 0),     # the GEMM path (score pass still writes X^T)
+])
+def test_blocks_mean_score(rmm, T, H, N, r, block, t_gemv):
+    X = rmm_synth.activations(T, H, rmm_synth.seed_for(9, T, 5))
+    W = rmm_synth.weights(N, H, rmm_synth.seed_for(9, T, 6), std=0.02)
+    Y, idx, _ = run_mean_blocks(rmm, X, W, r, block, t_gemv)
+    Yo, blocks = oracle.linear_blocks(X, W, r, block=block, block_score="mean")
+    assert idx.tolist() == expand(blocks, block).tolist()
+    assert_close(Y, Yo, f"mean blocks T={T} H={H} block={block}")
+
+
+def test_blocks_mean_then_max_on_one_workspace(rmm):
+    """A mean-score call leaves the workspace's score vector at zero for the next call."""
+    T, H, N, block = 4, 1024, 256, 64
+    X = rmm_synth.activations(T, H, 131)
+    W = rmm_synth.weights(N, H, 132)
+    Wt = rmm.rmm_transpose_weight(W.cuda())
+    ws = rmm.new_workspace(rmm.rmm_linear_workspace_bytes(T, H, N, rmm.options(block_size=block, t_gemv=0)))
+    for score, t_gemv in ((1, 0), (0, 0), (1, 16), (0, 16)):
+        opts = rmm.options(block_size=block, block_score=score, t_gemv=t_gemv)
+        idx = torch.empty(8 * block, dtype=torch.int32, device="cuda")
+        Y = rmm.rmm_linear(X.cuda(), Wt, 0.5, idx_out=idx, workspace=ws, opts=opts)
+        torch.cuda.synchronize()
+        Yo, blocks = oracle.linear_blocks(X, W, 0.5, block=block, block_score="mean" if score else "max")
+        assert idx.cpu().numpy().tolist() == expand(blocks, block).tolist()
+        assert_close(Y.cpu(), Yo, f"score={score} t_gemv={t_gemv}")
+
+
+def test_blocks_mean_rejects_long_chunks(rmm):
+    X = torch.zeros(17, 512, dtype=torch.bfloat16, device="cuda")
+    Wt = torch.zeros(512, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(rmm.RmmError):
+        rmm.rmm_linear(X, Wt, 0.5, opts=rmm.options(block_size=64, block_score=1))
+    with pytest.raises(rmm.RmmError):  # a block score needs blocks
+        rmm.rmm_linear(X[:1].contiguous(), Wt, 0.5, opts=rmm.options(block_score=1))
