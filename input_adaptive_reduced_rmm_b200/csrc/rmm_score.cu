@@ -127,6 +127,85 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// The score pass with the X^T copy, transposing in registers (H % 8 == 0,
+// X 16-byte aligned).  A CTA of 4 warps covers 64 tokens x 128 channels (about
+// seven CTAs per SM: one wave for the prefill shapes);
+// lane (g, half) of warp w loads 8 channels x 8 tokens (eight 16-byte loads,
+// all in flight), transposes the 8 x 8 block of bf16 with byte permutes and
+// stores 8 rows of X^T, 8 tokens each; lanes g and g + 16 fill the two halves
+// of one 32-byte sector.  No shared-memory tile.
+constexpr int kXtThreads = 128;
+constexpr int kXtTokens = 16 * (kXtThreads / 32);
+
+__global__ void __launch_bounds__(kXtThreads)
+    score_xt_kernel(const uint16_t* __restrict__ X, int T, int H, uint32_t* __restrict__ s32,
+                    uint16_t* __restrict__ Xt, int ldT) {
+    __shared__ uint32_t red[kXtThreads / 32][128];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane & 15, half = lane >> 4;
+    const int h = blockIdx.x * 128 + 8 * g;                   // first of the thread's 8 channels
+    const int tb = blockIdx.y * kXtTokens + 16 * warp + 8 * half;  // first of its 8 tokens
+    const bool hok = h < H;                                   // H % 8 == 0: all 8 channels valid
+    uint4 q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        q[i] = (hok && tb + i < T) ? ld_nc_v4(X + (size_t)(tb + i) * H + h) : make_uint4(0u, 0u, 0u, 0u);
+    uint32_t mx[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) mx[c] = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t w[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            mx[2 * m] = max(mx[2 * m], w[m] & 0x7FFFu);
+            mx[2 * m + 1] = max(mx[2 * m + 1], (w[m] >> 16) & 0x7FFFu);
+        }
+    }
+    // 8 x 8 transpose: o[j] holds channel h + j for tokens tb .. tb + 7
+    uint32_t o[8][4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+        const uint32_t a[4] = {q[2 * n].x, q[2 * n].y, q[2 * n].z, q[2 * n].w};
+        const uint32_t bb[4] = {q[2 * n + 1].x, q[2 * n + 1].y, q[2 * n + 1].z, q[2 * n + 1].w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            o[2 * m][n] = __byte_perm(a[m], bb[m], 0x5410);      // low halves: channel 2m
+            o[2 * m + 1][n] = __byte_perm(a[m], bb[m], 0x7632);  // high halves: channel 2m+1
+        }
+    }
+    if (hok && tb < T) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            uint16_t* dst = Xt + (size_t)(h + j) * ldT + tb;
+            if (tb + 8 <= T) {
+                *reinterpret_cast<uint4*>(dst) = make_uint4(o[j][0], o[j][1], o[j][2], o[j][3]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (tb + i < T) dst[i] = (uint16_t)((i & 1) ? (o[j][i >> 1] >> 16) : (o[j][i >> 1] & 0xFFFFu));
+            }
+        }
+    }
+    // channel maxima: the two token halves of a lane pair, then the 8 warps
+#pragma unroll
+    for (int c = 0; c < 8; ++c) mx[c] = max(mx[c], __shfl_xor_sync(0xffffffffu, mx[c], 16));
+    if (half == 0) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) red[warp][8 * g + c] = mx[c];
+    }
+    __syncthreads();
+    if (tid < 128) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int w = 0; w < kXtThreads / 32; ++w) m = max(m, red[w][tid]);
+        const int hh = blockIdx.x * 128 + tid;
+        if (s32 && hh < H && m > 0) atomicMax(s32 + hh, m);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_score(const uint16_t* X, int T, int H, uint32_t* s32, uint16_t* Xt, int ldT,
@@ -140,6 +219,12 @@ cudaError_t launch_score(const uint16_t* X, int T, int H, uint32_t* s32, uint16_
     if (ty < 1) ty = 1;
     dim3 grid(strips, ty);
     const bool vec = (H % 8 == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
+    if (Xt && vec) {
+        const int by = (T + kXtTokens - 1) / kXtTokens;
+        if (by <= 65535)
+            return launch_pdl(score_xt_kernel, dim3((H + 127) / 128, by), dim3(kXtThreads), 0, stream, X, T, H, s32,
+                              Xt, ldT);
+    }
     auto kern = Xt ? (vec ? score_kernel<true, true> : score_kernel<true, false>)
                    : (vec ? score_kernel<false, true> : score_kernel<false, false>);
     return launch_pdl(kern, grid, dim3(kThreads), 0, stream, X, T, H, s32, Xt, ldT);
