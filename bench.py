@@ -196,6 +196,13 @@ def oracle_sample(rows_per_proj: int, seed: int):
     return flops, secs, desc
 
 
+def step_config(world: int) -> dict:
+    """The workload description both arms print."""
+    return {"workload": WORKLOAD, "T": T_PREFILL, "r": R, "parallelism": f"replicas x{world}",
+            "calls_per_step": "q+k+v grouped, o, gate+up grouped, down",
+            "l2": "inputs larger than L2 (0.55 GB of weights and activations per step)"}
+
+
 def run_reference(args, world, rank):
     """The oracle timed on the host cores: each step is a bounded sample of the workload."""
     if rank != 0:
@@ -214,7 +221,7 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": WORKLOAD, "sample_rows_per_projection": rows},
+        "data": "synthetic", "config": step_config(args.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -740,9 +747,7 @@ def run_rmm(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "T": T_PREFILL, "r": R, "parallelism": f"replicas x{world}",
-                   "calls_per_step": "q+k+v grouped, o, gate+up grouped, down",
-                   "l2": "inputs larger than L2 (0.55 GB of weights and activations per step)"},
+        "config": step_config(world),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": STEP_GEMM_DRAM_BYTES,
                      "traffic_unit": "bytes (ncu dram read + write) over the step's 4 GEMM launches",
@@ -856,12 +861,13 @@ def main():
     if args.single:
         run_single(args)
         return
+    if args.impl == "reference":
+        # the oracle on the host cores: rank 0 alone, no process group, no GPU
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return
     world, rank, local = dist_setup()
     try:
-        if args.impl == "reference":
-            run_reference(args, world, rank)
-        else:
-            run_rmm(args, world, rank, local)
+        run_rmm(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist
