@@ -166,3 +166,19 @@ def test_ctx_rejects_unsupported(rmm):
         rmm.rmm_attn_ctx(Q1, Kt, V, means, L, 0.5, 0.5, 48)  # block 48
     with pytest.raises(rmm.RmmError):
         rmm.rmm_ctx_block_means(Kt, L, block, blk_begin=3, blk_end=5)  # past ceil(L / block)
+
+
+@pytest.mark.parametrize("L,block,r_ctx", [(65536, 32, 0.125), (4000, 256, 0.5), (65535, 64, 0.5)])
+def test_ctx_large_block_counts(rmm, L, block, r_ctx):
+    """2048 blocks of 32 keys (the most the block select sorts), a ragged 256-key last
+    block, and a ragged cache just under 64K keys."""
+    B, Hq, Hkv, T = 1, 4, 1, 1
+    seed = rmm_synth.seed_for(14, L % 1000, block)
+    Q = rmm_synth.normal((B, Hq, T, D), seed)
+    K = rmm_synth.normal((B, Hkv, L, D), seed + 1)
+    V = rmm_synth.normal((B, Hkv, L, D), seed + 2)
+    O, idx, blocks, k, kc, _ = run_ctx(rmm, Q, K, V, 0.5, r_ctx, block)
+    Oo, io, bo = oracle.attention_ctx(Q, K, V, k, block, kc, causal=True)
+    assert np.array_equal(idx, io)
+    assert np.array_equal(blocks, bo)
+    assert_close(O, Oo, f"L={L} block={block} r_ctx={r_ctx}")
