@@ -51,7 +51,7 @@ typedef void* rmm_stream_t;
 typedef enum {
     RMM_OK = 0,
     RMM_ERR_INVALID_ARG = 1, /* null pointer, bad size, r outside (0,1], misaligned pointer */
-    RMM_ERR_UNSUPPORTED = 2, /* a valid shape this build does not handle (e.g. d != 128) */
+    RMM_ERR_UNSUPPORTED = 2, /* a valid shape the library does not handle (e.g. d != 128) */
     RMM_ERR_WORKSPACE = 3,   /* workspace null or smaller than the *_workspace_bytes() query */
     RMM_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
     RMM_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (reported by rmm_get_status) */

@@ -36,7 +36,7 @@ namespace rmm {
 
 namespace {
 
-constexpr int D = 128;        // head dimension handled by this build
+constexpr int D = 128;        // the head dimension the kernels handle
 constexpr int kThreads = 256;
 constexpr int SB = 1024;      // keys per sub-block
 constexpr int RMAX = 8;       // query rows per CTA (at most)
