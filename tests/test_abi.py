@@ -115,3 +115,46 @@ def test_binding_fails_loudly_without_library(tmp_path):
     )
     out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT)
     assert "raised" in out.stdout
+
+
+def test_context_block_entry_points_validate_on_the_host(lib):
+    """rmm_ctx_block_means / rmm_attn_ctx reject bad arguments before anything is enqueued
+    (the fake pointers below are never dereferenced)."""
+    from input_adaptive_reduced_rmm_b200 import rmm
+
+    L = rmm.lib()
+    fake = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never touched
+    # block means: null pointers, a block size outside {32, 64, 128, 256}, a range past ceil(L/block)
+    assert L.rmm_ctx_block_means(None, 1, 1, 128, 256, 256, 64, 0, 4, None, None) == rmm.RMM_ERR_INVALID_ARG
+    assert L.rmm_ctx_block_means(fake, 1, 1, 128, 256, 256, 48, 0, 1, fake, None) == rmm.RMM_ERR_INVALID_ARG
+    assert L.rmm_ctx_block_means(fake, 1, 1, 128, 256, 256, 64, 3, 5, fake, None) == rmm.RMM_ERR_INVALID_ARG
+    assert L.rmm_ctx_block_means(fake, 1, 1, 128, 256, 256, 64, 2, 2, fake, None) == rmm.RMM_ERR_INVALID_ARG
+    # attention: no block means, a bad block, r_ctx out of (0, 1]
+    args = lambda means, block, r_ctx: (fake, fake, fake, means, 1, 4, 1, 1, 256, 256, 128, 0.5, r_ctx, block, 1,
+                                        1.0, fake, None, None, fake, 1 << 20, None, None)
+    assert L.rmm_attn_ctx(*args(None, 64, 0.5)) == rmm.RMM_ERR_INVALID_ARG
+    assert L.rmm_attn_ctx(*args(fake, 48, 0.5)) == rmm.RMM_ERR_INVALID_ARG
+    assert L.rmm_attn_ctx(*args(fake, 64, 1.5)) == rmm.RMM_ERR_INVALID_ARG
+    assert L.rmm_attn_ctx(*args(fake, 64, 0.0)) == rmm.RMM_ERR_INVALID_ARG
+
+
+def test_context_block_workspace_sizes(lib):
+    from input_adaptive_reduced_rmm_b200 import rmm
+
+    w1 = rmm.rmm_attn_ctx_workspace_bytes(1, 32, 8, 1, 4096, 64, 0.5)
+    w2 = rmm.rmm_attn_ctx_workspace_bytes(1, 32, 8, 1, 65536, 64, 0.5)
+    assert 0 < w1 <= w2
+    assert rmm.rmm_attn_ctx_workspace_bytes(1, 32, 8, 1, 4096, 48, 0.5) == 0   # block size
+    assert rmm.rmm_attn_ctx_workspace_bytes(1, 32, 8, 1, 4096, 64, 0.0) == 0   # r_ctx
+    assert rmm.rmm_attn_ctx_workspace_bytes(1, 32, 8, 1, 4096, 64, 0.5, d=64) == 0
+
+
+def test_option_fields_are_validated(lib):
+    """Option values outside their ranges make every size query return 0 (and every call
+    RMM_ERR_INVALID_ARG): a block score without blocks, unknown scores, paths and producers."""
+    from input_adaptive_reduced_rmm_b200 import rmm
+
+    assert rmm.rmm_linear_workspace_bytes(4, 1024, 1024, rmm.options(block_size=64, block_score=1)) > 0
+    for bad in (rmm.options(block_score=1), rmm.options(block_size=64, block_score=2), rmm.options(attn_path=3),
+                rmm.options(gemm_producer=3), rmm.options(block_size=-1)):
+        assert rmm.rmm_linear_workspace_bytes(4, 1024, 1024, bad) == 0
