@@ -839,6 +839,38 @@ def run_single_attn(args):
                                       "call_us": 1e3 * ms, "tflops": flops / (ms * 1e-3) / 1e12}}), flush=True)
 
 
+def run_single_ctx(args):
+    """One rmm_attn_ctx call timed alone (profiling aid): --single-ctx B,Hq,Hkv,L,block,r,r_ctx
+    (decode, T = 1, d = 128; the block means are made once, untimed)."""
+    from input_adaptive_reduced_rmm_b200 import rmm
+
+    B, Hq, Hkv, L, block, r, r_ctx = args.single_ctx.split(",")
+    B, Hq, Hkv, L, block, r, r_ctx = int(B), int(Hq), int(Hkv), int(L), int(block), float(r), float(r_ctx)
+    dev = torch.device("cuda", 0)
+    D, T = 128, 1
+    Q = rmm_synth.normal((B, Hq, T, D), 31).to(dev)
+    Kt = rmm_synth.normal((B, Hkv, D, L), 32).to(dev)
+    V = rmm_synth.normal((B, Hkv, L, D), 33).to(dev)
+    O = torch.empty_like(Q)
+    means = rmm.rmm_ctx_block_means(Kt, L, block)
+    ws = rmm.new_workspace(rmm.rmm_attn_ctx_workspace_bytes(B, Hq, Hkv, T, L, block, r_ctx), dev)
+    for _ in range(args.warmup):
+        rmm.rmm_attn_ctx(Q, Kt, V, means, L, r, r_ctx, block, O=O, workspace=ws)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        rmm.rmm_attn_ctx(Q, Kt, V, means, L, r, r_ctx, block, O=O, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    if rmm.rmm_get_status(ws) != rmm.RMM_OK:
+        raise RuntimeError("device status not OK")
+    print(json.dumps({"single_ctx": {"B": B, "Hq": Hq, "Hkv": Hkv, "L": L, "block": block, "r": r, "r_ctx": r_ctx,
+                                     "call_us": 1e3 * statistics.median(ts)}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -850,6 +882,8 @@ def main():
     ap.add_argument("--skip-secondary", action="store_true")
     ap.add_argument("--single", default=None, help="T,H,N,r: time one rmm_linear shape alone")
     ap.add_argument("--single-attn", default=None, help="B,Hq,Hkv,T,L,r: time one rmm_attn_qk call alone")
+    ap.add_argument("--single-ctx", default=None,
+                    help="B,Hq,Hkv,L,block,r,r_ctx: time one rmm_attn_ctx decode call alone")
     ap.add_argument("--gemm-producer", type=int, default=0)
     ap.add_argument("--block-size", type=int, default=0, help="with --single: block-granular kept sets")
     args = ap.parse_args()
@@ -857,6 +891,9 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.single_attn:
         run_single_attn(args)
+        return
+    if args.single_ctx:
+        run_single_ctx(args)
         return
     if args.single:
         run_single(args)
