@@ -23,13 +23,16 @@
 // Kernels:
 //   ctx_means_kernel   one CTA per (block, KV head), thread c sums row c of
 //                      the d-major K^T cache over the block (16-byte loads)
-//   ctx_score_kernel   one thread per (set, block): the set's query rows
-//                      staged in shared memory 16 at a time, four fmaf chains
-//                      in flight; the best dot written as an order-preserving
-//                      32-bit key (-0 and +0 share a key)
-//   ctx_select_kernel  one CTA per set: bitonic sort of (key desc, block asc)
-//                      over up to 2048 blocks, then the kept blocks listed in
-//                      ascending order by one block-wide scan
+//   ctx_score_kernel   a CTA per (set, 32 blocks): their mean keys and the
+//                      set's query rows staged in shared memory, a thread per
+//                      (block, row slot) running fmaf chains; the best dot
+//                      written as an order-preserving 32-bit key (-0 and +0
+//                      share a key)
+//   ctx_select_reg_kernel  one CTA per set, a thread per block (up to 1024):
+//                      bitonic sort of (key desc, block asc) in registers,
+//                      shuffles inside a warp, shared memory across warps;
+//                      then the kept blocks listed ascending by one scan
+//   ctx_select_kernel  the same sort in shared memory for 1025-2048 blocks
 // The attention itself is the split pass of rmm_attn.cu over the kept blocks.
 #include <math.h>
 
@@ -77,10 +80,17 @@ __device__ __forceinline__ uint32_t float_key(float f) {
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// CTA = 32 blocks x 4 row slots (128 threads): the 32 blocks' mean keys and
+// 16 query rows at a time are staged in shared memory (rows padded to 129
+// floats: conflict-free column reads), thread (block, slot) runs the fmaf
+// chain of rows slot, slot + 4, ... over the 128 dims in order and keeps the
+// best; the 4 slots' bests are folded by shuffles (a max: exact).
+constexpr int kScoreBlocks = 32;
 __global__ void __launch_bounds__(128)
     ctx_score_kernel(const uint16_t* __restrict__ Q, const float* __restrict__ means, int Hq, int Hkv, int T,
                      int nblk, int nblk_stride, int per_query_head, uint32_t* __restrict__ keys) {
-    __shared__ float qs[16][D];
+    __shared__ float qs[16][D + 1];
+    __shared__ float mt[kScoreBlocks][D + 1];
     const int nsets = per_query_head ? Hq : Hkv;
     const int set = blockIdx.y % nsets;
     const int b = blockIdx.y / nsets;
@@ -89,11 +99,24 @@ __global__ void __launch_bounds__(128)
     const int q_lo = per_query_head ? set : set * G;
     const int nq = per_query_head ? 1 : G;
     const int R = nq * T;
-    const int j = blockIdx.x * 128 + threadIdx.x;
-    const bool valid = j < nblk;
-    const float4* m4 = reinterpret_cast<const float4*>(means + ((size_t)(b * Hkv + g) * nblk_stride + (valid ? j : 0)) * D);
+    const int tid = threadIdx.x;
+    const int bl = tid >> 2, slot = tid & 3;
+    const int j0 = blockIdx.x * kScoreBlocks;
+    const int j = j0 + bl;
     pdl_wait();
     pdl_launch_dependents();
+    // the 32 mean keys: 128 threads x 8 float4, coalesced
+    const float4* m4 = reinterpret_cast<const float4*>(means + ((size_t)(b * Hkv + g) * nblk_stride + j0) * D);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int e = tid + 128 * u;  // float4 index in the tile: block e / 32, dims 4 * (e % 32) ..
+        const int eb = e >> 5, ec = (e & 31) * 4;
+        const float4 v = (j0 + eb < nblk) ? __ldg(m4 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+        mt[eb][ec] = v.x;
+        mt[eb][ec + 1] = v.y;
+        mt[eb][ec + 2] = v.z;
+        mt[eb][ec + 3] = v.w;
+    }
     float best = -INFINITY;
     for (int r0 = 0; r0 < R; r0 += 16) {
         __syncthreads();
@@ -101,13 +124,13 @@ __global__ void __launch_bounds__(128)
         uint4 piece[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            const int e = threadIdx.x + 128 * u, rr = e / 16, r = r0 + rr;
+            const int e = tid + 128 * u, rr = e / 16, r = r0 + rr;
             piece[u] = r < R ? ld_nc_v4(Q + (((size_t)b * Hq + q_lo + r / T) * T + r % T) * D + (e % 16) * 8)
                              : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            const int e = threadIdx.x + 128 * u, rr = e / 16, c = (e % 16) * 8;
+            const int e = tid + 128 * u, rr = e / 16, c = (e % 16) * 8;
             const uint32_t w[4] = {piece[u].x, piece[u].y, piece[u].z, piece[u].w};
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
@@ -117,30 +140,65 @@ __global__ void __launch_bounds__(128)
         }
         __syncthreads();
         const int nr = min(16, R - r0);
-        if (valid) {
-            for (int rr = 0; rr < nr; rr += 4) {
-                float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
-#pragma unroll 8
-                for (int c4 = 0; c4 < D / 4; ++c4) {
-                    const float4 mv = __ldg(m4 + c4);
-                    const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int c = 4 * c4 + u;
-                        a0 = fmaf(qs[rr][c], mm[u], a0);
-                        a1 = fmaf(qs[rr + 1][c], mm[u], a1);
-                        a2 = fmaf(qs[rr + 2][c], mm[u], a2);
-                        a3 = fmaf(qs[rr + 3][c], mm[u], a3);
-                    }
-                }
-                if (a0 > best) best = a0;
-                if (rr + 1 < nr && a1 > best) best = a1;
-                if (rr + 2 < nr && a2 > best) best = a2;
-                if (rr + 3 < nr && a3 > best) best = a3;
-            }
+        for (int rr = slot; rr < nr; rr += 4) {
+            float acc = 0.0f;
+#pragma unroll 16
+            for (int c = 0; c < D; ++c) acc = fmaf(qs[rr][c], mt[bl][c], acc);
+            if (acc > best) best = acc;
         }
     }
-    if (valid) keys[(size_t)blockIdx.y * nblk + j] = float_key(best);
+    best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 1));
+    best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 2));
+    if (slot == 0 && j < nblk) keys[(size_t)blockIdx.y * nblk + j] = float_key(best);
+}
+
+// One CTA of P threads per set (P = the power of two >= nblk, at most 1024):
+// thread i holds element i of (key desc, block asc) packed in 64 bits; a
+// bitonic sort in registers, partners within a warp by shuffle and across
+// warps through shared memory (two barriers per such stage); the first kc
+// elements are the kept blocks, listed ascending by one block-wide scan.
+__global__ void __launch_bounds__(kSelThreads)
+    ctx_select_reg_kernel(const uint32_t* __restrict__ keys, int nblk, int kc, int32_t* __restrict__ blocks) {
+    __shared__ uint64_t xs[kSelThreads];
+    __shared__ uint8_t flag[kSelThreads];
+    __shared__ int warp_sum[kSelThreads / 32];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int P = blockDim.x;
+    const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+    const uint32_t* key = keys + (size_t)blockIdx.x * nblk;
+    uint64_t v = i < nblk ? ((uint64_t)(~key[i]) << 32) | (uint32_t)i : ~0ull;
+    flag[i] = 0;
+    for (int k2 = 2; k2 <= P; k2 <<= 1)
+        for (int jj = k2 >> 1; jj > 0; jj >>= 1) {
+            uint64_t o;
+            if (jj >= 32) {
+                xs[i] = v;
+                __syncthreads();
+                o = xs[i ^ jj];
+                __syncthreads();
+            } else {
+                o = __shfl_xor_sync(0xffffffffu, v, jj);
+            }
+            // the lower index of a pair takes the smaller value in an ascending run
+            const bool take_min = ((i & k2) == 0) == (i < (i ^ jj));
+            v = take_min ? (o < v ? o : v) : (o < v ? v : o);
+        }
+    __syncthreads();
+    if (i < kc) flag[(uint32_t)v] = 1;
+    __syncthreads();
+    const int cnt = flag[i];
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    int pos = incl - cnt;
+    for (int w = 0; w < warp; ++w) pos += warp_sum[w];
+    if (cnt) blocks[(size_t)blockIdx.x * kc + pos] = i;
 }
 
 __global__ void __launch_bounds__(kSelThreads)
@@ -217,11 +275,15 @@ cudaError_t launch_attn_ctx(const uint16_t* Q, const uint16_t* Kt, const uint16_
     cudaError_t e = cudaSuccess;
     if (!select_here) e = launch_attn_dims(Q, B, Hq, Hkv, T, k, per_query_head, p.nsets, idx, sc, stream);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(ctx_score_kernel, dim3((nblk + 127) / 128, B * p.nsets), dim3(128), 0, stream, Q, means, Hq, Hkv,
-                   T, nblk, nblk_stride, per_query_head, keys);
+    e = launch_pdl(ctx_score_kernel, dim3((nblk + kScoreBlocks - 1) / kScoreBlocks, B * p.nsets), dim3(128), 0,
+                   stream, Q, means, Hq, Hkv, T, nblk, nblk_stride, per_query_head, keys);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(ctx_select_kernel, dim3(B * p.nsets), dim3(kSelThreads), (size_t)P * sizeof(uint64_t), stream,
-                   (const uint32_t*)keys, nblk, P, kc, blocks);
+    if (P <= kSelThreads)
+        e = launch_pdl(ctx_select_reg_kernel, dim3(B * p.nsets), dim3(P < 32 ? 32 : P), 0, stream,
+                       (const uint32_t*)keys, nblk, kc, blocks);
+    else
+        e = launch_pdl(ctx_select_kernel, dim3(B * p.nsets), dim3(kSelThreads), (size_t)P * sizeof(uint64_t), stream,
+                       (const uint32_t*)keys, nblk, P, kc, blocks);
     if (e != cudaSuccess) return e;
     return launch_attn_split_ctx(Q, Kt, V, B, Hq, Hkv, T, L, ldL, k, causal, scale, per_query_head, O, idx,
                                  (int)select_here, blocks, bc_shift, kc, partials, p, stream);
