@@ -252,6 +252,18 @@ __global__ void __launch_bounds__(kThreads, kRows == 4 ? 2 : 1)
         for (int c = 0; c < 8; ++c) acc[r][c] = 0.0f;
 
     for (int l0 = l_begin; l0 < l_end; l0 += SB) {
+        // with context blocks, the sub-block's scattered V rows start towards L2
+        // now, so that the P.V pass after the logits finds them there: line q of
+        // the sub-block (a V row is two 128-byte lines) is requested by thread
+        // q mod 256.  (For contiguous keys the same prefetch competes with the
+        // K loads on the critical path and measured slower: not done.)
+        if constexpr (kCtx) {
+            const int nk = min(SB, l_end - l0);
+            for (int q = tid; q < 2 * nk; q += kThreads) {
+                const int lv = key_pos(l0 + (q >> 1));
+                if (lv < L) prefetch_l2(vbase + (size_t)lv * D + (q & 1) * 64);
+            }
+        }
         // ---- logits: thread owns keys l0 + 4*tid .. +3
         const int l = l0 + tid * 4;
         const int lp = l < l_end ? key_pos(l) : L;  // cache position of the thread's first key
