@@ -3,9 +3,9 @@
  *
  * The method (Reduced Matrix Multiplication: Input-Adaptive Matrix-Product
  * Reduction for LLM Inference, Lan, Li, Zhou -- abstract): a training-free,
- * input-adaptive reduction of each Transformer matrix product that keeps
- * only informative slices along the contraction dimension, controlled by one
- * retention ratio r.  For a projection Y = X W^T (X [T,H] activations,
+ * input-adaptive reduction of each Transformer matrix product: the slices
+ * of the contraction dimension that the current input makes most significant
+ * are kept, their share set by one retention ratio r.  For a projection Y = X W^T (X [T,H] activations,
  * W [N,H] weights; cf-1.com post on input-adaptive matrix-product reduction,
  * §2) the library
  *   1. scores every contraction index h by s_h = max_t |X[t,h]| (post §5.1:

@@ -12,8 +12,9 @@ and marshals numpy arrays of bf16 bit patterns (uint16) into it.
 Every function follows the method as the pages describe it:
 
 * Reduced Matrix Multiplication: Input-Adaptive Matrix-Product Reduction for
-  LLM Inference (Lan, Li, Zhou), abstract -- keep informative slices along the
-  contraction dimension at retention ratio r;
+  LLM Inference (Lan, Li, Zhou), abstract -- each product keeps the slices of
+  its contraction dimension that the input makes most significant, at
+  retention ratio r;
 * Input-adaptive matrix-product reduction for LLM inference (cf-1.com post),
   §2 (Y ~= X @ W_sub^T), §5.1-§5.3 (score, top-k, gather + smaller product),
   §6.1 (top-k then sort; keep ratio 1 reproduces the full product),

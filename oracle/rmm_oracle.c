@@ -14,8 +14,9 @@
  *
  *   Reduced Matrix Multiplication: Input-Adaptive Matrix-Product Reduction for
  *   LLM Inference (Lan, Li, Zhou), abstract: a training-free, input-adaptive
- *   method that keeps informative slices along the contraction dimension of
- *   each Transformer matrix product, with one retention ratio r.
+ *   method; each Transformer matrix product keeps the slices of its
+ *   contraction dimension that the current input makes most significant, in
+ *   a share set by one retention ratio r.
  *
  *   Input-adaptive matrix-product reduction for LLM inference (cf-1.com post):
  *     §2   the linear map Y = X @ W^T is replaced by Y ~= X @ W_sub^T over a
