@@ -585,3 +585,73 @@ def test_block_mean_linear_full_ratio_is_dense_and_keeps_the_loud_block():
     X2[:, 128:192] = (X2[:, 128:192].float() * 50).to(torch.bfloat16)  # block 2 is loud
     _, b2 = oracle.linear_blocks(X2, W, 0.25, block=64, block_score="mean")
     assert b2.tolist() == [2]
+
+
+# ---------------------------------------------------------------- invariances
+# Relabelling the contraction index, exact rescaling and reordering keys are
+# symmetries of the method's definitions; a dropped or swapped index anywhere
+# in the oracle breaks one of them.
+
+
+def test_linear_is_equivariant_under_a_column_permutation():
+    """Distinct scores (no ties): permuting X's and W's columns by p permutes the kept
+    set by p and leaves Y unchanged."""
+    T, H, N = 5, 96, 40
+    g = np.random.default_rng(121)
+    # small random entries, and one distinct, exactly representable maximum per column
+    X = (rmm_synth.activations(T, H, 122).float() * 0.01)
+    X[2] = torch.tensor(g.permutation(H) + 1, dtype=torch.float32) / 16
+    X = X.to(torch.bfloat16)
+    W = rmm_synth.weights(N, H, 123)
+    s = oracle.score(X)
+    assert len(set(s.tolist())) == H, "the test wants distinct scores"
+    perm = g.permutation(H)
+    Xp, Wp = X[:, perm].contiguous(), W[:, perm].contiguous()
+    for r in (0.25, 0.5, 0.8):
+        Y, idx = oracle.linear(X, W, r)
+        Yp, idxp = oracle.linear(Xp, Wp, r)
+        assert sorted(perm[idxp].tolist()) == idx.tolist()
+        assert np.max(np.abs(Y - Yp)) <= 1e-12 * max(1.0, np.abs(Y).max())
+
+
+def test_linear_scales_exactly_with_a_power_of_two():
+    X = rmm_synth.activations(4, 128, 124)
+    W = rmm_synth.weights(32, 128, 125)
+    Y, idx = oracle.linear(X, W, 0.5)
+    Y2, idx2 = oracle.linear((X.float() * 2).to(torch.bfloat16), W, 0.5)
+    assert idx.tolist() == idx2.tolist()
+    assert np.array_equal(Y2, 2 * Y)
+
+
+def test_attention_is_invariant_under_a_key_permutation():
+    """Non-causal attention: reordering the cache's keys (K and V together) changes
+    nothing; with the causal mask of a decode step (T = 1) neither."""
+    B, Hq, Hkv, T, L, d = 1, 4, 2, 1, 50, 32
+    Q = rmm_synth.normal((B, Hq, T, d), 126)
+    K = rmm_synth.normal((B, Hkv, L, d), 127)
+    V = rmm_synth.normal((B, Hkv, L, d), 128)
+    perm = np.random.default_rng(129).permutation(L)
+    Kp, Vp = K[:, :, perm].contiguous(), V[:, :, perm].contiguous()
+    for causal in (False, True):
+        O, idx = oracle.attention(Q, K, V, 16, causal=causal)
+        Op, idxp = oracle.attention(Q, Kp, Vp, 16, causal=causal)
+        assert np.array_equal(idx, idxp)
+        assert np.max(np.abs(O - Op)) <= 1e-12
+
+
+def test_context_blocks_follow_their_keys_under_a_block_permutation():
+    """Non-causal: reordering whole blocks of keys reorders the block scores the same way,
+    so the kept set maps through the permutation and O is unchanged."""
+    B, Hq, Hkv, T, bc, nb, d = 1, 4, 1, 2, 32, 8, 32
+    L = bc * nb
+    Q = rmm_synth.normal((B, Hq, T, d), 130)
+    K = rmm_synth.normal((B, Hkv, L, d), 131)
+    V = rmm_synth.normal((B, Hkv, L, d), 132)
+    bperm = np.random.default_rng(133).permutation(nb)
+    pos = (bperm[:, None] * bc + np.arange(bc)[None, :]).reshape(-1)  # new block j holds old block bperm[j]
+    Kp, Vp = K[:, :, pos].contiguous(), V[:, :, pos].contiguous()
+    O, idx, blocks = oracle.attention_ctx(Q, K, V, 16, bc, 3, causal=False)
+    Op, idxp, blocksp = oracle.attention_ctx(Q, Kp, Vp, 16, bc, 3, causal=False)
+    assert np.array_equal(idx, idxp)
+    assert sorted(bperm[blocksp[0, 0]].tolist()) == blocks[0, 0].tolist()
+    assert np.max(np.abs(O - Op)) <= 1e-12
