@@ -201,6 +201,8 @@ __global__ void __launch_bounds__(kSelThreads)
     if (cnt) blocks[(size_t)blockIdx.x * kc + pos] = i;
 }
 
+// The same selection for 1025-2048 blocks: the sort in shared memory (P
+// entries, up to two per thread), a barrier per stage.
 __global__ void __launch_bounds__(kSelThreads)
     ctx_select_kernel(const uint32_t* __restrict__ keys, int nblk, int P, int kc, int32_t* __restrict__ blocks) {
     extern __shared__ uint64_t v[];  // P entries
