@@ -192,8 +192,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_tiles = (T + BQ - 1) / BQ;
-    const int tile = n_tiles - 1 - (int)blockIdx.x;  // the longest (latest) tiles first
-    const int h = blockIdx.y, b = blockIdx.z;
+    // heads vary fastest in launch order, so the longest (latest) tiles of every
+    // head are launched before any shorter tile: a short tail
+    const int tile = n_tiles - 1 - (int)blockIdx.y;
+    const int h = blockIdx.x, b = blockIdx.z;
     const int G = Hq / Hkv;
     const int g = h / G;
     const int nsets = per_query_head ? Hq : Hkv;
@@ -473,7 +475,7 @@ cudaError_t launch_attn_tc(const uint16_t* Q, const uint16_t* Kt, const uint16_t
     const size_t smem = attn_tc_smem_bytes(kp);
     cudaError_t e = ensure_smem_limit(attn_tc_kernel, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((T + BQ - 1) / BQ, Hq, B);
+    dim3 grid(Hq, (T + BQ - 1) / BQ, B);
     return launch_pdl(attn_tc_kernel, grid, dim3(kThreadsTc), smem, stream, Q, Kt, V, Hq, Hkv, T, L, ldL, k, kp,
                       causal, scale * 1.4426950408889634f, per_query_head, idx, O, status);
 }
