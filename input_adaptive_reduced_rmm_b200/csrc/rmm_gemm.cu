@@ -11,6 +11,13 @@
 // here the kept slices go straight from their home rows into shared memory,
 // and no compacted copy exists anywhere in HBM.
 //
+// Two kernels live here.  The default is the CTA-pair kernel (namespace
+// `pair`, described at its definition): a cluster of two CTAs computes a
+// 256 x 512 tile with tcgen05 cta_group::2, its operands gathered by cp.async
+// or, for kept sets made of whole 64-slice runs, loaded by TMA tile copies.
+// The single-CTA kernel described next is kept for comparison (rmm_options.
+// gemm_producer 1 and 2).
+//
 // A kept slice h is one contiguous row of W^T [H, N] and one contiguous row of
 // X^T [H, T] (written by the score pass).  For a 128 x 256 output tile and a
 // K-block of 64 kept slices the operands are 64 rows x 256 columns of W^T
