@@ -49,27 +49,42 @@ _f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
 _f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
 
 
-def build(force: bool = False) -> str:
-    """Compile rmm_oracle.c into _build/liboracle.so (plain gcc, no fast-math, no FMA contraction)."""
-    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
-        return _LIB
-    os.makedirs(os.path.dirname(_LIB), exist_ok=True)
-    tmp = _LIB + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
-           _SRC, "-o", tmp, "-lm"]
+_LIB_OMP = os.path.join(_HERE, "_build", "liboracle_omp.so")
+
+
+def build(force: bool = False, parallel: bool = False) -> str:
+    """Compile rmm_oracle.c into _build/liboracle.so (plain gcc, no fast-math, no FMA contraction);
+    parallel=True: the same source with OpenMP (output rows spread over the host's threads, each
+    row computed as in the plain build) into _build/liboracle_omp.so."""
+    out = _LIB_OMP if parallel else _LIB
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(_SRC):
+        return out
+    os.makedirs(os.path.dirname(out), exist_ok=True)
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+    cmd += ["-fopenmp"] if parallel else []
+    cmd += [_SRC, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, _LIB)
-    return _LIB
+    os.replace(tmp, out)
+    return out
 
 
 _lib = None
+_lib_omp = None
 
 
-def _load():
-    global _lib
-    if _lib is not None:
+def parallel_threads() -> int:
+    """Threads the OpenMP build's product loop uses on this host."""
+    return int(_load(parallel=True).oracle_threads())
+
+
+def _load(parallel: bool = False):
+    global _lib, _lib_omp
+    if parallel and _lib_omp is not None:
+        return _lib_omp
+    if not parallel and _lib is not None:
         return _lib
-    lib = ctypes.CDLL(build())
+    lib = ctypes.CDLL(build(parallel=parallel))
     L, D, I, P = ctypes.c_long, ctypes.c_double, ctypes.c_int, ctypes.c_void_p
     lib.oracle_k_for.argtypes = [L, D]
     lib.oracle_k_for.restype = I
@@ -101,7 +116,12 @@ def _load():
     lib.oracle_rmsnorm.restype = I
     lib.oracle_swiglu.argtypes = [_u16p, _u16p, L, _f64p]
     lib.oracle_swiglu.restype = I
-    _lib = lib
+    lib.oracle_threads.argtypes = []
+    lib.oracle_threads.restype = I
+    if parallel:
+        _lib_omp = lib
+    else:
+        _lib = lib
     return lib
 
 
@@ -172,8 +192,9 @@ def reduced_product(X, W, idx, rows=None, cols=None) -> np.ndarray:
     return Y
 
 
-def linear(X, W, r: float, rows=None, cols=None):
-    """(Y fp64 [nrows, ncols], idx int32 [k]) of the reduced linear map Y ~= X[:,S] W[:,S]^T."""
+def linear(X, W, r: float, rows=None, cols=None, parallel: bool = False):
+    """(Y fp64 [nrows, ncols], idx int32 [k]) of the reduced linear map Y ~= X[:,S] W[:,S]^T.
+    parallel=True runs the OpenMP build (same bits, rows spread over the host's threads)."""
     x, w = _bits(X), _bits(W)
     T, H = x.shape
     N = w.shape[0]
@@ -184,7 +205,7 @@ def linear(X, W, r: float, rows=None, cols=None):
     cp, nc, _kc = _rows(cols)
     Y = np.zeros((nr if rows is not None else T, nc if cols is not None else N), dtype=np.float64)
     idx = np.zeros(k, dtype=np.int32)
-    _check(_load().oracle_linear(x, w, T, H, N, float(r), rp, nr, cp, nc, Y, idx), "oracle_linear")
+    _check(_load(parallel).oracle_linear(x, w, T, H, N, float(r), rp, nr, cp, nc, Y, idx), "oracle_linear")
     return Y, idx
 
 

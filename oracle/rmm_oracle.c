@@ -52,6 +52,9 @@
  */
 #include <math.h>
 #include <stdint.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 #include <stdlib.h>
 #include <string.h>
 
@@ -176,29 +179,43 @@ int oracle_reduced_product(const uint16_t* X, const uint16_t* W, long T, long H,
         if (cols && (cols[c] < 0 || cols[c] >= N)) return ORACLE_ERR_ARG;
     if (!all_finite(X, T * H) || !all_finite(W, N * H)) return ORACLE_ERR_NONFINITE;
 
-    double* xk = (double*)malloc(sizeof(double) * (size_t)k);
-    double* wk = (double*)malloc(sizeof(double) * (size_t)k);
-    if (!xk || !wk) {
+    /* One output row per iteration; with the OpenMP build (the parallel CPU
+     * baseline) rows are spread over the host's threads, each row still
+     * computed by one thread in the order below, so the results are the
+     * same bits as the single-threaded build's. */
+    int nomem = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : nomem)
+    for (long r = 0; r < nrows; ++r) {
+        double* xk = (double*)malloc(sizeof(double) * (size_t)k);
+        double* wk = (double*)malloc(sizeof(double) * (size_t)k);
+        if (!xk || !wk) {
+            nomem = 1;
+        } else {
+            long t = rows ? (long)rows[r] : r;
+            /* gather the kept slices of this activation row */
+            for (long j = 0; j < k; ++j) xk[j] = bf16_to_double(X[t * H + idx[j]]);
+            for (long c = 0; c < ncols; ++c) {
+                long n = cols ? (long)cols[c] : c;
+                /* gather the same kept slices of the weight row, then the smaller dot product */
+                for (long j = 0; j < k; ++j) wk[j] = bf16_to_double(W[n * H + idx[j]]);
+                double acc = 0.0;
+                for (long j = 0; j < k; ++j) acc += xk[j] * wk[j];
+                Y[r * ncols + c] = acc;
+            }
+        }
         free(xk);
         free(wk);
-        return ORACLE_ERR_NOMEM;
     }
-    for (long r = 0; r < nrows; ++r) {
-        long t = rows ? (long)rows[r] : r;
-        /* gather the kept slices of this activation row */
-        for (long j = 0; j < k; ++j) xk[j] = bf16_to_double(X[t * H + idx[j]]);
-        for (long c = 0; c < ncols; ++c) {
-            long n = cols ? (long)cols[c] : c;
-            /* gather the same kept slices of the weight row, then the smaller dot product */
-            for (long j = 0; j < k; ++j) wk[j] = bf16_to_double(W[n * H + idx[j]]);
-            double acc = 0.0;
-            for (long j = 0; j < k; ++j) acc += xk[j] * wk[j];
-            Y[r * ncols + c] = acc;
-        }
-    }
-    free(xk);
-    free(wk);
-    return 0;
+    return nomem ? ORACLE_ERR_NOMEM : 0;
+}
+
+/* Threads the product loop may use: 1 in the plain build. */
+int oracle_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }
 
 /* ---- block-granular kept sets (§5.2, §6.1 demo) ------------------------ */

@@ -655,3 +655,14 @@ def test_context_blocks_follow_their_keys_under_a_block_permutation():
     assert np.array_equal(idx, idxp)
     assert sorted(bperm[blocksp[0, 0]].tolist()) == blocks[0, 0].tolist()
     assert np.max(np.abs(O - Op)) <= 1e-12
+
+
+def test_openmp_build_gives_the_same_bits():
+    """The parallel CPU baseline: each output row computed by one thread in the same
+    order as the plain build, so the two builds agree bit for bit."""
+    X = rmm_synth.activations(37, 512, 141)
+    W = rmm_synth.weights(300, 512, 142)
+    Y1, i1 = oracle.linear(X, W, 0.5)
+    Y2, i2 = oracle.linear(X, W, 0.5, parallel=True)
+    assert np.array_equal(i1, i2) and np.array_equal(Y1, Y2)
+    assert oracle.parallel_threads() >= 1
