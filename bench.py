@@ -175,24 +175,27 @@ def host_inputs():
     return _host_inputs
 
 
-def oracle_sample(rows_per_proj: int, seed: int):
-    """Time the CPU oracle on `rows_per_proj` token rows of every projection (full score/select).
+def oracle_sample(rows_per_proj: int, seed: int, parallel: bool = False):
+    """Time the CPU oracle on `rows_per_proj` token rows of every projection (full score/select);
+    parallel=True: its OpenMP build (output rows over the host's threads, same bits).
 
     Returns (flops, seconds, sample description)."""
     import oracle
 
-    oracle.build()
+    oracle.build(parallel=parallel)
     acts, weights = host_inputs()
     g = torch.Generator().manual_seed(seed)
     flops, secs = 0, 0.0
     for name, H, N, s in PROJ:
         rows = torch.randperm(T_PREFILL, generator=g)[:rows_per_proj].tolist()
         t0 = time.perf_counter()
-        oracle.linear(acts[s], weights[name], R, rows=rows)
+        oracle.linear(acts[s], weights[name], R, rows=rows, parallel=parallel)
         secs += time.perf_counter() - t0
         flops += metrics.reduced_linear_flops(rows_per_proj, N, metrics.k_for(H, R))
+    kind = (f"fp64 C oracle, OpenMP build on {oracle.parallel_threads()} threads" if parallel
+            else "single-threaded fp64 C oracle")
     desc = (f"{rows_per_proj} of {T_PREFILL} token rows per projection, all 7 projections, "
-            "score and kept set over the full batch; single-threaded fp64 C oracle")
+            f"score and kept set over the full batch; {kind}")
     return flops, secs, desc
 
 
@@ -735,10 +738,17 @@ def run_rmm(args, world, rank, local):
         extra.update(time_ffn_demo(dev))
         extra.update(time_layer(dev, host_inputs()[1]))
 
-    cpu = None
+    cpu = cpu_par = None
     if rank == 0 and not args.skip_cpu_baseline:
         f, t, desc = oracle_sample(args.cpu_rows, seed=1)
         cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc}
+        # the same oracle's OpenMP build on all host threads (a reported baseline too)
+        import oracle
+
+        threads = oracle.parallel_threads()
+        f, t, desc = oracle_sample(args.cpu_rows * max(1, min(threads, 16)) // 2, seed=2, parallel=True)
+        cpu_par = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle-openmp",
+                   "sample": desc}
 
     if rank != 0:
         return
@@ -758,6 +768,7 @@ def run_rmm(args, world, rank, local):
                   "effective_tflops_at_reduced_flops": step_flops / (dense_ms * 1e-3) / 1e12},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "cpu_baseline": cpu,
+        "cpu_baseline_parallel": cpu_par,
         "gpu_launches": launches_per_step(dev) * K,
         "clocks": clk,
         "per_call": per_call,
