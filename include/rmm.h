@@ -109,8 +109,9 @@ typedef struct rmm_options {
 /* Human-readable name of a status code (static storage). */
 const char* rmm_status_string(rmm_status status);
 
-/* Number of kept slices for retention ratio r: ceil(r*H) in double, clamped
- * to [1, H].  Returns -1 if r is not in (0, 1] or H < 1. */
+/* Number of kept slices for retention ratio r (paper abstract: one retention
+ * ratio sets the share of each product that is kept): ceil(r*H) in double,
+ * clamped to [1, H].  Returns -1 if r is not in (0, 1] or H < 1. */
 int rmm_k_for(int H, double r);
 
 /* Zero-fill a workspace (device memory, `bytes` long) on `stream`.  Needed
@@ -167,19 +168,25 @@ rmm_status rmm_linear_group(const void* X, int T, int H, double r, int count, co
                             const int* Ns, void* const* Ys, int32_t* idx_out, void* workspace,
                             size_t workspace_bytes, rmm_stream_t stream, const rmm_options* options);
 
-/* Step 1 alone: s_out[h] = max_t |X[t,h]| as the bf16 magnitude key
- * (bit pattern with the sign cleared; -0 and +0 both give 0).  X bf16 [T, H],
+/* Step 1 alone, the score (cf-1.com post §5.1: a cheap importance score of
+ * every contraction index from the current activations; §8: one score for the
+ * whole batch): s_out[h] = max_t |X[t,h]| as the bf16 magnitude key (bit
+ * pattern with the sign cleared; -0 and +0 both give 0).  X bf16 [T, H],
  * s_out uint32 [H].  T >= 1. */
 rmm_status rmm_score(const void* X, int T, int H, uint32_t* s_out, void* workspace,
                      size_t workspace_bytes, rmm_stream_t stream);
 
-/* Step 2 alone: the k indices of the largest scores under (score desc, index
- * asc), written to idx_out [k] in ascending order.  s: uint32 [H], each
- * < 65536; 1 <= k <= H <= 65535. */
+/* Step 2 alone, the kept set (cf-1.com post §5.2: scores turned into a top-k
+ * set; §6.1: the top-k indices sorted so the kept slices keep their order):
+ * the k indices of the largest scores under (score desc, index asc), written
+ * to idx_out [k] in ascending order.  s: uint32 [H], each < 65536;
+ * 1 <= k <= H <= 65535. */
 rmm_status rmm_select(const uint32_t* s, int H, int k, int32_t* idx_out, void* workspace,
                       size_t workspace_bytes, rmm_stream_t stream);
 
-/* Step 3 alone, for a given kept set: Y[t,n] = sum_{j<k} X[t,idx[j]] * Wt[idx[j],n].
+/* Step 3 alone, the reduced product for a given kept set (cf-1.com post §5.3:
+ * the gathered slices in one smaller dense product; §2: the output keeps its
+ * shape): Y[t,n] = sum_{j<k} X[t,idx[j]] * Wt[idx[j],n].
  * idx: int32 [k], distinct values in [0, H) (any order).  Same layouts and
  * path choice as rmm_linear. */
 rmm_status rmm_gemm_reduced(const void* X, const void* Wt, const int32_t* idx, int k, int T,
@@ -258,9 +265,8 @@ rmm_status rmm_attn_ctx(const void* Q, const void* Kt, const void* V, const floa
 /* The decode-sized reduced linear map without a workspace.  The pages have
  * no counterpart to this entry point; it exists for callers that cannot give
  * the library device memory of its own: a plugin whose host framework owns
- * every allocation and only lends it input and output buffers, a serving loop
- * with a fixed memory budget, code being recorded into a CUDA graph (where a
- * cudaMalloc would break the capture).
+ * every allocation and only lends it input and output buffers, or a serving
+ * loop under a fixed memory budget that must not grow once it has started.
  * Computes exactly what rmm_linear computes on its split-K GEMV path
  * (score -> kept set -> reduced product), but all intermediates live in a
  * fixed 4 MiB array inside the library: every GPU that loads the library

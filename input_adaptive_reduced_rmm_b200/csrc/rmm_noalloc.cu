@@ -1,19 +1,19 @@
 // rmm_noalloc.cu -- the decode-sized reduced linear map with library-owned scratch.
 //
 // Some callers cannot hand the library a workspace: they run where allocating
-// device memory is not allowed or not safe -- a plugin whose host framework owns
-// every allocation and only lends it input and output buffers, an inference
-// loop with a fixed memory budget that must not grow at run time, or code that
-// is being recorded into a CUDA graph, where a cudaMalloc would break the
-// capture.  rmm_linear_decode_noalloc serves them: the same score -> kept set ->
-// split-K GEMV path as rmm_linear for T <= 16, but every intermediate (partial
-// score vector, the kept list, the split partial sums) lives in
-// one file-scope __device__ array of fixed size that every GPU loading the
-// library holds until the process exits.  Nothing is allocated or freed.
+// device memory is not theirs to do -- a plugin whose host framework owns every
+// allocation and only lends it input and output buffers, or an inference loop
+// under a fixed memory budget that must not grow once serving has started.
+// rmm_linear_decode_noalloc serves them: the same score -> kept set -> split-K
+// GEMV path as rmm_linear for T <= 16, but every intermediate (the score
+// vector, the kept list, the split partial sums) lives in one file-scope
+// __device__ array of fixed size that every GPU loading the library holds
+// until the process exits.  Nothing is allocated or freed.
 //
 // Host code never uses the array's name as a device address: on first use on
 // a device (with that device current) the address is obtained once with
 // cudaGetSymbolAddress, checked, cached per device, and passed to the kernels.
+// That first call on a device should come before any stream capture.
 #include <string.h>
 
 #include <mutex>
@@ -25,7 +25,6 @@ namespace rmm {
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB per device
-constexpr size_t kNoAllocStatusBytes = 256;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -50,8 +49,9 @@ rmm_status noalloc_scratch(uint8_t** out) {
     return RMM_OK;
 }
 
-// Zero the words a call needs to start at zero (status word, score vector);
-// the scratch keeps whatever the previous call left there.
+// Zero the words a call needs to start at zero (the score vector, which the
+// score pass folds into with atomicMax); the scratch keeps whatever the
+// previous call left there.
 __global__ void noalloc_clear_kernel(unsigned* words, int n) {
     pdl_wait();
     pdl_launch_dependents();
@@ -80,8 +80,8 @@ extern "C" rmm_status rmm_linear_decode_noalloc(const void* X, const void* Wt, i
     rmm_status st = noalloc_scratch(&scratch);
     if (st != RMM_OK) return st;
 
-    // scratch layout: status | score vector | kept list | split partials
-    const size_t off_s32 = kNoAllocStatusBytes;
+    // scratch layout: score vector | kept list | split partials
+    const size_t off_s32 = 0;
     const size_t off_idx = off_s32 + up256((size_t)H * sizeof(uint32_t));
     const size_t off_partials = off_idx + up256(((size_t)H + 2 * kGemmBK) * sizeof(int32_t));
     if (off_partials >= kNoAllocScratchBytes) return RMM_ERR_UNSUPPORTED;
@@ -115,7 +115,7 @@ extern "C" rmm_status rmm_linear_decode_noalloc(const void* X, const void* Wt, i
     }
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // status word and score vector: they must start at zero
+    // the score vector must start at zero
     noalloc_clear_kernel<<<(int)((off_idx / 4 + 255) / 256), 256, 0, s>>>(reinterpret_cast<unsigned*>(scratch),
                                                                          (int)(off_idx / 4));
     if (cudaGetLastError() != cudaSuccess) return RMM_ERR_CUDA;

@@ -145,12 +145,46 @@ def _bf16_cuda(t, name):
         raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
 
 
+def _need(t, name, dtype=torch.bfloat16, shape=None, min_numel=None):
+    """Structure of a tensor handed to a kernel: dtype, contiguity, exact shape or
+    least element count.  The device is checked separately (_on_cuda), after every
+    tensor's structure, so that a wrong-sized output is named as such."""
+    if t is None:
+        return
+    if t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, needs at least {min_numel}")
+
+
+def _on_cuda(**tensors):
+    for name, t in tensors.items():
+        if t is not None and not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _dims(t, name, n):
+    if t.dim() != n:
+        raise ValueError(f"{name} must have {n} dimensions, has {t.dim()}")
+
+
 def rmm_status_string(status: int) -> str:
     return lib().rmm_status_string(int(status)).decode()
 
 
 def rmm_k_for(H: int, r: float) -> int:
     return int(lib().rmm_k_for(int(H), float(r)))
+
+
+def _kept_count(H: int, r: float, opts=None) -> int:
+    """Entries the library writes to idx_out for a linear call: ceil(r*H) kept slices, or
+    with block-granular sets (blocks of b slices, b dividing H) ceil(r*H/b) whole blocks."""
+    b = int(opts.block_size) if opts is not None else 0
+    if b > 0:
+        return max(0, rmm_k_for(int(H) // b, r) * b)
+    return max(0, rmm_k_for(H, r))
 
 
 def new_workspace(nbytes: int, device=None) -> torch.Tensor:
@@ -185,19 +219,23 @@ def rmm_linear_workspace_bytes(T: int, H: int, N: int, opts: rmm_options | None 
 def rmm_linear(X: torch.Tensor, Wt: torch.Tensor, r: float, Y: torch.Tensor | None = None,
                idx_out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                opts: rmm_options | None = None, stream=None) -> torch.Tensor:
-    """Y ~= X[:,S] W[:,S]^T with S the ceil(r*H) kept slices.  X [T,H], Wt [H,N] bf16."""
-    _bf16_cuda(X, "X")
-    _bf16_cuda(Wt, "Wt")
+    """Y ~= X[:,S] W[:,S]^T with S the ceil(r*H) kept slices.  X [T,H], Wt [H,N] bf16;
+    idx_out (optional) int32 with room for the kept list (H entries always suffice)."""
+    _dims(X, "X", 2)
+    _dims(Wt, "Wt", 2)
     T, H = X.shape
     H2, N = Wt.shape
     if H2 != H:
         raise ValueError("X and Wt disagree on H")
+    _need(X, "X")
+    _need(Wt, "Wt")
+    _need(Y, "Y", shape=(T, N))
+    _need(idx_out, "idx_out", torch.int32, min_numel=_kept_count(H, r, opts))
+    _on_cuda(X=X, Wt=Wt, Y=Y, idx_out=idx_out)
     if Y is None:
         Y = torch.empty(T, N, dtype=torch.bfloat16, device=X.device)
     if workspace is None:
         workspace = new_workspace(rmm_linear_workspace_bytes(T, H, N, opts), X.device)
-    if idx_out is not None and (idx_out.dtype != torch.int32 or not idx_out.is_cuda):
-        raise ValueError("idx_out must be an int32 CUDA tensor")
     _check(lib().rmm_linear(_ptr(X), _ptr(Wt), T, H, N, float(r), _ptr(Y), _ptr(idx_out),
                             _ptr(workspace), workspace.numel(), _stream(stream), _opt(opts)),
            "rmm_linear")
@@ -212,14 +250,24 @@ def rmm_linear_group_workspace_bytes(T: int, H: int, Ns, opts: rmm_options | Non
 def rmm_linear_group(X: torch.Tensor, Wts, r: float, Ys=None, idx_out: torch.Tensor | None = None,
                      workspace: torch.Tensor | None = None, opts: rmm_options | None = None, stream=None):
     """Projections of one activation matrix sharing one kept set: [X[:,S] W_p[:,S]^T for each W_p^T in Wts]."""
-    _bf16_cuda(X, "X")
+    _dims(X, "X", 2)
+    _need(X, "X")
     T, H = X.shape
     Ns = []
     for i, Wt in enumerate(Wts):
-        _bf16_cuda(Wt, f"Wts[{i}]")
+        _dims(Wt, f"Wts[{i}]", 2)
+        _need(Wt, f"Wts[{i}]")
         if Wt.shape[0] != H:
             raise ValueError("X and a weight disagree on H")
         Ns.append(Wt.shape[1])
+    if Ys is not None:
+        if len(Ys) != len(Ns):
+            raise ValueError("Ys and Wts differ in length")
+        for i, Y in enumerate(Ys):
+            _need(Y, f"Ys[{i}]", shape=(T, Ns[i]))
+    _need(idx_out, "idx_out", torch.int32, min_numel=_kept_count(H, r, opts))
+    _on_cuda(X=X, idx_out=idx_out, **{f"Wts[{i}]": W for i, W in enumerate(Wts)},
+             **{f"Ys[{i}]": Y for i, Y in enumerate(Ys or [])})
     if Ys is None:
         Ys = [torch.empty(T, n, dtype=torch.bfloat16, device=X.device) for n in Ns]
     if workspace is None:
@@ -237,8 +285,11 @@ def rmm_linear_group(X: torch.Tensor, Wts, r: float, Ys=None, idx_out: torch.Ten
 def rmm_score(X: torch.Tensor, s_out: torch.Tensor | None = None,
               workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """s[h] = max_t |X[t,h]| as the bf16 magnitude key (int32 tensor holding uint32 values)."""
-    _bf16_cuda(X, "X")
+    _dims(X, "X", 2)
+    _need(X, "X")
     T, H = X.shape
+    _need(s_out, "s_out", torch.int32, min_numel=H)
+    _on_cuda(X=X, s_out=s_out)
     if s_out is None:
         s_out = torch.empty(H, dtype=torch.int32, device=X.device)
     if workspace is None:
@@ -250,9 +301,10 @@ def rmm_score(X: torch.Tensor, s_out: torch.Tensor | None = None,
 
 def rmm_select(s: torch.Tensor, k: int, idx_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """The k best indices of s under (score desc, index asc), ascending (int32)."""
-    if s.dtype != torch.int32 or not s.is_cuda:
-        raise ValueError("s must be an int32 CUDA tensor (uint32 scores)")
+    _need(s, "s", torch.int32)
     H = s.numel()
+    _need(idx_out, "idx_out", torch.int32, min_numel=int(k))
+    _on_cuda(s=s, idx_out=idx_out)
     if idx_out is None:
         idx_out = torch.empty(int(k), dtype=torch.int32, device=s.device)
     _check(lib().rmm_select(_ptr(s), H, int(k), _ptr(idx_out), None, 0, _stream(stream)), "rmm_select")
@@ -263,12 +315,17 @@ def rmm_gemm_reduced(X: torch.Tensor, Wt: torch.Tensor, idx: torch.Tensor, Y: to
                      workspace: torch.Tensor | None = None, opts: rmm_options | None = None,
                      stream=None) -> torch.Tensor:
     """Y[t,n] = sum_j X[t, idx_j] * Wt[idx_j, n] for a given kept list."""
-    _bf16_cuda(X, "X")
-    _bf16_cuda(Wt, "Wt")
-    if idx.dtype != torch.int32 or not idx.is_cuda:
-        raise ValueError("idx must be an int32 CUDA tensor")
+    _dims(X, "X", 2)
+    _dims(Wt, "Wt", 2)
     T, H = X.shape
-    N = Wt.shape[1]
+    H2, N = Wt.shape
+    if H2 != H:
+        raise ValueError("X and Wt disagree on H")
+    _need(X, "X")
+    _need(Wt, "Wt")
+    _need(idx, "idx", torch.int32)
+    _need(Y, "Y", shape=(T, N))
+    _on_cuda(X=X, Wt=Wt, idx=idx, Y=Y)
     if Y is None:
         Y = torch.empty(T, N, dtype=torch.bfloat16, device=X.device)
     if workspace is None:
@@ -288,13 +345,20 @@ def rmm_attn_qk(Q: torch.Tensor, Kt: torch.Tensor, V: torch.Tensor, L: int, r: f
                 causal: bool = True, scale: float | None = None, O: torch.Tensor | None = None,
                 idx_out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                 opts: rmm_options | None = None, stream=None) -> torch.Tensor:
-    """Reduced attention.  Q [B,Hq,T,d]; Kt [B,Hkv,d,ldL] (d-major keys); V [B,Hkv,ldL,d]."""
-    for t, n in ((Q, "Q"), (Kt, "Kt"), (V, "V")):
-        _bf16_cuda(t, n)
+    """Reduced attention.  Q [B,Hq,T,d]; Kt [B,Hkv,d,ldL] (d-major keys); V [B,Hkv,ldL,d];
+    idx_out (optional) int32 with room for [B, sets, ceil(r*d)] (sets = Hkv, or Hq per query head)."""
+    _dims(Q, "Q", 4)
+    _dims(Kt, "Kt", 4)
     B, Hq, T, d = Q.shape
     _, Hkv, d2, ldL = Kt.shape
-    if d2 != d or V.shape != (B, Hkv, ldL, d):
+    if d2 != d or Kt.shape[0] != B or tuple(V.shape) != (B, Hkv, ldL, d):
         raise ValueError("Q, Kt, V shapes disagree")
+    for t, n in ((Q, "Q"), (Kt, "Kt"), (V, "V")):
+        _need(t, n)
+    _need(O, "O", shape=tuple(Q.shape))
+    nsets = Hq if (opts is not None and opts.attn_per_query_head) else Hkv
+    _need(idx_out, "idx_out", torch.int32, min_numel=B * nsets * max(0, rmm_k_for(d, r)))
+    _on_cuda(Q=Q, Kt=Kt, V=V, O=O, idx_out=idx_out)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if O is None:
@@ -325,8 +389,8 @@ def rmm_ctx_block_means(Kt: torch.Tensor, L: int, block: int, means: torch.Tenso
     B, Hkv, d, ldL = Kt.shape
     if means is None:
         means = new_ctx_means(Kt, block)
-    if means.dtype != torch.float32 or not means.is_cuda or not means.is_contiguous():
-        raise ValueError("means must be a contiguous fp32 CUDA tensor")
+    _need(means, "means", torch.float32, shape=(B, Hkv, ctx_num_blocks(ldL, block), d))
+    _on_cuda(means=means)
     if blk_end is None:
         blk_end = ctx_num_blocks(L, block)
     _check(lib().rmm_ctx_block_means(_ptr(Kt), B, Hkv, d, int(L), ldL, int(block), int(blk_begin), int(blk_end),
@@ -345,14 +409,21 @@ def rmm_attn_ctx(Q: torch.Tensor, Kt: torch.Tensor, V: torch.Tensor, means: torc
                  blocks_out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                  opts: rmm_options | None = None, stream=None) -> torch.Tensor:
     """Reduced attention over the kept head dimensions and the kept context blocks."""
-    for t, n in ((Q, "Q"), (Kt, "Kt"), (V, "V")):
-        _bf16_cuda(t, n)
+    _dims(Q, "Q", 4)
+    _dims(Kt, "Kt", 4)
     B, Hq, T, d = Q.shape
     _, Hkv, d2, ldL = Kt.shape
-    if d2 != d or V.shape != (B, Hkv, ldL, d):
+    if d2 != d or Kt.shape[0] != B or tuple(V.shape) != (B, Hkv, ldL, d):
         raise ValueError("Q, Kt, V shapes disagree")
-    if means.dtype != torch.float32 or not means.is_cuda or not means.is_contiguous():
-        raise ValueError("means must be a contiguous fp32 CUDA tensor")
+    for t, n in ((Q, "Q"), (Kt, "Kt"), (V, "V")):
+        _need(t, n)
+    _need(means, "means", torch.float32, shape=(B, Hkv, ctx_num_blocks(ldL, block), d))
+    _need(O, "O", shape=tuple(Q.shape))
+    nsets = Hq if (opts is not None and opts.attn_per_query_head) else Hkv
+    _need(idx_out, "idx_out", torch.int32, min_numel=B * nsets * max(0, rmm_k_for(d, r)))
+    _need(blocks_out, "blocks_out", torch.int32,
+          min_numel=B * nsets * max(0, rmm_k_for(ctx_num_blocks(L, block), r_ctx)))
+    _on_cuda(Q=Q, Kt=Kt, V=V, means=means, O=O, idx_out=idx_out, blocks_out=blocks_out)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if O is None:
@@ -368,13 +439,22 @@ def rmm_attn_ctx(Q: torch.Tensor, Kt: torch.Tensor, V: torch.Tensor, means: torc
 
 def rmm_linear_decode_noalloc(X: torch.Tensor, Wt: torch.Tensor, r: float, Y: torch.Tensor,
                               idx_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """The decode-sized reduced linear map (T <= 16) with no workspace: for callers that
-    cannot allocate device memory.  Y must be given (the binding allocates nothing)."""
-    _bf16_cuda(X, "X")
-    _bf16_cuda(Wt, "Wt")
-    _bf16_cuda(Y, "Y")
+    """The decode-sized reduced linear map (T <= 16) with no workspace, for callers that may
+    not allocate device memory.  Y [T, N] must be given (the binding allocates nothing);
+    idx_out (optional) int32 with room for ceil(r*H) entries."""
+    _dims(X, "X", 2)
+    _dims(Wt, "Wt", 2)
     T, H = X.shape
-    N = Wt.shape[1]
+    H2, N = Wt.shape
+    if H2 != H:
+        raise ValueError("X and Wt disagree on H")
+    _need(X, "X")
+    _need(Wt, "Wt")
+    if Y is None:
+        raise ValueError("Y must be given")
+    _need(Y, "Y", shape=(T, N))
+    _need(idx_out, "idx_out", torch.int32, min_numel=max(0, rmm_k_for(H, r)))
+    _on_cuda(X=X, Wt=Wt, Y=Y, idx_out=idx_out)
     _check(lib().rmm_linear_decode_noalloc(_ptr(X), _ptr(Wt), T, H, N, float(r), _ptr(Y), _ptr(idx_out),
                                            _stream(stream)), "rmm_linear_decode_noalloc")
     return Y

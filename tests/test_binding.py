@@ -53,3 +53,46 @@ def test_options_struct_matches_the_header(rmm):
     o = rmm.options(block_size=64, block_score=1, attn_path=2)
     assert (o.block_size, o.block_score, o.attn_path, o.t_gemv) == (64, 1, 2, 16)
     assert ctypes.sizeof(rmm.rmm_options) == 8 * 4 + 2 * ctypes.sizeof(ctypes.c_void_p)
+
+
+def test_wrong_sizes_are_refused_before_the_call(rmm):
+    """A wrong-sized output or kept-list buffer would let a kernel write past its end:
+    the binding names the mismatch instead of calling the library."""
+    X = torch.zeros(4, 64, dtype=torch.bfloat16)
+    Wt = torch.zeros(64, 32, dtype=torch.bfloat16)
+    bad = [
+        dict(Y=torch.zeros(4, 16, dtype=torch.bfloat16)),                  # Y not [T, N]
+        dict(Y=torch.zeros(4, 32, dtype=torch.bfloat16), idx_out=torch.zeros(3, dtype=torch.int32)),  # k = 32
+        dict(Y=torch.zeros(4, 32, dtype=torch.bfloat16), idx_out=torch.zeros(64, dtype=torch.int64)),
+    ]
+    for kw in bad:
+        for fn in (rmm.rmm_linear, rmm.rmm_linear_decode_noalloc):
+            with pytest.raises(ValueError):
+                fn(X, Wt, 0.5, **kw)
+    with pytest.raises(ValueError, match="disagree on H"):
+        rmm.rmm_linear_decode_noalloc(X, torch.zeros(32, 32, dtype=torch.bfloat16), 0.5,
+                                      torch.zeros(4, 32, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="Y must be given"):
+        rmm.rmm_linear_decode_noalloc(X, Wt, 0.5, None)
+    with pytest.raises(ValueError, match="expected"):
+        rmm.rmm_linear_group(X, [Wt, Wt], 0.5, Ys=[torch.zeros(4, 32, dtype=torch.bfloat16),
+                                                 torch.zeros(4, 31, dtype=torch.bfloat16)])
+    with pytest.raises(ValueError, match="at least 64"):
+        rmm.rmm_score(X, s_out=torch.zeros(63, dtype=torch.int32))
+    with pytest.raises(ValueError, match="at least 10"):
+        rmm.rmm_select(torch.zeros(64, dtype=torch.int32), 10, idx_out=torch.zeros(9, dtype=torch.int32))
+    with pytest.raises(ValueError, match="expected"):
+        rmm.rmm_gemm_reduced(X, Wt, torch.zeros(8, dtype=torch.int32), Y=torch.zeros(4, 33, dtype=torch.bfloat16))
+    Q = torch.zeros(1, 4, 2, 128, dtype=torch.bfloat16)
+    Kt = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    V = torch.zeros(1, 2, 64, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="expected"):
+        rmm.rmm_attn_qk(Q, Kt, V, 64, 0.5, O=torch.zeros(1, 4, 1, 128, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="at least 128"):  # 1 batch x 2 sets x 64 kept dims
+        rmm.rmm_attn_qk(Q, Kt, V, 64, 0.5, idx_out=torch.zeros(127, dtype=torch.int32))
+    with pytest.raises(ValueError, match="expected"):
+        rmm.rmm_attn_ctx(Q, Kt, V, torch.zeros(1, 2, 2, 128), 64, 0.5, 0.5, 16)  # needs 4 blocks of 16
+    # the right sizes pass every structural check and stop at the device check
+    with pytest.raises(ValueError, match="CUDA"):
+        rmm.rmm_linear_decode_noalloc(X, Wt, 0.5, torch.zeros(4, 32, dtype=torch.bfloat16),
+                                      idx_out=torch.zeros(32, dtype=torch.int32))
