@@ -1,22 +1,25 @@
 """Benchmark of the reduced-matrix-multiplication hot path on B200.
 
 One step = one pass of the reduced linear map over the seven projections of a
-Llama-3-8B-shaped layer (q, k, v, o: 4096 -> 4096/1024/1024/4096; gate, up:
-4096 -> 14336; down: 14336 -> 4096) on a prefill batch of T = 2048 tokens at
+Llama-3-70B-shaped layer (q, k, v, o: 8192 -> 8192/1024/1024/8192; gate, up:
+8192 -> 28672; down: 28672 -> 8192) on a prefill batch of T = 4096 tokens at
 retention r = 0.5, with random-init bf16 weights ~N(0, 0.02) pre-transposed
 once and synthetic activations N(0, 1) with 2 % of the channels x20.  As in
 the layer, q/k/v read one activation matrix and gate/up another, so each of
 those sets is one rmm_linear_group call (one score, one kept set, one grouped
 tcgen05 GEMM launch); o and down are rmm_linear calls: four C-ABI calls, three
-kernels each, per step.
+or four kernels each, per step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rmm|reference]
 
 Prints one JSON line (rank 0).  value = effective TFLOP/s = sum 2*T*N*k over
 all ranks' steps / max-over-ranks device time.  Extra keys: the dominant
-kernel's roofline, the dense cuBLAS comparison, the end-to-end number through
-the public call with host buffers, the oracle timed on the host cores, the
-decode (T = 1) GEMV and attention rows, and SM clocks sampled during timing.
+kernel's roofline, the dense cuBLAS comparison (seven products, and the same
+with q|k|v and gate|up concatenated into one product each), the end-to-end
+number through the public call with host buffers, the oracle timed on the host
+cores, the r sweep, the same step on Llama-3-8B shapes (T = 2048), and the
+decode (T = 1) GEMV, attention, FFN-demo and decoder-layer rows, with SM clocks
+sampled during timing.
 """
 from __future__ import annotations
 
@@ -38,21 +41,48 @@ if ROOT not in sys.path:
 import rmm_synth  # noqa: E402
 from input_adaptive_reduced_rmm_b200 import metrics  # noqa: E402
 
-T_PREFILL = 2048
 R = 0.5
-# DRAM bytes (read + write) of one step's four GEMM launches from one ncu capture of
-# this kernel (profiles/gemm_pair_step_traffic_llama3_8b_T2048_r0.5.md); set to None
-# whenever the GEMM kernel changes until it is captured again.
-STEP_GEMM_DRAM_BYTES = 361_726_464
-PROJ = [  # (name, H, N, activation stream)
-    ("q", 4096, 4096, 0), ("k", 4096, 1024, 0), ("v", 4096, 1024, 0), ("o", 4096, 4096, 1),
-    ("gate", 4096, 14336, 2), ("up", 4096, 14336, 2), ("down", 14336, 4096, 3),
-]
-ACT_H = {0: 4096, 1: 4096, 2: 4096, 3: 14336}
+R_SWEEP = [0.125 * i for i in range(1, 9)]
 CALLS = [(0, ["q", "k", "v"]), (1, ["o"]), (2, ["gate", "up"]), (3, ["down"])]  # (activation, members)
-PROJ_BY_NAME = {n: (H, N) for n, H, N, _ in PROJ}
-WORKLOAD = "llama3-8b 7 projections (q,k,v,o,gate,up,down), prefill T=2048, r=0.5"
 METRIC = "reduced-GEMM effective TFLOP/s (2*T*N*k / time)"
+
+
+class Workload:
+    """The seven projections of one decoder layer at a prefill batch of T tokens:
+    (name, contraction size, output size, activation stream) per projection."""
+
+    def __init__(self, label, cfg, T, H, Nq, Nkv, F):
+        self.label, self.cfg, self.T = label, cfg, T
+        self.proj = [("q", H, Nq, 0), ("k", H, Nkv, 0), ("v", H, Nkv, 0), ("o", Nq, H, 1),
+                     ("gate", H, F, 2), ("up", H, F, 2), ("down", F, H, 3)]
+        self.act_h = {0: H, 1: Nq, 2: H, 3: F}
+        self.shape = {n: (h, N) for n, h, N, _ in self.proj}
+
+    def name(self, r):
+        return f"{self.label} 7 projections (q,k,v,o,gate,up,down), prefill T={self.T}, r={r}"
+
+    def k(self, n, r):
+        return metrics.k_for(self.shape[n][0], r)
+
+    def flops(self, r):
+        return sum(metrics.reduced_linear_flops(self.T, N, metrics.k_for(h, r)) for _, h, N, _ in self.proj)
+
+    def dense_flops(self):
+        return sum(metrics.gemm_flops(self.T, N, h) for _, h, N, _ in self.proj)
+
+    def resident_gb(self):
+        w = sum(h * N * 2 for _, h, N, _ in self.proj)
+        a = sum(self.T * h * 2 for h in self.act_h.values()) + sum(self.T * N * 2 for _, _, N, _ in self.proj)
+        return (w + a) / 1e9
+
+
+LLAMA70 = Workload("llama3-70b", 4, 4096, 8192, 8192, 1024, 28672)
+LLAMA8 = Workload("llama3-8b", 1, 2048, 4096, 4096, 1024, 14336)
+HEADLINE = LLAMA70
+# DRAM bytes (read + write) of one step's four GEMM launches at r = 0.5, from one
+# ncu capture of the current GEMM kernel per workload; an entry is removed whenever
+# the GEMM kernel changes, until it is captured again.
+STEP_GEMM_DRAM_BYTES = {"llama3-8b": 361_726_464}
 
 
 def load_peaks():
@@ -161,62 +191,67 @@ def barrier(world):
 
 # ------------------------------------------------------------------ oracle (CPU baseline)
 
-_host_inputs = None
+_host = {}
 
 
-def host_inputs():
-    """The step's activations and weights on the host (bf16), generated once."""
-    global _host_inputs
-    if _host_inputs is None:
-        acts = {s: rmm_synth.activations(T_PREFILL, h, rmm_synth.seed_for(1, 70 + s, 0)) for s, h in ACT_H.items()}
-        weights = {n: rmm_synth.weights(N, H, rmm_synth.seed_for(1, 80 + i, 1), std=0.02)
-                   for i, (n, H, N, _) in enumerate(PROJ)}
-        _host_inputs = (acts, weights)
-    return _host_inputs
+def host_inputs(wl):
+    """The workload's activations and weights drawn on the host (bf16), once: what the
+    reference arm (no GPU) times the oracle on."""
+    if wl.label not in _host:
+        acts = {s: rmm_synth.activations(wl.T, h, rmm_synth.seed_for(wl.cfg, 70 + s, 0))
+                for s, h in wl.act_h.items()}
+        weights = {n: rmm_synth.weights(N, h, rmm_synth.seed_for(wl.cfg, 80 + i, 1), std=0.02)
+                   for i, (n, h, N, _) in enumerate(wl.proj)}
+        _host[wl.label] = (acts, weights)
+    return _host[wl.label]
 
 
-def oracle_sample(rows_per_proj: int, seed: int, parallel: bool = False):
-    """Time the CPU oracle on `rows_per_proj` token rows of every projection (full score/select);
-    parallel=True: its OpenMP build (output rows over the host's threads, same bits).
+def oracle_sample(wl, inputs, rows_per_proj: int, seed: int, parallel: bool = False):
+    """Time the CPU oracle on `rows_per_proj` token rows of every projection (its score and
+    kept set over the full batch); parallel=True: its OpenMP build (output rows over the
+    host's threads, same bits).  inputs = (activations, weights W [N, H]) on the host.
 
     Returns (flops, seconds, sample description)."""
     import oracle
 
     oracle.build(parallel=parallel)
-    acts, weights = host_inputs()
+    acts, weights = inputs
     g = torch.Generator().manual_seed(seed)
     flops, secs = 0, 0.0
-    for name, H, N, s in PROJ:
-        rows = torch.randperm(T_PREFILL, generator=g)[:rows_per_proj].tolist()
+    for name, h, N, s in wl.proj:
+        rows = torch.randperm(wl.T, generator=g)[:rows_per_proj].tolist()
         t0 = time.perf_counter()
         oracle.linear(acts[s], weights[name], R, rows=rows, parallel=parallel)
         secs += time.perf_counter() - t0
-        flops += metrics.reduced_linear_flops(rows_per_proj, N, metrics.k_for(H, R))
+        flops += metrics.reduced_linear_flops(rows_per_proj, N, metrics.k_for(h, R))
     kind = (f"fp64 C oracle, OpenMP build on {oracle.parallel_threads()} threads" if parallel
             else "single-threaded fp64 C oracle")
-    desc = (f"{rows_per_proj} of {T_PREFILL} token rows per projection, all 7 projections, "
+    desc = (f"{rows_per_proj} of {wl.T} token rows per projection, all 7 projections of {wl.label}, "
             f"score and kept set over the full batch; {kind}")
     return flops, secs, desc
 
 
-def step_config(world: int) -> dict:
+def step_config(wl, world: int) -> dict:
     """The workload description both arms print."""
-    return {"workload": WORKLOAD, "T": T_PREFILL, "r": R, "parallelism": f"replicas x{world}",
+    return {"workload": wl.name(R), "T": wl.T, "r": R, "parallelism": f"replicas x{world}",
             "calls_per_step": "q+k+v grouped, o, gate+up grouped, down",
-            "l2": "inputs larger than L2 (0.55 GB of weights and activations per step)"}
+            "l2": f"inputs larger than L2 ({wl.resident_gb():.2f} GB of weights and activations per step)"}
 
 
 def run_reference(args, world, rank):
-    """The oracle timed on the host cores: each step is a bounded sample of the workload."""
+    """The oracle timed on the host cores: each step is a bounded sample of the workload
+    (inputs drawn on the host with the same recipe)."""
     if rank != 0:
         return
-    rows = 2
+    wl = HEADLINE
+    inputs = host_inputs(wl)
+    rows = 1
     for _ in range(args.warmup):
-        oracle_sample(1, seed=999)
+        oracle_sample(wl, inputs, 1, seed=999)
     times, total_flops = [], 0
     sample = ""
     for s in range(args.steps):
-        f, t, sample = oracle_sample(rows, seed=s)
+        f, t, sample = oracle_sample(wl, inputs, rows, seed=s)
         times.append(t)
         total_flops += f
     value = total_flops / sum(times) / 1e12
@@ -224,7 +259,7 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": step_config(args.gpus),
+        "data": "synthetic", "config": step_config(wl, args.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -233,29 +268,175 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ GPU arm
 
-def make_inputs(dev):
+def device_inputs(wl, dev):
+    """Activations and pre-transposed weights W^T [H, N] drawn on the device (same recipe as
+    the host draws, the device's generator)."""
     from input_adaptive_reduced_rmm_b200 import rmm
 
-    hacts, hweights = host_inputs()
-    acts = {s: a.to(dev) for s, a in hacts.items()}
+    acts = {s: rmm_synth.activations(wl.T, h, rmm_synth.seed_for(wl.cfg, 70 + s, 0), device=dev)
+            for s, h in wl.act_h.items()}
     Wts = {}
-    for name, H, N, _ in PROJ:
-        Wts[name] = rmm.rmm_transpose_weight(hweights[name].to(dev))
+    for i, (n, h, N, _) in enumerate(wl.proj):
+        W = rmm_synth.weights(N, h, rmm_synth.seed_for(wl.cfg, 80 + i, 1), std=0.02, device=dev)
+        Wts[n] = rmm.rmm_transpose_weight(W)
+        del W
     torch.cuda.synchronize()
     return acts, Wts
 
 
-def time_decode(dev, peaks):
-    """Secondary row: one decode step (T = 1) over the same seven projections, grouped like
-    the prefill step, at r = 0.5; L2 flushed before every timed step."""
+class PrefillStep:
+    """The four calls of one step (q+k+v grouped, o, gate+up grouped, down) with their
+    buffers and workspaces, allocated once."""
+
+    def __init__(self, wl, acts, Wts, dev, opts=None):
+        from input_adaptive_reduced_rmm_b200 import rmm
+
+        self.rmm, self.wl, self.acts, self.Wts, self.opts = rmm, wl, acts, Wts, opts
+        self.Ys = {n: torch.empty(wl.T, N, dtype=torch.bfloat16, device=dev) for n, _, N, _ in wl.proj}
+        self.ws = {c: rmm.new_workspace(rmm.rmm_linear_group_workspace_bytes(
+            wl.T, wl.act_h[s], [wl.shape[n][1] for n in names], opts), dev) for c, (s, names) in enumerate(CALLS)}
+
+    def __call__(self, r=R, events=None):
+        """One step; events = {call: (begin, end)} records the product kernel of each call."""
+        rmm = self.rmm
+        for c, (s, names) in enumerate(CALLS):
+            o = self.opts
+            if events is not None:
+                base = self.opts
+                o = rmm.options(product_events=events[c],
+                                block_size=base.block_size if base is not None else 0)
+            rmm.rmm_linear_group(self.acts[s], [self.Wts[n] for n in names], r, Ys=[self.Ys[n] for n in names],
+                                 workspace=self.ws[c], opts=o)
+
+    def check_status(self, what):
+        for c in self.ws:
+            if self.rmm.rmm_get_status(self.ws[c]) != self.rmm.RMM_OK:
+                raise RuntimeError(f"device status not OK ({what})")
+
+
+def time_steps(fn, steps, warmup):
+    """Device time (ms) of `steps` back-to-back calls after `warmup` untimed ones."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        fn()
+    t1.record()
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / steps
+
+
+def product_times(step, r, steps):
+    """Per-call product-kernel time (ms, mean over `steps` steps), from the events the library
+    records around each product launch; the step runs `steps` times for it."""
+    evs = [{c: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for c in range(len(CALLS))} for _ in range(steps)]
+    for i in range(steps):
+        step(r, events=evs[i])
+    torch.cuda.synchronize()
+    return {c: sum(evs[i][c][0].elapsed_time(evs[i][c][1]) for i in range(steps)) / steps
+            for c in range(len(CALLS))}
+
+
+class DenseSteps:
+    """cuBLAS (torch.matmul) on the same shapes, inputs and stream: the seven products one by
+    one, and the like-for-like form with q|k|v and gate|up concatenated into one product each
+    (as the reduced step groups them)."""
+
+    def __init__(self, wl, acts, Wts, dev):
+        self.wl, self.acts, self.Wts = wl, acts, Wts
+        self.Ys = {n: torch.empty(wl.T, N, dtype=torch.bfloat16, device=dev) for n, _, N, _ in wl.proj}
+        self.Wcat = {0: torch.cat([Wts["q"], Wts["k"], Wts["v"]], dim=1),
+                     2: torch.cat([Wts["gate"], Wts["up"]], dim=1)}
+        self.Ycat = {s: torch.empty(wl.T, W.shape[1], dtype=torch.bfloat16, device=dev) for s, W in self.Wcat.items()}
+
+    def seven(self):
+        for n, _, _, s in self.wl.proj:
+            torch.matmul(self.acts[s], self.Wts[n], out=self.Ys[n])
+
+    def grouped(self):
+        torch.matmul(self.acts[0], self.Wcat[0], out=self.Ycat[0])
+        torch.matmul(self.acts[1], self.Wts["o"], out=self.Ys["o"])
+        torch.matmul(self.acts[2], self.Wcat[2], out=self.Ycat[2])
+        torch.matmul(self.acts[3], self.Wts["down"], out=self.Ys["down"])
+
+    def times(self, steps, warmup):
+        t7 = time_steps(self.seven, steps, warmup)
+        tg = time_steps(self.grouped, steps, warmup)
+        return {"seven_products_ms": t7, "grouped_ms": tg, "best_ms": min(t7, tg),
+                "tflops_best": self.wl.dense_flops() / (min(t7, tg) * 1e-3) / 1e12}
+
+    def release(self):
+        del self.Wcat, self.Ycat, self.Ys
+
+
+def launches_per_step(wl, r, dev) -> int:
+    """Our kernels launched by one step: per call the score pass, the select, the CTA-pair
+    GEMM, and the fold of the split last wave when the call's tiles leave a partial wave
+    that the GEMM splits (more than one K-range per tile)."""
+    pairs = torch.cuda.get_device_properties(dev).multi_processor_count // 2
+    n = 0
+    for s, names in CALLS:
+        nkb = -(-metrics.k_for(wl.act_h[s], r) // 64)
+        tiles = sum(-(-wl.T // 256) * -(-wl.shape[m][1] // 512) for m in names)
+        rem = tiles % pairs
+        split = min(pairs // rem, 8, nkb) if rem else 1
+        n += 3 + (1 if split > 1 else 0)
+    return n
+
+
+def prefill_row(wl, dev, peaks, steps, warmup):
+    """Secondary row: the same step on another workload (value, GEMM fraction, speedup
+    over the faster dense form)."""
+    acts, Wts = device_inputs(wl, dev)
+    step = PrefillStep(wl, acts, Wts, dev)
+    ms = time_steps(step, steps, warmup)
+    gms = product_times(step, R, steps)
+    step.check_status(wl.label)
+    dense = DenseSteps(wl, acts, Wts, dev)
+    dt = dense.times(steps, warmup)
+    dense.release()
+    flops = wl.flops(R)
+    gemm_ms = sum(gms.values())
+    out = {"workload": wl.name(R), "ms_per_step": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+           "gemm_us": 1e3 * gemm_ms, "gemm_tflops": flops / (gemm_ms * 1e-3) / 1e12,
+           "gemm_frac_of_peak": flops / (gemm_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+           "gemm_dram_bytes": STEP_GEMM_DRAM_BYTES.get(wl.label),
+           "dense": dt, "speedup_vs_dense": dt["best_ms"] / ms}
+    del step, acts, Wts
+    torch.cuda.empty_cache()
+    return out
+
+
+def r_sweep(wl, step, dense_ms, peaks, steps, warmup):
+    """The headline step at every retention ratio of the sweep: effective TFLOP/s of the
+    step and of its GEMM launches, speedup over the faster dense form, and 1/r."""
+    rows = []
+    for r in R_SWEEP:
+        ms = time_steps(lambda: step(r), steps, warmup)
+        gms = sum(product_times(step, r, steps).values())
+        f = wl.flops(r)
+        rows.append({"r": r, "ms_per_step": ms, "tflops": f / (ms * 1e-3) / 1e12,
+                     "gemm_tflops": f / (gms * 1e-3) / 1e12,
+                     "gemm_frac_of_peak": f / (gms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                     "speedup_vs_dense": dense_ms / ms, "ideal_speedup": 1.0 / r})
+    step.check_status("r sweep")
+    return rows
+
+
+def time_decode(wl, dev, peaks):
+    """Secondary row: one decode step (T = 1) over the workload's seven projections, grouped
+    like the prefill step, at r = 0.5; L2 flushed before every timed step."""
     from input_adaptive_reduced_rmm_b200 import rmm
 
-    acts = {s: rmm_synth.activations(1, h, 500 + s).to(dev) for s, h in ACT_H.items()}
-    Wts = {n: rmm.rmm_transpose_weight(rmm_synth.weights(N, H, 600 + i, std=0.02).to(dev))
-           for i, (n, H, N, _) in enumerate(PROJ)}
-    Ys = {n: torch.empty(1, N, dtype=torch.bfloat16, device=dev) for n, H, N, _ in PROJ}
+    acts = {s: rmm_synth.activations(1, h, 500 + s, device=dev) for s, h in wl.act_h.items()}
+    Wts = {n: rmm.rmm_transpose_weight(rmm_synth.weights(N, h, 600 + i, std=0.02, device=dev))
+           for i, (n, h, N, _) in enumerate(wl.proj)}
+    Ys = {n: torch.empty(1, N, dtype=torch.bfloat16, device=dev) for n, h, N, _ in wl.proj}
     ws = {c: rmm.new_workspace(rmm.rmm_linear_group_workspace_bytes(
-        1, ACT_H[s], [PROJ_BY_NAME[n][1] for n in names]), dev) for c, (s, names) in enumerate(CALLS)}
+        1, wl.act_h[s], [wl.shape[n][1] for n in names]), dev) for c, (s, names) in enumerate(CALLS)}
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
     def step():
@@ -264,7 +445,7 @@ def time_decode(dev, peaks):
                                  workspace=ws[c])
 
     def dense_step():
-        for n, H, N, s in PROJ:
+        for n, h, N, s in wl.proj:
             torch.matmul(acts[s], Wts[n], out=Ys[n])
 
     def timed(fn, iters=20):
@@ -326,65 +507,43 @@ def time_decode(dev, peaks):
             kern_ms += sum(ev_g[c][0].elapsed_time(ev_g[c][1]) for c in ev_g)
     kern_ms /= iters
     del graph
-    kept_bytes = sum(metrics.gemv_bytes(1, H, N, metrics.k_for(H, R)) for _, H, N, _ in PROJ)
-    dense_bytes = sum(N * H * 2 + H * 2 + N * 2 for _, H, N, _ in PROJ)
-    out = {"decode_gemv": {
-        "workload": "T=1, same 7 projections (q+k+v, o, gate+up, down), r=0.5, CUDA-graph replay, "
-                    "L2 flushed before each step",
+    for c in ws:
+        if rmm.rmm_get_status(ws[c]) != rmm.RMM_OK:
+            raise RuntimeError("device status not OK (decode step)")
+    kept_bytes = sum(metrics.gemv_bytes(1, h, N, metrics.k_for(h, R)) for _, h, N, _ in wl.proj)
+    dense_bytes = sum(N * h * 2 + h * 2 + N * 2 for _, h, N, _ in wl.proj)
+    out = {
+        "workload": f"T=1, the 7 projections of {wl.label} (q+k+v, o, gate+up, down), r=0.5, CUDA-graph "
+                    "replay, L2 flushed before each step",
         "step_us": 1e3 * call_ms,
         "kernel_us": 1e3 * kern_ms,
         "kernel_gbs": kept_bytes / (kern_ms * 1e-3) / 1e9,
         "kernel_frac_of_hbm": kept_bytes / (kern_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "step_gbs": kept_bytes / (call_ms * 1e-3) / 1e9,
+        "step_frac_of_hbm": kept_bytes / (call_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "dense_us": 1e3 * dense_ms,
         "dense_gbs": dense_bytes / (dense_ms * 1e-3) / 1e9,
         "speedup_vs_dense": dense_ms / call_ms,
-    }}
+    }
     del Wts, ws, flush
     torch.cuda.empty_cache()
     return out
 
 
-def time_blocks(dev, acts, Wts, Ys, dense_ms, steps, warmup, block=64):
+def time_blocks(wl, dev, acts, Wts, dense_ms, steps, warmup, block=64):
     """Secondary row: the same prefill step with block-granular kept sets (blocks of
     `block` consecutive slices scored by their largest slice score; with 64-slice runs
     the GEMM stages its operands by TMA tile copies)."""
     from input_adaptive_reduced_rmm_b200 import rmm
 
-    ks = {n: metrics.k_for(H // block, R) * block for n, H, _, _ in PROJ}
-    flops = sum(metrics.reduced_linear_flops(T_PREFILL, N, ks[n]) for n, _, N, _ in PROJ)
-    evs = {c: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(steps)] for c in range(len(CALLS))}
-    opts = {c: [rmm.options(block_size=block, product_events=evs[c][i]) for i in range(steps)]
-            for c in range(len(CALLS))}
-    plain = rmm.options(block_size=block)
-    ws = {c: rmm.new_workspace(rmm.rmm_linear_group_workspace_bytes(
-        T_PREFILL, ACT_H[s], [PROJ_BY_NAME[n][1] for n in names], plain), dev) for c, (s, names) in enumerate(CALLS)}
-
-    def step(i=None):
-        for c, (s, names) in enumerate(CALLS):
-            rmm.rmm_linear_group(acts[s], [Wts[n] for n in names], R, Ys=[Ys[n] for n in names],
-                                 workspace=ws[c], opts=plain if i is None else opts[c][i])
-
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(steps):
-        step()
-    t1.record()
-    torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / steps
-    for i in range(steps):
-        step(i)
-    torch.cuda.synchronize()
-    for c in ws:
-        if rmm.rmm_get_status(ws[c]) != rmm.RMM_OK:
-            raise RuntimeError("device status not OK (block-granular step)")
-    gemm_ms = sum(b.elapsed_time(e) for c in evs for b, e in evs[c]) / steps
+    ks = {n: metrics.k_for(h // block, R) * block for n, h, _, _ in wl.proj}
+    flops = sum(metrics.reduced_linear_flops(wl.T, N, ks[n]) for n, _, N, _ in wl.proj)
+    step = PrefillStep(wl, acts, Wts, dev, opts=rmm.options(block_size=block))
+    ms = time_steps(step, steps, warmup)
+    gemm_ms = sum(product_times(step, R, steps).values())
+    step.check_status("block-granular step")
     return {"blocks": {
-        "workload": f"the prefill step (T={T_PREFILL}, r={R}) with {block}-slice block-granular kept sets",
+        "workload": f"the prefill step ({wl.label}, T={wl.T}, r={R}) with {block}-slice block-granular kept sets",
         "ms_per_step": ms,
         "tflops": flops / (ms * 1e-3) / 1e12,
         "gemm_us": 1e3 * gemm_ms,
@@ -510,23 +669,7 @@ def time_ffn_demo(dev):
     return out
 
 
-def launches_per_step(dev) -> int:
-    """Our kernels launched by one step: per call the score pass, the select, the CTA-pair
-    GEMM, and the fold of the split last wave when the call's tiles leave a partial wave
-    that the GEMM splits (more than one K-range per tile)."""
-    pairs = torch.cuda.get_device_properties(dev).multi_processor_count // 2
-    n = 0
-    for s, names in CALLS:
-        H = ACT_H[s]
-        nkb = -(-metrics.k_for(H, R) // 64)
-        tiles = sum(-(-T_PREFILL // 256) * -(-PROJ_BY_NAME[m][1] // 512) for m in names)
-        rem = tiles % pairs
-        split = min(pairs // rem, 8, nkb) if rem else 1
-        n += 3 + (1 if split > 1 else 0)
-    return n
-
-
-def time_layer(dev, hweights):
+def time_layer(dev):
     """Secondary row: one Llama-3-8B decoder layer (hidden 4096, 32 query / 8 KV heads,
     MLP 14336, B = 1): prefill of T = 2048 tokens, then 128 decode steps against the
     growing KV cache, r = 0.5; against the same layer with dense products (cuBLAS) and
@@ -536,11 +679,13 @@ def time_layer(dev, hweights):
     from input_adaptive_reduced_rmm_b200.layer import DecoderLayer, DenseLayer, LayerDims
 
     dims = LayerDims()
-    Tp, steps = T_PREFILL, 128
-    W = {n: hweights[n] for n in ("q", "k", "v", "o", "gate", "up", "down")}
+    wl = LLAMA8
+    Tp, steps = wl.T, 128
+    W = {n: rmm_synth.weights(N, h, rmm_synth.seed_for(3, 80 + i, 1), std=0.02, device=dev)
+         for i, (n, h, N, _) in enumerate(wl.proj)}
     layers = {"rmm": DecoderLayer(dims, W, Tp + steps, R, dev), "dense": DenseLayer(dims, W, Tp + steps, dev)}
-    xp = rmm_synth.activations(Tp, dims.H, 700).to(dev)
-    xd = rmm_synth.activations(steps, dims.H, 701).to(dev)
+    xp = rmm_synth.activations(Tp, dims.H, 700, device=dev)
+    xd = rmm_synth.activations(steps, dims.H, 701, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     out = {}
     for name, layer in layers.items():
@@ -609,7 +754,8 @@ def time_layer(dev, hweights):
     return {"layer": {
         "workload": "Llama-3-8B decoder layer (RMSNorm, q/k/v, reduced attention over the head dim, o, "
                     "residual, RMSNorm, gate/up, SwiGLU, down, residual), B=1, prefill T=2048 then 128 "
-                    "decode steps, r=0.5; dense = cuBLAS products + SDPA attention, same glue kernels",
+                    "decode steps, r=0.5; dense = cuBLAS products (q|k|v and gate|up concatenated, one product each) "
+                    "+ SDPA attention, the same norm kernels, torch's silu(g)*u",
         "rmm": r_, "dense": d_,
         "prefill_speedup_vs_dense": d_["prefill_us"] / r_["prefill_us"],
         "decode_speedup_vs_dense": d_["decode_128_steps_us"] / r_["decode_128_steps_us"],
@@ -619,35 +765,18 @@ def time_layer(dev, hweights):
 
 
 def run_rmm(args, world, rank, local):
-    from input_adaptive_reduced_rmm_b200 import rmm
-
     dev = torch.device("cuda", local if world > 1 else 0)
     peaks = load_peaks()
-    acts, Wts = make_inputs(dev)
-    ks = {n: metrics.k_for(H, R) for n, H, _, _ in PROJ}
-    step_flops = sum(metrics.reduced_linear_flops(T_PREFILL, N, ks[n]) for n, _, N, _ in PROJ)
-    Ys = {n: torch.empty(T_PREFILL, N, dtype=torch.bfloat16, device=dev) for n, _, N, _ in PROJ}
-    ws = {}
-    for c, (s, names) in enumerate(CALLS):
-        ws[c] = rmm.new_workspace(rmm.rmm_linear_group_workspace_bytes(
-            T_PREFILL, ACT_H[s], [PROJ_BY_NAME[n][1] for n in names]), dev)
+    wl = HEADLINE
+    acts, Wts = device_inputs(wl, dev)
+    step_flops = wl.flops(R)
+    step = PrefillStep(wl, acts, Wts, dev)
     K, W = args.steps, args.warmup
-    evs = {c: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-           for c in range(len(CALLS))}
-    opt_timed = {c: [rmm.options(product_events=evs[c][i]) for i in range(K)] for c in range(len(CALLS))}
-
-    def step(i=None):
-        for c, (s, names) in enumerate(CALLS):
-            o = opt_timed[c][i] if i is not None else None
-            rmm.rmm_linear_group(acts[s], [Wts[n] for n in names], R, Ys=[Ys[n] for n in names],
-                                 workspace=ws[c], opts=o)
 
     for _ in range(W):
         step()
     torch.cuda.synchronize()
-    for c in ws:
-        if rmm.rmm_get_status(ws[c]) != rmm.RMM_OK:
-            raise RuntimeError("device status not OK after warm-up")
+    step.check_status("warm-up")
 
     clocks = ClockSampler(local if world > 1 else 0)
     clocks.start()
@@ -669,44 +798,31 @@ def run_rmm(args, world, rank, local):
     # pass is timed on its own and only its per-kernel split is used)
     barrier(world)
     torch.cuda.synchronize()
-    for i in range(K):
-        step(i)
-    torch.cuda.synchronize()
+    gemm_ms = product_times(step, R, K)
     barrier(world)
     clk = clocks.stop()
+    step.check_status("timed steps")
 
     # dominant kernel: the reduced GEMM launches, timed by events the library
     # records around each product launch inside the timed region
-    gemm_ms = {c: sum(b.elapsed_time(e) for b, e in evs[c]) / K for c in range(len(CALLS))}
     gemm_total_ms = sum(gemm_ms.values())
     achieved = step_flops / (gemm_total_ms * 1e-3) / 1e12
     per_call = {}
     for c, (s, names) in enumerate(CALLS):
-        f = sum(metrics.reduced_linear_flops(T_PREFILL, PROJ_BY_NAME[n][1], ks[n]) for n in names)
-        per_call["+".join(names)] = {"H": ACT_H[s], "N": [PROJ_BY_NAME[n][1] for n in names], "k": ks[names[0]],
+        f = sum(metrics.reduced_linear_flops(wl.T, wl.shape[n][1], wl.k(n, R)) for n in names)
+        per_call["+".join(names)] = {"H": wl.act_h[s], "N": [wl.shape[n][1] for n in names], "k": wl.k(names[0], R),
                                      "gemm_us": 1e3 * gemm_ms[c], "gemm_tflops": f / (gemm_ms[c] * 1e-3) / 1e12}
 
-    # dense cuBLAS product of the same shapes, same stream, same inputs
-    def dense_step():
-        for n, H, N, s in PROJ:
-            torch.matmul(acts[s], Wts[n], out=Ys[n])
-
-    for _ in range(W):
-        dense_step()
-    torch.cuda.synchronize()
-    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    d0.record()
-    for _ in range(K):
-        dense_step()
-    d1.record()
-    torch.cuda.synchronize()
-    dense_ms = d0.elapsed_time(d1) / K
-    dense_flops = sum(metrics.gemm_flops(T_PREFILL, N, H) for _, H, N, _ in PROJ)
+    # dense cuBLAS products of the same shapes, same stream, same inputs
+    dense = DenseSteps(wl, acts, Wts, dev)
+    dense_t = dense.times(K, W)
+    dense.release()
+    dense_ms = dense_t["best_ms"]
 
     # end to end through the public calls with host buffers: H2D of the step's
     # activations, the four calls, D2H of the seven outputs, every step
     host_acts = {s: a.cpu().pin_memory() for s, a in acts.items()}
-    host_Y = {n: torch.empty(T_PREFILL, N, dtype=torch.bfloat16).pin_memory() for n, _, N, _ in PROJ}
+    host_Y = {n: torch.empty(wl.T, N, dtype=torch.bfloat16).pin_memory() for n, _, N, _ in wl.proj}
     h2d = sum(a.numel() * 2 for a in host_acts.values())
     d2h = sum(y.numel() * 2 for y in host_Y.values())
 
@@ -715,7 +831,7 @@ def run_rmm(args, world, rank, local):
             acts[s].copy_(a, non_blocking=True)
         step()
         for n in host_Y:
-            host_Y[n].copy_(Ys[n], non_blocking=True)
+            host_Y[n].copy_(step.Ys[n], non_blocking=True)
 
     for _ in range(W):
         e2e_step()
@@ -729,26 +845,40 @@ def run_rmm(args, world, rank, local):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = job_throughput(step_flops * K, world, e2e_ms) / 1e12
+    del host_Y
 
     extra = {}
     if not args.skip_secondary:
-        extra.update(time_blocks(dev, acts, Wts, Ys, dense_ms, K, W))
-        extra.update(time_decode(dev, peaks))
-        extra.update(time_attn_decode(dev, peaks))
-        extra.update(time_ffn_demo(dev))
-        extra.update(time_layer(dev, host_inputs()[1]))
+        sweep_steps = max(5, K // 2)
+        extra["r_sweep"] = r_sweep(wl, step, dense_ms, peaks, sweep_steps, 3)
+        extra.update(time_blocks(wl, dev, acts, Wts, dense_ms, sweep_steps, 3))
 
     cpu = cpu_par = None
     if rank == 0 and not args.skip_cpu_baseline:
-        f, t, desc = oracle_sample(args.cpu_rows, seed=1)
+        # the oracle on the step's own inputs, copied to the host (W back to [N, H])
+        inputs = ({s: a.cpu() for s, a in acts.items()}, {n: Wt.t().contiguous().cpu() for n, Wt in Wts.items()})
+        f, t, desc = oracle_sample(wl, inputs, args.cpu_rows, seed=1)
         cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc}
         # the same oracle's OpenMP build on all host threads (a reported baseline too)
         import oracle
 
         threads = oracle.parallel_threads()
-        f, t, desc = oracle_sample(args.cpu_rows * max(1, min(threads, 16)) // 2, seed=2, parallel=True)
+        f, t, desc = oracle_sample(wl, inputs, args.cpu_rows * max(1, min(threads, 16)) // 2, seed=2,
+                                   parallel=True)
         cpu_par = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle-openmp",
                    "sample": desc}
+        del inputs
+
+    launches = launches_per_step(wl, R, dev)
+    del step, acts, Wts
+    torch.cuda.empty_cache()
+    if not args.skip_secondary:
+        extra["prefill_llama3_8b"] = prefill_row(LLAMA8, dev, peaks, K, W)
+        extra["decode_gemv"] = time_decode(LLAMA70, dev, peaks)
+        extra["decode_gemv_llama3_8b"] = time_decode(LLAMA8, dev, peaks)
+        extra.update(time_attn_decode(dev, peaks))
+        extra.update(time_ffn_demo(dev))
+        extra.update(time_layer(dev))
 
     if rank != 0:
         return
@@ -757,24 +887,38 @@ def run_rmm(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": step_config(world),
+        "config": step_config(wl, world),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": STEP_GEMM_DRAM_BYTES,
+                     "frac": achieved / peak, "traffic": STEP_GEMM_DRAM_BYTES.get(wl.label),
                      "traffic_unit": "bytes (ncu dram read + write) over the step's 4 GEMM launches",
                      "kernel": "gemm_pair_kernel (tcgen05 cta_group::2 reduced GEMM), the 4 launches of a step",
                      "peak_source": f"{peaks['source']} bf16 burst"},
         "speedup_vs_dense": dense_ms / (ms_max / K),
-        "dense": {"ms_per_step": dense_ms, "tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
+        "dense": {**dense_t, "tflops": dense_t["tflops_best"],
                   "effective_tflops_at_reduced_flops": step_flops / (dense_ms * 1e-3) / 1e12},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "cpu_baseline": cpu,
         "cpu_baseline_parallel": cpu_par,
-        "gpu_launches": launches_per_step(dev) * K,
+        "gpu_launches": launches * K,
         "clocks": clk,
         "per_call": per_call,
     }
     line.update(extra)
     print(json.dumps(line), flush=True)
+
+
+def run_profile_step(args):
+    """The headline step alone, --warmup then --steps times (profiling aid: nothing else
+    runs, so an ncu capture holds only the step's own buffers)."""
+    dev = torch.device("cuda", 0)
+    wl = HEADLINE
+    acts, Wts = device_inputs(wl, dev)
+    step = PrefillStep(wl, acts, Wts, dev)
+    ms = time_steps(step, args.steps, args.warmup)
+    step.check_status("profile step")
+    print(json.dumps({"profile_step": {"workload": wl.name(R), "ms_per_step": ms,
+                                       "tflops": wl.flops(R) / (ms * 1e-3) / 1e12,
+                                       "launches_per_step": launches_per_step(wl, R, dev)}}), flush=True)
 
 
 def run_single(args):
@@ -888,13 +1032,14 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["rmm", "reference"], default="rmm")
-    ap.add_argument("--cpu-rows", type=int, default=24)
+    ap.add_argument("--cpu-rows", type=int, default=8)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-secondary", action="store_true")
     ap.add_argument("--single", default=None, help="T,H,N,r: time one rmm_linear shape alone")
     ap.add_argument("--single-attn", default=None, help="B,Hq,Hkv,T,L,r: time one rmm_attn_qk call alone")
     ap.add_argument("--single-ctx", default=None,
                     help="B,Hq,Hkv,L,block,r,r_ctx: time one rmm_attn_ctx decode call alone")
+    ap.add_argument("--profile-step", action="store_true", help="run only the headline step (profiling aid)")
     ap.add_argument("--gemm-producer", type=int, default=0)
     ap.add_argument("--block-size", type=int, default=0, help="with --single: block-granular kept sets")
     args = ap.parse_args()
@@ -908,6 +1053,9 @@ def main():
         return
     if args.single:
         run_single(args)
+        return
+    if args.profile_step:
+        run_profile_step(args)
         return
     if args.impl == "reference":
         # the oracle on the host cores: rank 0 alone, no process group, no GPU

@@ -154,12 +154,16 @@ class DecoderLayer:
 
 class DenseLayer:
     """The same layer with dense products (cuBLAS through torch.matmul) and dense
-    attention (torch scaled_dot_product_attention): the comparison, not the product."""
+    attention (torch scaled_dot_product_attention): the comparison, not the product.
+    Like the reduced layer, which runs q/k/v and gate/up as one grouped launch each,
+    it runs q|k|v and gate|up as one product each over concatenated weights."""
 
     def __init__(self, dims: LayerDims, weights: dict, max_len: int, device):
         self.d = dims
         self.dev = device
-        self.Wt = {n: weights[n].to(device).t().contiguous() for n in ("q", "k", "v", "o", "gate", "up", "down")}
+        Wt = {n: weights[n].to(device).t().contiguous() for n in ("q", "k", "v", "o", "gate", "up", "down")}
+        self.Wt = {"qkv": torch.cat([Wt["q"], Wt["k"], Wt["v"]], dim=1), "o": Wt["o"],
+                   "gate_up": torch.cat([Wt["gate"], Wt["up"]], dim=1), "down": Wt["down"]}
         self.K = torch.zeros(1, dims.Hkv, max_len, D_HEAD, dtype=torch.bfloat16, device=device)
         self.V = torch.zeros(1, dims.Hkv, max_len, D_HEAD, dtype=torch.bfloat16, device=device)
         self.pos = 0
@@ -177,7 +181,7 @@ class DenseLayer:
         with op("rmsnorm"):
             _, xn = rmm.rmm_add_rmsnorm(x, eps=dm.eps)
         with op("qkv"):
-            q, k, v = xn @ self.Wt["q"], xn @ self.Wt["k"], xn @ self.Wt["v"]
+            q, k, v = (xn @ self.Wt["qkv"]).split([dm.q_cols, dm.kv_cols, dm.kv_cols], dim=1)
         with op("kv_append"):
             Q = q.view(T, dm.Hq, D_HEAD).transpose(0, 1).unsqueeze(0)
             self.K[0, :, L0:L] = k.view(T, dm.Hkv, D_HEAD).transpose(0, 1)
@@ -193,9 +197,9 @@ class DenseLayer:
         with op("add_rmsnorm"):
             h2, xn2 = rmm.rmm_add_rmsnorm(x, yo, eps=dm.eps)
         with op("gate_up"):
-            g, u = xn2 @ self.Wt["gate"], xn2 @ self.Wt["up"]
+            g, u = (xn2 @ self.Wt["gate_up"]).split([dm.F, dm.F], dim=1)
         with op("swiglu"):
-            hh = rmm.rmm_swiglu(g, u)
+            hh = torch.nn.functional.silu(g) * u
         with op("down"):
             yd = hh @ self.Wt["down"]
         with op("residual"):

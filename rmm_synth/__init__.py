@@ -18,6 +18,10 @@ weights or datasets are used):
 
 Values are drawn in fp32 with ``torch.Generator`` on the CPU and rounded to
 bf16 with round-to-nearest-even.  Seeds follow ``1000*config + 10*case + stream``.
+``device="cuda"`` draws the same recipe with the device's generator instead
+(other numbers, same distribution): the benchmark's large workloads use it so
+that gigabytes of weights are not drawn on the host; parity tests use the CPU
+draws so that both sides see identical bytes.
 """
 from __future__ import annotations
 
@@ -40,29 +44,29 @@ def seed_for(config: int, case: int, stream: int) -> int:
     return 1000 * int(config) + 10 * int(case) + int(stream)
 
 
-def _gen(seed: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
+def _gen(seed: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
     g.manual_seed(int(seed))
     return g
 
 
 def activations(T: int, H: int, seed: int, outlier_frac: float = 0.02,
-                outlier_scale: float = 20.0) -> torch.Tensor:
+                outlier_scale: float = 20.0, device="cpu") -> torch.Tensor:
     """X [T, H] bf16: N(0,1) with ``round(outlier_frac*H)`` seeded outlier columns x ``outlier_scale``."""
-    g = _gen(seed)
-    x = torch.randn(T, H, generator=g, dtype=torch.float32)
+    g = _gen(seed, device)
+    x = torch.randn(T, H, generator=g, dtype=torch.float32, device=device)
     n_out = int(round(outlier_frac * H))
     if n_out > 0:
-        cols = torch.randperm(H, generator=g)[:n_out]
+        cols = torch.randperm(H, generator=g, device=device)[:n_out]
         x[:, cols] *= outlier_scale
     return x.to(torch.bfloat16)
 
 
-def weights(N: int, H: int, seed: int, std: float | None = None) -> torch.Tensor:
+def weights(N: int, H: int, seed: int, std: float | None = None, device="cpu") -> torch.Tensor:
     """W [N, H] bf16 ~ N(0, std^2); ``std=None`` means 1/sqrt(H)."""
-    g = _gen(seed)
+    g = _gen(seed, device)
     s = (1.0 / math.sqrt(H)) if std is None else float(std)
-    w = torch.randn(N, H, generator=g, dtype=torch.float32) * s
+    w = torch.randn(N, H, generator=g, dtype=torch.float32, device=device) * s
     return w.to(torch.bfloat16)
 
 

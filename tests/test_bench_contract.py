@@ -28,7 +28,7 @@ def test_reference_arm_prints_one_contract_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["steps"] == 3 and d["warmup"] == 3
     assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True and d["value"] > 0
-    assert d["config"]["workload"].startswith("llama3-8b") and d["config"]["T"] == 2048
+    assert d["config"]["workload"].startswith("llama3-70b") and d["config"]["T"] == 4096
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
