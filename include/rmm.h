@@ -322,6 +322,19 @@ rmm_status rmm_qkv_heads(const void* Yq, const void* Yk, const void* Yv, int T, 
  * A[t, h*d + j] = O[h, t, j] for O [Hq, T, d] (batch 1), d == 128. */
 rmm_status rmm_heads_to_tokens(const void* O, int Hq, int T, int d, void* A, rmm_stream_t stream);
 
+/* ---------------------------------------------------------------- self-test
+ *
+ * y[i] = 2^x[i] as the tensor-core attention's softmax computes half of its
+ * exponentials: on the FMA pipe, by a round-to-nearest split x = n + f
+ * (|f| <= 1/2), the Taylor series of e^(f ln 2) to degree 4 and n added to
+ * the exponent.  The softmax only evaluates x <= 8; below -126 the result is
+ * 2^-126.  Stated bound: relative error below 6e-5 on [-126, 8].  It exists so
+ * that the bound can be checked directly; x and y are fp32 device buffers of
+ * n elements (n >= 1).  The pages have no counterpart: the exponential is an
+ * implementation detail of the softmax (cf-1.com post §3.3 keeps softmax.V
+ * exact in form). */
+rmm_status rmm_selftest_exp2_fma(const float* x, float* y, int n, rmm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -630,4 +630,9 @@ rmm_status rmm_heads_to_tokens(const void* O, int Hq, int T, int d, void* A, rmm
                                               num_sms_current(), static_cast<cudaStream_t>(stream)));
 }
 
+rmm_status rmm_selftest_exp2_fma(const float* x, float* y, int n, rmm_stream_t stream) {
+    if (!x || !y || n < 1) return RMM_ERR_INVALID_ARG;
+    return cuda_status(launch_exp2_fma(x, y, n, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

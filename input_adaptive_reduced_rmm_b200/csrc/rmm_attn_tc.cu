@@ -459,12 +459,23 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (warp == kMmaWarp) tmem_dealloc(tmem, TMEM_COLS);
 }
 
+// The FMA-pipe exponential on its own, for its direct test.
+__global__ void exp2_fma_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) y[i] = poly_exp2(x[i]);
+}
+
 size_t attn_tc_smem_bytes(int kp) {
     const int ks = kp <= 96 ? 3 : 2;
     return 1024 + P_BYTES + (size_t)ks * V_BYTES + (size_t)(1 + ks) * kp * 256 + D * sizeof(int) + sizeof(Bars);
 }
 
 }  // namespace
+
+cudaError_t launch_exp2_fma(const float* x, float* y, int n, cudaStream_t stream) {
+    const int blocks = (n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184;
+    exp2_fma_kernel<<<blocks, 256, 0, stream>>>(x, y, n);
+    return cudaGetLastError();
+}
 
 bool attn_tc_supported(int T, int k) { return T >= kAttnTcMinT && k >= 1 && k <= D; }
 

@@ -71,6 +71,7 @@ cudaError_t launch_gemv(const uint16_t* X, int T, int H, const int32_t* idx, int
 // least kAttnTcMinT tokens, kept sets from the attention select kernel
 constexpr int kAttnTcMinT = 16;
 bool attn_tc_supported(int T, int k);
+cudaError_t launch_exp2_fma(const float* x, float* y, int n, cudaStream_t stream);
 cudaError_t launch_attn_tc(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq, int Hkv, int T,
                            int L, int ldL, int k, int causal, float scale, int per_query_head, const int32_t* idx,
                            uint16_t* O, int* status, cudaStream_t stream);

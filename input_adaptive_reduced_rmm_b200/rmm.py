@@ -30,7 +30,7 @@ EXPORTED = (
     "rmm_select", "rmm_gemm_reduced", "rmm_attn_workspace_bytes", "rmm_attn_qk",
     "rmm_linear_decode_noalloc", "rmm_linear_group", "rmm_linear_group_workspace_bytes",
     "rmm_add_rmsnorm", "rmm_swiglu", "rmm_qkv_heads", "rmm_heads_to_tokens",
-    "rmm_ctx_block_means", "rmm_attn_ctx_workspace_bytes", "rmm_attn_ctx",
+    "rmm_ctx_block_means", "rmm_attn_ctx_workspace_bytes", "rmm_attn_ctx", "rmm_selftest_exp2_fma",
 )
 
 
@@ -112,6 +112,7 @@ def lib() -> ctypes.CDLL:
         "rmm_ctx_block_means": (I, [P, I, I, I, I, I, I, I, I, P, P]),
         "rmm_attn_ctx_workspace_bytes": (Z, [I, I, I, I, I, I, I, D, OP]),
         "rmm_attn_ctx": (I, [P, P, P, P, I, I, I, I, I, I, I, D, D, I, I, F, P, P, P, P, Z, P, OP]),
+        "rmm_selftest_exp2_fma": (I, [P, P, I, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -508,3 +509,14 @@ def rmm_heads_to_tokens(O: torch.Tensor, A: torch.Tensor | None = None, stream=N
         A = torch.empty(T, Hq * d, dtype=torch.bfloat16, device=O.device)
     _check(lib().rmm_heads_to_tokens(_ptr(O), Hq, T, d, _ptr(A), _stream(stream)), "rmm_heads_to_tokens")
     return A
+
+
+def rmm_selftest_exp2_fma(x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """2^x by the FMA-pipe exponential of the tensor-core softmax (fp32, elementwise)."""
+    _need(x, "x", torch.float32)
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", torch.float32, shape=tuple(x.shape))
+    _on_cuda(x=x, y=y)
+    _check(lib().rmm_selftest_exp2_fma(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "rmm_selftest_exp2_fma")
+    return y

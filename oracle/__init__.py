@@ -174,10 +174,11 @@ def select(s, k: int) -> np.ndarray:
     return idx
 
 
-def reduced_product(X, W, idx, rows=None, cols=None) -> np.ndarray:
+def reduced_product(X, W, idx, rows=None, cols=None, parallel: bool = False) -> np.ndarray:
     """Y[r, c] = sum_{j} X[t_r, idx_j] * W[n_c, idx_j] in fp64.  W is [N, H].
 
     rows / cols (optional) select the token rows and output features computed.
+    parallel=True runs the OpenMP build (same bits, rows spread over the host's threads).
     """
     x, w = _bits(X), _bits(W)
     T, H = x.shape
@@ -187,7 +188,7 @@ def reduced_product(X, W, idx, rows=None, cols=None) -> np.ndarray:
     rp, nr, _kr = _rows(rows)
     cp, nc, _kc = _rows(cols)
     Y = np.zeros((nr if rows is not None else T, nc if cols is not None else N), dtype=np.float64)
-    _check(_load().oracle_reduced_product(x, w, T, H, N, idx, len(idx), rp, nr, cp, nc, Y),
+    _check(_load(parallel).oracle_reduced_product(x, w, T, H, N, idx, len(idx), rp, nr, cp, nc, Y),
            "oracle_reduced_product")
     return Y
 

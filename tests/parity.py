@@ -39,3 +39,24 @@ def sample_indices(n, count, seed):
 
 def bits_u16(t):
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def tile_rows(T, tile=128, seed=0):
+    """One row in every `tile`-row tile (at a seeded offset), plus the first and last rows."""
+    rng = np.random.default_rng(seed)
+    rows = {0, T - 1}
+    for t0 in range(0, T, tile):
+        rows.add(int(t0 + rng.integers(0, min(tile, T - t0))))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def row_head_pairs(rows, Hq, Hkv, heads_per_row=1):
+    """(row, query head) pairs to check: each row on `heads_per_row` heads, rotating over
+    the KV groups and over the heads inside a group, so the sample touches every group."""
+    G = Hq // Hkv
+    pairs = []
+    for i, t in enumerate(rows):
+        for j in range(heads_per_row):
+            g = (i * heads_per_row + j) % Hkv
+            pairs.append((int(t), g * G + (i + j) % G))
+    return pairs

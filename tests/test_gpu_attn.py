@@ -13,7 +13,7 @@ import torch
 
 import oracle
 import rmm_synth
-from parity import assert_close, sample_indices
+from parity import assert_close, row_head_pairs, sample_indices, tile_rows
 
 pytestmark = pytest.mark.gpu
 D = 128
@@ -93,16 +93,44 @@ def test_attention_tie_heavy_queries(rmm):
     assert_close(O, Oo, "ties")
 
 
-def check_large(rmm, cfg, B, Hq, Hkv, T, L, r, nrows):
+def oracle_kept_sets(Q, K, V, k):
+    """The oracle's kept head-dimension sets for Q (per KV group): they depend on Q alone, so
+    the oracle runs them against the cache's first T keys and computes one output row."""
+    T = Q.shape[2]
+    _, io = oracle.attention(Q, K[:, :, :T], V[:, :, :T], k, causal=True, t_rows=[0])
+    return io
+
+
+def check_pairs(O, Q, K, V, k, idx, pairs, what, causal=True):
+    """O[b, h, t] against the oracle for each sampled (t, h), with the kept sets given (one
+    oracle call per query head: that head and its KV group alone)."""
+    B, Hq, T, d = Q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    by_head = {}
+    for t, h in pairs:
+        by_head.setdefault(h, []).append(t)
+    got, ref = [], []
+    for h, rows in sorted(by_head.items()):
+        g = h // G
+        Oo, _ = oracle.attention(Q[:, h:h + 1].contiguous(), K[:, g:g + 1].contiguous(), V[:, g:g + 1].contiguous(),
+                                 k, causal=causal, t_rows=rows, idx_in=idx[:, g:g + 1])
+        got.append(O[:, h, rows].double().numpy())
+        ref.append(Oo[:, 0])
+    assert_close(np.concatenate(got, axis=1), np.concatenate(ref, axis=1), what)
+
+
+def check_large(rmm, cfg, B, Hq, Hkv, T, L, r, heads_per_row=2, opts=None):
+    """Kept sets in full; O on one query row of every 128-row query tile (plus the first and
+    last rows), each on `heads_per_row` query heads spread over the KV groups."""
     seed = rmm_synth.seed_for(cfg, T % 100, L % 97)
     Q = rmm_synth.normal((B, Hq, T, D), seed)
     K = rmm_synth.normal((B, Hkv, L, D), seed + 1)
     V = rmm_synth.normal((B, Hkv, L, D), seed + 2)
-    O, idx, k = run_attn(rmm, Q, K, V, r, True)
-    rows = sample_indices(T, nrows, seed=L + T)
-    Oo, io = oracle.attention(Q, K, V, k, causal=True, t_rows=rows)
-    assert np.array_equal(idx, io)
-    assert_close(O[:, :, rows], Oo, f"cfg{cfg} T={T} L={L} r={r}")
+    O, idx, k = run_attn(rmm, Q, K, V, r, True, opts=opts)
+    assert np.array_equal(idx, oracle_kept_sets(Q, K, V, k)), "kept sets"
+    rows = tile_rows(T, 128, seed=L + T)
+    check_pairs(O, Q, K, V, k, idx, row_head_pairs(rows, Hq, Hkv, heads_per_row), f"cfg{cfg} T={T} L={L} r={r}")
 
 
 @pytest.mark.parametrize("L", [4096, 16384, 32768])
@@ -110,13 +138,22 @@ def check_large(rmm, cfg, B, Hq, Hkv, T, L, r, nrows):
 @pytest.mark.parametrize("r", [0.25, 0.5])
 def test_attention_llama3_8b(rmm, L, T, r):
     """Batch 1, 32 query / 8 KV heads, d = 128, decode and a prefill chunk of 512."""
-    check_large(rmm, 2, 1, 32, 8, T, L, r, nrows=3)
+    check_large(rmm, 2, 1, 32, 8, T, L, r, heads_per_row=8 if T == 1 else 2)
 
 
-@pytest.mark.parametrize("T", [1, 512])
-def test_attention_llama3_70b(rmm, T):
-    """64 query / 8 KV heads, d = 128, KV length 65536."""
-    check_large(rmm, 4, 1, 64, 8, T, 65536, 0.5, nrows=2)
+@pytest.mark.parametrize("r", [0.25, 0.5])
+def test_attention_layer_prefill_shape(rmm, r):
+    """The decoder layer's own prefill attention: T = L = 2048, causal, 32 query / 8 KV
+    heads (16 query tiles per head on the tensor cores)."""
+    check_large(rmm, 3, 1, 32, 8, 2048, 2048, r, heads_per_row=4)
+
+
+@pytest.mark.parametrize("T", [1, 4096])
+@pytest.mark.parametrize("r", [0.125, 0.25, 0.5, 1.0])
+def test_attention_llama3_70b(rmm, T, r):
+    """64 query / 8 KV heads, d = 128, KV length 65536; decode and a 4096-token chunk
+    (32 query tiles per head) across the retention sweep."""
+    check_large(rmm, 4, 1, 64, 8, T, 65536, r, heads_per_row=8 if T == 1 else 1)
 
 
 @pytest.mark.parametrize("path", [1, 2])
@@ -153,3 +190,26 @@ def test_attention_rejects_bad_head_dim(rmm):
     rc = L.rmm_attn_qk(p(Q), p(Kt), p(V), 1, 2, 1, 1, 16, 16, 64, 0.5, 1, 1.0 / math.sqrt(64), p(Q), None,
                        p(ws), ws.numel(), rmm._stream(None), None)
     assert rc == rmm.RMM_ERR_UNSUPPORTED
+
+
+def test_fma_exponential_meets_its_stated_bound(rmm):
+    """The softmax's FMA-pipe 2^x against the exact value (fp64 on the host) over its whole
+    input range [-126, 8]: relative error below the stated 6e-5, every integer exact, and
+    the hardware 2^x (torch.exp2) within the same bound; below -126 it clamps to 2^-126."""
+    g = torch.Generator().manual_seed(11)
+    dense = torch.linspace(-126.0, 8.0, 1 << 20, dtype=torch.float64)
+    rand = torch.rand(1 << 20, generator=g, dtype=torch.float64) * 134.0 - 126.0
+    near = (torch.arange(-126, 9, dtype=torch.float64)[:, None] +
+            torch.tensor([-0.5, -0.4999999, -1e-6, 0.0, 1e-6, 0.4999999, 0.5], dtype=torch.float64)[None, :]).reshape(-1)
+    x = torch.cat([dense, rand, near]).clamp(-126.0, 8.0).to(torch.float32)
+    y = rmm.rmm_selftest_exp2_fma(x.cuda())
+    hw = torch.exp2(x.cuda())
+    torch.cuda.synchronize()
+    exact = torch.exp2(x.double())
+    rel = ((y.cpu().double() - exact) / exact).abs()
+    assert float(rel.max()) < 6e-5, f"max relative error {float(rel.max()):.3e}"
+    ints = torch.arange(-126, 9, dtype=torch.float32)
+    assert torch.equal(rmm.rmm_selftest_exp2_fma(ints.cuda()).cpu(), torch.exp2(ints.double()).float())
+    assert float(((hw.cpu().double() - exact) / exact).abs().max()) < 6e-5
+    low = rmm.rmm_selftest_exp2_fma(torch.tensor([-130.0, -1000.0, -126.0], device="cuda")).cpu()
+    assert torch.equal(low, torch.full((3,), 2.0 ** -126))

@@ -13,7 +13,7 @@ import torch
 
 import oracle
 import rmm_synth
-from parity import assert_close, bits_u16
+from parity import assert_close, bits_u16, tile_rows
 
 pytestmark = pytest.mark.gpu
 D = 128
@@ -45,17 +45,25 @@ def cpu(t):
     return t.detach().cpu()
 
 
-def check_step(tr, W, r, Hq, Hkv):
-    """Per-op parity of one forward call, from its trace."""
+def check_step(tr, W, r, Hq, Hkv, rows=None):
+    """Per-op parity of one forward call, from its trace.  Kept sets are compared in full
+    (their scores run over every token row); float outputs on the token rows `rows`
+    (None: all of them), each computed by the oracle from the GPU's own inputs."""
     T, H = tr["x"].shape
+    rs = slice(None) if rows is None else rows
+    par = rows is not None
+
+    def prod(X, Wn, idx):
+        return oracle.reduced_product(X, Wn, idx, rows=rows, parallel=par)
+
     k_h = oracle.k_for(H, r)
     # RMSNorm
-    assert_close(tr["xn"], oracle.rmsnorm(cpu(tr["x"])), "rmsnorm")
+    assert_close(cpu(tr["xn"])[rs], oracle.rmsnorm(cpu(tr["x"])[rs]), "rmsnorm")
     # q, k, v: one kept set from xn
     idx = oracle.select(oracle.score(cpu(tr["xn"])), k_h)
     assert cpu(tr["idx_qkv"])[:k_h].numpy().tolist() == idx.tolist(), "q/k/v kept set"
     for n in ("q", "k", "v"):
-        assert_close(tr["y" + n], oracle.reduced_product(cpu(tr["xn"]), W[n], idx), f"{n} projection")
+        assert_close(cpu(tr["y" + n])[rs], prod(cpu(tr["xn"]), W[n], idx), f"{n} projection")
     # heads and the KV-cache append: exact relayouts
     L0, L = tr["L0"], tr["L"]
     yq, yk, yv = cpu(tr["yq"]), cpu(tr["yk"]), cpu(tr["yv"])
@@ -67,49 +75,57 @@ def check_step(tr, W, r, Hq, Hkv):
     k_d = oracle.k_for(D, r)
     Kc = Kt[:, :, :L].permute(0, 2, 1).contiguous().unsqueeze(0)
     Vc = V[:, :L].contiguous().unsqueeze(0)
-    O_ref, idx_a = oracle.attention(cpu(tr["Q"]).unsqueeze(0), Kc, Vc, k_d, causal=True)
+    O_ref, idx_a = oracle.attention(cpu(tr["Q"]).unsqueeze(0), Kc, Vc, k_d, causal=True, t_rows=rows)
     assert np.array_equal(cpu(tr["idx_attn"]).numpy(), idx_a[0]), "attention kept sets"
-    assert_close(tr["O"], O_ref[0], "attention")
+    assert_close(cpu(tr["O"])[:, rs], O_ref[0], "attention")
     assert torch.equal(cpu(tr["a"]), cpu(tr["O"]).transpose(0, 1).reshape(T, Hq * D)), "heads to tokens"
     # o projection
     k_o = oracle.k_for(Hq * D, r)
     idx = oracle.select(oracle.score(cpu(tr["a"])), k_o)
     assert cpu(tr["idx_o"])[:k_o].numpy().tolist() == idx.tolist(), "o kept set"
-    assert_close(tr["yo"], oracle.reduced_product(cpu(tr["a"]), W["o"], idx), "o projection")
+    assert_close(cpu(tr["yo"])[rs], prod(cpu(tr["a"]), W["o"], idx), "o projection")
     # residual add (exact: both addends are bf16, their fp32 sum rounds once) + RMSNorm
     h2 = (cpu(tr["x"]).float() + cpu(tr["yo"]).float()).to(torch.bfloat16)
     assert np.array_equal(bits_u16(tr["h2"]), bits_u16(h2)), "residual add"
-    assert_close(tr["xn2"], oracle.rmsnorm(cpu(tr["h2"])), "rmsnorm after attention")
+    assert_close(cpu(tr["xn2"])[rs], oracle.rmsnorm(cpu(tr["h2"])[rs]), "rmsnorm after attention")
     # gate, up (one kept set), SwiGLU, down
     idx = oracle.select(oracle.score(cpu(tr["xn2"])), k_h)
     assert cpu(tr["idx_gu"])[:k_h].numpy().tolist() == idx.tolist(), "gate/up kept set"
     for n, key in (("gate", "g"), ("up", "u")):
-        assert_close(tr[key], oracle.reduced_product(cpu(tr["xn2"]), W[n], idx), f"{n} projection")
-    assert_close(tr["hh"], oracle.swiglu(cpu(tr["g"]), cpu(tr["u"])), "swiglu")
+        assert_close(cpu(tr[key])[rs], prod(cpu(tr["xn2"]), W[n], idx), f"{n} projection")
+    assert_close(cpu(tr["hh"])[rs], oracle.swiglu(cpu(tr["g"])[rs], cpu(tr["u"])[rs]), "swiglu")
     F = tr["hh"].shape[1]
     k_f = oracle.k_for(F, r)
     idx = oracle.select(oracle.score(cpu(tr["hh"])), k_f)
     assert cpu(tr["idx_down"])[:k_f].numpy().tolist() == idx.tolist(), "down kept set"
-    assert_close(tr["yd"], oracle.reduced_product(cpu(tr["hh"]), W["down"], idx), "down projection")
+    assert_close(cpu(tr["yd"])[rs], prod(cpu(tr["hh"]), W["down"], idx), "down projection")
     out = (cpu(tr["h2"]).float() + cpu(tr["yd"]).float()).to(torch.bfloat16)
     assert np.array_equal(bits_u16(tr["out"]), bits_u16(out)), "final residual add"
 
 
-def oracle_layer_prefill(x, W, r, Hq, Hkv, tr):
+def oracle_layer_prefill(x, W, r, Hq, Hkv, tr, rows=None):
     """The layer on an empty cache in oracle arithmetic (fp64 ops, bf16 between ops),
-    following the GPU's kept sets from the trace."""
+    following the GPU's kept sets from the trace.  rows (None: all) restricts the output
+    to those token rows: keys and values are still projected for every token (each row
+    attends to all earlier ones), queries and everything after attention only for `rows`."""
     T, H = x.shape
     k_h, k_o, k_f = oracle.k_for(H, r), oracle.k_for(Hq * D, r), oracle.k_for(W["down"].shape[1], r)
+    par = rows is not None
+    rs = slice(None) if rows is None else rows
     xn = bf16(oracle.rmsnorm(x))
     i_qkv = cpu(tr["idx_qkv"])[:k_h].numpy()
-    yq, yk, yv = (bf16(oracle.reduced_product(xn, W[n], i_qkv)) for n in ("q", "k", "v"))
+    yk, yv = (bf16(oracle.reduced_product(xn, W[n], i_qkv, parallel=par)) for n in ("k", "v"))
+    yq = torch.zeros(T, Hq * D, dtype=torch.bfloat16)  # rows not asked for stay zero: the kept sets are given
+    yq[rs] = bf16(oracle.reduced_product(xn, W["q"], i_qkv, rows=rows, parallel=par))
     Q = yq.view(T, Hq, D).transpose(0, 1).contiguous().unsqueeze(0)
     K = yk.view(T, Hkv, D).transpose(0, 1).contiguous().unsqueeze(0)
     V = yv.view(T, Hkv, D).transpose(0, 1).contiguous().unsqueeze(0)
-    O, _ = oracle.attention(Q, K, V, oracle.k_for(D, r), causal=True, idx_in=cpu(tr["idx_attn"]).numpy()[None])
-    a = bf16(O[0]).transpose(0, 1).reshape(T, Hq * D).contiguous()
+    O, _ = oracle.attention(Q, K, V, oracle.k_for(D, r), causal=True, idx_in=cpu(tr["idx_attn"]).numpy()[None],
+                            t_rows=rows)
+    n = O.shape[2]
+    a = bf16(O[0]).transpose(0, 1).reshape(n, Hq * D).contiguous()
     yo = bf16(oracle.reduced_product(a, W["o"], cpu(tr["idx_o"])[:k_o].numpy()))
-    h2 = (x.float() + yo.float()).to(torch.bfloat16)
+    h2 = (x[rs].float() + yo.float()).to(torch.bfloat16)
     xn2 = bf16(oracle.rmsnorm(h2))
     i_gu = cpu(tr["idx_gu"])[:k_h].numpy()
     g, u = (bf16(oracle.reduced_product(xn2, W[n], i_gu)) for n in ("gate", "up"))
@@ -135,6 +151,35 @@ def test_layer_prefill_then_decode(rmm, T):
     # decode steps: one token at a time against the growing cache
     for step in range(3):
         xt = rmm_synth.activations(1, H, rmm_synth.seed_for(3, T, 10 + step))
+        tr = {}
+        layer.forward(xt.cuda(), trace=tr)
+        torch.cuda.synchronize()
+        assert tr["L"] == T + step + 1
+        check_step(tr, W, r, Hq, Hkv)
+
+
+def test_layer_llama3_8b_full_size(rmm):
+    """The decoder layer at its Llama-3-8B size (hidden 4096, 32 query / 8 KV heads, d = 128,
+    MLP 14336), prefill of T = 2048 tokens then decode steps against the 2048+ cache, r = 0.5.
+    Kept sets in full; float outputs on one token row per 128-row tile (the products' and the
+    attention's query tiles) and the first and last rows."""
+    from input_adaptive_reduced_rmm_b200.layer import DecoderLayer, LayerDims
+
+    H, Hq, Hkv, F, r, T = 4096, 32, 8, 14336, 0.5, 2048
+    W = make_weights(H, Hq, Hkv, F, 77)
+    dims = LayerDims(H=H, Hq=Hq, Hkv=Hkv, F=F)
+    layer = DecoderLayer(dims, W, max_len=T + 8, r=r, device=torch.device("cuda"))
+    x = rmm_synth.activations(T, H, rmm_synth.seed_for(3, 77, 9))
+    tr = {}
+    y = layer.forward(x.cuda(), trace=tr)
+    torch.cuda.synchronize()
+    rows = tile_rows(T, 128, seed=7)
+    check_step(tr, W, r, Hq, Hkv, rows=rows)
+    assert_close(cpu(y)[rows], oracle_layer_prefill(x, W, r, Hq, Hkv, tr, rows=rows),
+                 "layer output (prefill T=2048, GPU kept sets)")
+    del tr
+    for step in range(3):
+        xt = rmm_synth.activations(1, H, rmm_synth.seed_for(3, 77, 10 + step))
         tr = {}
         layer.forward(xt.cuda(), trace=tr)
         torch.cuda.synchronize()

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import rmm_synth
-from parity import assert_close, bits_u16, sample_indices
+from parity import assert_close, bits_u16, sample_indices, tile_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -171,13 +171,16 @@ def _inputs(cfg, T, H, N):
 
 
 def check_projection(rmm, cfg, T, H, N, r, nrows=12, ncols=384):
+    """Kept set in full; Y on a row sample with one row in every 128-row M tile (and
+    `nrows` more at random) and a column sample with one column in every 512-column N
+    tile of the CTA-pair GEMM (and `ncols` more at random)."""
     X, W = _inputs(cfg, T, H, N)
     Y, idx = run_linear(rmm, X, W, r)
     k = oracle.k_for(H, r)
     io = oracle.select(oracle.score(X), k)
     assert np.array_equal(idx, io), "kept set differs"
-    rows = sample_indices(T, nrows, seed=T + N)
-    cols = sample_indices(N, ncols, seed=H + N)
+    rows = np.union1d(sample_indices(T, nrows, seed=T + N), tile_rows(T, 128, seed=T))
+    cols = np.union1d(sample_indices(N, ncols, seed=H + N), tile_rows(N, 512, seed=N))
     Yo = oracle.reduced_product(X, W, io, rows=rows, cols=cols)
     assert_close(Y[rows][:, cols], Yo, f"cfg{cfg} T={T} H={H} N={N} r={r}")
 

@@ -665,4 +665,7 @@ def test_openmp_build_gives_the_same_bits():
     Y1, i1 = oracle.linear(X, W, 0.5)
     Y2, i2 = oracle.linear(X, W, 0.5, parallel=True)
     assert np.array_equal(i1, i2) and np.array_equal(Y1, Y2)
+    rows = [36, 0, 5]
+    assert np.array_equal(oracle.reduced_product(X, W, i1, rows=rows),
+                          oracle.reduced_product(X, W, i1, rows=rows, parallel=True))
     assert oracle.parallel_threads() >= 1
