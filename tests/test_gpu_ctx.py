@@ -162,8 +162,8 @@ def test_ctx_rejects_unsupported(rmm):
     with pytest.raises(rmm.RmmError):
         rmm.rmm_attn_ctx(Q, Kt, V, means, L, 0.5, 0.5, block)  # T = 17 > 16
     Q1 = torch.zeros(B, Hq, 1, D, dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(rmm.RmmError):
-        rmm.rmm_attn_ctx(Q1, Kt, V, means, L, 0.5, 0.5, 48)  # block 48
+    with pytest.raises(rmm.RmmError):  # block 48 (the means buffer sized for it)
+        rmm.rmm_attn_ctx(Q1, Kt, V, rmm.new_ctx_means(Kt, 48), L, 0.5, 0.5, 48)
     with pytest.raises(rmm.RmmError):
         rmm.rmm_ctx_block_means(Kt, L, block, blk_begin=3, blk_end=5)  # past ceil(L / block)
 
