@@ -82,7 +82,7 @@ HEADLINE = LLAMA70
 # DRAM bytes (read + write) of one step's four GEMM launches at r = 0.5, from one
 # ncu capture of the current GEMM kernel per workload; an entry is removed whenever
 # the GEMM kernel changes, until it is captured again.
-STEP_GEMM_DRAM_BYTES = {"llama3-8b": 361_726_464}
+STEP_GEMM_DRAM_BYTES = {}
 
 
 def load_peaks():
