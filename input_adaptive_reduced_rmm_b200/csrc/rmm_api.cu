@@ -334,6 +334,59 @@ rmm_status linear_group(const void* X, int T, int H, double r, int count, const 
 }
 
 }  // namespace
+
+// A 3-D tiled map over a bf16 tensor [n2][n1][n0] (innermost n0, row stride
+// ld1 elements, plane stride ld2 elements): box = 64 x box1 x 1 elements,
+// 128-byte swizzle; loads read zeros outside the tensor.  Cached like the
+// 2-D maps.
+bool tiled_map_3d(const void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint64_t ld1, uint64_t ld2,
+                  uint32_t box1, CUtensorMap* out) {
+    struct Key3 {
+        const void* ptr;
+        uint64_t n0, n1, n2, ld1, ld2, box1;
+        bool operator==(const Key3& o) const {
+            return ptr == o.ptr && n0 == o.n0 && n1 == o.n1 && n2 == o.n2 && ld1 == o.ld1 && ld2 == o.ld2 &&
+                   box1 == o.box1;
+        }
+    };
+    struct Hash3 {
+        size_t operator()(const Key3& k) const {
+            size_t h = std::hash<const void*>()(k.ptr);
+            h ^= std::hash<uint64_t>()(((k.n0 * 1000003ull + k.n1) * 7919ull + k.n2) * 31ull + k.ld1 * 131ull +
+                                       k.ld2 * 17ull + k.box1) + 0x9e3779b9 + (h << 6) + (h >> 2);
+            return h;
+        }
+    };
+    static std::mutex mu;
+    static std::unordered_map<Key3, CUtensorMap, Hash3> cache;
+    const Key3 key{base, n0, n1, n2, ld1, ld2, box1};
+    {
+        std::lock_guard<std::mutex> g(mu);
+        auto it = cache.find(key);
+        if (it != cache.end()) {
+            *out = it->second;
+            return true;
+        }
+    }
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    CUtensorMap m;
+    memset(&m, 0, sizeof m);
+    const cuuint64_t dims[3] = {n0, n1, n2};
+    const cuuint64_t strides[2] = {ld1 * sizeof(uint16_t), ld2 * sizeof(uint16_t)};
+    const cuuint32_t box[3] = {64, box1, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    std::lock_guard<std::mutex> g(mu);
+    if (cache.size() > 4096) cache.clear();
+    cache[key] = m;
+    *out = m;
+    return true;
+}
+
 }  // namespace rmm
 
 using namespace rmm;

@@ -30,9 +30,10 @@
 //   8    MMA: one thread keeps two S blocks ahead of the softmax and issues
 //        P_j V_j as soon as P_j is written; tcgen05.commit releases buffers.
 //   9-11 producers: the query tile once (kept dims gathered), then per key
-//        block the kp kept rows of K^T and 128 rows of V with 16-byte
-//        cp.async (zero-filled past the valid keys), three stages (two when
-//        128 kept dims leave no room).
+//        block the kp kept rows of K^T with 16-byte cp.async (zero-filled past
+//        the valid keys) and the 128 x 128 V tile with two TMA tile loads
+//        (a 3-D map over [head][key][dim]: keys past L read as zero), three
+//        stages (two when 128 kept dims leave no room).
 // Every wait is bounded: on expiry the kernel records RMM_ERR_TIMEOUT, every
 // role leaves its loop, in-flight tensor-core work drains, TMEM is freed.
 #include <math.h>
@@ -172,9 +173,10 @@ __device__ __forceinline__ float row_exp64(uint32_t scol, int key0, int L, int c
 }
 
 __global__ void __launch_bounds__(kThreadsTc, 1)
-    attn_tc_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ Kt, const uint16_t* __restrict__ V,
-                   int Hq, int Hkv, int T, int L, int ldL, int k, int kp, int causal, float scale_log2,
-                   int per_query_head, const int32_t* __restrict__ idx, uint16_t* __restrict__ O, int* status) {
+    attn_tc_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ Kt,
+                   const __grid_constant__ CUtensorMap vmap, int Hq, int Hkv, int T, int L, int ldL, int k, int kp,
+                   int causal, float scale_log2, int per_query_head, const int32_t* __restrict__ idx,
+                   uint16_t* __restrict__ O, int* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -209,7 +211,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (tid == 0) {
         mbar_init(smem_addr(&bars->q_full), kProdThreads);
         for (int s = 0; s < ks; ++s) {
-            mbar_init(smem_addr(&bars->kv_full[s]), kProdThreads);
+            // the producers' cp.async arrivals + one arrival that expects the V tile's bytes
+            mbar_init(smem_addr(&bars->kv_full[s]), kProdThreads + 1);
             mbar_init(smem_addr(&bars->kv_empty[s]), 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -232,6 +235,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
+    if (tid == 32 * (kMmaWarp + 1)) tma_prefetch_desc(&vmap);
     pdl_wait();  // Q, the caches and the kept sets come from the preceding kernels
     pdl_launch_dependents();
 
@@ -267,13 +271,23 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         fence_proxy_async_smem();
         mbar_arrive(smem_addr(&bars->q_full));
         const uint16_t* Kg = Kt + ((size_t)b * Hkv + g) * D * ldL;
-        const uint16_t* Vg = V + ((size_t)b * Hkv + g) * ldL * D;
+        const int vplane = b * Hkv + g;
+        int issued = 0;  // key blocks whose loads were issued
         for (int j = 0; j < nkb; ++j) {
             const int s = j % ks;
             const uint32_t ph = (uint32_t)(j / ks) & 1u;
             if (!mbar_wait(smem_addr(&bars->kv_empty[s]), ph ^ 1u, status, abort_flag)) break;
             const int kb0 = j * BKV;
-            const uint32_t kst = smem_addr(sK + s * QK_BYTES), vst = smem_addr(sV + s * V_BYTES);
+            const uint32_t full = smem_addr(&bars->kv_full[s]);
+            if (pt == 0) {
+                // V: two 64-dim x 128-key boxes, the swizzled layout the P.V MMA reads
+                // (keys past L are outside the map and read as zero; P is 0 there)
+                mbar_arrive_expect_tx(full, V_BYTES);
+                const uint32_t vst = smem_addr(sV + s * V_BYTES);
+                tma_load_3d(vst, &vmap, full, 0, kb0, vplane);
+                tma_load_3d(vst + V_CHUNK, &vmap, full, 64, kb0, vplane);
+            }
+            const uint32_t kst = smem_addr(sK + s * QK_BYTES);
             for (int it = pt; it < kp * 16; it += kProdThreads) {
                 const int jr = it >> 4, c16 = it & 15;
                 const int key = kb0 + c16 * 8;
@@ -281,15 +295,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 const bool ok = dim >= 0 && key < ldL;
                 cp_async_16(kst + swz(jr, c16, kp * 128), ok ? Kg + (size_t)dim * ldL + key : Kg, ok ? 16u : 0u);
             }
-            for (int it = pt; it < BKV * 16; it += kProdThreads) {
-                const int kr = it >> 4, c16 = it & 15;
-                const int key = kb0 + kr;
-                const bool ok = key < L;  // V past the valid keys reads as zero (P is 0 there)
-                cp_async_16(vst + swz(kr, c16, V_CHUNK), ok ? Vg + (size_t)key * D + c16 * 8 : Vg, ok ? 16u : 0u);
-            }
-            cp_async_arrive_noinc(smem_addr(&bars->kv_full[s]));
+            cp_async_arrive_noinc(full);
+            issued = j + 1;
         }
         cp_async_wait_all();
+        // no V tile may still be landing in shared memory when the CTA leaves
+        // (after an abort; otherwise every issued block was consumed): wait,
+        // bounded, for the last phase of each stage that was issued
+        if (pt == 0) {
+            volatile int no_abort = 0;
+            for (int j = max(0, issued - ks); j < issued; ++j)
+                mbar_wait(smem_addr(&bars->kv_full[j % ks]), (uint32_t)(j / ks) & 1u, status, &no_abort);
+        }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         bool ok = __all_sync(0xffffffffu, mbar_wait(smem_addr(&bars->q_full), 0, status, abort_flag));
@@ -484,10 +501,14 @@ cudaError_t launch_attn_tc(const uint16_t* Q, const uint16_t* Kt, const uint16_t
                            uint16_t* O, int* status, cudaStream_t stream) {
     const int kp = (k + 15) / 16 * 16;
     const size_t smem = attn_tc_smem_bytes(kp);
+    // V [B * Hkv][ldL][d] as [plane][key][dim], only the L valid keys of a plane
+    CUtensorMap vmap;
+    if (!tiled_map_3d(V, D, (uint64_t)L, (uint64_t)B * Hkv, D, (uint64_t)ldL * D, BKV, &vmap))
+        return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem_limit(attn_tc_kernel, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(Hq, (T + BQ - 1) / BQ, B);
-    return launch_pdl(attn_tc_kernel, grid, dim3(kThreadsTc), smem, stream, Q, Kt, V, Hq, Hkv, T, L, ldL, k, kp,
+    return launch_pdl(attn_tc_kernel, grid, dim3(kThreadsTc), smem, stream, Q, Kt, vmap, Hq, Hkv, T, L, ldL, k, kp,
                       causal, scale * 1.4426950408889634f, per_query_head, idx, O, status);
 }
 

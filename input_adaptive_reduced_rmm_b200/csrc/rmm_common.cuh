@@ -241,6 +241,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// A 3-D tile load (box from the map) into shared memory at coordinates (c0
+// innermost, c1, c2), completing `bytes` of transaction on the barrier.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                            int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+        : "memory");
+}
+
 // A 2-D tile store (box from the map) from shared memory at coordinates (c0
 // innermost, c1); elements outside the tensor are not written.  The source
 // must be visible to the async proxy (fence_proxy_async_smem) first.

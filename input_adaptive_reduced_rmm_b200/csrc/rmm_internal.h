@@ -71,6 +71,11 @@ cudaError_t launch_gemv(const uint16_t* X, int T, int H, const int32_t* idx, int
 // least kAttnTcMinT tokens, kept sets from the attention select kernel
 constexpr int kAttnTcMinT = 16;
 bool attn_tc_supported(int T, int k);
+// A 3-D tiled map over a bf16 tensor [n2][n1][n0] with row / plane strides ld1 /
+// ld2 elements, box 64 x box1 x 1, 128-byte swizzle, zero fill outside
+// (defined in rmm_api.cu).
+bool tiled_map_3d(const void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint64_t ld1, uint64_t ld2,
+                  uint32_t box1, CUtensorMap* out);
 cudaError_t launch_exp2_fma(const float* x, float* y, int n, cudaStream_t stream);
 cudaError_t launch_attn_tc(const uint16_t* Q, const uint16_t* Kt, const uint16_t* V, int B, int Hq, int Hkv, int T,
                            int L, int ldL, int k, int causal, float scale, int per_query_head, const int32_t* idx,
