@@ -82,7 +82,7 @@ HEADLINE = LLAMA70
 # DRAM bytes (read + write) of one step's four GEMM launches at r = 0.5, from one
 # ncu capture of the current GEMM kernel per workload; an entry is removed whenever
 # the GEMM kernel changes, until it is captured again.
-STEP_GEMM_DRAM_BYTES = {}
+STEP_GEMM_DRAM_BYTES = {"llama3-8b": 361_726_464, "llama3-70b": 2_843_581_696}
 
 
 def load_peaks():
@@ -921,6 +921,31 @@ def run_profile_step(args):
                                        "launches_per_step": launches_per_step(wl, R, dev)}}), flush=True)
 
 
+def run_profile_decode(args):
+    """The decode step (T = 1, the seven projections of --profile-decode's workload, grouped
+    like the prefill step) eagerly, --warmup then --steps times (profiling aid)."""
+    from input_adaptive_reduced_rmm_b200 import rmm
+
+    wl = {"llama3-8b": LLAMA8, "llama3-70b": LLAMA70}[args.profile_decode]
+    dev = torch.device("cuda", 0)
+    acts = {s: rmm_synth.activations(1, h, 500 + s, device=dev) for s, h in wl.act_h.items()}
+    Wts = {n: rmm.rmm_transpose_weight(rmm_synth.weights(N, h, 600 + i, std=0.02, device=dev))
+           for i, (n, h, N, _) in enumerate(wl.proj)}
+    Ys = {n: torch.empty(1, N, dtype=torch.bfloat16, device=dev) for n, h, N, _ in wl.proj}
+    ws = {c: rmm.new_workspace(rmm.rmm_linear_group_workspace_bytes(
+        1, wl.act_h[s], [wl.shape[n][1] for n in names]), dev) for c, (s, names) in enumerate(CALLS)}
+
+    def step():
+        for c, (s, names) in enumerate(CALLS):
+            rmm.rmm_linear_group(acts[s], [Wts[n] for n in names], R, Ys=[Ys[n] for n in names], workspace=ws[c])
+
+    ms = time_steps(step, args.steps, args.warmup)
+    for c in ws:
+        if rmm.rmm_get_status(ws[c]) != rmm.RMM_OK:
+            raise RuntimeError("device status not OK (decode profile)")
+    print(json.dumps({"profile_decode": {"workload": wl.label, "ms_per_step_eager": ms}}), flush=True)
+
+
 def run_single(args):
     """One rmm_linear shape timed alone (profiling aid): --single T,H,N,r."""
     from input_adaptive_reduced_rmm_b200 import rmm
@@ -1040,6 +1065,8 @@ def main():
     ap.add_argument("--single-ctx", default=None,
                     help="B,Hq,Hkv,L,block,r,r_ctx: time one rmm_attn_ctx decode call alone")
     ap.add_argument("--profile-step", action="store_true", help="run only the headline step (profiling aid)")
+    ap.add_argument("--profile-decode", default=None, choices=["llama3-8b", "llama3-70b"],
+                    help="run only the decode (T = 1) step of that workload, eagerly (profiling aid)")
     ap.add_argument("--gemm-producer", type=int, default=0)
     ap.add_argument("--block-size", type=int, default=0, help="with --single: block-granular kept sets")
     args = ap.parse_args()
@@ -1056,6 +1083,9 @@ def main():
         return
     if args.profile_step:
         run_profile_step(args)
+        return
+    if args.profile_decode:
+        run_profile_decode(args)
         return
     if args.impl == "reference":
         # the oracle on the host cores: rank 0 alone, no process group, no GPU
