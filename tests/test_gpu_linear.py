@@ -53,8 +53,11 @@ def test_score_bit_exact(rmm, T, H, kind):
     assert np.array_equal(s.cpu().numpy().astype(np.uint32), oracle.score(X).astype(np.uint32))
 
 
-@pytest.mark.parametrize("H", [1, 2, 7, 12, 64, 65, 127, 128, 129, 1000, 4096, 14336, 28672, 65535])
+@pytest.mark.parametrize("H", [1, 2, 7, 12, 64, 65, 127, 128, 129, 1000, 4096, 14336, 16384, 16385, 20001, 28672,
+                               40961, 65535])
 def test_select_bit_exact(rmm, H):
+    """One CTA up to H = 16384, a cluster of CTAs above (16385: 8 slices of 2049 keys,
+    the last one short; 20001 and 40961: ragged slices)."""
     rng = np.random.default_rng(H)
     for trial in range(3):
         if trial == 0:
