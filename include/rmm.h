@@ -97,6 +97,16 @@ typedef struct rmm_options {
      * slices ascending, then one correctly rounded division by T*block_size).
      * 1 requires T <= 16 (RMM_ERR_UNSUPPORTED otherwise). */
     int block_score;
+    /* Gated-MLP epilogue for a group of two products of the same width (gate
+     * and up of a SwiGLU MLP, the gated FFN of the cf-1.com post §6.1):
+     * nonzero makes rmm_linear_group write Ys[0][t,n] = bf16(silu(g) * u) with
+     * g = bf16(Y_gate[t,n]), u = bf16(Y_up[t,n]), silu(z) = z / (1 + e^-z), the
+     * same bits as rmm_swiglu applied to the two products; Ys[1] serves as
+     * scratch (its contents unspecified).  On the split-K GEMV path the fold
+     * of the split partial sums applies it (no extra launch); otherwise the
+     * SwiGLU kernel runs after the products.  Requires count == 2 and
+     * Ns[0] == Ns[1] (RMM_ERR_INVALID_ARG otherwise). */
+    int swiglu_pair;
     /* Optional pair of cudaEvent_t handles (NULL: none) recorded on the
      * stream immediately before and after the reduced-product kernel (GEMV or
      * GEMM) of rmm_linear / rmm_gemm_reduced, so that a caller can time that

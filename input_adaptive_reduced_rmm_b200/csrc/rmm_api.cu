@@ -54,7 +54,7 @@ int num_sms_current() {
 }
 
 const rmm_options& opts_or_default(const rmm_options* o) {
-    static const rmm_options d = {16, 0, 0, 0, 0, 0, 0, 0, nullptr, nullptr};
+    static const rmm_options d = {16, 0, 0, 0, 0, 0, 0, 0, 0, nullptr, nullptr};
     return o ? *o : d;
 }
 
@@ -66,6 +66,7 @@ bool opts_valid(const rmm_options* o) {
     if (o->attn_path < 0 || o->attn_path > 2) return false;
     if (o->block_size < 0) return false;
     if (o->block_score < 0 || o->block_score > 1 || (o->block_score == 1 && o->block_size == 0)) return false;
+    if (o->swiglu_pair < 0 || o->swiglu_pair > 1) return false;
     return true;
 }
 
@@ -204,15 +205,30 @@ rmm_status run_product_kernels(const void* X, int T, int H, int count, const voi
                                cudaStream_t s) {
     int* status = reinterpret_cast<int*>(ws);
     const int sms = num_sms_current();
+    // the gated-MLP epilogue when it is not fused into the GEMV fold:
+    // Ys[0] = bf16(silu(Ys[0]) * Ys[1]) after the products
+    auto swiglu_after = [&]() -> rmm_status {
+        return cuda_status(launch_swiglu(static_cast<const uint16_t*>(Ys[0]), static_cast<const uint16_t*>(Ys[1]),
+                                         (size_t)T * Ns[0], static_cast<uint16_t*>(Ys[0]), sms, s));
+    };
     if (L.gemv) {
         GemvGroup g = L.plan;
         for (int p = 0; p < count; ++p) {
             g.Wt[p] = static_cast<const uint16_t*>(Wts[p]);
             g.Y[p] = static_cast<uint16_t*>(Ys[p]);
         }
+        g.swiglu = o.swiglu_pair;  // fused into the fold of the split partials
         (void)status;
-        return cuda_status(launch_gemv(static_cast<const uint16_t*>(X), T, H, idx_padded, k, g,
-                                       reinterpret_cast<float*>(ws + L.partials), sms, s));
+        rmm_status st = cuda_status(launch_gemv(static_cast<const uint16_t*>(X), T, H, idx_padded, k, g,
+                                                reinterpret_cast<float*>(ws + L.partials), sms, s));
+        if (st == RMM_OK && o.swiglu_pair && g.splits[0] == 1) st = swiglu_after();  // no fold to fuse into
+        return st;
+    }
+    if (o.swiglu_pair) {
+        rmm_options o2 = o;
+        o2.swiglu_pair = 0;
+        rmm_status st = run_product_kernels(X, T, H, count, Wts, Ns, Ys, idx_padded, k, ws, L, o2, s);
+        return st == RMM_OK ? swiglu_after() : st;
     }
     if (o.gemm_producer == 1 && count != 1) return RMM_ERR_UNSUPPORTED;
     GemmGroup g;
@@ -285,6 +301,7 @@ rmm_status linear_group(const void* X, int T, int H, double r, int count, const 
                         size_t workspace_bytes, rmm_stream_t stream, const rmm_options* options) {
     if (!group_args_ok(X, T, H, count, Wts, Ns, Ys) || !opts_valid(options)) return RMM_ERR_INVALID_ARG;
     const rmm_options& o = opts_or_default(options);
+    if (o.swiglu_pair && (count != 2 || Ns[0] != Ns[1])) return RMM_ERR_INVALID_ARG;
     const int bsz = o.block_size;
     if (!block_size_ok(H, bsz)) return RMM_ERR_UNSUPPORTED;
     const bool mean_blocks = bsz > 0 && o.block_score == 1;
@@ -315,8 +332,11 @@ rmm_status linear_group(const void* X, int T, int H, double r, int count, const 
         if (e == cudaSuccess && pad_to > k) e = launch_pad_idx(idx, k, H, idx, pad_to, s);
     } else if (L.gemv && k == H) {
         // every slice kept (ratio 1): the kept list is 0..H-1 whatever the
-        // scores, so neither score nor select runs
-        e = launch_pad_idx(nullptr, k, H, idx, pad_to, s, idx_out);
+        // scores, so neither score nor select runs, and the GEMV reads the
+        // identity list implicitly; the list is written only when asked for
+        e = idx_out ? launch_pad_idx(nullptr, k, H, idx, pad_to, s, idx_out) : cudaSuccess;
+        if (e != cudaSuccess) return RMM_ERR_CUDA;
+        return run_products(X, T, H, count, Wts, Ns, Ys, nullptr, k, ws, L, o, s);
     } else if (L.gemv && T == 1) {
         // one token: the select kernel reads the score straight from X
         e = launch_select(static_cast<const uint16_t*>(X), T, nullptr, 0, H, k, idx, pad_to, idx_out, nullptr, s);
@@ -501,6 +521,7 @@ rmm_status rmm_gemm_reduced(const void* X, const void* Wt, const int32_t* idx, i
     if (!group_args_ok(X, T, H, 1, Wts, &N, Ys) || !idx || k < 1 || k > H || !opts_valid(options))
         return RMM_ERR_INVALID_ARG;
     const rmm_options& o = opts_or_default(options);
+    if (o.swiglu_pair) return RMM_ERR_INVALID_ARG;  // a pair epilogue needs a group of two
     const int sms = num_sms_current();
     const LinearLayout L = linear_layout(T, H, &N, 1, k, o, sms);
     if (!workspace || workspace_bytes < L.total || !aligned16(workspace)) return RMM_ERR_WORKSPACE;

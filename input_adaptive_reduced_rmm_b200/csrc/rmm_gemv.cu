@@ -123,8 +123,8 @@ __global__ void __launch_bounds__(kThreads, (TT <= 4) ? 3 : 1)
     const int nr = max(0, min(k, j0 + rows) - j0);
     const int n0 = cb * COLS;
 
-    // 1. the split's kept indices
-    for (int i = tid; i < nr; i += kThreads) sidx[i] = __ldg(idx + j0 + i);
+    // 1. the split's kept indices (idx null: every slice kept, the identity list)
+    for (int i = tid; i < nr; i += kThreads) sidx[i] = idx ? __ldg(idx + j0 + i) : j0 + i;
     __syncthreads();
 
     // 2. the first batch of weight pieces in flight, then the X values beside them
@@ -224,17 +224,12 @@ __global__ void __launch_bounds__(kThreads, (TT <= 4) ? 3 : 1)
 // columns of one member and one token; its 8 thread groups take consecutive
 // ranges of the splits (four splits' loads in flight at a time) and the range
 // sums are added in range order.
-__global__ void __launch_bounds__(kThreads)
-    gemv_fold_kernel(const __grid_constant__ GemvGroup g, int T, const float* __restrict__ partials) {
-    __shared__ float4 gs[kFoldGroups][kFoldCols / 8][2];
-    pdl_wait();
-    pdl_launch_dependents();
-    const int tid = threadIdx.x;
-    const int p = member_of(g.fold_start, g.count, blockIdx.x);
-    const int c = tid % (kFoldCols / 8);
-    const int n = (blockIdx.x - g.fold_start[p]) * kFoldCols + c * 8;
-    const int grp = tid / (kFoldCols / 8);
-    const int t = blockIdx.y;
+// With g.swiglu the grid covers member 0's column blocks and each CTA folds
+// both members at the same columns, then writes Y[0] = bf16(silu(g) * u) from
+// the bf16-rounded gate and up values (the arithmetic of swiglu_kernel).
+__device__ __forceinline__ void fold_member(const GemvGroup& g, int p, int t, int n, int c, int grp, int T,
+                                            const float* __restrict__ partials, float4 (*gs)[kFoldCols / 8][2],
+                                            float (&tot)[8]) {
     const int N = g.N[p], S = g.splits[p];
     const bool live = n < N;
     float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -263,16 +258,46 @@ __global__ void __launch_bounds__(kThreads)
     gs[grp][c][0] = make_float4(s[0], s[1], s[2], s[3]);
     gs[grp][c][1] = make_float4(s[4], s[5], s[6], s[7]);
     __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) tot[e] = 0.f;
     if (grp == 0 && live) {
-        float tot[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int q = 0; q < kFoldGroups; ++q) {
             const float4 a = gs[q][c][0], d = gs[q][c][1];
             tot[0] += a.x; tot[1] += a.y; tot[2] += a.z; tot[3] += a.w;
             tot[4] += d.x; tot[5] += d.y; tot[6] += d.z; tot[7] += d.w;
         }
-        store_bf16x8(g.Y[p] + (size_t)t * g.ld[p] + n, tot);
     }
+    __syncthreads();  // gs may be reused by the next member
+}
+
+__global__ void __launch_bounds__(kThreads)
+    gemv_fold_kernel(const __grid_constant__ GemvGroup g, int T, const float* __restrict__ partials) {
+    __shared__ float4 gs[kFoldGroups][kFoldCols / 8][2];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int tid = threadIdx.x;
+    const int p = member_of(g.fold_start, g.count, blockIdx.x);
+    const int c = tid % (kFoldCols / 8);
+    const int n = (blockIdx.x - g.fold_start[p]) * kFoldCols + c * 8;
+    const int grp = tid / (kFoldCols / 8);
+    const int t = blockIdx.y;
+    const bool live = n < g.N[p];
+    float tot[8];
+    fold_member(g, p, t, n, c, grp, T, partials, gs, tot);
+    if (g.swiglu) {
+        float up[8];
+        fold_member(g, 1, t, n, c, grp, T, partials, gs, up);
+        if (grp == 0 && live) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float gv = bf16_bits_to_float(float_to_bf16_bits(tot[e]));
+                const float uv = bf16_bits_to_float(float_to_bf16_bits(up[e]));
+                tot[e] = gv / (1.0f + expf(-gv)) * uv;
+            }
+        }
+    }
+    if (grp == 0 && live) store_bf16x8(g.Y[p] + (size_t)t * g.ld[p] + n, tot);
 }
 
 template <int TT>
@@ -290,8 +315,9 @@ cudaError_t launch_tt(const uint16_t* X, int T, int H, const int32_t* idx, int k
     e = launch_pdl(kern, dim3(g.item_start[g.count], g.splits[0]), dim3(kThreads), smem, stream, X, T, H, idx, k, g,
                    partials);
     if (e != cudaSuccess || g.splits[0] == 1) return e;
-    return launch_pdl(gemv_fold_kernel, dim3(g.fold_start[g.count], T), dim3(kThreads), 0, stream, g, T,
-                      static_cast<const float*>(partials));
+    // with the SwiGLU epilogue only member 0's column blocks (each folds both members)
+    return launch_pdl(gemv_fold_kernel, dim3(g.fold_start[g.swiglu ? 1 : g.count], T), dim3(kThreads), 0, stream, g,
+                      T, static_cast<const float*>(partials));
 }
 
 // Splits before rounding to whole rows; never decreases as k grows.  Measured

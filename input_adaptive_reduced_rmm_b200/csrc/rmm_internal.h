@@ -54,6 +54,7 @@ struct GemvGroup {
     size_t partial_off[kMaxGroupGemv];  // float offsets of each member's split partials
     int cols;                           // outputs per column block
     int count;
+    int swiglu;                         // 1: members 0 and 1 are gate and up; Y[0] = bf16(silu(g) * u)
 };
 int gemv_cols_for(int T);
 // Fills the plan; returns the bytes of split partial sums the group needs.
@@ -64,6 +65,7 @@ size_t gemv_smem_bytes(int cols, int T);  // dynamic shared memory of one CTA
 constexpr size_t kGemvMaxSmemBytes = 200 * 1024;
 // The product (and, with more than one split, the fold of the split partials
 // in a second launch).  partials: the planned bytes, no initial contents.
+// idx null: every slice kept (k == H), read as the identity list.
 cudaError_t launch_gemv(const uint16_t* X, int T, int H, const int32_t* idx, int k, const GemvGroup& g,
                         float* partials, int num_sms, cudaStream_t stream);
 

@@ -8,9 +8,10 @@ the current token); §6.2: the down projection's work drops with the keep
 ratio while gate and up stay full.  The demo's sizes are H = 1024, M = 4096.
 
 Every op runs in the package's kernels through the C ABI: gate and up as one
-reduced-product group at ratio 1 (every slice kept: the full products), the
-SwiGLU kernel, then the down projection with mean-magnitude block-granular
-kept sets.  This module only sequences the calls and owns the buffers.
+reduced-product group at ratio 1 (every slice kept: the full products) with
+the SwiGLU applied as the split products are folded (or, unfused, the SwiGLU
+kernel after them), then the down projection with mean-magnitude
+block-granular kept sets.  This module only sequences the calls and owns the buffers.
 """
 from __future__ import annotations
 
@@ -27,7 +28,7 @@ class FfnBlockReduce:
     [kb], h [T, M])."""
 
     def __init__(self, W_gate: torch.Tensor, W_up: torch.Tensor, W_down: torch.Tensor, block: int = 64,
-                 keep: float = 0.5):
+                 keep: float = 0.5, fused_swiglu: bool = True):
         self.M, self.H = W_gate.shape
         if W_up.shape != (self.M, self.H) or W_down.shape != (self.H, self.M):
             raise ValueError("gate/up must be [M, H] and down [H, M]")
@@ -37,6 +38,10 @@ class FfnBlockReduce:
         self.Wd_t = rmm.rmm_transpose_weight(W_down)
         self.kb = rmm.rmm_k_for(self.M // self.block, self.keep)
         self.opts_down = rmm.options(block_size=self.block, block_score=1)
+        # gate and up with the SwiGLU applied as they are folded (h written directly;
+        # the up buffer is scratch), or the three steps one by one (gate, up kept)
+        self.fused = bool(fused_swiglu)
+        self.opts_gu = rmm.options(swiglu_pair=True) if self.fused else None
         self._bufs = {}
 
     def _buffers(self, T: int, dev):
@@ -53,14 +58,21 @@ class FfnBlockReduce:
             self._bufs[T] = b
         return self._bufs[T]
 
-    def forward(self, x: torch.Tensor):
+    def forward(self, x: torch.Tensor, want_blocks: bool = True):
+        """(y, kept blocks, h); want_blocks=False returns (y, None, h) and launches nothing
+        beyond the FFN itself (the kept block ids are derived from the kept slices by a
+        tensor op)."""
         T = x.shape[0]
         b = self._buffers(T, x.device)
-        rmm.rmm_linear_group(x, [self.Wg_t, self.Wu_t], 1.0, Ys=[b["gate"], b["up"]], workspace=b["ws_gu"])
-        rmm.rmm_swiglu(b["gate"], b["up"], out=b["h"])
+        if self.fused:
+            rmm.rmm_linear_group(x, [self.Wg_t, self.Wu_t], 1.0, Ys=[b["h"], b["up"]], workspace=b["ws_gu"],
+                                 opts=self.opts_gu)
+        else:
+            rmm.rmm_linear_group(x, [self.Wg_t, self.Wu_t], 1.0, Ys=[b["gate"], b["up"]], workspace=b["ws_gu"])
+            rmm.rmm_swiglu(b["gate"], b["up"], out=b["h"])
         rmm.rmm_linear(b["h"], self.Wd_t, self.keep, Y=b["y"], idx_out=b["idx"], workspace=b["ws_d"],
                        opts=self.opts_down)
-        blocks = b["idx"].view(self.kb, self.block)[:, 0] // self.block
+        blocks = b["idx"].view(self.kb, self.block)[:, 0] // self.block if want_blocks else None
         return b["y"], blocks, b["h"]
 
     def forward_dense(self, x: torch.Tensor):

@@ -4,6 +4,7 @@
       -> heads + KV-cache append -> reduced attention (head-dim sets) -> o
       -> residual add + RMSNorm -> gate, up (one kept set) -> SwiGLU -> down
       -> residual add
+(without a trace, SwiGLU is applied as gate and up are produced)
 
 The anatomy (RMSNorm, a residual stream through every block, a SwiGLU MLP)
 follows the 'Numerical Linear Algebra for LLMs' paper digest (ai-feeds.com),
@@ -58,6 +59,7 @@ class DecoderLayer:
         self.pos = 0
         self._ws = {}
         self._bufs = {}
+        self._opts_swiglu = rmm.options(swiglu_pair=True)
 
     # workspaces and activations are kept per token count, so repeated calls
     # (decode steps) allocate nothing
@@ -124,13 +126,22 @@ class DecoderLayer:
             h2, xn2 = rmm.rmm_add_rmsnorm(x, yo, eps=dm.eps, Hsum=self._buf("h2", (T, H)),
                                           Y=self._buf("xn2", (T, H)))
         idx_gu = self._idx("gu", H)
-        with op("gate_up"):
-            g, u = self._buf("g", (T, F)), self._buf("u", (T, F))
-            rmm.rmm_linear_group(xn2, [self.Wt["gate"], self.Wt["up"]], r, Ys=[g, u], idx_out=idx_gu,
-                                 workspace=self._ws_for(("gu", T), rmm.rmm_linear_group_workspace_bytes(
-                                     T, H, [F, F])))
-        with op("swiglu"):
-            hh = rmm.rmm_swiglu(g, u, out=self._buf("hh", (T, F)))
+        ws_gu = self._ws_for(("gu", T), rmm.rmm_linear_group_workspace_bytes(T, H, [F, F]))
+        g, u = self._buf("g", (T, F)), self._buf("u", (T, F))
+        if trace is None:
+            # SwiGLU applied as gate/up are produced (folded into the decode GEMV's
+            # split sums; after the products on the GEMM path): hh directly, the
+            # same bits as the two steps below
+            with op("gate_up_swiglu"):
+                hh = self._buf("hh", (T, F))
+                rmm.rmm_linear_group(xn2, [self.Wt["gate"], self.Wt["up"]], r, Ys=[hh, u], idx_out=idx_gu,
+                                     workspace=ws_gu, opts=self._opts_swiglu)
+        else:
+            with op("gate_up"):
+                rmm.rmm_linear_group(xn2, [self.Wt["gate"], self.Wt["up"]], r, Ys=[g, u], idx_out=idx_gu,
+                                     workspace=ws_gu)
+            with op("swiglu"):
+                hh = rmm.rmm_swiglu(g, u, out=self._buf("hh", (T, F)))
         idx_d = self._idx("down", F)
         with op("down"):
             yd = rmm.rmm_linear(hh, self.Wt["down"], r, Y=self._buf("yd", (T, H)), idx_out=idx_d,

@@ -50,6 +50,7 @@ class rmm_options(ctypes.Structure):
         ("attn_path", ctypes.c_int),
         ("block_size", ctypes.c_int),
         ("block_score", ctypes.c_int),
+        ("swiglu_pair", ctypes.c_int),
         ("product_event_begin", ctypes.c_void_p),
         ("product_event_end", ctypes.c_void_p),
     ]
@@ -57,14 +58,16 @@ class rmm_options(ctypes.Structure):
 
 def options(t_gemv: int = 16, attn_per_query_head: bool = False, gemv_splits: int = 0,
             debug_timeout_test: bool = False, gemm_producer: int = 0, attn_path: int = 0,
-            block_size: int = 0, block_score: int = 0, product_events=None) -> rmm_options:
+            block_size: int = 0, block_score: int = 0, swiglu_pair: bool = False,
+            product_events=None) -> rmm_options:
     """An rmm_options struct; product_events = (begin, end) torch.cuda.Event pair (enable_timing);
     attn_path 0 = auto, 1 = CUDA-core split pass, 2 = tensor cores; block_size 0 = single-slice
     kept sets, else blocks of that many consecutive slices; block_score 0 = max of the slice
-    scores, 1 = mean magnitude of the block (T <= 16)."""
+    scores, 1 = mean magnitude of the block (T <= 16); swiglu_pair: for a group of two products
+    of one width (gate, up), Ys[0] receives bf16(silu(gate) * up) and Ys[1] is scratch."""
     o = rmm_options(int(t_gemv), int(bool(attn_per_query_head)), int(gemv_splits),
                     int(bool(debug_timeout_test)), int(gemm_producer), int(attn_path), int(block_size),
-                    int(block_score), None, None)
+                    int(block_score), int(bool(swiglu_pair)), None, None)
     if product_events is not None:
         b, e = product_events
         for ev in (b, e):

@@ -52,7 +52,8 @@ def test_options_struct_matches_the_header(rmm):
     assert names == [f[0] for f in rmm.rmm_options._fields_]
     o = rmm.options(block_size=64, block_score=1, attn_path=2)
     assert (o.block_size, o.block_score, o.attn_path, o.t_gemv) == (64, 1, 2, 16)
-    assert ctypes.sizeof(rmm.rmm_options) == 8 * 4 + 2 * ctypes.sizeof(ctypes.c_void_p)
+    assert ctypes.sizeof(rmm.rmm_options) == 9 * 4 + 4 + 2 * ctypes.sizeof(ctypes.c_void_p)  # 4 bytes of padding
+    assert rmm.options(swiglu_pair=True).swiglu_pair == 1
 
 
 def test_wrong_sizes_are_refused_before_the_call(rmm):

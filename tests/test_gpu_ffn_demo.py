@@ -35,11 +35,17 @@ def demo():
 @pytest.mark.parametrize("keep", [0.5, 0.25])
 def test_ffn_demo_per_op(demo, T, keep):
     cls, (Wg, Wu, Wd) = demo
-    f = cls(Wg.cuda(), Wu.cuda(), Wd.cuda(), block=BLOCK, keep=keep)
+    f = cls(Wg.cuda(), Wu.cuda(), Wd.cuda(), block=BLOCK, keep=keep, fused_swiglu=False)
     x = rmm_synth.normal((T, H), 144 + T)
     y, blocks, h = f.forward(x.cuda())
     torch.cuda.synchronize()
     b = f._bufs[T]
+    # the fused form (SwiGLU applied as gate/up are folded) gives the same h, kept blocks and y
+    ff = cls(Wg.cuda(), Wu.cuda(), Wd.cuda(), block=BLOCK, keep=keep)
+    y2, blocks2, h2 = ff.forward(x.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(h2.view(torch.int16), h.view(torch.int16))
+    assert torch.equal(blocks2, blocks) and torch.equal(y2.view(torch.int16), y.view(torch.int16))
     assert_close(b["gate"].cpu(), oracle.linear(x, Wg, 1.0)[0], "gate (full)")
     assert_close(b["up"].cpu(), oracle.linear(x, Wu, 1.0)[0], "up (full)")
     assert_close(h.cpu(), oracle.swiglu(b["gate"].cpu(), b["up"].cpu()), "swiglu")

@@ -299,3 +299,39 @@ def test_watchdog_reports_timeout_and_context_survives(rmm):
     assert rmm.rmm_get_status(ws) == rmm.RMM_OK
     Yo, _ = oracle.linear(X, W, 0.5)
     assert_close(Y.cpu(), Yo, "after watchdog")
+
+
+# ---------------------------------------------------------------- gated-MLP epilogue
+
+@pytest.mark.parametrize("T,r,splits", [(1, 1.0, 0), (1, 0.5, 0), (4, 0.5, 0), (16, 0.25, 0), (1, 0.5, 1),
+                                        (40, 0.5, 0), (300, 1.0, 0)])
+def test_swiglu_pair_epilogue_matches_the_two_steps(rmm, T, r, splits):
+    """options.swiglu_pair on a gate/up group writes the same bits as the two products followed
+    by rmm_swiglu: fused into the fold of the split-K GEMV (T <= 16), run after the products
+    when the GEMV has one split (nothing to fold) and on the tensor-core GEMM path."""
+    H, F = 1024, 3072
+    X = rmm_synth.activations(T, H, rmm_synth.seed_for(1, 170 + T, 0)).cuda()
+    Wg = rmm.rmm_transpose_weight(rmm_synth.weights(F, H, 171, std=0.02).cuda())
+    Wu = rmm.rmm_transpose_weight(rmm_synth.weights(F, H, 172, std=0.02).cuda())
+    g, u = rmm.rmm_linear_group(X, [Wg, Wu], r, opts=rmm.options(gemv_splits=splits))
+    ref = rmm.rmm_swiglu(g, u)
+    h = torch.full((T, F), float("nan"), dtype=torch.bfloat16, device="cuda")
+    scratch = torch.empty(T, F, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(rmm.rmm_k_for(H, r), dtype=torch.int32, device="cuda")
+    rmm.rmm_linear_group(X, [Wg, Wu], r, Ys=[h, scratch], idx_out=idx,
+                         opts=rmm.options(gemv_splits=splits, swiglu_pair=True))
+    torch.cuda.synchronize()
+    assert torch.equal(h.view(torch.int16), ref.view(torch.int16))
+    assert np.array_equal(idx.cpu().numpy(), oracle.select(oracle.score(X.cpu()), rmm.rmm_k_for(H, r)))
+
+
+def test_swiglu_pair_needs_a_pair_of_equal_widths(rmm):
+    X = torch.zeros(1, 64, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
+    W2 = torch.zeros(64, 32, dtype=torch.bfloat16, device="cuda")
+    o = rmm.options(swiglu_pair=True)
+    for Wts in ([W], [W, W2], [W, W, W]):
+        with pytest.raises(rmm.RmmError):
+            rmm.rmm_linear_group(X, Wts, 0.5, opts=o)
+    with pytest.raises(rmm.RmmError):
+        rmm.rmm_gemm_reduced(X, W, torch.arange(8, dtype=torch.int32, device="cuda"), opts=o)
