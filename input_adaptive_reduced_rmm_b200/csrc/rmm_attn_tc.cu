@@ -15,16 +15,18 @@
 // Operands in shared memory, 128-byte swizzled: the gathered query tile and
 // the key block are MN-major (a kept dim is one row of 128 tokens / keys --
 // the d-major key cache makes each kept dim of a key block one contiguous
-// 256-byte segment); V blocks are MN-major (a key is one row of d values);
-// P is written by the softmax threads as a K-major operand (each thread owns
-// one query row).  TMEM holds two S buffers (columns 0-127, 128-255) and O
-// (256-383).
+// 256-byte segment); V blocks are MN-major (a key is one row of d values).
+// TMEM holds two S buffers (columns 0-127, 128-255), O (256-383) and P
+// (384-447): the softmax threads write P_j there, two bf16 keys per 32-bit
+// column, each thread its own row, and the P.V product reads it as its A
+// operand straight from tensor memory (K-major by definition), so P never
+// passes through shared memory.
 //
 // Warp roles (384 threads):
 //   0-7  softmax: warps q and q+4 own query rows 32q .. 32q+31 (their TMEM
 //        lanes), one row per thread, and split the 128 columns; reads S_j,
-//        masks, keeps a running reference max m and sum l; P_j to shared
-//        memory.  O is rescaled in TMEM only when a row's block max exceeds m
+//        masks, keeps a running reference max m and sum l; P_j to TMEM.
+//        O is rescaled in TMEM only when a row's block max exceeds m
 //        by more than 2^8 (the reference max is then raised), so P stays below
 //        256 and most blocks need no rescale.  At the end O / l goes to HBM.
 //   8    MMA: one thread keeps two S blocks ahead of the softmax and issues
@@ -48,7 +50,7 @@ namespace {
 constexpr int D = 128;
 constexpr int BQ = 128;   // query rows per CTA (= TMEM lanes)
 constexpr int BKV = 128;  // keys per block
-constexpr int KV_STAGES_MAX = 3;  // key/value stages: 3 when they fit (kp <= 96), else 2
+constexpr int KV_STAGES_MAX = 3;  // key/value stages: 3 when they fit with the static arrays (kp <= 112), else 2
 constexpr int kSoftmaxWarps = 8;  // two per TMEM lane quarter, each on 64 of the 128 columns
 constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
 constexpr int kMmaWarp = kSoftmaxWarps;
@@ -57,10 +59,8 @@ constexpr int kProdThreads = 32 * kProdWarps;
 constexpr int kThreadsTc = 32 * (kSoftmaxWarps + 1 + kProdWarps);  // 12 warps: three per SM sub-partition
 constexpr int V_CHUNK = BKV * 128;     // 64 dims x 128 key rows (bytes)
 constexpr int V_BYTES = 2 * V_CHUNK;   // 32 KB
-constexpr int P_ATOM = BQ * 128;       // 128 rows x 64 keys (bytes)
-constexpr int P_BYTES = 2 * P_ATOM;    // 32 KB
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_S0 = 0, TM_O = 256;
+constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_P = 384;  // P: 128 keys as 64 packed columns
 constexpr float kRescaleLog2 = 8.0f;   // rescale O when a block max exceeds the reference by 2^8
 
 struct __align__(8) Bars {
@@ -139,17 +139,18 @@ __device__ __forceinline__ float row_max64(uint32_t scol, int key0, int L, int c
 }
 
 // Softmax pass 2 for the same 64 columns: p = 2^(s * scale_log2 - m) (one FMA
-// and one hardware exp2; masked logits give 0), their sum, and P (bf16) as
-// one 64-key atom of the K-major A operand: row i at prow, 16-byte chunks
-// XOR-swizzled by row.
+// and an exponential, half of them on the FMA pipe; masked logits give 0),
+// their sum, and P (bf16) into the 32 TMEM columns at pcol of the row's lane
+// (column c holds keys 2c and 2c+1 of the 64), written 32 keys at a time.
 template <bool kMask>
 __device__ __forceinline__ float row_exp64(uint32_t scol, int key0, int L, int causal, int pos, float scale_log2,
-                                           float neg_m, uint32_t prow, int i) {
+                                           float neg_m, uint32_t pcol) {
     uint32_t r[2][32];
     tmem_ld_32x32b_x32(scol, r[0]);
     tmem_ld_32x32b_x32(scol + 32, r[1]);
     tmem_ld_wait();
     float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    uint32_t pk[2][16];
 #pragma unroll
     for (int c8 = 0; c8 < 8; ++c8) {
         float p[8];
@@ -165,10 +166,13 @@ __device__ __forceinline__ float row_exp64(uint32_t scol, int key0, int L, int c
             p[e] = v;
             sm[e] += v;
         }
-        const uint4 w = make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
-                                   pack_bf16x2(p[6], p[7]));
-        st_shared_v4(prow + ((c8 ^ (i & 7)) << 4), w);
+        pk[c8 >> 2][(c8 & 3) * 4 + 0] = pack_bf16x2(p[0], p[1]);
+        pk[c8 >> 2][(c8 & 3) * 4 + 1] = pack_bf16x2(p[2], p[3]);
+        pk[c8 >> 2][(c8 & 3) * 4 + 2] = pack_bf16x2(p[4], p[5]);
+        pk[c8 >> 2][(c8 & 3) * 4 + 3] = pack_bf16x2(p[6], p[7]);
+        if ((c8 & 3) == 3) tmem_st_32x32b_x16(pcol + (c8 >> 2) * 16, pk[c8 >> 2]);
     }
+    tmem_st_wait();
     return ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
 }
 
@@ -181,9 +185,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     const int QK_BYTES = kp * 256;  // a gathered query tile or key block
-    const int ks = kp <= 96 ? 3 : 2;   // key/value stages
-    uint8_t* sP = smem;                                   // 32 KB (1024-aligned)
-    uint8_t* sV = sP + P_BYTES;                           // ks x 32 KB
+    const int ks = kp <= 112 ? 3 : 2;   // key/value stages
+    uint8_t* sV = smem;                                   // ks x 32 KB (1024-aligned)
     uint8_t* sQ = sV + ks * V_BYTES;                      // kp x 256
     uint8_t* sK = sQ + QK_BYTES;                          // ks x kp x 256
     int* sidx = reinterpret_cast<int*>(sK + ks * QK_BYTES);  // kp kept dims
@@ -246,10 +249,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         for (int j = pt; j < kp; j += kProdThreads) sidx[j] = j < k ? __ldg(S + j) : -1;
         asm volatile("bar.sync 1, %0;" ::"r"(kProdThreads));
         // the query tile: 128 tokens x 128 dims staged row-major in the (not yet
-        // used) P buffer with coalesced 16-byte copies, then the kp kept dims
-        // gathered from there into the MN-major operand, 8 tokens per chunk
+        // used) first V stage with coalesced 16-byte copies, then the kp kept
+        // dims gathered from there into the MN-major operand, 8 tokens per chunk
         const uint16_t* Qh = Q + ((size_t)b * Hq + h) * T * D;
-        const uint32_t qstage = smem_addr(sP);
+        const uint32_t qstage = smem_addr(sV);
         for (int it = pt; it < BQ * 16; it += kProdThreads) {
             const int tr = it >> 4, c16 = it & 15;
             const bool ok = t0 + tr < T;
@@ -257,7 +260,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
         cp_async_wait_all();
         asm volatile("bar.sync 1, %0;" ::"r"(kProdThreads));
-        const uint16_t* qs = reinterpret_cast<const uint16_t*>(sP);
+        const uint16_t* qs = reinterpret_cast<const uint16_t*>(sV);
         for (int it = pt; it < kp * 16; it += kProdThreads) {
             const int jr = it >> 4, c16 = it & 15;
             const int dim = sidx[jr];
@@ -269,6 +272,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             st_shared_v4(smem_addr(sQ) + swz(jr, c16, kp * 128), w);
         }
         fence_proxy_async_smem();
+        asm volatile("bar.sync 1, %0;" ::"r"(kProdThreads));  // staging read before V lands there
         mbar_arrive(smem_addr(&bars->q_full));
         const uint16_t* Kg = Kt + ((size_t)b * Hkv + g) * D * ldL;
         const int vplane = b * Hkv + g;
@@ -344,14 +348,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 ok = false;
                 break;
             }
-            fence_proxy_async_smem();  // P written by the softmax threads
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t pbase = smem_addr(sP), vbase = smem_addr(sV + sp * V_BYTES);
+                const uint32_t vbase = smem_addr(sV + sp * V_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < BKV / 16; ++kk)
-                    umma_f16(tmem + TM_O, smem_desc_sw128(pbase + (kk >> 2) * P_ATOM + (kk & 3) * 32, 16, 1024),
-                             smem_desc_sw128(vbase + kk * 2048, V_CHUNK, 1024), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_f16_tmem_a(tmem + TM_O, tmem + TM_P + kk * 8, smem_desc_sw128(vbase + kk * 2048, V_CHUNK, 1024),
+                                    idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(smem_addr(&bars->p_empty));
                 umma_commit(smem_addr(&bars->kv_empty[sp]));
             }
@@ -431,13 +434,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 tmem_st_wait();
             }
             m_use = m_new;
-            const uint32_t prow = smem_addr(sP) + half * P_ATOM + i * 128;
-            const float rs = full ? row_exp64<false>(scol, key0, L, causal, pos, scale_log2, neg_m, prow, i)
-                                  : row_exp64<true>(scol, key0, L, causal, pos, scale_log2, neg_m, prow, i);
+            const uint32_t pcol = tmem + lane_base + TM_P + half * 32;
+            const float rs = full ? row_exp64<false>(scol, key0, L, causal, pos, scale_log2, neg_m, pcol)
+                                  : row_exp64<true>(scol, key0, L, causal, pos, scale_log2, neg_m, pcol);
             tc_fence_before();
             mbar_arrive(smem_addr(&bars->s_empty[sb]));  // S_j fully read
             l_half = l_half * alpha + rs;
-            fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(smem_addr(&bars->p_full));
         }
@@ -482,8 +484,8 @@ __global__ void exp2_fma_kernel(const float* __restrict__ x, float* __restrict__
 }
 
 size_t attn_tc_smem_bytes(int kp) {
-    const int ks = kp <= 96 ? 3 : 2;
-    return 1024 + P_BYTES + (size_t)ks * V_BYTES + (size_t)(1 + ks) * kp * 256 + D * sizeof(int) + sizeof(Bars);
+    const int ks = kp <= 112 ? 3 : 2;
+    return 1024 + (size_t)ks * V_BYTES + (size_t)(1 + ks) * kp * 256 + D * sizeof(int) + sizeof(Bars);
 }
 
 }  // namespace
