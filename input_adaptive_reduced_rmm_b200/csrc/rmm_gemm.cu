@@ -75,7 +75,6 @@ constexpr int kRowsA = BK / (2 * kProducerWarps);  // X^T double-row copies per 
 static_assert(BK % (2 * kProducerWarps) == 0, "row copies must divide evenly over the producer warps");
 constexpr int kProducerThreads = 32 * kProducerWarps;
 constexpr int kEpilogueWarps = 4;
-constexpr int kFirstEpilogueWarp = kProducerWarps;
 constexpr int kMmaWarp = kProducerWarps + kEpilogueWarps;
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 
@@ -754,8 +753,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         for (int u = cluster_id; u < num_units; u += num_clusters) {
             const Unit ux = decode_unit(group, u, m_tiles, nkb);
             const TileCoord tc = ux.tc;
-            const int N = group.N[tc.p];
-            uint16_t* __restrict__ Y = group.Y[tc.p];
             if (!mbar_wait(smem_addr(&bars->tfull), acc_phase, status, abort_flag)) {
                 st_shared_cluster_u32(peer_abort, 1);
                 break;
