@@ -262,7 +262,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         asm volatile("bar.sync 1, %0;" ::"r"(kProdThreads));
         const uint16_t* qs = reinterpret_cast<const uint16_t*>(sV);
         for (int it = pt; it < kp * 16; it += kProdThreads) {
-            const int jr = it >> 4, c16 = it & 15;
+            // consecutive lanes take consecutive kept dims of one 8-token chunk:
+            // their reads fall in different banks (lanes on one dim and different
+            // chunks would all hit one bank: the staged rows are 256 B apart)
+            const int jr = it % kp, c16 = it / kp;
             const int dim = sidx[jr];
             uint16_t v[8];
 #pragma unroll
