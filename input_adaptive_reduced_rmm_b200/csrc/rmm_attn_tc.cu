@@ -16,11 +16,11 @@
 // the key block are MN-major (a kept dim is one row of 128 tokens / keys --
 // the d-major key cache makes each kept dim of a key block one contiguous
 // 256-byte segment); V blocks are MN-major (a key is one row of d values).
-// TMEM holds two S buffers (columns 0-127, 128-255), O (256-383) and P
-// (384-447): the softmax threads write P_j there, two bf16 keys per 32-bit
-// column, each thread its own row, and the P.V product reads it as its A
-// operand straight from tensor memory (K-major by definition), so P never
-// passes through shared memory.
+// TMEM holds two S buffers (columns 0-127, 128-255), O (256-383), P
+// (384-447) and the softmax warps' row exchange (448-453).  The softmax
+// threads write P_j there, two bf16 keys per 32-bit column, each thread its
+// own row, and the P.V product reads it as its A operand straight from tensor
+// memory (K-major by definition), so P never passes through shared memory.
 //
 // Warp roles (384 threads):
 //   0-7  softmax: warps q and q+4 own query rows 32q .. 32q+31 (their TMEM
@@ -35,7 +35,7 @@
 //        block the kp kept rows of K^T with 16-byte cp.async (zero-filled past
 //        the valid keys) and the 128 x 128 V tile with two TMA tile loads
 //        (a 3-D map over [head][key][dim]: keys past L read as zero), three
-//        stages (two when 128 kept dims leave no room).
+//        stages.
 // Every wait is bounded: on expiry the kernel records RMM_ERR_TIMEOUT, every
 // role leaves its loop, in-flight tensor-core work drains, TMEM is freed.
 #include <math.h>
@@ -50,7 +50,7 @@ namespace {
 constexpr int D = 128;
 constexpr int BQ = 128;   // query rows per CTA (= TMEM lanes)
 constexpr int BKV = 128;  // keys per block
-constexpr int KV_STAGES_MAX = 3;  // key/value stages: 3 when they fit with the static arrays (kp <= 112), else 2
+constexpr int KV_STAGES_MAX = 3;  // key/value stages (231 KB of shared memory at kp = 128)
 constexpr int kSoftmaxWarps = 8;  // two per TMEM lane quarter, each on 64 of the 128 columns
 constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
 constexpr int kMmaWarp = kSoftmaxWarps;
@@ -61,6 +61,9 @@ constexpr int V_CHUNK = BKV * 128;     // 64 dims x 128 key rows (bytes)
 constexpr int V_BYTES = 2 * V_CHUNK;   // 32 KB
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_P = 384;  // P: 128 keys as 64 packed columns
+// The two softmax warps of a lane quarter exchange row values through TMEM
+// columns TM_X .. TM_X+5: block maxima [block parity][half], then row sums [half].
+constexpr uint32_t TM_X = 448;
 constexpr float kRescaleLog2 = 8.0f;   // rescale O when a block max exceeds the reference by 2^8
 
 struct __align__(8) Bars {
@@ -185,15 +188,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     const int QK_BYTES = kp * 256;  // a gathered query tile or key block
-    const int ks = kp <= 112 ? 3 : 2;   // key/value stages
+    const int ks = KV_STAGES_MAX;   // key/value stages
     uint8_t* sV = smem;                                   // ks x 32 KB (1024-aligned)
     uint8_t* sQ = sV + ks * V_BYTES;                      // kp x 256
     uint8_t* sK = sQ + QK_BYTES;                          // ks x kp x 256
     int* sidx = reinterpret_cast<int*>(sK + ks * QK_BYTES);  // kp kept dims
     Bars* bars = reinterpret_cast<Bars*>(sidx + D);
     volatile int* abort_flag = &bars->abort_flag;
-    __shared__ float red_max[2][2][BQ];  // [block parity][half][row]: the halves' row maxima
-    __shared__ float red_sum[2][BQ];     // [half][row]: the halves' row sums at the end
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_tiles = (T + BQ - 1) / BQ;
@@ -377,7 +378,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         // ------------------------------------------------------------ softmax + epilogue
         // warps q and q + 4 share TMEM lanes 32q .. 32q+31 (query rows) and take
         // columns 0-63 and 64-127 of S, of P (one atom each) and of O; the row max
-        // is combined through shared memory with one barrier per pair and block,
+        // is combined through TMEM (columns TM_X..) with one barrier per pair and block,
         // the row sums are kept per half and added at the end
         const int quarter = warp & 3, half = warp >> 2;
         const int i = quarter * 32 + lane;  // query row inside the tile = TMEM lane
@@ -404,14 +405,19 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint32_t scol = tmem + lane_base + TM_S0 + sb * BKV + half * 64;
             const float m_mine = full ? row_max64<false>(scol, key0, L, causal, pos)
                                       : row_max64<true>(scol, key0, L, causal, pos);
-            red_max[j & 1][half][i] = m_mine;
+            tmem_st_32x32b_x1(tmem + lane_base + TM_X + (j & 1) * 2 + half, __float_as_uint(m_mine));
+            tmem_st_wait();
+            tc_fence_before();
             // meet the partner warp (bounded, like every wait here)
             mbar_arrive(pair_mb);
             if (!__all_sync(0xffffffffu, mbar_wait(pair_mb, (uint32_t)(pair_phase++) & 1u, status, abort_flag))) {
                 ok = false;
                 break;
             }
-            const float m_blk = fmaxf(m_mine, red_max[j & 1][half ^ 1][i]) * scale_log2;
+            tc_fence_after();
+            const float m_blk = fmaxf(m_mine, __uint_as_float(tmem_ld_32x32b_x1(
+                                                  tmem + lane_base + TM_X + (j & 1) * 2 + (half ^ 1)))) *
+                                scale_log2;
             const bool resc = m_blk > m_use + kRescaleLog2;
             const float m_new = resc ? m_blk : m_use;
             const float alpha = resc ? exp2f(m_use - m_new) : 1.0f;  // exp2(-inf) = 0 on the first block
@@ -448,12 +454,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
         const bool done = ok && __all_sync(0xffffffffu, mbar_wait(smem_addr(&bars->o_full), 0, status, abort_flag));
         // the two halves' row sums
-        red_sum[half][i] = l_half;
+        tmem_st_32x32b_x1(tmem + lane_base + TM_X + 4 + half, __float_as_uint(l_half));
+        tmem_st_wait();
+        tc_fence_before();
         mbar_arrive(pair_mb);
         const bool met = __all_sync(0xffffffffu, mbar_wait(pair_mb, (uint32_t)pair_phase & 1u, status, abort_flag));
         if (done && met) {
             tc_fence_after();
-            const float inv = 1.0f / (red_sum[0][i] + red_sum[1][i]);
+            const float l_other = __uint_as_float(tmem_ld_32x32b_x1(tmem + lane_base + TM_X + 4 + (half ^ 1)));
+            const float inv = 1.0f / (half == 0 ? l_half + l_other : l_other + l_half);  // half 0's sum first
             uint16_t* orow = O + (((size_t)b * Hq + h) * T + (t < T ? t : 0)) * D + half * 64;
 #pragma unroll 1
             for (int q = 0; q < 2; ++q) {
@@ -487,7 +496,7 @@ __global__ void exp2_fma_kernel(const float* __restrict__ x, float* __restrict__
 }
 
 size_t attn_tc_smem_bytes(int kp) {
-    const int ks = kp <= 112 ? 3 : 2;
+    const int ks = KV_STAGES_MAX;
     return 1024 + (size_t)ks * V_BYTES + (size_t)(1 + ks) * kp * 256 + D * sizeof(int) + sizeof(Bars);
 }
 
